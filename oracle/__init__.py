@@ -1,0 +1,197 @@
+"""CPU oracle for the FMDQ differential linear layer -- TEST INFRASTRUCTURE.
+
+Plain, slow and exact restatement of DSTAR's fine-grained mixed-precision
+differential quantization (section 3.1, Eqs. 1-5; computation-flow steps 1-5
+of Fig. 5) and of the MPU epilogue (section 4.2 inverse quantization and
+accumulation units; section 4.3 reverse differential).  Only the tests, the
+smoke check and the CPU-baseline leg of the benchmark may import this module.
+It shares no code with the CUDA library and never calls it.
+
+Every function takes and returns numpy arrays.  Floating-point inputs are fp32
+arrays; bf16 data is widened exactly with :func:`bf16_to_f32` first.
+
+Parity status of each function (what pins it, see tests/test_oracle_pins.py):
+  quantize      -- worked PoT example (section 3.1, step 1), boundary cases,
+                   rounding ties, closed form under forced 8/2 bits, slice
+                   reassembly over every code, layout invariants.
+  acc_slices    -- the value-70 example of section 3.1 step 2, equality with
+                   acc_direct, the non-identity without shifts.
+  acc_direct    -- equality with a numpy int64 matmul of the shifted codes.
+  epilogue_f32  -- bounded against epilogue_f64 and against the dense fp64
+                   product within the quantization error bound.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+TILE = 16
+ST_NONFINITE = 1
+ST_RANGE = 2
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        i64 = ctypes.c_int64
+        ci = ctypes.c_int
+        lib.fmdq_orc_quantize.argtypes = [P, P, i64, i64, ci, ci, ci] + [P] * 11
+        lib.fmdq_orc_quantize.restype = ci
+        lib.fmdq_orc_acc_slices.argtypes = [i64, i64, i64] + [P] * 10
+        lib.fmdq_orc_acc_slices.restype = None
+        lib.fmdq_orc_acc_direct.argtypes = [i64, i64, i64] + [P] * 6
+        lib.fmdq_orc_acc_direct.restype = None
+        lib.fmdq_orc_epilogue_f32.argtypes = [i64, i64, P, P, ci, P, P, ci, P, P]
+        lib.fmdq_orc_epilogue_f32.restype = None
+        lib.fmdq_orc_epilogue_f64.argtypes = [i64, i64, P, P, ci, P, P, P, P]
+        lib.fmdq_orc_epilogue_f64.restype = None
+        lib.fmdq_orc_bf16_to_f32.argtypes = [P, i64, P]
+        lib.fmdq_orc_f32_to_bf16.argtypes = [P, i64, P]
+        lib.fmdq_orc_slice_digit.argtypes = [ctypes.c_uint32, ci, ci]
+        lib.fmdq_orc_slice_digit.restype = ci
+        lib.fmdq_orc_pot_max.restype = ci
+        _lib = lib
+    return _lib
+
+
+def _p(a: np.ndarray | None):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def pot_max() -> int:
+    return _load().fmdq_orc_pot_max()
+
+
+def bf16_to_f32(h: np.ndarray) -> np.ndarray:
+    h = np.ascontiguousarray(h, dtype=np.uint16)
+    out = np.empty(h.shape, np.float32)
+    _load().fmdq_orc_bf16_to_f32(_p(h), h.size, _p(out))
+    return out
+
+
+def f32_to_bf16(f: np.ndarray) -> np.ndarray:
+    f = np.ascontiguousarray(f, dtype=np.float32)
+    out = np.empty(f.shape, np.uint16)
+    _load().fmdq_orc_f32_to_bf16(_p(f), f.size, _p(out))
+    return out
+
+
+def slice_digit(field: int, j: int, b: int) -> int:
+    return _load().fmdq_orc_slice_digit(field, j, b)
+
+
+class Quantized:
+    """Everything steps 1-4 produce for one call."""
+
+    def __init__(self, M, K):
+        T = M // TILE
+        cap = 4 * K
+        self.M, self.K, self.T, self.cap = M, K, T, cap
+        self.codes = np.zeros((M, K), np.int8)
+        self.bits = np.zeros((T, K), np.int8)
+        self.fpot = np.zeros((T, K), np.int8)
+        self.pot = np.zeros((T, K), np.int16)
+        self.g_ref = np.zeros(T, np.int32)
+        self.count = np.zeros(T, np.int32)
+        self.rec_word = np.zeros((T, cap), np.uint32)
+        self.rec_k = np.zeros((T, cap), np.uint16)
+        self.rec_tag = np.zeros((T, cap), np.int8)
+        self.rec_j = np.zeros((T, cap), np.uint8)
+        self.shift = np.zeros((T, cap), np.int8)
+        self.status = 0
+
+
+def quantize(x_t: np.ndarray, x_prev: np.ndarray, lb: int, t0: int = 0, force_bits: int = 0) -> Quantized:
+    """Steps 1-4 of the computation flow for fp32 inputs [M x K], base = 2^lb."""
+    x_t = np.ascontiguousarray(x_t, np.float32)
+    x_prev = np.ascontiguousarray(x_prev, np.float32)
+    M, K = x_t.shape
+    assert x_prev.shape == (M, K) and M % TILE == 0
+    q = Quantized(M, K)
+    q.status = _load().fmdq_orc_quantize(
+        _p(x_t), _p(x_prev), M, K, lb, t0, force_bits, _p(q.codes), _p(q.bits), _p(q.fpot), _p(q.pot),
+        _p(q.g_ref), _p(q.count), _p(q.rec_word), _p(q.rec_k), _p(q.rec_tag), _p(q.rec_j), _p(q.shift))
+    return q
+
+
+def _mask(T, tiles):
+    if tiles is None:
+        return None
+    m = np.zeros(T, np.uint8)
+    m[np.asarray(tiles, dtype=np.int64)] = 1
+    return m
+
+
+def acc_slices(q: Quantized, w_q: np.ndarray, tiles=None) -> np.ndarray:
+    """Step 5: shift-aligned accumulation over the encoded stream (int64 [M x N])."""
+    w_q = np.ascontiguousarray(w_q, np.int8)
+    N, K = w_q.shape
+    assert K == q.K
+    acc = np.zeros((q.M, N), np.int64)
+    _load().fmdq_orc_acc_slices(q.M, q.K, N, _p(q.rec_word), _p(q.rec_k), _p(q.rec_tag), _p(q.rec_j),
+                                _p(q.count), _p(q.bits), _p(q.g_ref), _p(w_q), _p(_mask(q.T, tiles)),
+                                _p(acc))
+    return acc
+
+
+def acc_direct(q: Quantized, w_q: np.ndarray, tiles=None) -> np.ndarray:
+    """The accumulator by its definition, sum_k code * 2^(g_ref - FPoT) * w (int64 [M x N])."""
+    w_q = np.ascontiguousarray(w_q, np.int8)
+    N, K = w_q.shape
+    assert K == q.K
+    acc = np.zeros((q.M, N), np.int64)
+    _load().fmdq_orc_acc_direct(q.M, q.K, N, _p(q.codes), _p(q.fpot), _p(q.g_ref), _p(w_q),
+                                _p(_mask(q.T, tiles)), _p(acc))
+    return acc
+
+
+def epilogue_f32(acc: np.ndarray, g_ref: np.ndarray, lb: int, w_scale: np.ndarray, y_prev: np.ndarray,
+                 out_bf16: bool, tiles=None) -> np.ndarray:
+    """Y_t = Y_{t-1} + dequant(acc) in the fixed fp32 order; fp32 array of the output values."""
+    acc = np.ascontiguousarray(acc, np.int64)
+    M, N = acc.shape
+    w_scale = np.ascontiguousarray(w_scale, np.float32)
+    y_prev = np.ascontiguousarray(y_prev, np.float32)
+    g_ref = np.ascontiguousarray(g_ref, np.int32)
+    out = np.zeros((M, N), np.float32)
+    _load().fmdq_orc_epilogue_f32(M, N, _p(acc), _p(g_ref), lb, _p(w_scale), _p(y_prev), int(out_bf16),
+                                  _p(_mask(M // TILE, tiles)), _p(out))
+    return out
+
+
+def epilogue_f64(acc: np.ndarray, g_ref: np.ndarray, lb: int, w_scale: np.ndarray, y_prev: np.ndarray,
+                 tiles=None) -> np.ndarray:
+    acc = np.ascontiguousarray(acc, np.int64)
+    M, N = acc.shape
+    w_scale = np.ascontiguousarray(w_scale, np.float32)
+    y_prev = np.ascontiguousarray(y_prev, np.float32)
+    g_ref = np.ascontiguousarray(g_ref, np.int32)
+    out = np.zeros((M, N), np.float64)
+    _load().fmdq_orc_epilogue_f64(M, N, _p(acc), _p(g_ref), lb, _p(w_scale), _p(y_prev),
+                                  _p(_mask(M // TILE, tiles)), _p(out))
+    return out
+
+
+def linear(x_t, x_prev, y_prev, w_q, w_scale, lb, t0=0, force_bits=0, out_bf16=True, tiles=None,
+           path="direct"):
+    """The whole differential linear: returns (Quantized, acc, y_out)."""
+    q = quantize(x_t, x_prev, lb, t0, force_bits)
+    acc = acc_direct(q, w_q, tiles) if path == "direct" else acc_slices(q, w_q, tiles)
+    y = epilogue_f32(acc, q.g_ref, lb, w_scale, y_prev, out_bf16, tiles)
+    return q, acc, y
+
+
+def n_threads() -> int:
+    return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
