@@ -1,0 +1,507 @@
+// K2+K3: the shift-aligned slice GEMM on tcgen05 tensor cores with the fused
+// dequantize / reverse-differential epilogue (DSTAR section 3.1 step 5,
+// section 4.2 "Design of MPU" inverse quantization and accumulation units,
+// section 4.3 "Operator Mapping": cached outputs added to the partial sum).
+//
+// The paper's MPU streams 2-bit slices in ascending FPoT order and shifts the
+// partial sum by the FPoT difference between groups.  Here every shift is
+// folded into the operand before the contraction: slice j of channel k in
+// tile T enters with weight 2^(g_ref(T) - FPoT(T,k) + 2j), so the sum of a
+// channel's slices is v = q * 2^(g_ref - FPoT), an exact integer that the
+// quantizer splits into int8 planes v = A0 + 256 A1.  The tensor cores then
+// compute D_p = A_p W^T (int8 x int8 -> int32, exact), and the epilogue forms
+// acc = D_0 + 256 D_1 in 64-bit integers -- bit for bit the accumulator that
+// ascending-FPoT shift-and-add produces -- then
+//   Y_t = Y_{t-1} + ((float)acc * 2^(-lb - g_ref)) * w_scale[n]   (fp32, in this order).
+//
+// Structure (one CTA per SM, persistent over 128 x BN output tiles):
+//   warp 0      TMA producer: A0 chunk (128 x 128 B), W chunk (BN x 128 B) and,
+//               for K chunks where plane 1 is nonzero, the A1 chunk
+//   warp 1      TMEM allocator and MMA issuer (one thread): M=128, N=BN, K=32
+//   warps 2..5  epilogue: tcgen05.ld of their 32 TMEM lanes (= rows), y_prev
+//               loads issued before the accumulator is ready, fp32 epilogue,
+//               bf16/fp32 stores of Y_t to y_out (and y_prev when distinct)
+// TMEM holds 512 columns = 512/BN accumulator slots; a one-plane tile takes one
+// slot, a two-plane tile two, so the epilogue of one tile overlaps the MMAs
+// of the next.  Tiles whose planes do not fit in two int8 planes are left to
+// the slice-stream kernel below.  Every wait is bounded (wait_parity).
+#include <cuda_bf16.h>
+
+#include "fmdq_device.cuh"
+
+namespace fmdq {
+
+namespace {
+
+constexpr int kGThreads = 192;
+constexpr int kA0Bytes = kBlockM * kChunkK;  // 16 KB
+constexpr int kA1Bufs = 2;
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int kStages = BN == 256 ? 4 : 6;
+  static constexpr int kWBytes = BN * kChunkK;
+  static constexpr int kStageBytes = kA0Bytes + kWBytes;
+  static constexpr int kSlots = 512 / BN;
+  static constexpr int kGroups = BN / 32;
+  // shared memory map (offsets from a 1024-aligned base)
+  static constexpr int kOffA1 = kStages * kStageBytes;
+  static constexpr int kOffBar = kOffA1 + kA1Bufs * kA0Bytes;
+  static constexpr int kNumBars = 2 * kStages + kA1Bufs + 2 * kSlots + 1;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kBytes = kOffMisc + 64 + 1024;  // + alignment slack
+};
+
+struct BlockInfo {
+  int nplanes;  // 0: skip (all tiles of the row block go to the slice kernel), 1 or 2
+  uint32_t mask[2];
+};
+
+// Identical on every role: what the quantizer decided for this 128-row block.
+__device__ __forceinline__ BlockInfo block_info(const GemmParams& p, int rb) {
+  BlockInfo bi;
+  bi.mask[0] = bi.mask[1] = 0;
+  const int T = (int)(p.M / kTile);
+  int np = 0;
+  bool any = false;
+  for (int t = rb * 8; t < min(rb * 8 + 8, T); ++t) {
+    const int pl = p.planes[t];
+    if (pl <= 2) {
+      any = true;
+      np = max(np, pl);
+    }
+    for (int w = 0; w < (int)p.mask_words && w < 2; ++w) bi.mask[w] |= p.mask1[(int64_t)t * p.mask_words + w];
+  }
+  bi.nplanes = !any ? 0 : (np == 2 && (bi.mask[0] | bi.mask[1])) ? 2 : 1;
+  return bi;
+}
+
+__device__ __forceinline__ bool chunk_has_plane1(const BlockInfo& bi, int c) {
+  return bi.nplanes == 2 && ((bi.mask[c >> 5] >> (c & 31)) & 1u);
+}
+
+__device__ __forceinline__ float exp2_exact(int e) { return __int_as_float((127 + e) << 23); }
+
+template <bool OUT_BF16>
+struct OutT;
+template <>
+struct OutT<true> {
+  using T = __nv_bfloat16;
+};
+template <>
+struct OutT<false> {
+  using T = float;
+};
+
+// y = y_prev + ((float)acc * p2) * ws  -- fp32, no contraction
+__device__ __forceinline__ float epi(int64_t acc, bool wide, float p2, float ws, float yp) {
+  const float a = wide ? __ll2float_rn(acc) : __int2float_rn((int)acc);
+  return __fadd_rn(yp, __fmul_rn(__fmul_rn(a, p2), ws));
+}
+
+}  // namespace
+
+size_t gemm_smem_bytes(int bn) { return bn == 256 ? GemmCfg<256>::kBytes : GemmCfg<128>::kBytes; }
+
+template <int BN, bool OUT_BF16>
+__global__ void __launch_bounds__(kGThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CUtensorMap tm_a1,
+                const __grid_constant__ CUtensorMap tm_w, const GemmParams p) {
+  using C = GemmCfg<BN>;
+  using TOut = typename OutT<OUT_BF16>::T;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* full = bars;                       // [kStages] TMA -> MMA
+  uint64_t* empty = full + C::kStages;         // [kStages] MMA -> TMA
+  uint64_t* a1_empty = empty + C::kStages;     // [kA1Bufs] MMA -> TMA
+  uint64_t* tm_full = a1_empty + kA1Bufs;      // [kSlots] MMA -> epilogue
+  uint64_t* tm_empty = tm_full + C::kSlots;    // [kSlots] epilogue -> MMA
+  uint64_t* drain = tm_empty + C::kSlots;      // MMA completion at exit
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int num_tiles = p.tiles_m * p.tiles_n;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::kStages; ++i) mbar_init(&full[i], 1), mbar_init(&empty[i], 1);
+    for (int i = 0; i < kA1Bufs; ++i) mbar_init(&a1_empty[i], 1);
+    for (int i = 0; i < C::kSlots; ++i) mbar_init(&tm_full[i], 1), mbar_init(&tm_empty[i], 4);
+    mbar_init(drain, 1);
+    *s_abort = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tm_a0);
+    prefetch_tmap(&tm_a1);
+    prefetch_tmap(&tm_w);
+  }
+  if (warp == 1) {
+    tmem_alloc(s_tmem, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *s_tmem;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (elect_one()) {
+      uint32_t it = 0, a1_it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const int rb = tile / p.tiles_n, nb = tile % p.tiles_n;
+        const BlockInfo bi = block_info(p, rb);
+        if (bi.nplanes == 0) continue;
+        for (int c = 0; c < p.num_chunks; ++c, ++it) {
+          const int s = it % C::kStages;
+          if (!wait_parity(&empty[s], ((it / C::kStages) & 1) ^ 1, s_abort, p.status, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          const bool use1 = chunk_has_plane1(bi, c);
+          if (use1 && !wait_parity(&a1_empty[a1_it % kA1Bufs], ((a1_it / kA1Bufs) & 1) ^ 1, s_abort, p.status,
+                                   kWaitLimitNs)) {
+            // nothing was loaded into this stage; the MMA side leaves on the abort flag
+            ok = false;
+            break;
+          }
+          uint8_t* a0 = smem + s * C::kStageBytes;
+          uint8_t* wb = a0 + kA0Bytes;
+          mbar_arrive_expect_tx(&full[s], C::kStageBytes + (use1 ? kA0Bytes : 0));
+          tma_load_2d(a0, &tm_a0, &full[s], c * kChunkK, rb * kBlockM);
+          tma_load_2d(wb, &tm_w, &full[s], c * kChunkK, nb * BN);
+          if (use1) {
+            uint8_t* a1 = smem + C::kOffA1 + (a1_it % kA1Bufs) * kA0Bytes;
+            tma_load_2d(a1, &tm_a1, &full[s], c * kChunkK, rb * kBlockM);
+            ++a1_it;
+          }
+        }
+      }
+      // drain: every stage filled must have landed before the block can exit
+      const uint32_t first = it > (uint32_t)C::kStages ? it - C::kStages : 0;
+      for (uint32_t j = first; j < it; ++j)
+        wait_parity(&full[j % C::kStages], (j / C::kStages) & 1, s_abort, p.status, kWaitLimitNs, true);
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------------- MMA
+    if (elect_one()) {
+      constexpr uint32_t idesc = idesc_i8(BN);
+      uint32_t it = 0, a1_it = 0, slot_it = 0;
+      bool ok = true, issued = false;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const int rb = tile / p.tiles_n;
+        const BlockInfo bi = block_info(p, rb);
+        if (bi.nplanes == 0) continue;
+        // acquire accumulator slots
+        uint32_t slot[2];
+        for (int q = 0; q < bi.nplanes && ok; ++q) {
+          const uint32_t si = slot_it + q;
+          slot[q] = si % C::kSlots;
+          ok = wait_parity(&tm_empty[slot[q]], ((si / C::kSlots) & 1) ^ 1, s_abort, p.status, kWaitLimitNs);
+        }
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + slot[0] * BN;
+        const uint32_t d1 = tmem_base + (bi.nplanes == 2 ? slot[1] : slot[0]) * BN;
+        bool first1 = true;
+        for (int c = 0; c < p.num_chunks; ++c, ++it) {
+          const int s = it % C::kStages;
+          if (!wait_parity(&full[s], (it / C::kStages) & 1, s_abort, p.status, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t da = smem_desc_k_sw128(smem + s * C::kStageBytes);
+          const uint64_t dw = smem_desc_k_sw128(smem + s * C::kStageBytes + kA0Bytes);
+#pragma unroll
+          for (int kk = 0; kk < kChunkK / 32; ++kk)
+            mma_i8(d0, da + 2 * kk, dw + 2 * kk, idesc, (c > 0 || kk > 0) ? 1u : 0u);
+          if (chunk_has_plane1(bi, c)) {
+            const uint64_t d_a1 = smem_desc_k_sw128(smem + C::kOffA1 + (a1_it % kA1Bufs) * kA0Bytes);
+#pragma unroll
+            for (int kk = 0; kk < kChunkK / 32; ++kk)
+              mma_i8(d1, d_a1 + 2 * kk, dw + 2 * kk, idesc, (!first1 || kk > 0) ? 1u : 0u);
+            first1 = false;
+            mma_commit(&a1_empty[a1_it % kA1Bufs]);
+            ++a1_it;
+          }
+          mma_commit(&empty[s]);
+          issued = true;
+        }
+        if (!ok) break;
+        for (int q = 0; q < bi.nplanes; ++q) mma_commit(&tm_full[slot[q]]);
+        slot_it += bi.nplanes;
+      }
+      // drain: all MMAs this thread issued complete before TMEM and SMEM go away
+      if (issued) {
+        mma_commit(drain);
+        wait_parity(drain, 0, s_abort, p.status, kWaitLimitNs, true);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31 are this warp's
+    uint32_t slot_it = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      const int rb = tile / p.tiles_n, nb = tile % p.tiles_n;
+      const BlockInfo bi = block_info(p, rb);
+      if (bi.nplanes == 0) continue;
+      const int64_t row = (int64_t)rb * kBlockM + quarter * 32 + lane;
+      const bool in_range = row < p.M;
+      const int t = (int)(row / kTile);
+      const int pl = in_range ? p.planes[t] : 3;
+      const bool row_ok = in_range && pl <= 2;
+      const float p2 = row_ok ? exp2_exact(-p.lb - p.g_ref[t]) : 0.f;
+      const int64_t n_base = (int64_t)nb * BN;
+      const TOut* yp_row = reinterpret_cast<const TOut*>(p.y_prev) + (row_ok ? row : 0) * p.ld_yp;
+
+      // issue the y_prev loads of the whole tile before the accumulator is ready
+      constexpr int kVecPerGroup = 32 * (int)sizeof(TOut) / 16;  // 16-byte vectors per 32 columns
+      constexpr int kPre = OUT_BF16 ? C::kGroups : 1;             // groups prefetched
+      uint4 ypv[kPre][kVecPerGroup];
+      if constexpr (OUT_BF16) {
+#pragma unroll
+        for (int g = 0; g < kPre; ++g)
+#pragma unroll
+          for (int v = 0; v < kVecPerGroup; ++v) {
+            const int64_t n = n_base + g * 32 + v * (16 / (int)sizeof(TOut));
+            ypv[g][v] = (row_ok && n < p.N) ? __ldg(reinterpret_cast<const uint4*>(yp_row + n)) : make_uint4(0, 0, 0, 0);
+          }
+      }
+
+      uint32_t slot[2];
+      int ok = 1;
+      for (int q = 0; q < bi.nplanes; ++q) {
+        const uint32_t si = slot_it + q;
+        slot[q] = si % C::kSlots;
+        // one lane polls; the warp follows its verdict (tcgen05.ld needs the whole warp)
+        if (lane == 0 && ok)
+          ok = wait_parity(&tm_full[slot[q]], (si / C::kSlots) & 1, s_abort, p.status, kWaitLimitNs) ? 1 : 0;
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+      const uint32_t t0 = tmem_base + lane_off + slot[0] * BN;
+      const uint32_t t1 = tmem_base + lane_off + (bi.nplanes == 2 ? slot[1] : slot[0]) * BN;
+
+#pragma unroll
+      for (int g = 0; g < C::kGroups; ++g) {
+        uint32_t d0[32], d1[32];
+        tmem_ld32(t0 + g * 32, d0);
+        if (bi.nplanes == 2) tmem_ld32(t1 + g * 32, d1);
+        tmem_ld_wait();
+        const int64_t n0 = n_base + g * 32;
+        uint4 yv[kVecPerGroup];
+        if constexpr (OUT_BF16) {
+#pragma unroll
+          for (int v = 0; v < kVecPerGroup; ++v) yv[v] = ypv[g][v];
+        } else {
+#pragma unroll
+          for (int v = 0; v < kVecPerGroup; ++v) {
+            const int64_t n = n0 + v * 4;
+            yv[v] = (row_ok && n < p.N) ? __ldg(reinterpret_cast<const uint4*>(yp_row + n)) : make_uint4(0, 0, 0, 0);
+          }
+        }
+        if (row_ok && n0 < p.N) {
+          const bool wide = pl == 2;
+          float y[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int64_t acc = wide ? (int64_t)(int32_t)d0[i] + (int64_t)(int32_t)d1[i] * 256 : (int64_t)(int32_t)d0[i];
+            float ypf;
+            if constexpr (OUT_BF16) {
+              const uint32_t w = reinterpret_cast<const uint32_t*>(yv)[i >> 1];
+              ypf = __uint_as_float((i & 1) ? (w & 0xFFFF0000u) : (w << 16));
+            } else {
+              ypf = __uint_as_float(reinterpret_cast<const uint32_t*>(yv)[i]);
+            }
+            const float ws = (n0 + i < p.N) ? __ldg(p.w_scale + n0 + i) : 0.f;
+            y[i] = epi(acc, wide, p2, ws, ypf);
+            if (p.debug_acc && n0 + i < p.N) p.debug_acc[row * p.N + n0 + i] = acc;
+          }
+          const int64_t nv_rem = (p.N - n0) * (int64_t)sizeof(TOut) / 16;
+          const int nv = nv_rem < kVecPerGroup ? (int)nv_rem : kVecPerGroup;
+          uint4 ov[kVecPerGroup];
+          if constexpr (OUT_BF16) {
+#pragma unroll
+            for (int v = 0; v < kVecPerGroup; ++v) {
+              uint32_t w[4];
+#pragma unroll
+              for (int h = 0; h < 4; ++h) {
+                const __nv_bfloat162 b2 = __floats2bfloat162_rn(y[v * 8 + 2 * h], y[v * 8 + 2 * h + 1]);
+                w[h] = *reinterpret_cast<const uint32_t*>(&b2);
+              }
+              ov[v] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+          } else {
+#pragma unroll
+            for (int v = 0; v < kVecPerGroup; ++v)
+              ov[v] = make_uint4(__float_as_uint(y[4 * v]), __float_as_uint(y[4 * v + 1]), __float_as_uint(y[4 * v + 2]),
+                                 __float_as_uint(y[4 * v + 3]));
+          }
+          TOut* yo = reinterpret_cast<TOut*>(p.y_out) + row * p.ld_yo + n0;
+          TOut* yq = reinterpret_cast<TOut*>(p.y_prev) + row * p.ld_yp + n0;
+#pragma unroll
+          for (int v = 0; v < kVecPerGroup; ++v) {
+            if (v < nv) {
+              reinterpret_cast<uint4*>(yo)[v] = ov[v];
+              if (p.y_distinct) reinterpret_cast<uint4*>(yq)[v] = ov[v];
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0)
+        for (int q = 0; q < bi.nplanes; ++q) mbar_arrive(&tm_empty[slot[q]]);
+      slot_it += bi.nplanes;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Slice-stream kernel: the paper's accumulation order literally.  One block
+// per (tile, 256 output columns); every thread owns one output column and
+// the 16 tokens of the tile.  It walks the tile's encoded stream in order:
+// when the FPoT changes it shifts the 16 running sums left by the difference,
+// then adds digit x w[n][k] (section 3.1 step 5, Fig. 6).  The sums end in
+// units of the last FPoT and are shifted to g_ref, then the same fp32
+// epilogue as the tensor-core kernel is applied.  Used for tiles whose
+// shift-folded operands need more than two int8 planes, and for every tile
+// under DSTAR_FLAG_SLICE_PATH.
+// ---------------------------------------------------------------------------
+template <bool OUT_BF16>
+__global__ void __launch_bounds__(256) slice_gemm_kernel(const SliceParams p) {
+  using TOut = typename OutT<OUT_BF16>::T;
+  __shared__ uint2 s_rec[256];
+  extern __shared__ int8_t s_bits[];  // [K]
+  const int64_t T = p.M / kTile;
+  const int64_t nblk = (p.N + 255) / 256;
+  for (int64_t item = blockIdx.x; item < T * nblk; item += gridDim.x) {
+    const int64_t t = item / nblk;
+    const int64_t n = (item % nblk) * 256 + threadIdx.x;
+    if (!p.all_tiles && p.planes[t] <= 2) continue;  // uniform across the block
+    __syncthreads();
+    for (int64_t k = threadIdx.x; k < p.K; k += 256) s_bits[k] = p.bits[t * p.K + k];
+    const int cnt = p.count[t];
+    int64_t acc[kTile];
+#pragma unroll
+    for (int i = 0; i < kTile; ++i) acc[i] = 0;
+    int prev = 0;
+    for (int r0 = 0; r0 < cnt; r0 += 256) {
+      __syncthreads();
+      if (r0 + (int)threadIdx.x < cnt) s_rec[threadIdx.x] = p.records[t * p.record_cap + r0 + threadIdx.x];
+      __syncthreads();
+      const int rn = min(256, cnt - r0);
+      for (int r = 0; r < rn; ++r) {
+        const uint2 rec = s_rec[r];
+        const int k = (int)(rec.y & 0xFFFFu);
+        const int tag = (int)(int8_t)((rec.y >> 16) & 0xFFu);
+        const int j = (int)(rec.y >> 24);
+        if (r0 + r > 0 && tag != prev) {
+          const int sh = tag - prev;
+#pragma unroll
+          for (int i = 0; i < kTile; ++i) acc[i] *= ((int64_t)1 << sh);
+        }
+        prev = tag;
+        const int top = (j == (s_bits[k] >> 1) - 1);
+        const int64_t w = (n < p.N) ? (int64_t)p.w_q[n * p.ld_w + k] : 0;
+#pragma unroll
+        for (int i = 0; i < kTile; ++i) {
+          int d = (int)((rec.x >> (2 * i)) & 3u);
+          if (top && d >= 2) d -= 4;
+          acc[i] += (int64_t)d * w;
+        }
+      }
+    }
+    if (cnt > 0 && p.g_ref[t] != prev) {
+      const int sh = p.g_ref[t] - prev;
+#pragma unroll
+      for (int i = 0; i < kTile; ++i) acc[i] *= ((int64_t)1 << sh);
+    }
+    if (n < p.N) {
+      const float p2 = exp2_exact(-p.lb - p.g_ref[t]);
+      const float ws = p.w_scale[n];
+#pragma unroll
+      for (int i = 0; i < kTile; ++i) {
+        const int64_t row = t * kTile + i;
+        TOut* yp = reinterpret_cast<TOut*>(p.y_prev) + row * p.ld_yp + n;
+        TOut* yo = reinterpret_cast<TOut*>(p.y_out) + row * p.ld_yo + n;
+        float ypf;
+        if constexpr (OUT_BF16) ypf = __bfloat162float(*yp);
+        else ypf = *yp;
+        const float y = epi(acc[i], true, p2, ws, ypf);
+        TOut o;
+        if constexpr (OUT_BF16) o = __float2bfloat16_rn(y);
+        else o = y;
+        *yo = o;
+        if (p.y_distinct) *yp = o;
+        if (p.debug_acc) p.debug_acc[row * p.N + n] = acc[i];
+      }
+    }
+  }
+}
+
+// Self-test of the bounded wait: one thread waits on a barrier that nothing
+// completes; the wait must give up after limit_us and record TIMEOUT.
+__global__ void selftest_wait_kernel(uint32_t* status, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+    wait_parity(&bar, 0, &abort_flag, status, limit_ns);
+  }
+}
+
+template <int BN, bool BF>
+static int launch_gemm_t(const GemmParams& p, const void* a0, const void* a1, const void* w, int num_sms,
+                         void* stream) {
+  const int tiles = p.tiles_m * p.tiles_n;
+  const int grid = tiles < num_sms ? tiles : num_sms;
+  if (grid == 0) return 0;
+  const int smem = GemmCfg<BN>::kBytes;
+  cudaError_t e = cudaFuncSetAttribute(gemm_kernel<BN, BF>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return (int)e;
+  gemm_kernel<BN, BF><<<grid, kGThreads, smem, (cudaStream_t)stream>>>(
+      *static_cast<const CUtensorMap*>(a0), *static_cast<const CUtensorMap*>(a1),
+      *static_cast<const CUtensorMap*>(w), p);
+  return (int)cudaGetLastError();
+}
+
+int launch_gemm(const GemmParams& p, const void* a0, const void* a1, const void* w, int bn, int out_bf16,
+                int num_sms, void* stream) {
+  if (bn == 256) return out_bf16 ? launch_gemm_t<256, true>(p, a0, a1, w, num_sms, stream)
+                                 : launch_gemm_t<256, false>(p, a0, a1, w, num_sms, stream);
+  return out_bf16 ? launch_gemm_t<128, true>(p, a0, a1, w, num_sms, stream)
+                  : launch_gemm_t<128, false>(p, a0, a1, w, num_sms, stream);
+}
+
+int launch_slice_gemm(const SliceParams& p, int out_bf16, int num_sms, void* stream) {
+  const int64_t T = p.M / kTile;
+  const int64_t items = T * ((p.N + 255) / 256);
+  if (items == 0) return 0;
+  const int64_t grid = items < 4LL * num_sms ? items : 4LL * num_sms;
+  const size_t smem = (size_t)p.K;
+  if (out_bf16) slice_gemm_kernel<true><<<(unsigned)grid, 256, smem, (cudaStream_t)stream>>>(p);
+  else slice_gemm_kernel<false><<<(unsigned)grid, 256, smem, (cudaStream_t)stream>>>(p);
+  return (int)cudaGetLastError();
+}
+
+int launch_selftest_wait(uint32_t* status, uint32_t limit_us, void* stream) {
+  selftest_wait_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(status, (uint64_t)limit_us * 1000ull);
+  return (int)cudaGetLastError();
+}
+
+}  // namespace fmdq

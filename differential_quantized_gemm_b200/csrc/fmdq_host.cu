@@ -1,0 +1,453 @@
+// Host side of the C ABI declared in include/dstar_fmdq.h: argument checks,
+// workspace layout, TMA descriptors and kernel launches on the caller's
+// stream.  Nothing here allocates device memory.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "fmdq_internal.h"
+
+namespace fmdq {
+
+namespace {
+
+thread_local char g_last_error[256] = {0};
+
+int fail(int code, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int ok() {
+  g_last_error[0] = 0;
+  return DSTAR_OK;
+}
+
+int cuda_fail(int e, const char* what) {
+  return fail(DSTAR_ERR_CUDA, "%s: %s", what, cudaGetErrorString((cudaError_t)e));
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+size_t elem_size(int dtype) { return dtype == DSTAR_F32 ? 4 : dtype == DSTAR_BF16 ? 2 : 1; }
+
+// device properties, cached per device ordinal
+struct DevInfo {
+  int sms = 0;
+  int major = 0, minor = 0;
+  bool valid = false;
+};
+std::mutex g_dev_mu;
+DevInfo g_dev[64];
+
+int device_info(DevInfo* out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(DSTAR_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (!g_dev[dev].valid) {
+    DevInfo d;
+    if ((e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess)
+      return cuda_fail(e, "cudaDeviceGetAttribute");
+    d.valid = true;
+    g_dev[dev] = d;
+  }
+  *out = g_dev[dev];
+  if (out->major != 10 || out->minor != 0)
+    return fail(DSTAR_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a", dev,
+                out->major, out->minor);
+  return DSTAR_OK;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda)
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D int8 tensor map: rows x cols with a row pitch of ld bytes, box of
+// box_rows x 128 bytes, 128-byte swizzle, zero fill outside the matrix.
+int make_map_i8(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t ld, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(DSTAR_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)ld};
+  const cuuint32_t box[2] = {(cuuint32_t)kChunkK, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(DSTAR_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return DSTAR_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_mat(const dstar_mat* m, const char* name, int64_t rows, int64_t cols, bool want_float) {
+  if (!m) return fail(DSTAR_ERR_INVALID_ARG, "%s is NULL", name);
+  if (want_float && m->dtype != DSTAR_F32 && m->dtype != DSTAR_BF16)
+    return fail(DSTAR_ERR_INVALID_ARG, "%s: dtype must be F32 or BF16", name);
+  if (!want_float && m->dtype != DSTAR_I8) return fail(DSTAR_ERR_INVALID_ARG, "%s: dtype must be I8", name);
+  if (m->rows != rows || m->cols != cols)
+    return fail(DSTAR_ERR_INVALID_ARG, "%s: shape %lldx%lld, expected %lldx%lld", name, (long long)m->rows,
+                (long long)m->cols, (long long)rows, (long long)cols);
+  if (rows > 0 && cols > 0) {
+    if (!m->data) return fail(DSTAR_ERR_INVALID_ARG, "%s: data is NULL", name);
+    if (m->ld < cols) return fail(DSTAR_ERR_INVALID_ARG, "%s: ld < cols", name);
+    if (!aligned16(m->data) || (m->ld * (int64_t)elem_size(m->dtype)) % 16 != 0)
+      return fail(DSTAR_ERR_INVALID_ARG, "%s: data and row pitch must be 16-byte aligned", name);
+  }
+  return DSTAR_OK;
+}
+
+bool overlap(const dstar_mat* a, const dstar_mat* b) {
+  if (!a->data || !b->data || a->rows == 0 || b->rows == 0) return false;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a->data), b0 = reinterpret_cast<uintptr_t>(b->data);
+  const uintptr_t a1 = a0 + (size_t)((a->rows - 1) * a->ld + a->cols) * elem_size(a->dtype);
+  const uintptr_t b1 = b0 + (size_t)((b->rows - 1) * b->ld + b->cols) * elem_size(b->dtype);
+  return a0 < b1 && b0 < a1;
+}
+
+int base_log2(float base, int* lb) {
+  if (!(base > 0.f) || !std::isfinite(base)) return fail(DSTAR_ERR_INVALID_ARG, "base_scale must be positive and finite");
+  int e;
+  const float f = std::frexp(base, &e);
+  if (f != 0.5f) return fail(DSTAR_ERR_INVALID_ARG, "base_scale must be an exact power of two");
+  *lb = e - 1;
+  if (*lb < DSTAR_BASE_LOG2_MIN || *lb > DSTAR_BASE_LOG2_MAX)
+    return fail(DSTAR_ERR_INVALID_ARG, "base_scale 2^%d outside [2^%d, 2^%d]", *lb, DSTAR_BASE_LOG2_MIN,
+                DSTAR_BASE_LOG2_MAX);
+  return DSTAR_OK;
+}
+
+int check_cfg(const dstar_tile_cfg* c, int64_t M, int64_t K) {
+  if (!c) return fail(DSTAR_ERR_INVALID_ARG, "tile_cfg is NULL");
+  if (c->tile_tokens != DSTAR_TILE_TOKENS) return fail(DSTAR_ERR_INVALID_ARG, "tile_tokens must be 16");
+  if (c->force_bits != 0 && c->force_bits != 2 && c->force_bits != 4 && c->force_bits != 6 && c->force_bits != 8)
+    return fail(DSTAR_ERR_INVALID_ARG, "force_bits must be 0, 2, 4, 6 or 8");
+  if (c->thr0_log2 < -100 || c->thr0_log2 > 100) return fail(DSTAR_ERR_INVALID_ARG, "thr0_log2 out of [-100, 100]");
+  if (c->flags & ~(DSTAR_FLAG_NO_XPREV_REFRESH | DSTAR_FLAG_SLICE_PATH))
+    return fail(DSTAR_ERR_INVALID_ARG, "unknown flag bits 0x%x", c->flags);
+  const WsLayout L = ws_layout(M, K);
+  if (!c->workspace) return fail(DSTAR_ERR_WORKSPACE, "workspace is NULL");
+  if (reinterpret_cast<uintptr_t>(c->workspace) & 255u) return fail(DSTAR_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  if (c->workspace_bytes < L.total)
+    return fail(DSTAR_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", c->workspace_bytes, L.total);
+  if ((c->debug_codes && !aligned16(c->debug_codes)) || (c->debug_acc && !aligned16(c->debug_acc)))
+    return fail(DSTAR_ERR_INVALID_ARG, "debug buffers must be 16-byte aligned");
+  return DSTAR_OK;
+}
+
+int check_mk(int64_t M, int64_t K) {
+  if (M < 0 || M % kTile != 0) return fail(DSTAR_ERR_INVALID_ARG, "M=%lld must be a non-negative multiple of 16", (long long)M);
+  if (K <= 0 || K % 32 != 0 || K > DSTAR_K_MAX)
+    return fail(DSTAR_ERR_INVALID_ARG, "K=%lld must be a positive multiple of 32 up to %d", (long long)K, DSTAR_K_MAX);
+  return DSTAR_OK;
+}
+
+template <typename T>
+T* ws_ptr(const dstar_tile_cfg* c, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(c->workspace) + off);
+}
+
+int do_quantize(const dstar_mat* x_t, dstar_mat* x_prev, int lb, const dstar_tile_cfg* c, int64_t M, int64_t K,
+                void* stream) {
+  const WsLayout L = ws_layout(M, K);
+  QuantParams q{};
+  q.x_t = x_t->data;
+  q.x_prev = x_prev->data;
+  q.ld_xt = x_t->ld;
+  q.ld_xp = x_prev->ld;
+  q.M = M, q.K = K;
+  q.lb = lb, q.t0 = c->thr0_log2, q.force_bits = c->force_bits, q.flags = c->flags;
+  q.status = ws_ptr<uint32_t>(c, L.status);
+  q.plane0 = ws_ptr<int8_t>(c, L.plane0);
+  q.plane1 = ws_ptr<int8_t>(c, L.plane1);
+  q.fpot = ws_ptr<int8_t>(c, L.fpot);
+  q.bits = ws_ptr<int8_t>(c, L.bits);
+  q.g_ref = ws_ptr<int32_t>(c, L.g_ref);
+  q.planes = ws_ptr<int32_t>(c, L.planes);
+  q.count = ws_ptr<int32_t>(c, L.count);
+  q.mask1 = ws_ptr<uint32_t>(c, L.mask1);
+  q.records = ws_ptr<uint2>(c, L.records);
+  q.record_cap = L.record_cap;
+  q.mask_words = L.mask_words;
+  q.debug_codes = c->debug_codes;
+  const int e = launch_quantize(q, x_t->dtype == DSTAR_BF16, stream);
+  if (e) return cuda_fail(e, "quantize launch");
+  return DSTAR_OK;
+}
+
+// Output tile width: the one with the least wave-quantised work (ties -> 256).
+int choose_bn(int64_t M, int64_t N, int sms) {
+  const int64_t tm = (M + kBlockM - 1) / kBlockM;
+  const int64_t t256 = tm * ((N + 255) / 256), t128 = tm * ((N + 127) / 128);
+  const int64_t c256 = (t256 + sms - 1) / sms * 256, c128 = (t128 + sms - 1) / sms * 128;
+  return c128 < c256 ? 128 : 256;
+}
+
+int do_gemm(const dstar_mat* w_q, const float* w_scale, dstar_mat* y_prev, int lb, const dstar_tile_cfg* c,
+            dstar_mat* y_out, int64_t M, int64_t K, int64_t N, const DevInfo& dev, void* stream) {
+  if (N == 0 || M == 0) return DSTAR_OK;
+  const WsLayout L = ws_layout(M, K);
+  const bool bf16 = y_prev->dtype == DSTAR_BF16;
+  const bool distinct = y_out->data != y_prev->data;
+  const bool slice_all = (c->flags & DSTAR_FLAG_SLICE_PATH) != 0;
+  if (!slice_all) {
+    const int bn = choose_bn(M, N, dev.sms);
+    CUtensorMap ma0, ma1, mw;
+    int r;
+    if ((r = make_map_i8(&ma0, ws_ptr<void>(c, L.plane0), M, K, K, kBlockM)) != DSTAR_OK) return r;
+    if ((r = make_map_i8(&ma1, ws_ptr<void>(c, L.plane1), M, K, K, kBlockM)) != DSTAR_OK) return r;
+    if ((r = make_map_i8(&mw, w_q->data, N, K, w_q->ld, bn)) != DSTAR_OK) return r;
+    GemmParams g{};
+    g.M = M, g.N = N, g.K = K;
+    g.lb = lb;
+    g.flags = c->flags;
+    g.g_ref = ws_ptr<int32_t>(c, L.g_ref);
+    g.planes = ws_ptr<int32_t>(c, L.planes);
+    g.mask1 = ws_ptr<uint32_t>(c, L.mask1);
+    g.mask_words = L.mask_words;
+    g.w_scale = w_scale;
+    g.y_prev = y_prev->data;
+    g.ld_yp = y_prev->ld;
+    g.y_out = y_out->data;
+    g.ld_yo = y_out->ld;
+    g.y_distinct = distinct;
+    g.status = ws_ptr<uint32_t>(c, L.status);
+    g.debug_acc = c->debug_acc;
+    g.tiles_m = (int)((M + kBlockM - 1) / kBlockM);
+    g.tiles_n = (int)((N + bn - 1) / bn);
+    g.num_chunks = (int)((K + kChunkK - 1) / kChunkK);
+    const int e = launch_gemm(g, &ma0, &ma1, &mw, bn, bf16, dev.sms, stream);
+    if (e) return cuda_fail(e, "slice-GEMM launch");
+  }
+  SliceParams s{};
+  s.M = M, s.N = N, s.K = K;
+  s.lb = lb;
+  s.w_q = static_cast<const int8_t*>(w_q->data);
+  s.ld_w = w_q->ld;
+  s.records = ws_ptr<const uint2>(c, L.records);
+  s.record_cap = L.record_cap;
+  s.count = ws_ptr<const int32_t>(c, L.count);
+  s.bits = ws_ptr<const int8_t>(c, L.bits);
+  s.g_ref = ws_ptr<const int32_t>(c, L.g_ref);
+  s.planes = ws_ptr<const int32_t>(c, L.planes);
+  s.w_scale = w_scale;
+  s.y_prev = y_prev->data;
+  s.ld_yp = y_prev->ld;
+  s.y_out = y_out->data;
+  s.ld_yo = y_out->ld;
+  s.y_distinct = distinct;
+  s.all_tiles = slice_all;
+  s.debug_acc = c->debug_acc;
+  const int e = launch_slice_gemm(s, bf16, dev.sms, stream);
+  if (e) return cuda_fail(e, "slice-stream launch");
+  return DSTAR_OK;
+}
+
+int check_gemm_args(const dstar_mat* w_q, const float* w_scale, dstar_mat* y_prev, dstar_mat* y_out, int64_t M,
+                    int64_t K, int64_t* N_out) {
+  if (!w_q) return fail(DSTAR_ERR_INVALID_ARG, "w_q is NULL");
+  const int64_t N = w_q->rows;
+  if (N < 0 || N % 16 != 0) return fail(DSTAR_ERR_INVALID_ARG, "N=%lld must be a non-negative multiple of 16", (long long)N);
+  int r;
+  if ((r = check_mat(w_q, "w_q", N, K, false)) != DSTAR_OK) return r;
+  if ((r = check_mat(y_prev, "y_prev", M, N, true)) != DSTAR_OK) return r;
+  if ((r = check_mat(y_out, "y_out", M, N, true)) != DSTAR_OK) return r;
+  if (y_out->dtype != y_prev->dtype) return fail(DSTAR_ERR_INVALID_ARG, "y_out and y_prev must share a dtype");
+  if (N > 0 && M > 0) {
+    if (!w_scale) return fail(DSTAR_ERR_INVALID_ARG, "w_scale is NULL");
+    if (reinterpret_cast<uintptr_t>(w_scale) & 3u) return fail(DSTAR_ERR_INVALID_ARG, "w_scale must be 4-byte aligned");
+    const bool same = y_out->data == y_prev->data && y_out->ld == y_prev->ld;
+    if (!same && overlap(y_out, y_prev)) return fail(DSTAR_ERR_INVALID_ARG, "y_out partially overlaps y_prev");
+  }
+  *N_out = N;
+  return DSTAR_OK;
+}
+
+}  // namespace
+
+WsLayout ws_layout(int64_t M, int64_t K) {
+  WsLayout L{};
+  const int64_t T = M / kTile;
+  const int64_t chunks = (K + kChunkK - 1) / kChunkK;
+  L.mask_words = (chunks + 31) / 32;
+  L.record_cap = 4 * K;
+  size_t o = 0;
+  L.status = o, o = align256(o + 256);
+  L.plane0 = o, o = align256(o + (size_t)(M * K));
+  L.plane1 = o, o = align256(o + (size_t)(M * K));
+  L.fpot = o, o = align256(o + (size_t)(T * K));
+  L.bits = o, o = align256(o + (size_t)(T * K));
+  L.g_ref = o, o = align256(o + (size_t)T * 4);
+  L.planes = o, o = align256(o + (size_t)T * 4);
+  L.count = o, o = align256(o + (size_t)T * 4);
+  L.mask1 = o, o = align256(o + (size_t)(T * L.mask_words) * 4);
+  L.records = o, o = align256(o + (size_t)(T * L.record_cap) * 8);
+  L.total = o;
+  return L;
+}
+
+}  // namespace fmdq
+
+using namespace fmdq;
+
+extern "C" {
+
+int dstar_fmdq_version(void) { return DSTAR_FMDQ_VERSION; }
+
+const char* dstar_fmdq_error_string(int code) {
+  switch (code) {
+    case DSTAR_OK: return "ok";
+    case DSTAR_ERR_INVALID_ARG: return "invalid argument";
+    case DSTAR_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case DSTAR_ERR_CUDA: return "CUDA error";
+    case DSTAR_ERR_UNSUPPORTED: return "unsupported device";
+    default: return "unknown error";
+  }
+}
+
+const char* dstar_fmdq_last_error(void) { return g_last_error; }
+
+int dstar_fmdq_workspace_size(int64_t M, int64_t K, size_t* bytes) {
+  if (!bytes) return fail(DSTAR_ERR_INVALID_ARG, "bytes is NULL");
+  if (M < 0 || K < 0 || K > DSTAR_K_MAX) return fail(DSTAR_ERR_INVALID_ARG, "bad M or K");
+  *bytes = ws_layout(M, K).total;
+  return ok();
+}
+
+int dstar_fmdq_workspace_layout(int64_t M, int64_t K, dstar_fmdq_ws_layout* out) {
+  if (!out) return fail(DSTAR_ERR_INVALID_ARG, "out is NULL");
+  if (M < 0 || K < 0 || K > DSTAR_K_MAX) return fail(DSTAR_ERR_INVALID_ARG, "bad M or K");
+  const WsLayout L = ws_layout(M, K);
+  out->total = L.total;
+  out->status = L.status;
+  out->plane0 = L.plane0;
+  out->plane1 = L.plane1;
+  out->fpot = L.fpot;
+  out->bits = L.bits;
+  out->g_ref = L.g_ref;
+  out->planes = L.planes;
+  out->count = L.count;
+  out->mask1 = L.mask1;
+  out->records = L.records;
+  out->mask_words = L.mask_words;
+  out->record_cap = L.record_cap;
+  return ok();
+}
+
+int dstar_fmdq_workspace_init(void* workspace, size_t bytes, void* stream) {
+  if (!workspace || bytes < 256) return fail(DSTAR_ERR_WORKSPACE, "workspace is NULL or smaller than 256 bytes");
+  const cudaError_t e = cudaMemsetAsync(workspace, 0, 256, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  return ok();
+}
+
+int dstar_fmdq_quantize(const dstar_mat* x_t, dstar_mat* x_prev, float base_scale, const dstar_tile_cfg* tile_cfg,
+                        void* stream) {
+  int r;
+  if (!x_t || !x_prev) return fail(DSTAR_ERR_INVALID_ARG, "x_t or x_prev is NULL");
+  const int64_t M = x_t->rows, K = x_t->cols;
+  if ((r = check_mk(M, K)) != DSTAR_OK) return r;
+  if ((r = check_mat(x_t, "x_t", M, K, true)) != DSTAR_OK) return r;
+  if ((r = check_mat(x_prev, "x_prev", M, K, true)) != DSTAR_OK) return r;
+  if (x_t->dtype != x_prev->dtype) return fail(DSTAR_ERR_INVALID_ARG, "x_t and x_prev must share a dtype");
+  if (!(x_t->data == x_prev->data && x_t->ld == x_prev->ld) && overlap(x_t, x_prev))
+    return fail(DSTAR_ERR_INVALID_ARG, "x_t partially overlaps x_prev");
+  int lb = 0;
+  if ((r = base_log2(base_scale, &lb)) != DSTAR_OK) return r;
+  if ((r = check_cfg(tile_cfg, M, K)) != DSTAR_OK) return r;
+  if (M == 0) return ok();
+  DevInfo dev;
+  if ((r = device_info(&dev)) != DSTAR_OK) return r;
+  if ((r = do_quantize(x_t, x_prev, lb, tile_cfg, M, K, stream)) != DSTAR_OK) return r;
+  return ok();
+}
+
+int dstar_fmdq_slice_gemm(const dstar_mat* w_q, const float* w_scale, dstar_mat* y_prev, float base_scale,
+                          const dstar_tile_cfg* tile_cfg, dstar_mat* y_out, void* stream) {
+  int r;
+  if (!w_q || !y_prev) return fail(DSTAR_ERR_INVALID_ARG, "w_q or y_prev is NULL");
+  const int64_t M = y_prev->rows, K = w_q->cols;
+  if ((r = check_mk(M, K)) != DSTAR_OK) return r;
+  int64_t N = 0;
+  if ((r = check_gemm_args(w_q, w_scale, y_prev, y_out, M, K, &N)) != DSTAR_OK) return r;
+  int lb = 0;
+  if ((r = base_log2(base_scale, &lb)) != DSTAR_OK) return r;
+  if ((r = check_cfg(tile_cfg, M, K)) != DSTAR_OK) return r;
+  if (M == 0 || N == 0) return ok();
+  DevInfo dev;
+  if ((r = device_info(&dev)) != DSTAR_OK) return r;
+  if ((r = do_gemm(w_q, w_scale, y_prev, lb, tile_cfg, y_out, M, K, N, dev, stream)) != DSTAR_OK) return r;
+  return ok();
+}
+
+int dstar_fmdq_linear(const dstar_mat* x_t, dstar_mat* x_prev, dstar_mat* y_prev, const dstar_mat* w_q,
+                      const float* w_scale, float base_scale, const dstar_tile_cfg* tile_cfg, dstar_mat* y_out,
+                      void* stream) {
+  int r;
+  if (!x_t || !x_prev) return fail(DSTAR_ERR_INVALID_ARG, "x_t or x_prev is NULL");
+  const int64_t M = x_t->rows, K = x_t->cols;
+  if ((r = check_mk(M, K)) != DSTAR_OK) return r;
+  if ((r = check_mat(x_t, "x_t", M, K, true)) != DSTAR_OK) return r;
+  if ((r = check_mat(x_prev, "x_prev", M, K, true)) != DSTAR_OK) return r;
+  if (x_t->dtype != x_prev->dtype) return fail(DSTAR_ERR_INVALID_ARG, "x_t and x_prev must share a dtype");
+  if (!(x_t->data == x_prev->data && x_t->ld == x_prev->ld) && overlap(x_t, x_prev))
+    return fail(DSTAR_ERR_INVALID_ARG, "x_t partially overlaps x_prev");
+  int64_t N = 0;
+  if ((r = check_gemm_args(w_q, w_scale, y_prev, y_out, M, K, &N)) != DSTAR_OK) return r;
+  int lb = 0;
+  if ((r = base_log2(base_scale, &lb)) != DSTAR_OK) return r;
+  if ((r = check_cfg(tile_cfg, M, K)) != DSTAR_OK) return r;
+  if (M == 0) return ok();
+  DevInfo dev;
+  if ((r = device_info(&dev)) != DSTAR_OK) return r;
+  if ((r = do_quantize(x_t, x_prev, lb, tile_cfg, M, K, stream)) != DSTAR_OK) return r;
+  if ((r = do_gemm(w_q, w_scale, y_prev, lb, tile_cfg, y_out, M, K, N, dev, stream)) != DSTAR_OK) return r;
+  return ok();
+}
+
+int dstar_fmdq_status(void* workspace, void* stream, uint32_t* status) {
+  if (!workspace || !status) return fail(DSTAR_ERR_INVALID_ARG, "workspace or status is NULL");
+  cudaError_t e = cudaMemcpyAsync(status, workspace, sizeof(uint32_t), cudaMemcpyDeviceToHost, (cudaStream_t)stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(workspace, 0, sizeof(uint32_t), (cudaStream_t)stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the status word");
+  return ok();
+}
+
+int dstar_fmdq_selftest_wait(void* workspace, uint32_t limit_us, void* stream) {
+  if (!workspace) return fail(DSTAR_ERR_WORKSPACE, "workspace is NULL");
+  DevInfo dev;
+  int r;
+  if ((r = device_info(&dev)) != DSTAR_OK) return r;
+  const int e = launch_selftest_wait(static_cast<uint32_t*>(workspace), limit_us, stream);
+  if (e) return cuda_fail(e, "self-test launch");
+  return ok();
+}
+
+}  // extern "C"

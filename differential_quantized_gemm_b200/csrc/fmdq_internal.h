@@ -1,0 +1,102 @@
+// Internal definitions shared by the host dispatcher and the kernels of the
+// FMDQ differential linear library (not part of the C ABI).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/dstar_fmdq.h"
+
+namespace fmdq {
+
+constexpr int kTile = DSTAR_TILE_TOKENS;  // tokens per sub-channel
+constexpr int kBlockM = 128;               // rows of one tensor-core tile (8 token tiles)
+constexpr int kChunkK = 128;               // int8 columns per K chunk (one 128-byte swizzle row)
+constexpr int kPotMax = DSTAR_POT_MAX;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded waits give up after 2 s
+
+// Plane split of a shift-folded operand v = q * 2^(g_ref - FPoT):
+// v = A0 + 256 * A1 with A0 = the low byte of v read as signed, A1 the rest.
+// One plane holds v in [-128, 127]; two planes hold v in [-128*257, 127*257].
+constexpr int64_t kPlane1Lo = -128, kPlane1Hi = 127;
+constexpr int64_t kPlane2Lo = -128 * 257, kPlane2Hi = 127 * 257;
+
+struct QuantParams {
+  const void* x_t;
+  void* x_prev;
+  int64_t ld_xt, ld_xp;
+  int64_t M, K;
+  int lb, t0, force_bits;
+  uint32_t flags;
+  uint32_t* status;
+  int8_t* plane0;
+  int8_t* plane1;
+  int8_t* fpot;
+  int8_t* bits;
+  int32_t* g_ref;
+  int32_t* planes;
+  int32_t* count;
+  uint32_t* mask1;
+  uint2* records;
+  int64_t record_cap;
+  int64_t mask_words;
+  int8_t* debug_codes;
+};
+
+struct GemmParams {
+  int64_t M, N, K;
+  int lb;
+  uint32_t flags;
+  const int32_t* g_ref;
+  const int32_t* planes;
+  const uint32_t* mask1;
+  int64_t mask_words;
+  const float* w_scale;
+  void* y_prev;
+  int64_t ld_yp;
+  void* y_out;
+  int64_t ld_yo;
+  int y_distinct;  // y_out is a different buffer: write both
+  uint32_t* status;
+  int64_t* debug_acc;
+  int tiles_m, tiles_n, num_chunks;
+};
+
+struct SliceParams {
+  int64_t M, N, K;
+  int lb;
+  const int8_t* w_q;
+  int64_t ld_w;
+  const uint2* records;
+  int64_t record_cap;
+  const int32_t* count;
+  const int8_t* bits;
+  const int32_t* g_ref;
+  const int32_t* planes;
+  const float* w_scale;
+  void* y_prev;
+  int64_t ld_yp;
+  void* y_out;
+  int64_t ld_yo;
+  int y_distinct;
+  int all_tiles;  // 1: every tile; 0: only tiles that need more than two planes
+  int64_t* debug_acc;
+};
+
+// Workspace sections (byte offsets from the workspace base).
+struct WsLayout {
+  size_t total, status, plane0, plane1, fpot, bits, g_ref, planes, count, mask1, records;
+  int64_t mask_words, record_cap;
+};
+WsLayout ws_layout(int64_t M, int64_t K);
+
+// Launchers (return cudaError_t as int).
+int launch_quantize(const QuantParams& p, int in_bf16, void* stream);
+int launch_gemm(const GemmParams& p, const void* tmap_a0, const void* tmap_a1, const void* tmap_w, int bn,
+                int out_bf16, int num_sms, void* stream);
+int launch_slice_gemm(const SliceParams& p, int out_bf16, int num_sms, void* stream);
+int launch_selftest_wait(uint32_t* status, uint32_t spin_limit, void* stream);
+size_t quantize_smem_bytes(int64_t K);
+size_t gemm_smem_bytes(int bn);
+
+}  // namespace fmdq

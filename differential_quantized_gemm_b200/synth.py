@@ -130,7 +130,12 @@ def _dx(cfg: int, spec: LayerSpec, rng, sigma: float | None) -> np.ndarray:
         sig = np.exp(rng.uniform(math.log(1e-3), math.log(1.0), size=T)).astype(np.float32)
         return rng.standard_normal((M, K), dtype=np.float32) * np.repeat(sig, 16)[:, None]
     if cfg == 4:
-        B, F, Pn = M // (16 * 256), 16, 256
+        # tokens ordered (batch, frame, patch); 256 patches per frame at full size,
+        # fewer for small test cases, always whole 16-token tiles per frame
+        F = 16
+        Pn = min(256, max(16, (M // F) // 16 * 16))
+        B = M // (F * Pn)
+        assert B * F * Pn == M, "video workload needs M = batch x 16 frames x patches"
         z = rng.standard_normal((B, F, Pn, K), dtype=np.float32)
         e = np.empty_like(z)
         e[:, 0] = 0.05 * z[:, 0]
@@ -196,7 +201,9 @@ def adversarial_layer(M: int, K: int, N: int, seed: int, spread: int = 24, dtype
     rng = _rng(seed, 7, 7)
     w_q, w_scale = _weights(rng, K, N)
     x_prev = rng.standard_normal((M, K), dtype=np.float32)
-    mag = np.exp2(rng.uniform(-8, -8 + spread, size=(M // 16, K))).astype(np.float32)
+    # each tile draws its own spread in [0, spread]: some tiles are narrow, some wide
+    tile_spread = rng.uniform(0, spread, size=(M // 16, 1))
+    mag = np.exp2(-8 + tile_spread * rng.uniform(0, 1, size=(M // 16, K))).astype(np.float32)
     dx = rng.standard_normal((M, K), dtype=np.float32) * np.repeat(mag, 16, axis=0)
     spec = LayerSpec("adversarial", M, K, N, dtype, lb)
     w_deq_t = w_q.astype(np.float32).T * w_scale[None, :]
@@ -207,3 +214,34 @@ def adversarial_layer(M: int, K: int, N: int, seed: int, spread: int = 24, dtype
         return LayerInputs(spec, xt_b, xp_b, to_bf16_bits(xp_f @ w_deq_t), w_q, w_scale)
     x_t = (x_prev + dx).astype(np.float32)
     return LayerInputs(spec, x_t, x_prev, (x_prev @ w_deq_t).astype(np.float32), w_q, w_scale)
+
+
+class SweepChain:
+    """Consecutive calls of one layer of the timestep sweep with the caches
+    carried: X at each listed step is the previous X plus sigma_t * N(0, 1)
+    (rounded to bf16), starting from X_{-1} ~ N(0, 1); the cached output
+    starts from the dense product and is carried by each side itself."""
+
+    def __init__(self, layer: int, steps: list[int], M: int = 8192, force_bits: int = 0):
+        self.layer, self.step_list, self.force_bits = layer, list(steps), force_bits
+        spec = config_layers(5)[layer]
+        self.spec = LayerSpec(spec.name, M, spec.K, spec.N, "bf16", spec.lb, spec.t0, force_bits)
+
+    def steps(self):
+        spec = self.spec
+        rng_w = _rng(5, self.layer, 101)
+        rng_x = _rng(5, self.layer, 202)
+        w_q, w_scale = _weights(rng_w, spec.K, spec.N)
+        x = to_bf16_bits(rng_x.standard_normal((spec.M, spec.K), dtype=np.float32))
+        xf = bf16_bits_to_f32(x)
+        y = to_bf16_bits(xf @ (w_q.astype(np.float32).T * w_scale[None, :]))
+        for s in self.step_list:
+            sig = 0.03 if self.force_bits else sweep_sigma(s)
+            z = _rng(5, self.layer, 303, s).standard_normal((spec.M, spec.K), dtype=np.float32)
+            x_new = to_bf16_bits(bf16_bits_to_f32(x) + np.float32(sig) * z)
+            yield LayerInputs(spec, x_new, x, y, w_q, w_scale)
+            x = x_new
+
+
+def sweep_chain(layer: int, steps: list[int], M: int = 8192, force_bits: int = 0) -> SweepChain:
+    return SweepChain(layer, steps, M, force_bits)

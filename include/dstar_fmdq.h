@@ -1,0 +1,207 @@
+/*
+ * dstar_fmdq.h -- C ABI of the B200 (sm_100a) FMDQ differential linear layer.
+ *
+ * FMDQ is the fine-grained mixed-precision differential quantization of
+ * DSTAR ("DSTAR: Accelerating Diffusion Transformers via Spatial and Temporal
+ * Redundancy Reduction"), section 3.1.  One call computes, for a linear layer
+ * Y = X W with int8 weights,
+ *
+ *   dX  = X_t - X_{t-1}                                  (section 2.2, Eq. 1)
+ *   per sub-channel (16 tokens x 1 channel): M_i = max|dX|, PoT (Eq. 3),
+ *        bit width b in {2,4,6,8} from the thresholds Thr_0 * 2^(2N),
+ *        FPoT (Eq. 4), scale s_i = base * 2^FPoT (Eq. 5), codes q = rne(dX s_i)
+ *   2-bit slices of every code, their FPoT lowered by 2 per slice, grouped by
+ *        FPoT and encoded with shift counts               (section 3.1, steps 2-4)
+ *   acc = shift-aligned accumulation of slice x weight    (section 3.1, step 5)
+ *   Y_t = Y_{t-1} + acc * 2^(-lb-g_ref) * w_scale          (section 4.2 inverse
+ *        quantization and accumulation units; section 4.3 reverse differential)
+ *
+ * and refreshes the caches (x_prev <- X_t, y_prev <- Y_t).
+ *
+ * Conventions for every entry point
+ *   - All matrices are row-major in DEVICE memory and owned by the caller; the
+ *     library allocates nothing and keeps no global state.  Scratch lives in a
+ *     caller-owned device workspace (dstar_fmdq_workspace_size bytes).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  All work is enqueued asynchronously on it; nothing synchronises
+ *     except dstar_fmdq_status.
+ *   - Return value: DSTAR_OK or a negative DSTAR_ERR_* code, decided on the host
+ *     before anything is enqueued (arguments) or right after (launch errors).
+ *     dstar_fmdq_last_error() gives a one-line reason for the calling thread.
+ *   - Data-dependent problems found on the device (non-finite dX, PoT above its
+ *     maximum, an exhausted wait) set bits of the workspace's sticky status
+ *     word, read and cleared by dstar_fmdq_status.  When a bit is set the
+ *     outputs of the calls since the last read are unspecified.
+ *   - The entry points are reentrant; two calls that share a workspace must be
+ *     ordered on the device (same stream, or events).
+ */
+#ifndef DSTAR_FMDQ_H
+#define DSTAR_FMDQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DSTAR_FMDQ_VERSION 1
+
+#if defined(__GNUC__)
+#define DSTAR_API __attribute__((visibility("default")))
+#else
+#define DSTAR_API
+#endif
+
+/* return codes */
+#define DSTAR_OK 0
+#define DSTAR_ERR_INVALID_ARG (-1) /* bad pointer, shape, dtype, alignment, parameter */
+#define DSTAR_ERR_WORKSPACE (-2)   /* workspace missing, misaligned or too small */
+#define DSTAR_ERR_CUDA (-3)        /* a CUDA runtime call or launch failed */
+#define DSTAR_ERR_UNSUPPORTED (-4) /* the current device is not sm_100 */
+
+/* sticky device status bits (dstar_fmdq_status) */
+#define DSTAR_STATUS_NONFINITE 1u /* some dX was NaN or infinite; that sub-channel was zeroed */
+#define DSTAR_STATUS_RANGE 2u     /* some PoT exceeded DSTAR_POT_MAX and was clamped */
+#define DSTAR_STATUS_TIMEOUT 4u   /* a bounded device wait ran out; the kernel returned early */
+
+/* element types of dstar_mat */
+#define DSTAR_F32 0
+#define DSTAR_BF16 1
+#define DSTAR_I8 2
+
+/* tile_cfg.flags */
+#define DSTAR_FLAG_NO_XPREV_REFRESH 1u /* leave x_prev untouched (caller swaps buffers) */
+#define DSTAR_FLAG_SLICE_PATH 2u       /* compute every tile with the slice-stream kernel */
+
+/* limits of this implementation */
+#define DSTAR_TILE_TOKENS 16   /* tokens per sub-channel (the only supported tile) */
+#define DSTAR_POT_MAX 32       /* largest PoT (Eq. 3); larger ones clamp and set RANGE */
+#define DSTAR_K_MAX 8192       /* input channels */
+#define DSTAR_BASE_LOG2_MIN (-32)
+#define DSTAR_BASE_LOG2_MAX 32
+
+/* A row-major matrix in device memory: element (r, c) is at
+ * data + (r * ld + c) * sizeof(element).  ld is in elements. */
+typedef struct {
+  void* data;
+  int32_t dtype; /* DSTAR_F32, DSTAR_BF16 or DSTAR_I8 */
+  int32_t reserved;
+  int64_t rows, cols, ld;
+} dstar_mat;
+
+/* Per-call quantizer configuration (section 3.1, step 1) and scratch. */
+typedef struct {
+  int32_t tile_tokens; /* tokens per sub-channel; must be DSTAR_TILE_TOKENS */
+  int32_t thr0_log2;   /* t0: Thr_0 = base_scale * 2^t0; Thr_N = Thr_0 * 2^(2N) */
+  int32_t force_bits;  /* 0: bit width by the thresholds; 2, 4, 6 or 8: that width everywhere */
+  uint32_t flags;      /* DSTAR_FLAG_* */
+  void* workspace;     /* device memory, 256-byte aligned, dstar_fmdq_workspace_size bytes,
+                          initialised once with dstar_fmdq_workspace_init */
+  size_t workspace_bytes;
+  int8_t* debug_codes; /* optional device [M x K] int8 (ld = K): every code q */
+  int64_t* debug_acc;  /* optional device [M x N] int64 (ld = N): every exact accumulator */
+} dstar_tile_cfg;
+
+/* Byte offsets of the sections of a workspace for an (M, K) call.  The
+ * sections hold the quantizer's outputs and stay valid until the next call
+ * that uses the workspace:
+ *   fpot    int8  [T x K]  absolute FPoT of each sub-channel (Eq. 4)
+ *   bits    int8  [T x K]  its bit width
+ *   g_ref   int32 [T]      finest FPoT of each 16-token tile
+ *   count   int32 [T]      number of slice records of the tile
+ *   records 8-byte [T x record_cap] records of the tile in (FPoT, channel)
+ *           order: { uint32 word; uint16 k; int8 fpot; uint8 j }, where word
+ *           holds the 2-bit field of slice j of channel k for the 16 tokens
+ *           (token i in bits 2i..2i+1) -- the encoded stream of section 3.1
+ *           step 4; the shift before a record is its fpot minus the previous
+ *   planes  int32 [T]      tensor-core operand planes the tile needs
+ *   plane0/plane1 int8 [M x K]  shift-folded operands of the tensor-core GEMM
+ *   mask1   uint32 [T x mask_words]  K-chunks (128 wide) where plane 1 is nonzero
+ * T = M / 16. */
+typedef struct {
+  size_t total;
+  size_t status;
+  size_t plane0, plane1;
+  size_t fpot, bits;
+  size_t g_ref, planes, count;
+  size_t mask1;
+  size_t records;
+  int64_t mask_words;
+  int64_t record_cap;
+} dstar_fmdq_ws_layout;
+
+/* Workspace bytes needed by calls with M tokens and K input channels.
+ * Errors: INVALID_ARG for a NULL `bytes`, negative sizes, K > DSTAR_K_MAX. */
+DSTAR_API int dstar_fmdq_workspace_size(int64_t M, int64_t K, size_t* bytes);
+
+/* Section offsets of that workspace (see dstar_fmdq_ws_layout). */
+DSTAR_API int dstar_fmdq_workspace_layout(int64_t M, int64_t K, dstar_fmdq_ws_layout* out);
+
+/* Clear the status word of a fresh workspace (enqueued on `stream`).  Call once
+ * after allocating it; the other sections need no initialisation. */
+DSTAR_API int dstar_fmdq_workspace_init(void* workspace, size_t bytes, void* stream);
+
+/*
+ * The FMDQ differential linear (whole hot path).
+ *   x_t     [M x K] F32 or BF16: current input X_t (read only)
+ *   x_prev  [M x K] same dtype:  cached X_{t-1}; overwritten with X_t unless
+ *           DSTAR_FLAG_NO_XPREV_REFRESH (then the caller swaps buffers)
+ *   y_prev  [M x N] F32 or BF16: cached Y_{t-1}; holds Y_t afterwards
+ *   w_q     [N x K] I8 in [-127, 127]: weights, W_deq[k][n] = w_q[n][k] * w_scale[n]
+ *   w_scale [N] fp32 device array: per-output-channel weight scale
+ *   base_scale: the static base of Eq. 3 (section 3.1 "predefined static base");
+ *           an exact power of two 2^lb, lb in [DSTAR_BASE_LOG2_MIN, DSTAR_BASE_LOG2_MAX]
+ *   tile_cfg: quantizer settings and workspace (see dstar_tile_cfg)
+ *   y_out   [M x N] same dtype as y_prev: receives Y_t; may be y_prev itself
+ *           (same pointer and ld) or a disjoint buffer, never a partial overlap
+ * Shapes: M % 16 == 0 (M == 0 is a no-op), 0 < K <= DSTAR_K_MAX with K % 32 == 0,
+ * N >= 0 with N % 16 == 0.  Pointers 16-byte aligned, ld * element size a
+ * multiple of 16 bytes; w_q and w_scale are not written.
+ */
+DSTAR_API int dstar_fmdq_linear(const dstar_mat* x_t, dstar_mat* x_prev, dstar_mat* y_prev, const dstar_mat* w_q,
+                      const float* w_scale, float base_scale, const dstar_tile_cfg* tile_cfg,
+                      dstar_mat* y_out, void* stream);
+
+/*
+ * First stage alone (section 3.1 steps 1-4, the paper's QPU): dX, max-abs,
+ * PoT/bit width/FPoT, codes, 2-bit slices, FPoT-grouped encoded stream, plus
+ * the tensor-core operand planes; refreshes x_prev like dstar_fmdq_linear.
+ * Outputs go to the workspace sections listed in dstar_fmdq_ws_layout.
+ */
+DSTAR_API int dstar_fmdq_quantize(const dstar_mat* x_t, dstar_mat* x_prev, float base_scale,
+                        const dstar_tile_cfg* tile_cfg, void* stream);
+
+/*
+ * Second stage alone (section 3.1 step 5 and the section 4.2/4.3 epilogue):
+ * the shift-aligned slice GEMM over the workspace written by the last
+ * dstar_fmdq_quantize with the same (M, K) and workspace, then
+ * Y_t = Y_{t-1} + dequant(acc) into y_out and y_prev.  Same argument rules as
+ * dstar_fmdq_linear; M and K are taken from y_prev and w_q.
+ */
+DSTAR_API int dstar_fmdq_slice_gemm(const dstar_mat* w_q, const float* w_scale, dstar_mat* y_prev, float base_scale,
+                          const dstar_tile_cfg* tile_cfg, dstar_mat* y_out, void* stream);
+
+/* Synchronise `stream`, copy the workspace's sticky status word to *status
+ * (DSTAR_STATUS_* bits, 0 when clean) and clear it. */
+DSTAR_API int dstar_fmdq_status(void* workspace, void* stream, uint32_t* status);
+
+/* Device self-test of the bounded wait used by every pipeline wait in the
+ * library: launches one block whose thread waits on a barrier that nothing
+ * completes, with a wall-clock limit of `limit_us` microseconds; the wait gives
+ * up, the kernel sets DSTAR_STATUS_TIMEOUT in the workspace status word and
+ * returns normally (the context stays usable). */
+DSTAR_API int dstar_fmdq_selftest_wait(void* workspace, uint32_t limit_us, void* stream);
+
+/* Human-readable name of a return code; one-line reason for the last error of
+ * the calling thread (empty when none). */
+DSTAR_API const char* dstar_fmdq_error_string(int code);
+DSTAR_API const char* dstar_fmdq_last_error(void);
+
+DSTAR_API int dstar_fmdq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSTAR_FMDQ_H */

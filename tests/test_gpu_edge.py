@@ -1,0 +1,130 @@
+"""GPU edge cases: degenerate and ragged shapes, cache semantics, status word
+(non-finite input, PoT range, bounded-wait self-test), stage split, and
+stationarity (dX = 0 leaves Y unchanged, bit for bit)."""
+import numpy as np
+import pytest
+import torch
+
+from differential_quantized_gemm_b200 import _native as nat
+from differential_quantized_gemm_b200 import synth
+
+from gpu_helpers import full_parity, run_gpu, run_oracle, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _build():
+    from differential_quantized_gemm_b200 import build
+    build.build()
+    assert torch.cuda.is_available()
+
+
+def _sub(inp, M, K, N):
+    s = inp.spec
+    spec = synth.LayerSpec(s.name, M, K, N, s.dtype, s.lb, s.t0, s.force_bits)
+    return synth.LayerInputs(spec, np.ascontiguousarray(inp.x_t[:M, :K]), np.ascontiguousarray(inp.x_prev[:M, :K]),
+                             np.ascontiguousarray(inp.y_prev[:M, :N]), np.ascontiguousarray(inp.w_q[:N, :K]),
+                             np.ascontiguousarray(inp.w_scale[:N]))
+
+
+@pytest.mark.parametrize("M,K,N", [(16, 32, 16), (16, 1152, 48), (144, 96, 272), (128, 4608, 16), (48, 160, 400),
+                                   (272, 8192, 32)])
+def test_ragged_shapes(M, K, N):
+    base = synth.adversarial_layer(272, 8192, 400, seed=5, spread=10) if K == 8192 else \
+        synth.adversarial_layer(272, 4608, 400, seed=4, spread=10)
+    full_parity(_sub(base, M, K, N))
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_distinct_output_refreshes_y_prev(dtype):
+    inp = synth.adversarial_layer(160, 256, 96, seed=6, spread=8, dtype=dtype)
+    g, q, acc, y, _ = full_parity(inp, y_distinct=True)
+    assert np.array_equal(g["y_prev_after"].float().cpu().numpy(), g["y"])
+
+
+def test_no_xprev_refresh_flag():
+    inp = synth.make_layer(2, 0, M=128)
+    g = run_gpu(inp, flags=nat.FLAG_NO_XPREV_REFRESH)
+    after = g["x_prev_after"].cpu().view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(after, inp.x_prev)
+
+
+def test_stationary_input_keeps_output_bit_exact():
+    inp = synth.make_layer(3, 2, M=256)
+    inp.x_t = inp.x_prev.copy()
+    g = run_gpu(inp)
+    assert not g["codes"].any() and not g["acc"].any()
+    assert np.array_equal(g["y"], inp.as_f32("y_prev"))
+    # repeated calls with the same input keep Y unchanged
+    d = g["dev"]
+    for _ in range(3):
+        nat.linear(d["x_t"], d["x_prev"], d["y_prev"], d["w_q"], d["w_scale"], 2.0 ** -4, g["ws"])
+    torch.cuda.synchronize()
+    assert np.array_equal(d["y_prev"].float().cpu().numpy(), inp.as_f32("y_prev"))
+
+
+def test_stage_split_equals_linear():
+    inp = synth.make_layer(3, 3, M=256)
+    a = run_gpu(inp)
+    d = to_dev(inp)
+    ws = nat.Workspace(inp.spec.M, inp.spec.K)
+    nat.quantize(d["x_t"], d["x_prev"], 2.0 ** -4, ws)
+    nat.slice_gemm(d["w_q"], d["w_scale"], d["y_prev"], 2.0 ** -4, ws)
+    torch.cuda.synchronize()
+    assert np.array_equal(d["y_prev"].float().cpu().numpy(), a["y"])
+
+
+def test_nonfinite_input_sets_status_and_returns():
+    inp = synth.make_layer(2, 0, M=128)
+    x = synth.bf16_bits_to_f32(inp.x_t).copy()
+    x[5, 7] = np.nan
+    x[20, 100] = np.inf
+    inp.x_t = synth.to_bf16_bits(x)
+    g = run_gpu(inp)
+    assert g["status"] & nat.STATUS_NONFINITE
+    # the affected sub-channels are zeroed; the rest matches the oracle
+    q, acc, y = run_oracle(inp)
+    assert np.array_equal(g["codes"], q.codes)
+    assert np.array_equal(g["acc"], acc)
+
+
+def test_pot_range_sets_status():
+    inp = synth.make_layer(2, 0, M=64)
+    x = synth.bf16_bits_to_f32(inp.x_t).copy()
+    x[3, 3] = 2.0 ** 30  # PoT = 30 + 4 + 1 > 32 with base 2^-4
+    inp.x_t = synth.to_bf16_bits(x)
+    g = run_gpu(inp)
+    assert g["status"] & nat.STATUS_RANGE
+
+
+def test_bounded_wait_selftest_reports_timeout():
+    ws = nat.Workspace(16, 32)
+    assert nat.status(ws) == 0
+    nat.selftest_wait(ws, 2000)  # 2 ms limit on a barrier nothing completes
+    assert nat.status(ws) == nat.STATUS_TIMEOUT
+    # the context stays usable
+    inp = synth.make_layer(2, 0, M=64)
+    full_parity(_sub(inp, 64, 1152, 256))
+
+
+def test_empty_batch_noop():
+    d = {"x": torch.zeros(0, 64, dtype=torch.bfloat16, device="cuda"),
+         "y": torch.zeros(0, 32, dtype=torch.bfloat16, device="cuda")}
+    ws = nat.Workspace(16, 64)
+    w = torch.zeros(32, 64, dtype=torch.int8, device="cuda")
+    s = torch.ones(32, device="cuda")
+    nat.linear(d["x"], d["x"].clone(), d["y"], w, s, 1.0, ws)
+    torch.cuda.synchronize()
+    assert nat.status(ws) == 0
+
+
+def test_invalid_arguments_leave_buffers_untouched():
+    inp = synth.make_layer(2, 0, M=64)
+    d = to_dev(inp)
+    ws = nat.Workspace(64, 1152)
+    before = d["y_prev"].clone()
+    with pytest.raises(nat.DstarError, match="INVALID_ARG"):
+        nat.linear(d["x_t"], d["x_prev"], d["y_prev"], d["w_q"], d["w_scale"], 0.1, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(before, d["y_prev"])
