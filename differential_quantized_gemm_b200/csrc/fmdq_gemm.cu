@@ -33,9 +33,11 @@ namespace fmdq {
 
 namespace {
 
-constexpr int kGThreads = 192;
-constexpr int kA0Bytes = kBlockM * kChunkK;  // 16 KB
-constexpr int kA1Bufs = 2;
+constexpr int kEpiWarps = 8;                       // two per TMEM lane quarter, each half the columns
+constexpr int kGThreads = 64 + 32 * kEpiWarps;     // producer warp, MMA warp, epilogue warps
+constexpr int kA0Bytes = kBlockM * kChunkK;        // 16 KB
+constexpr int kMaxTileSlots = 64;                  // tiles per CTA whose block info is precomputed
+constexpr int kEpiBarrier = 1;                     // named barrier of the epilogue warps
 
 template <int BN>
 struct GemmCfg {
@@ -43,24 +45,30 @@ struct GemmCfg {
   static constexpr int kWBytes = BN * kChunkK;
   static constexpr int kStageBytes = kA0Bytes + kWBytes;
   static constexpr int kSlots = 512 / BN;
-  static constexpr int kGroups = BN / 32;
-  // shared memory map (offsets from a 1024-aligned base)
-  static constexpr int kOffA1 = kStages * kStageBytes;
-  static constexpr int kOffBar = kOffA1 + kA1Bufs * kA0Bytes;
-  static constexpr int kNumBars = 2 * kStages + kA1Bufs + 2 * kSlots + 1;
-  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr int kBytes = kOffMisc + 64 + 1024;  // + alignment slack
+  static constexpr int kHalfGroups = BN / 64;  // 32-column groups per epilogue warp
+  // small region first, then the 1024-aligned operand buffers
+  static constexpr int kNumBars = 2 * kStages + 1 + 2 * kSlots + 1;
+  static constexpr int kOffBar = 0;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;            // tmem base, abort flag
+  static constexpr int kOffWs = kOffMisc + 16;                       // [2][BN] fp32 weight scales
+  static constexpr int kOffInfo = kOffWs + 2 * BN * 4;               // [kMaxTileSlots] block info
+  static constexpr int kSmallBytes = kOffInfo + kMaxTileSlots * 16;
+  static constexpr int kOffStages = (kSmallBytes + 1023) & ~1023;
+  static constexpr int kOffA1 = kOffStages + kStages * kStageBytes;
+  static constexpr int kBytes = kOffA1 + kA0Bytes + 1024;            // + base alignment slack
 };
 
 struct BlockInfo {
-  int nplanes;  // 0: skip (all tiles of the row block go to the slice kernel), 1 or 2
+  int nplanes;  // 0: no tile of the row block uses the tensor cores; 1 or 2 planes
+  int any_slice;  // some tile of the row block goes through the slice stream
   uint32_t mask[2];
 };
 
-// Identical on every role: what the quantizer decided for this 128-row block.
-__device__ __forceinline__ BlockInfo block_info(const GemmParams& p, int rb) {
+// What the quantizer decided for a 128-row block (any thread, from global memory).
+__device__ __forceinline__ BlockInfo block_info_global(const GemmParams& p, int rb) {
   BlockInfo bi;
   bi.mask[0] = bi.mask[1] = 0;
+  bi.any_slice = 0;
   const int T = (int)(p.M / kTile);
   int np = 0;
   bool any = false;
@@ -69,6 +77,8 @@ __device__ __forceinline__ BlockInfo block_info(const GemmParams& p, int rb) {
     if (pl <= 2) {
       any = true;
       np = max(np, pl);
+    } else {
+      bi.any_slice = 1;
     }
     for (int w = 0; w < (int)p.mask_words && w < 2; ++w) bi.mask[w] |= p.mask1[(int64_t)t * p.mask_words + w];
   }
@@ -81,6 +91,10 @@ __device__ __forceinline__ bool chunk_has_plane1(const BlockInfo& bi, int c) {
 }
 
 __device__ __forceinline__ float exp2_exact(int e) { return __int_as_float((127 + e) << 23); }
+
+__device__ __forceinline__ void epi_barrier() {
+  asm volatile("bar.sync %0, %1;" ::"n"(kEpiBarrier), "n"(32 * kEpiWarps) : "memory");
+}
 
 template <bool OUT_BF16>
 struct OutT;
@@ -99,6 +113,68 @@ __device__ __forceinline__ float epi(int64_t acc, bool wide, float p2, float ws,
   return __fadd_rn(yp, __fmul_rn(__fmul_rn(a, p2), ws));
 }
 
+template <bool OUT_BF16>
+__device__ __forceinline__ float load_y(const void* base, int64_t off) {
+  if constexpr (OUT_BF16) return __bfloat162float(static_cast<const __nv_bfloat16*>(base)[off]);
+  else return static_cast<const float*>(base)[off];
+}
+
+template <bool OUT_BF16>
+__device__ __forceinline__ void store_y(void* base, int64_t off, float y) {
+  if constexpr (OUT_BF16) static_cast<__nv_bfloat16*>(base)[off] = __float2bfloat16_rn(y);
+  else static_cast<float*>(base)[off] = y;
+}
+
+// The paper's accumulation order literally, for one 16-token tile and one
+// output column n: walk the tile's encoded stream in (FPoT, channel) order;
+// when the FPoT changes, shift the 16 running sums left by the difference,
+// then add digit x w[n][k] (section 3.1 step 5, Fig. 6).  The sums end in
+// units of the last FPoT and are shifted to g_ref.
+template <bool OUT_BF16>
+__device__ void slice_stream_column(const uint2* recs, int cnt, const int8_t* bits_row, int g_ref,
+                                    const int8_t* w_row, int64_t t, int64_t n, int lb, float ws,
+                                    void* y_prev, int64_t ld_yp, void* y_out, int64_t ld_yo, int y_distinct,
+                                    int64_t* debug_acc, int64_t N) {
+  int64_t acc[kTile];
+#pragma unroll
+  for (int i = 0; i < kTile; ++i) acc[i] = 0;
+  int prev = 0;
+  for (int r = 0; r < cnt; ++r) {
+    const uint2 rec = recs[r];
+    const int k = (int)(rec.y & 0xFFFFu);
+    const int tag = (int)(int8_t)((rec.y >> 16) & 0xFFu);
+    const int j = (int)(rec.y >> 24);
+    if (r > 0 && tag != prev) {
+      const int sh = tag - prev;
+#pragma unroll
+      for (int i = 0; i < kTile; ++i) acc[i] *= ((int64_t)1 << sh);
+    }
+    prev = tag;
+    const bool top = j == (bits_row[k] >> 1) - 1;
+    const int64_t w = (int64_t)w_row[k];
+#pragma unroll
+    for (int i = 0; i < kTile; ++i) {
+      int d = (int)((rec.x >> (2 * i)) & 3u);
+      if (top && d >= 2) d -= 4;
+      acc[i] += (int64_t)d * w;
+    }
+  }
+  if (cnt > 0 && g_ref != prev) {
+    const int sh = g_ref - prev;
+#pragma unroll
+    for (int i = 0; i < kTile; ++i) acc[i] *= ((int64_t)1 << sh);
+  }
+  const float p2 = exp2_exact(-lb - g_ref);
+#pragma unroll
+  for (int i = 0; i < kTile; ++i) {
+    const int64_t row = t * kTile + i;
+    const float y = epi(acc[i], true, p2, ws, load_y<OUT_BF16>(y_prev, row * ld_yp + n));
+    store_y<OUT_BF16>(y_out, row * ld_yo + n, y);
+    if (y_distinct) store_y<OUT_BF16>(y_prev, row * ld_yp + n, y);
+    if (debug_acc) debug_acc[row * N + n] = acc[i];
+  }
+}
+
 }  // namespace
 
 size_t gemm_smem_bytes(int bn) { return bn == 256 ? GemmCfg<256>::kBytes : GemmCfg<128>::kBytes; }
@@ -114,26 +190,48 @@ __global__ void __launch_bounds__(kGThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* full = bars;                       // [kStages] TMA -> MMA
   uint64_t* empty = full + C::kStages;         // [kStages] MMA -> TMA
-  uint64_t* a1_empty = empty + C::kStages;     // [kA1Bufs] MMA -> TMA
-  uint64_t* tm_full = a1_empty + kA1Bufs;      // [kSlots] MMA -> epilogue
+  uint64_t* a1_empty = empty + C::kStages;     // MMA -> TMA (the plane-1 buffer)
+  uint64_t* tm_full = a1_empty + 1;            // [kSlots] MMA -> epilogue
   uint64_t* tm_empty = tm_full + C::kSlots;    // [kSlots] epilogue -> MMA
   uint64_t* drain = tm_empty + C::kSlots;      // MMA completion at exit
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+  float* s_ws = reinterpret_cast<float*>(smem + C::kOffWs);
+  int4* s_info = reinterpret_cast<int4*>(smem + C::kOffInfo);  // {nplanes, any_slice, mask0, mask1}
+  uint8_t* stages = smem + C::kOffStages;
+  uint8_t* a1buf = smem + C::kOffA1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int num_tiles = p.tiles_m * p.tiles_n;
+  const int my_tiles = num_tiles > (int)blockIdx.x ? (num_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  const int T = (int)(p.M / kTile);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kStages; ++i) mbar_init(&full[i], 1), mbar_init(&empty[i], 1);
-    for (int i = 0; i < kA1Bufs; ++i) mbar_init(&a1_empty[i], 1);
-    for (int i = 0; i < C::kSlots; ++i) mbar_init(&tm_full[i], 1), mbar_init(&tm_empty[i], 4);
+    mbar_init(a1_empty, 1);
+    for (int i = 0; i < C::kSlots; ++i) mbar_init(&tm_full[i], 1), mbar_init(&tm_empty[i], kEpiWarps);
     mbar_init(drain, 1);
     *s_abort = 0;
     fence_barrier_init();
     prefetch_tmap(&tm_a0);
     prefetch_tmap(&tm_a1);
     prefetch_tmap(&tm_w);
+  }
+  // block info of this CTA's first kMaxTileSlots tiles, loaded in parallel
+  for (int i = threadIdx.x; i < kMaxTileSlots; i += kGThreads) s_info[i] = make_int4(0, 0, 0, 0);
+  __syncthreads();
+  for (int i = threadIdx.x; i < min(my_tiles, kMaxTileSlots) * 8; i += kGThreads) {
+    const int slot = i >> 3, sub = i & 7;
+    const int rb = ((int)blockIdx.x + slot * (int)gridDim.x) / p.tiles_n;
+    const int t = rb * 8 + sub;
+    if (t < T) {
+      const int pl = p.planes[t];
+      int* e = reinterpret_cast<int*>(&s_info[slot]);
+      if (pl <= 2) atomicMax(&e[0], pl);
+      else atomicOr(&e[1], 1);
+      if (p.mask_words > 0) atomicOr(reinterpret_cast<unsigned*>(&e[2]), p.mask1[(int64_t)t * p.mask_words]);
+      if (p.mask_words > 1) atomicOr(reinterpret_cast<unsigned*>(&e[3]), p.mask1[(int64_t)t * p.mask_words + 1]);
+    }
   }
   if (warp == 1) {
     tmem_alloc(s_tmem, 512);
@@ -144,14 +242,27 @@ __global__ void __launch_bounds__(kGThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
 
+  auto info = [&](int slot, int rb) -> BlockInfo {
+    if (slot < kMaxTileSlots) {
+      const int4 e = s_info[slot];
+      BlockInfo bi;
+      bi.mask[0] = (uint32_t)e.z, bi.mask[1] = (uint32_t)e.w;
+      bi.any_slice = e.y;
+      bi.nplanes = e.x == 0 ? 0 : (e.x == 2 && (e.z | e.w)) ? 2 : 1;
+      return bi;
+    }
+    return block_info_global(p, rb);
+  };
+
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (elect_one()) {
       uint32_t it = 0, a1_it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      for (int slot = 0; slot < my_tiles && ok; ++slot) {
+        const int tile = (int)blockIdx.x + slot * (int)gridDim.x;
         const int rb = tile / p.tiles_n, nb = tile % p.tiles_n;
-        const BlockInfo bi = block_info(p, rb);
+        const BlockInfo bi = info(slot, rb);
         if (bi.nplanes == 0) continue;
         for (int c = 0; c < p.num_chunks; ++c, ++it) {
           const int s = it % C::kStages;
@@ -160,20 +271,17 @@ __global__ void __launch_bounds__(kGThreads, 1)
             break;
           }
           const bool use1 = chunk_has_plane1(bi, c);
-          if (use1 && !wait_parity(&a1_empty[a1_it % kA1Bufs], ((a1_it / kA1Bufs) & 1) ^ 1, s_abort, p.status,
-                                   kWaitLimitNs)) {
-            // nothing was loaded into this stage; the MMA side leaves on the abort flag
-            ok = false;
+          if (use1 && !wait_parity(a1_empty, (a1_it & 1) ^ 1, s_abort, p.status, kWaitLimitNs)) {
+            ok = false;  // nothing was loaded into this stage; the MMA side leaves on the abort flag
             break;
           }
-          uint8_t* a0 = smem + s * C::kStageBytes;
+          uint8_t* a0 = stages + s * C::kStageBytes;
           uint8_t* wb = a0 + kA0Bytes;
           mbar_arrive_expect_tx(&full[s], C::kStageBytes + (use1 ? kA0Bytes : 0));
           tma_load_2d(a0, &tm_a0, &full[s], c * kChunkK, rb * kBlockM);
           tma_load_2d(wb, &tm_w, &full[s], c * kChunkK, nb * BN);
           if (use1) {
-            uint8_t* a1 = smem + C::kOffA1 + (a1_it % kA1Bufs) * kA0Bytes;
-            tma_load_2d(a1, &tm_a1, &full[s], c * kChunkK, rb * kBlockM);
+            tma_load_2d(a1buf, &tm_a1, &full[s], c * kChunkK, rb * kBlockM);
             ++a1_it;
           }
         }
@@ -189,21 +297,21 @@ __global__ void __launch_bounds__(kGThreads, 1)
       constexpr uint32_t idesc = idesc_i8(BN);
       uint32_t it = 0, a1_it = 0, slot_it = 0;
       bool ok = true, issued = false;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int rb = tile / p.tiles_n;
-        const BlockInfo bi = block_info(p, rb);
+      for (int slot = 0; slot < my_tiles && ok; ++slot) {
+        const int tile = (int)blockIdx.x + slot * (int)gridDim.x;
+        const BlockInfo bi = info(slot, tile / p.tiles_n);
         if (bi.nplanes == 0) continue;
         // acquire accumulator slots
-        uint32_t slot[2];
+        uint32_t acc_slot[2];
         for (int q = 0; q < bi.nplanes && ok; ++q) {
           const uint32_t si = slot_it + q;
-          slot[q] = si % C::kSlots;
-          ok = wait_parity(&tm_empty[slot[q]], ((si / C::kSlots) & 1) ^ 1, s_abort, p.status, kWaitLimitNs);
+          acc_slot[q] = si % C::kSlots;
+          ok = wait_parity(&tm_empty[acc_slot[q]], ((si / C::kSlots) & 1) ^ 1, s_abort, p.status, kWaitLimitNs);
         }
         if (!ok) break;
         tc_fence_after();
-        const uint32_t d0 = tmem_base + slot[0] * BN;
-        const uint32_t d1 = tmem_base + (bi.nplanes == 2 ? slot[1] : slot[0]) * BN;
+        const uint32_t d0 = tmem_base + acc_slot[0] * BN;
+        const uint32_t d1 = tmem_base + (bi.nplanes == 2 ? acc_slot[1] : acc_slot[0]) * BN;
         bool first1 = true;
         for (int c = 0; c < p.num_chunks; ++c, ++it) {
           const int s = it % C::kStages;
@@ -212,25 +320,25 @@ __global__ void __launch_bounds__(kGThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint64_t da = smem_desc_k_sw128(smem + s * C::kStageBytes);
-          const uint64_t dw = smem_desc_k_sw128(smem + s * C::kStageBytes + kA0Bytes);
+          const uint64_t da = smem_desc_k_sw128(stages + s * C::kStageBytes);
+          const uint64_t dw = smem_desc_k_sw128(stages + s * C::kStageBytes + kA0Bytes);
 #pragma unroll
           for (int kk = 0; kk < kChunkK / 32; ++kk)
             mma_i8(d0, da + 2 * kk, dw + 2 * kk, idesc, (c > 0 || kk > 0) ? 1u : 0u);
           if (chunk_has_plane1(bi, c)) {
-            const uint64_t d_a1 = smem_desc_k_sw128(smem + C::kOffA1 + (a1_it % kA1Bufs) * kA0Bytes);
+            const uint64_t d_a1 = smem_desc_k_sw128(a1buf);
 #pragma unroll
             for (int kk = 0; kk < kChunkK / 32; ++kk)
               mma_i8(d1, d_a1 + 2 * kk, dw + 2 * kk, idesc, (!first1 || kk > 0) ? 1u : 0u);
             first1 = false;
-            mma_commit(&a1_empty[a1_it % kA1Bufs]);
+            mma_commit(a1_empty);
             ++a1_it;
           }
           mma_commit(&empty[s]);
           issued = true;
         }
         if (!ok) break;
-        for (int q = 0; q < bi.nplanes; ++q) mma_commit(&tm_full[slot[q]]);
+        for (int q = 0; q < bi.nplanes; ++q) mma_commit(&tm_full[acc_slot[q]]);
         slot_it += bi.nplanes;
       }
       // drain: all MMAs this thread issued complete before TMEM and SMEM go away
@@ -241,122 +349,137 @@ __global__ void __launch_bounds__(kGThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31 are this warp's
+    const int ew = warp - 2;           // 0 .. kEpiWarps-1
+    const int etid = threadIdx.x - 64; // 0 .. 32*kEpiWarps-1
+    const int quarter = warp & 3;      // TMEM lanes 32*quarter .. +31 are this warp's rows
+    const int half = ew >> 2;          // columns [half*BN/2, (half+1)*BN/2)
+    constexpr int kVecPerGroup = 32 * (int)sizeof(TOut) / 16;  // 16-byte vectors per 32 columns
     uint32_t slot_it = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+    int ok = 1;
+    // Every epilogue warp runs every iteration and both named barriers of it,
+    // also after a timed-out wait (ok == 0), so no warp can be left waiting
+    // at a barrier that another warp skipped.
+    for (int slot = 0; slot < my_tiles; ++slot) {
+      const int tile = (int)blockIdx.x + slot * (int)gridDim.x;
       const int rb = tile / p.tiles_n, nb = tile % p.tiles_n;
-      const BlockInfo bi = block_info(p, rb);
-      if (bi.nplanes == 0) continue;
-      const int64_t row = (int64_t)rb * kBlockM + quarter * 32 + lane;
-      const bool in_range = row < p.M;
-      const int t = (int)(row / kTile);
-      const int pl = in_range ? p.planes[t] : 3;
-      const bool row_ok = in_range && pl <= 2;
-      const float p2 = row_ok ? exp2_exact(-p.lb - p.g_ref[t]) : 0.f;
+      const BlockInfo bi = info(slot, rb);
       const int64_t n_base = (int64_t)nb * BN;
-      const TOut* yp_row = reinterpret_cast<const TOut*>(p.y_prev) + (row_ok ? row : 0) * p.ld_yp;
+      // weight scales of the tile's columns, double-buffered by tile parity
+      float* ws_t = s_ws + (slot & 1) * BN;
+      for (int i = etid; i < BN; i += 32 * kEpiWarps) ws_t[i] = (n_base + i < p.N) ? p.w_scale[n_base + i] : 0.f;
+      epi_barrier();
 
-      // issue the y_prev loads of the whole tile before the accumulator is ready
-      constexpr int kVecPerGroup = 32 * (int)sizeof(TOut) / 16;  // 16-byte vectors per 32 columns
-      constexpr int kPre = OUT_BF16 ? C::kGroups : 1;             // groups prefetched
-      uint4 ypv[kPre][kVecPerGroup];
-      if constexpr (OUT_BF16) {
+      if (ok && bi.nplanes > 0) {
+        const int64_t row = (int64_t)rb * kBlockM + quarter * 32 + lane;
+        const bool in_range = row < p.M;
+        const int t = (int)(row / kTile);
+        const int pl = in_range ? p.planes[t] : 3;
+        const bool row_ok = in_range && pl <= 2;
+        const float p2 = row_ok ? exp2_exact(-p.lb - p.g_ref[t]) : 0.f;
+        const int64_t n_half = n_base + half * (BN / 2);
+        const TOut* yp_row = reinterpret_cast<const TOut*>(p.y_prev) + (row_ok ? row : 0) * p.ld_yp;
+
+        // y_prev of this thread's row and columns, loaded before the accumulator is ready
+        uint4 ypv[C::kHalfGroups][kVecPerGroup];
 #pragma unroll
-        for (int g = 0; g < kPre; ++g)
+        for (int g = 0; g < C::kHalfGroups; ++g)
 #pragma unroll
           for (int v = 0; v < kVecPerGroup; ++v) {
-            const int64_t n = n_base + g * 32 + v * (16 / (int)sizeof(TOut));
-            ypv[g][v] = (row_ok && n < p.N) ? __ldg(reinterpret_cast<const uint4*>(yp_row + n)) : make_uint4(0, 0, 0, 0);
+            const int64_t n = n_half + g * 32 + v * (16 / (int)sizeof(TOut));
+            ypv[g][v] = (row_ok && n < p.N) ? __ldg(reinterpret_cast<const uint4*>(yp_row + n))
+                                            : make_uint4(0, 0, 0, 0);
           }
-      }
 
-      uint32_t slot[2];
-      int ok = 1;
-      for (int q = 0; q < bi.nplanes; ++q) {
-        const uint32_t si = slot_it + q;
-        slot[q] = si % C::kSlots;
-        // one lane polls; the warp follows its verdict (tcgen05.ld needs the whole warp)
-        if (lane == 0 && ok)
-          ok = wait_parity(&tm_full[slot[q]], (si / C::kSlots) & 1, s_abort, p.status, kWaitLimitNs) ? 1 : 0;
-      }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) break;
-      tc_fence_after();
-      const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-      const uint32_t t0 = tmem_base + lane_off + slot[0] * BN;
-      const uint32_t t1 = tmem_base + lane_off + (bi.nplanes == 2 ? slot[1] : slot[0]) * BN;
-
-#pragma unroll
-      for (int g = 0; g < C::kGroups; ++g) {
-        uint32_t d0[32], d1[32];
-        tmem_ld32(t0 + g * 32, d0);
-        if (bi.nplanes == 2) tmem_ld32(t1 + g * 32, d1);
-        tmem_ld_wait();
-        const int64_t n0 = n_base + g * 32;
-        uint4 yv[kVecPerGroup];
-        if constexpr (OUT_BF16) {
-#pragma unroll
-          for (int v = 0; v < kVecPerGroup; ++v) yv[v] = ypv[g][v];
-        } else {
-#pragma unroll
-          for (int v = 0; v < kVecPerGroup; ++v) {
-            const int64_t n = n0 + v * 4;
-            yv[v] = (row_ok && n < p.N) ? __ldg(reinterpret_cast<const uint4*>(yp_row + n)) : make_uint4(0, 0, 0, 0);
-          }
+        uint32_t acc_slot[2];
+        for (int q = 0; q < bi.nplanes; ++q) {
+          const uint32_t si = slot_it + q;
+          acc_slot[q] = si % C::kSlots;
+          // one lane polls; the warp follows its verdict (tcgen05.ld needs the whole warp)
+          if (lane == 0 && ok)
+            ok = wait_parity(&tm_full[acc_slot[q]], (si / C::kSlots) & 1, s_abort, p.status, kWaitLimitNs) ? 1 : 0;
         }
-        if (row_ok && n0 < p.N) {
-          const bool wide = pl == 2;
-          float y[32];
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (ok) {
+        tc_fence_after();
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        const uint32_t col_half = half * (BN / 2);
+        const uint32_t t0a = tmem_base + lane_off + acc_slot[0] * BN + col_half;
+        const uint32_t t1a = tmem_base + lane_off + (bi.nplanes == 2 ? acc_slot[1] : acc_slot[0]) * BN + col_half;
+        const float* ws_h = ws_t + half * (BN / 2);
+
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int64_t acc = wide ? (int64_t)(int32_t)d0[i] + (int64_t)(int32_t)d1[i] * 256 : (int64_t)(int32_t)d0[i];
-            float ypf;
-            if constexpr (OUT_BF16) {
-              const uint32_t w = reinterpret_cast<const uint32_t*>(yv)[i >> 1];
-              ypf = __uint_as_float((i & 1) ? (w & 0xFFFF0000u) : (w << 16));
-            } else {
-              ypf = __uint_as_float(reinterpret_cast<const uint32_t*>(yv)[i]);
+        for (int g = 0; g < C::kHalfGroups; ++g) {
+          uint32_t d0[32], d1[32];
+          tmem_ld32(t0a + g * 32, d0);
+          if (bi.nplanes == 2) tmem_ld32(t1a + g * 32, d1);
+          tmem_ld_wait();
+          const int64_t n0 = n_half + g * 32;
+          if (row_ok && n0 < p.N) {
+            const bool wide = pl == 2;
+            float y[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int64_t acc = wide ? (int64_t)(int32_t)d0[i] + (int64_t)(int32_t)d1[i] * 256
+                                       : (int64_t)(int32_t)d0[i];
+              float ypf;
+              if constexpr (OUT_BF16) {
+                const uint32_t w = reinterpret_cast<const uint32_t*>(ypv[g])[i >> 1];
+                ypf = __uint_as_float((i & 1) ? (w & 0xFFFF0000u) : (w << 16));
+              } else {
+                ypf = __uint_as_float(reinterpret_cast<const uint32_t*>(ypv[g])[i]);
+              }
+              y[i] = epi(acc, wide, p2, ws_h[g * 32 + i], ypf);
+              if (p.debug_acc && n0 + i < p.N) p.debug_acc[row * p.N + n0 + i] = acc;
             }
-            const float ws = (n0 + i < p.N) ? __ldg(p.w_scale + n0 + i) : 0.f;
-            y[i] = epi(acc, wide, p2, ws, ypf);
-            if (p.debug_acc && n0 + i < p.N) p.debug_acc[row * p.N + n0 + i] = acc;
-          }
-          const int64_t nv_rem = (p.N - n0) * (int64_t)sizeof(TOut) / 16;
-          const int nv = nv_rem < kVecPerGroup ? (int)nv_rem : kVecPerGroup;
-          uint4 ov[kVecPerGroup];
-          if constexpr (OUT_BF16) {
+            const int64_t nv_rem = (p.N - n0) * (int64_t)sizeof(TOut) / 16;
+            const int nv = nv_rem < kVecPerGroup ? (int)nv_rem : kVecPerGroup;
+            TOut* yo = reinterpret_cast<TOut*>(p.y_out) + row * p.ld_yo + n0;
+            TOut* yq = reinterpret_cast<TOut*>(p.y_prev) + row * p.ld_yp + n0;
 #pragma unroll
             for (int v = 0; v < kVecPerGroup; ++v) {
-              uint32_t w[4];
+              uint4 o;
+              if constexpr (OUT_BF16) {
+                uint32_t w[4];
 #pragma unroll
-              for (int h = 0; h < 4; ++h) {
-                const __nv_bfloat162 b2 = __floats2bfloat162_rn(y[v * 8 + 2 * h], y[v * 8 + 2 * h + 1]);
-                w[h] = *reinterpret_cast<const uint32_t*>(&b2);
+                for (int h = 0; h < 4; ++h) {
+                  const __nv_bfloat162 b2 = __floats2bfloat162_rn(y[v * 8 + 2 * h], y[v * 8 + 2 * h + 1]);
+                  w[h] = *reinterpret_cast<const uint32_t*>(&b2);
+                }
+                o = make_uint4(w[0], w[1], w[2], w[3]);
+              } else {
+                o = make_uint4(__float_as_uint(y[4 * v]), __float_as_uint(y[4 * v + 1]),
+                               __float_as_uint(y[4 * v + 2]), __float_as_uint(y[4 * v + 3]));
               }
-              ov[v] = make_uint4(w[0], w[1], w[2], w[3]);
-            }
-          } else {
-#pragma unroll
-            for (int v = 0; v < kVecPerGroup; ++v)
-              ov[v] = make_uint4(__float_as_uint(y[4 * v]), __float_as_uint(y[4 * v + 1]), __float_as_uint(y[4 * v + 2]),
-                                 __float_as_uint(y[4 * v + 3]));
-          }
-          TOut* yo = reinterpret_cast<TOut*>(p.y_out) + row * p.ld_yo + n0;
-          TOut* yq = reinterpret_cast<TOut*>(p.y_prev) + row * p.ld_yp + n0;
-#pragma unroll
-          for (int v = 0; v < kVecPerGroup; ++v) {
-            if (v < nv) {
-              reinterpret_cast<uint4*>(yo)[v] = ov[v];
-              if (p.y_distinct) reinterpret_cast<uint4*>(yq)[v] = ov[v];
+              if (v < nv) {
+                reinterpret_cast<uint4*>(yo)[v] = o;
+                if (p.y_distinct) reinterpret_cast<uint4*>(yq)[v] = o;
+              }
             }
           }
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0)
+          for (int q = 0; q < bi.nplanes; ++q) mbar_arrive(&tm_empty[acc_slot[q]]);
+        slot_it += bi.nplanes;
+        }  // ok
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0)
-        for (int q = 0; q < bi.nplanes; ++q) mbar_arrive(&tm_empty[slot[q]]);
-      slot_it += bi.nplanes;
+
+      // tiles of this row block whose operands need more than two planes:
+      // the slice stream, one output column per epilogue thread
+      if (ok && bi.any_slice) {
+        for (int t = rb * 8; t < min(rb * 8 + 8, T); ++t) {
+          if (p.planes[t] <= 2) continue;
+          for (int c = etid; c < BN; c += 32 * kEpiWarps) {
+            const int64_t n = n_base + c;
+            if (n >= p.N) continue;
+            slice_stream_column<OUT_BF16>(p.records + (int64_t)t * p.record_cap, p.count[t], p.bits + (int64_t)t * p.K,
+                                          p.g_ref[t], p.w_q + n * p.ld_w, t, n, p.lb, ws_t[c], p.y_prev, p.ld_yp,
+                                          p.y_out, p.ld_yo, p.y_distinct, p.debug_acc, p.N);
+          }
+        }
+      }
+      epi_barrier();  // the weight-scale buffer of this parity is free again
     }
   }
 
@@ -370,85 +493,24 @@ __global__ void __launch_bounds__(kGThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// Slice-stream kernel: the paper's accumulation order literally.  One block
-// per (tile, 256 output columns); every thread owns one output column and
-// the 16 tokens of the tile.  It walks the tile's encoded stream in order:
-// when the FPoT changes it shifts the 16 running sums left by the difference,
-// then adds digit x w[n][k] (section 3.1 step 5, Fig. 6).  The sums end in
-// units of the last FPoT and are shifted to g_ref, then the same fp32
-// epilogue as the tensor-core kernel is applied.  Used for tiles whose
-// shift-folded operands need more than two int8 planes, and for every tile
-// under DSTAR_FLAG_SLICE_PATH.
+// Slice-stream kernel: every tile through the paper's accumulation order
+// (slice_stream_column), one block per (tile, 256 output columns), one output
+// column per thread.  Used under DSTAR_FLAG_SLICE_PATH; in the default path
+// the tensor-core kernel's epilogue warps run the same routine for the tiles
+// that need it.
 // ---------------------------------------------------------------------------
 template <bool OUT_BF16>
 __global__ void __launch_bounds__(256) slice_gemm_kernel(const SliceParams p) {
-  using TOut = typename OutT<OUT_BF16>::T;
-  __shared__ uint2 s_rec[256];
-  extern __shared__ int8_t s_bits[];  // [K]
   const int64_t T = p.M / kTile;
   const int64_t nblk = (p.N + 255) / 256;
   for (int64_t item = blockIdx.x; item < T * nblk; item += gridDim.x) {
     const int64_t t = item / nblk;
     const int64_t n = (item % nblk) * 256 + threadIdx.x;
-    if (!p.all_tiles && p.planes[t] <= 2) continue;  // uniform across the block
-    __syncthreads();
-    for (int64_t k = threadIdx.x; k < p.K; k += 256) s_bits[k] = p.bits[t * p.K + k];
-    const int cnt = p.count[t];
-    int64_t acc[kTile];
-#pragma unroll
-    for (int i = 0; i < kTile; ++i) acc[i] = 0;
-    int prev = 0;
-    for (int r0 = 0; r0 < cnt; r0 += 256) {
-      __syncthreads();
-      if (r0 + (int)threadIdx.x < cnt) s_rec[threadIdx.x] = p.records[t * p.record_cap + r0 + threadIdx.x];
-      __syncthreads();
-      const int rn = min(256, cnt - r0);
-      for (int r = 0; r < rn; ++r) {
-        const uint2 rec = s_rec[r];
-        const int k = (int)(rec.y & 0xFFFFu);
-        const int tag = (int)(int8_t)((rec.y >> 16) & 0xFFu);
-        const int j = (int)(rec.y >> 24);
-        if (r0 + r > 0 && tag != prev) {
-          const int sh = tag - prev;
-#pragma unroll
-          for (int i = 0; i < kTile; ++i) acc[i] *= ((int64_t)1 << sh);
-        }
-        prev = tag;
-        const int top = (j == (s_bits[k] >> 1) - 1);
-        const int64_t w = (n < p.N) ? (int64_t)p.w_q[n * p.ld_w + k] : 0;
-#pragma unroll
-        for (int i = 0; i < kTile; ++i) {
-          int d = (int)((rec.x >> (2 * i)) & 3u);
-          if (top && d >= 2) d -= 4;
-          acc[i] += (int64_t)d * w;
-        }
-      }
-    }
-    if (cnt > 0 && p.g_ref[t] != prev) {
-      const int sh = p.g_ref[t] - prev;
-#pragma unroll
-      for (int i = 0; i < kTile; ++i) acc[i] *= ((int64_t)1 << sh);
-    }
-    if (n < p.N) {
-      const float p2 = exp2_exact(-p.lb - p.g_ref[t]);
-      const float ws = p.w_scale[n];
-#pragma unroll
-      for (int i = 0; i < kTile; ++i) {
-        const int64_t row = t * kTile + i;
-        TOut* yp = reinterpret_cast<TOut*>(p.y_prev) + row * p.ld_yp + n;
-        TOut* yo = reinterpret_cast<TOut*>(p.y_out) + row * p.ld_yo + n;
-        float ypf;
-        if constexpr (OUT_BF16) ypf = __bfloat162float(*yp);
-        else ypf = *yp;
-        const float y = epi(acc[i], true, p2, ws, ypf);
-        TOut o;
-        if constexpr (OUT_BF16) o = __float2bfloat16_rn(y);
-        else o = y;
-        *yo = o;
-        if (p.y_distinct) *yp = o;
-        if (p.debug_acc) p.debug_acc[row * p.N + n] = acc[i];
-      }
-    }
+    if (!p.all_tiles && p.planes[t] <= 2) continue;
+    if (n >= p.N) continue;
+    slice_stream_column<OUT_BF16>(p.records + t * p.record_cap, p.count[t], p.bits + t * p.K, p.g_ref[t],
+                                  p.w_q + n * p.ld_w, t, n, p.lb, p.w_scale[n], p.y_prev, p.ld_yp, p.y_out, p.ld_yo,
+                                  p.y_distinct, p.debug_acc, p.N);
   }
 }
 
@@ -472,8 +534,8 @@ static int launch_gemm_t(const GemmParams& p, const void* a0, const void* a1, co
   const int grid = tiles < num_sms ? tiles : num_sms;
   if (grid == 0) return 0;
   const int smem = GemmCfg<BN>::kBytes;
-  cudaError_t e = cudaFuncSetAttribute(gemm_kernel<BN, BF>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return (int)e;
+  const int e = ensure_max_smem((const void*)gemm_kernel<BN, BF>, smem);
+  if (e != 0) return e;
   gemm_kernel<BN, BF><<<grid, kGThreads, smem, (cudaStream_t)stream>>>(
       *static_cast<const CUtensorMap*>(a0), *static_cast<const CUtensorMap*>(a1),
       *static_cast<const CUtensorMap*>(w), p);
@@ -493,9 +555,8 @@ int launch_slice_gemm(const SliceParams& p, int out_bf16, int num_sms, void* str
   const int64_t items = T * ((p.N + 255) / 256);
   if (items == 0) return 0;
   const int64_t grid = items < 4LL * num_sms ? items : 4LL * num_sms;
-  const size_t smem = (size_t)p.K;
-  if (out_bf16) slice_gemm_kernel<true><<<(unsigned)grid, 256, smem, (cudaStream_t)stream>>>(p);
-  else slice_gemm_kernel<false><<<(unsigned)grid, 256, smem, (cudaStream_t)stream>>>(p);
+  if (out_bf16) slice_gemm_kernel<true><<<(unsigned)grid, 256, 0, (cudaStream_t)stream>>>(p);
+  else slice_gemm_kernel<false><<<(unsigned)grid, 256, 0, (cudaStream_t)stream>>>(p);
   return (int)cudaGetLastError();
 }
 

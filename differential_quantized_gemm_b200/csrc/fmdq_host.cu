@@ -242,8 +242,15 @@ int do_gemm(const dstar_mat* w_q, const float* w_scale, dstar_mat* y_prev, int l
     g.tiles_m = (int)((M + kBlockM - 1) / kBlockM);
     g.tiles_n = (int)((N + bn - 1) / bn);
     g.num_chunks = (int)((K + kChunkK - 1) / kChunkK);
+    g.w_q = static_cast<const int8_t*>(w_q->data);
+    g.ld_w = w_q->ld;
+    g.records = ws_ptr<const uint2>(c, L.records);
+    g.record_cap = L.record_cap;
+    g.count = ws_ptr<const int32_t>(c, L.count);
+    g.bits = ws_ptr<const int8_t>(c, L.bits);
     const int e = launch_gemm(g, &ma0, &ma1, &mw, bn, bf16, dev.sms, stream);
     if (e) return cuda_fail(e, "slice-GEMM launch");
+    return DSTAR_OK;  // tiles needing the slice stream are handled inside the GEMM kernel
   }
   SliceParams s{};
   s.M = M, s.N = N, s.K = K;
@@ -262,7 +269,7 @@ int do_gemm(const dstar_mat* w_q, const float* w_scale, dstar_mat* y_prev, int l
   s.y_out = y_out->data;
   s.ld_yo = y_out->ld;
   s.y_distinct = distinct;
-  s.all_tiles = slice_all;
+  s.all_tiles = 1;
   s.debug_acc = c->debug_acc;
   const int e = launch_slice_gemm(s, bf16, dev.sms, stream);
   if (e) return cuda_fail(e, "slice-stream launch");
@@ -289,7 +296,34 @@ int check_gemm_args(const dstar_mat* w_q, const float* w_scale, dstar_mat* y_pre
   return DSTAR_OK;
 }
 
+std::mutex g_attr_mu;
+struct AttrEntry {
+  int dev;
+  const void* func;
+  int bytes;
+};
+AttrEntry g_attr[64];
+int g_nattr = 0;
+
 }  // namespace
+
+int ensure_max_smem(const void* func, int bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return (int)e;
+  std::lock_guard<std::mutex> lk(g_attr_mu);
+  for (int i = 0; i < g_nattr; ++i)
+    if (g_attr[i].dev == dev && g_attr[i].func == func && g_attr[i].bytes >= bytes) return 0;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return (int)e;
+  for (int i = 0; i < g_nattr; ++i)
+    if (g_attr[i].dev == dev && g_attr[i].func == func) {
+      g_attr[i].bytes = bytes;
+      return 0;
+    }
+  if (g_nattr < 64) g_attr[g_nattr++] = AttrEntry{dev, func, bytes};
+  return 0;
+}
 
 WsLayout ws_layout(int64_t M, int64_t K) {
   WsLayout L{};

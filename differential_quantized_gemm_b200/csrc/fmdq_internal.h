@@ -60,6 +60,13 @@ struct GemmParams {
   uint32_t* status;
   int64_t* debug_acc;
   int tiles_m, tiles_n, num_chunks;
+  // encoded stream, for tiles whose operands need more than two planes
+  const int8_t* w_q;
+  int64_t ld_w;
+  const uint2* records;
+  int64_t record_cap;
+  const int32_t* count;
+  const int8_t* bits;
 };
 
 struct SliceParams {
@@ -97,6 +104,10 @@ int launch_gemm(const GemmParams& p, const void* tmap_a0, const void* tmap_a1, c
 int launch_slice_gemm(const SliceParams& p, int out_bf16, int num_sms, void* stream);
 int launch_selftest_wait(uint32_t* status, uint32_t spin_limit, void* stream);
 size_t quantize_smem_bytes(int64_t K);
+// Raise a kernel's dynamic shared-memory limit once per device (returns a
+// cudaError_t as int); later calls only look up the cache, so launches stay
+// legal inside stream capture.
+int ensure_max_smem(const void* func, int bytes);
 size_t gemm_smem_bytes(int bn);
 
 }  // namespace fmdq

@@ -1,17 +1,18 @@
 // K1: the FMDQ quantizer (DSTAR section 3.1 steps 1-4; the paper's QPU,
 // section 4.2 "Design of QPU", stages 1-5).
 //
-// One 256-thread block per 16-token tile.  Phase 1 streams the tile's rows of
-// X_t and X_{t-1} once with 16-byte loads (coalesced along channels), forms
-// dX in fp32, takes the per-channel max |dX| as an integer max over the
-// magnitude bits (stage 1 compares the value without its sign), derives PoT
-// (Eq. 3), the bit width (threshold bins, stage 2), FPoT (Eq. 4) and the codes
-// q = rne(dX * s_i) with s_i = base * 2^FPoT (Eq. 5, stage 3), and keeps the
-// codes in shared memory.  Phase 2 knows the tile's finest FPoT (g_ref) and
-// writes (a) the tensor-core operand planes: v = q * 2^(g_ref - FPoT), split
-// into int8 planes v = A0 + 256 A1, and (b) the encoded stream: one record per
-// 2-bit slice, grouped by slice FPoT ascending and channel ascending (stages
-// 4-5), located by a per-tag count and exclusive scan instead of a sort.
+// One 256-thread block per 16-token tile.  Phase 1: every thread owns a pair
+// of adjacent channels and walks the 16 tokens of the tile, so a warp reads
+// whole 128-byte row segments of X_t and X_{t-1} and the per-channel max
+// |dX| (stage 1: compare the magnitude bits, sign dropped) stays inside the
+// thread.  PoT (Eq. 3), the bit width (threshold bins, stage 2), FPoT (Eq. 4)
+// and the codes q = rne(dX * s_i) with s_i = base * 2^FPoT (Eq. 5, stage 3)
+// follow per channel; the 16 codes of a channel go to shared memory as one
+// 16-byte column.  Phase 2 knows the tile's finest FPoT (g_ref) and writes
+// (a) the tensor-core operand planes v = q * 2^(g_ref - FPoT), split into int8
+// planes v = A0 + 256 A1, and (b) the encoded stream: one record per 2-bit
+// slice, grouped by slice FPoT ascending then channel ascending (stages 4-5),
+// placed by per-tag counts and an exclusive scan rather than a sort.
 #include <cuda_bf16.h>
 
 #include "fmdq_device.cuh"
@@ -25,82 +26,115 @@ constexpr int kQWarps = kQThreads / 32;
 constexpr int kMaxTags = 64;  // tag spread within a tile is at most 6 + kPotMax + 6 < 64
 constexpr int kMaxMaskWords = (DSTAR_K_MAX / kChunkK + 31) / 32;
 
+// Two adjacent channels of one token row.
 template <typename TIn>
-struct In;
+struct Pair;
 template <>
-struct In<float> {
-  static constexpr int kVec = 4;
-  __device__ static void load(const void* base, int64_t off, float (&v)[4]) {
-    float4 f = *reinterpret_cast<const float4*>(static_cast<const float*>(base) + off);
-    v[0] = f.x, v[1] = f.y, v[2] = f.z, v[3] = f.w;
+struct Pair<__nv_bfloat16> {
+  using Raw = uint32_t;
+  __device__ static Raw load(const void* base, int64_t off) {
+    return *reinterpret_cast<const uint32_t*>(static_cast<const __nv_bfloat16*>(base) + off);
   }
-  __device__ static uint4 raw(const void* base, int64_t off) {
-    return *reinterpret_cast<const uint4*>(static_cast<const float*>(base) + off);
+  __device__ static void store(void* base, int64_t off, Raw r) {
+    *reinterpret_cast<uint32_t*>(static_cast<__nv_bfloat16*>(base) + off) = r;
   }
-  __device__ static void store_raw(void* base, int64_t off, uint4 r) {
-    *reinterpret_cast<uint4*>(static_cast<float*>(base) + off) = r;
-  }
-  __device__ static void widen(uint4 r, float (&v)[4]) {
-    v[0] = __uint_as_float(r.x), v[1] = __uint_as_float(r.y), v[2] = __uint_as_float(r.z),
-    v[3] = __uint_as_float(r.w);
-  }
+  // bf16 -> fp32 is exact: the bf16 bits are the high half of the fp32 word
+  __device__ static float lo(Raw r) { return __uint_as_float(r << 16); }
+  __device__ static float hi(Raw r) { return __uint_as_float(r & 0xFFFF0000u); }
 };
 template <>
-struct In<__nv_bfloat16> {
-  static constexpr int kVec = 8;
-  __device__ static uint4 raw(const void* base, int64_t off) {
-    return *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(base) + off);
+struct Pair<float> {
+  using Raw = uint2;
+  __device__ static Raw load(const void* base, int64_t off) {
+    return *reinterpret_cast<const uint2*>(static_cast<const float*>(base) + off);
   }
-  __device__ static void store_raw(void* base, int64_t off, uint4 r) {
-    *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(base) + off) = r;
+  __device__ static void store(void* base, int64_t off, Raw r) {
+    *reinterpret_cast<uint2*>(static_cast<float*>(base) + off) = r;
   }
-  // bf16 -> fp32 is exact: the bf16 bits are the high half of the fp32 word.
-  __device__ static void widen(uint4 r, float (&v)[8]) {
-    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      v[2 * i] = __uint_as_float(w[i] << 16);
-      v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
-  }
+  __device__ static float lo(Raw r) { return __uint_as_float(r.x); }
+  __device__ static float hi(Raw r) { return __uint_as_float(r.y); }
 };
 
 __device__ __forceinline__ float exp2_exact(int e) {  // 2^e for e in the normal range
   return __int_as_float((127 + e) << 23);
 }
 
+// Per-channel parameters from the magnitude bits of M_i (section 3.1 step 1).
+struct ColParams {
+  int fpot, bits;
+  float scale;
+  bool nonfinite;
+};
+
+__device__ __forceinline__ ColParams col_params(uint32_t mbits, int lb, float beta, int t0, int fb, int& flags) {
+  ColParams cp;
+  cp.nonfinite = mbits >= 0x7F800000u;
+  int P = 0;
+  // Eq. 3 with the static base: PoT = ceil(log2(M_i / base)), 0 when M_i <= base.
+  // M_i > base >= 2^-32 is a normal float: M_i = (1 + f) 2^x  ->  PoT = x - lb + (f != 0).
+  if (!cp.nonfinite && __uint_as_float(mbits) > beta)
+    P = (int)(mbits >> 23) - 127 - lb + ((mbits & 0x7FFFFFu) != 0u ? 1 : 0);
+  if (cp.nonfinite) flags |= 1;
+  if (P > kPotMax) {
+    P = kPotMax;
+    flags |= 2;
+  }
+  // bins Thr_N = base * 2^(t0 + 2N): PoT <= t0 -> 2 bits, <= t0+2 -> 4, <= t0+4 -> 6, else 8
+  cp.bits = fb ? fb : (P <= t0 ? 2 : P <= t0 + 2 ? 4 : P <= t0 + 4 ? 6 : 8);
+  cp.fpot = cp.bits - 2 - 2 * lb - P;          // Eq. 4 with PCeil = 2^(b-2)
+  cp.scale = exp2_exact(cp.bits - 2 - lb - P);  // Eq. 5: s_i = base * 2^FPoT
+  return cp;
+}
+
+// The 2-bit field j of the 16 codes of a channel (byte r of word w = token
+// 4w + r), gathered into one word: token i in bits 2i..2i+1.
+__device__ __forceinline__ uint32_t slice_word(const uint4 cw, int j) {
+  const uint32_t ws[4] = {cw.x, cw.y, cw.z, cw.w};
+  uint32_t out = 0;
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    uint32_t x = (ws[w] >> (2 * j)) & 0x03030303u;
+    x = (x | (x >> 6)) & 0x000F000Fu;
+    x = (x | (x >> 12)) & 0xFFu;
+    out |= x << (8 * w);
+  }
+  return out;
+}
+
+__device__ __forceinline__ int code_at(const uint4 cw, int r) {
+  const uint32_t w = r < 4 ? cw.x : r < 8 ? cw.y : r < 12 ? cw.z : cw.w;
+  return (int)(int8_t)(w >> (8 * (r & 3)));
+}
+
 }  // namespace
 
 size_t quantize_smem_bytes(int64_t K) {
-  const size_t cs = (size_t)K + 64;                         // padded code row stride
-  size_t b = 16 * cs + 4 * (size_t)K;                       // codes + 4 per-column bytes
+  size_t b = 16 * (size_t)K + 4 * (size_t)K;  // column-major codes + 4 per-column bytes
   b = (b + 15) & ~(size_t)15;
   b += sizeof(int) * (64 + 2 * kQWarps * kMaxTags) + sizeof(uint32_t) * kMaxMaskWords;
   return b;
 }
 
 template <typename TIn>
-__global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p) {
+__global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParams p) {
   extern __shared__ __align__(16) uint8_t smem[];
-  constexpr int VEC = In<TIn>::kVec;
-  constexpr int CB = 8 * VEC;  // channels covered by one warp pass (8 lanes x VEC)
+  using PR = Pair<TIn>;
 
   const int64_t K = p.K;
-  const int64_t cs = K + 64;
   const int t = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  int8_t* s_codes = reinterpret_cast<int8_t*>(smem);  // [16][cs]
-  int8_t* s_fpot = s_codes + 16 * cs;                  // [K]
+  int8_t* s_code = reinterpret_cast<int8_t*>(smem);  // [K][16]: the 16 codes of channel k
+  int8_t* s_fpot = s_code + 16 * K;                   // [K]
   int8_t* s_bits = s_fpot + K;
   int8_t* s_qmax = s_bits + K;
   int8_t* s_qmin = s_qmax + K;
-  int* s_small = reinterpret_cast<int*>(smem + ((16 * cs + 4 * K + 15) & ~(int64_t)15));
+  int* s_small = reinterpret_cast<int*>(smem + ((20 * K + 15) & ~(int64_t)15));
   int* s_hist = s_small + 64;                  // [warps][kMaxTags]
   int* s_off = s_hist + kQWarps * kMaxTags;    // [warps][kMaxTags]
   uint32_t* s_mask = reinterpret_cast<uint32_t*>(s_off + kQWarps * kMaxTags);
   // s_small: [0,8) warp max FPoT, [8,16) warp min FPoT, [16,24) warp plane need,
-  //          [24] flags (1 nonfinite, 2 range), [25] g_ref, [26] min FPoT, [27] planes
+  //          [24] flags (1 nonfinite, 2 range), [25] g_ref, [26] min FPoT, [27] planes, [28] records
 
   if (tid < kMaxMaskWords) s_mask[tid] = 0;
   if (tid == 0) s_small[24] = 0;
@@ -109,122 +143,58 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
   const int lb = p.lb, t0 = p.t0, fb = p.force_bits;
   const float beta = exp2_exact(lb);
   const bool refresh = !(p.flags & DSTAR_FLAG_NO_XPREV_REFRESH);
-  const int rsub = lane >> 3;  // this lane's rows: 4*rsub .. 4*rsub+3
-  const int csub = lane & 7;   // this lane's channels: VEC consecutive
-  const int nblk = (int)((K + CB - 1) / CB);
+  const int64_t row0 = (int64_t)t * kTile;
+  const int npairs = (int)(K / 2);
   int fmax = -1000, fmin = 1000;
   int flags = 0;
 
   // ---------------------------------------------------------------- phase 1
-  for (int blk = warp; blk < nblk; blk += kQWarps) {
-    const int64_t c0 = (int64_t)blk * CB + csub * VEC;
-    const bool valid = c0 < K;  // K % 32 == 0: a lane's VEC channels are all valid or all not
-    float dx[4][VEC];
-    uint4 xt_raw[4], xp_raw[4];
-    if (valid) {
+  for (int pr = tid; pr < npairs; pr += kQThreads) {
+    const int64_t c = 2 * (int64_t)pr;
+    typename PR::Raw rt[kTile], rp[kTile];
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int64_t row = (int64_t)t * kTile + rsub * 4 + r;
-        xt_raw[r] = In<TIn>::raw(p.x_t, row * p.ld_xt + c0);
-        xp_raw[r] = In<TIn>::raw(p.x_prev, row * p.ld_xp + c0);
-      }
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        float a[VEC], b[VEC];
-        In<TIn>::widen(xt_raw[r], a);
-        In<TIn>::widen(xp_raw[r], b);
-#pragma unroll
-        for (int c = 0; c < VEC; ++c) dx[r][c] = __fsub_rn(a[c], b[c]);  // Eq. 1, one fp32 subtraction
-        if (refresh) {
-          const int64_t row = (int64_t)t * kTile + rsub * 4 + r;
-          In<TIn>::store_raw(p.x_prev, row * p.ld_xp + c0, xt_raw[r]);
-        }
-      }
-    } else {
-#pragma unroll
-      for (int r = 0; r < 4; ++r)
-#pragma unroll
-        for (int c = 0; c < VEC; ++c) dx[r][c] = 0.f;
+    for (int r = 0; r < kTile; ++r) {
+      rt[r] = PR::load(p.x_t, (row0 + r) * p.ld_xt + c);
+      rp[r] = PR::load(p.x_prev, (row0 + r) * p.ld_xp + c);
     }
-
-    // stage 1: max |dX| of each channel over the 16 tokens, on the magnitude bits
-    uint32_t mb[VEC];
+    if (refresh) {
 #pragma unroll
-    for (int c = 0; c < VEC; ++c) {
-      uint32_t m = 0;
-#pragma unroll
-      for (int r = 0; r < 4; ++r) m = max(m, __float_as_uint(dx[r][c]) & 0x7FFFFFFFu);
-      m = max(m, __shfl_xor_sync(0xffffffffu, m, 8));
-      m = max(m, __shfl_xor_sync(0xffffffffu, m, 16));
-      mb[c] = m;
+      for (int r = 0; r < kTile; ++r) PR::store(p.x_prev, (row0 + r) * p.ld_xp + c, rt[r]);
     }
-
-    int8_t qv[4][VEC];
-    int fp_c[VEC], b_c[VEC], qmx_c[VEC], qmn_c[VEC];
+    float d0[kTile], d1[kTile];
+    uint32_t m0 = 0, m1 = 0;
 #pragma unroll
-    for (int c = 0; c < VEC; ++c) {
-      const bool nonfinite = mb[c] >= 0x7F800000u;
-      int P = 0;
-      // stage 2, Eq. 3 with the static base: PoT = ceil(log2(M_i / base)), 0 when M_i <= base.
-      // M_i > base >= 2^-32 is a normal float: M_i = (1 + f) 2^x  ->  PoT = x - lb + (f != 0).
-      if (!nonfinite && __uint_as_float(mb[c]) > beta)
-        P = (int)(mb[c] >> 23) - 127 - lb + ((mb[c] & 0x7FFFFFu) != 0u ? 1 : 0);
-      if (nonfinite && valid) flags |= 1;
-      if (P > kPotMax) {
-        P = kPotMax;
-        if (valid) flags |= 2;
-      }
-      // bins Thr_N = base * 2^(t0 + 2N): PoT <= t0 -> 2 bits, <= t0+2 -> 4, <= t0+4 -> 6, else 8
-      const int b = fb ? fb : (P <= t0 ? 2 : P <= t0 + 2 ? 4 : P <= t0 + 4 ? 6 : 8);
-      const int fpot = b - 2 - 2 * lb - P;         // Eq. 4 with PCeil = 2^(b-2)
-      const float s = exp2_exact(b - 2 - lb - P);  // Eq. 5: s_i = base * 2^FPoT
-      int qmx = -128, qmn = 127;
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int q = nonfinite ? 0 : __float2int_rn(__fmul_rn(dx[r][c], s));  // stage 3
-        qv[r][c] = (int8_t)q;
-        qmx = max(qmx, q);
-        qmn = min(qmn, q);
-      }
-      qmx = max(qmx, __shfl_xor_sync(0xffffffffu, qmx, 8));
-      qmx = max(qmx, __shfl_xor_sync(0xffffffffu, qmx, 16));
-      qmn = min(qmn, __shfl_xor_sync(0xffffffffu, qmn, 8));
-      qmn = min(qmn, __shfl_xor_sync(0xffffffffu, qmn, 16));
-      fp_c[c] = fpot, b_c[c] = b, qmx_c[c] = qmx, qmn_c[c] = qmn;
-      if (valid) fmax = max(fmax, fpot), fmin = min(fmin, fpot);
+    for (int r = 0; r < kTile; ++r) {
+      d0[r] = __fsub_rn(PR::lo(rt[r]), PR::lo(rp[r]));  // Eq. 1, one fp32 subtraction
+      d1[r] = __fsub_rn(PR::hi(rt[r]), PR::hi(rp[r]));
+      m0 = max(m0, __float_as_uint(d0[r]) & 0x7FFFFFFFu);  // stage 1 on the magnitude bits
+      m1 = max(m1, __float_as_uint(d1[r]) & 0x7FFFFFFFu);
     }
-
-    if (valid) {
+    const ColParams c0 = col_params(m0, lb, beta, t0, fb, flags);
+    const ColParams c1 = col_params(m1, lb, beta, t0, fb, flags);
+    uint32_t w0[4] = {0, 0, 0, 0}, w1[4] = {0, 0, 0, 0};
+    int qmx0 = -128, qmn0 = 127, qmx1 = -128, qmn1 = 127;
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int row = rsub * 4 + r;
-        if constexpr (VEC == 8) {
-          uint2 w;
-          w.x = (uint32_t)(uint8_t)qv[r][0] | ((uint32_t)(uint8_t)qv[r][1] << 8) |
-                ((uint32_t)(uint8_t)qv[r][2] << 16) | ((uint32_t)(uint8_t)qv[r][3] << 24);
-          w.y = (uint32_t)(uint8_t)qv[r][4] | ((uint32_t)(uint8_t)qv[r][5] << 8) |
-                ((uint32_t)(uint8_t)qv[r][6] << 16) | ((uint32_t)(uint8_t)qv[r][7] << 24);
-          *reinterpret_cast<uint2*>(s_codes + row * cs + c0) = w;
-          if (p.debug_codes)
-            *reinterpret_cast<uint2*>(p.debug_codes + ((int64_t)t * kTile + row) * K + c0) = w;
-        } else {
-          uint32_t w = (uint32_t)(uint8_t)qv[r][0] | ((uint32_t)(uint8_t)qv[r][1] << 8) |
-                       ((uint32_t)(uint8_t)qv[r][2] << 16) | ((uint32_t)(uint8_t)qv[r][3] << 24);
-          *reinterpret_cast<uint32_t*>(s_codes + row * cs + c0) = w;
-          if (p.debug_codes)
-            *reinterpret_cast<uint32_t*>(p.debug_codes + ((int64_t)t * kTile + row) * K + c0) = w;
-        }
-      }
-      if (rsub == 0) {
-#pragma unroll
-        for (int c = 0; c < VEC; ++c) {
-          s_fpot[c0 + c] = (int8_t)fp_c[c];
-          s_bits[c0 + c] = (int8_t)b_c[c];
-          s_qmax[c0 + c] = (int8_t)qmx_c[c];
-          s_qmin[c0 + c] = (int8_t)qmn_c[c];
-        }
-      }
+    for (int r = 0; r < kTile; ++r) {
+      const int q0 = c0.nonfinite ? 0 : __float2int_rn(__fmul_rn(d0[r], c0.scale));  // stage 3
+      const int q1 = c1.nonfinite ? 0 : __float2int_rn(__fmul_rn(d1[r], c1.scale));
+      w0[r >> 2] |= ((uint32_t)q0 & 0xFFu) << (8 * (r & 3));
+      w1[r >> 2] |= ((uint32_t)q1 & 0xFFu) << (8 * (r & 3));
+      qmx0 = max(qmx0, q0), qmn0 = min(qmn0, q0);
+      qmx1 = max(qmx1, q1), qmn1 = min(qmn1, q1);
+      if (p.debug_codes)
+        *reinterpret_cast<uint16_t*>(p.debug_codes + (row0 + r) * K + c) =
+            (uint16_t)(((uint32_t)q0 & 0xFFu) | (((uint32_t)q1 & 0xFFu) << 8));
     }
+    *reinterpret_cast<uint4*>(s_code + 16 * c) = make_uint4(w0[0], w0[1], w0[2], w0[3]);
+    *reinterpret_cast<uint4*>(s_code + 16 * c + 16) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+    auto two = [](int a, int b) { return (uint16_t)(((uint32_t)a & 0xFFu) | (((uint32_t)b & 0xFFu) << 8)); };
+    *reinterpret_cast<uint16_t*>(s_fpot + c) = two(c0.fpot, c1.fpot);
+    *reinterpret_cast<uint16_t*>(s_bits + c) = two(c0.bits, c1.bits);
+    *reinterpret_cast<uint16_t*>(s_qmax + c) = two(qmx0, qmx1);
+    *reinterpret_cast<uint16_t*>(s_qmin + c) = two(qmn0, qmn1);
+    fmax = max(fmax, max(c0.fpot, c1.fpot));
+    fmin = min(fmin, min(c0.fpot, c1.fpot));
   }
 
   // block reductions: finest / coarsest FPoT, flags
@@ -273,40 +243,44 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
   const int planes = s_small[27];
 
   // ------------------------------------------------- phase 2a: operand planes
-  if (planes <= 2) {
-    const int64_t vpr = K / 16;  // 16-byte vectors per row
-    for (int64_t v = tid; v < 16 * vpr; v += kQThreads) {
-      const int row = (int)(v / vpr);
-      const int64_t c = (v - row * vpr) * 16;
-      const uint4 qraw = *reinterpret_cast<const uint4*>(s_codes + row * cs + c);
-      const uint4 fraw = *reinterpret_cast<const uint4*>(s_fpot + c);
-      const uint32_t qw[4] = {qraw.x, qraw.y, qraw.z, qraw.w};
-      const uint32_t fw[4] = {fraw.x, fraw.y, fraw.z, fraw.w};
-      uint32_t a0w[4], a1w[4];
-      bool nz1 = false;
+  // Same channel-pair mapping: 2-byte stores, a warp writes 64 contiguous bytes per row.
+  if (planes == 1) {
+    for (int pr = tid; pr < npairs; pr += kQThreads) {
+      const int64_t c = 2 * (int64_t)pr;
+      const uint4 q0 = *reinterpret_cast<const uint4*>(s_code + 16 * c);
+      const uint4 q1 = *reinterpret_cast<const uint4*>(s_code + 16 * c + 16);
+      // a nonzero code of a one-plane tile has a shift <= 7; zero codes stay zero
+      const int S0 = min(g - s_fpot[c], 31), S1 = min(g - s_fpot[c + 1], 31);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        a0w[i] = 0, a1w[i] = 0;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int q = (int)(int8_t)(qw[i] >> (8 * j));
-          const int S = g - (int)(int8_t)(fw[i] >> (8 * j));
-          const int64_t val = (int64_t)q * ((int64_t)1 << S);  // shift-folded code, exact
-          const int a0 = (int)(int8_t)(val & 0xFF);
-          const int a1 = (int)((val - a0) >> 8);
-          a0w[i] |= (uint32_t)(uint8_t)a0 << (8 * j);
-          a1w[i] |= (uint32_t)(uint8_t)a1 << (8 * j);
-          nz1 |= a1 != 0;
-        }
+      for (int r = 0; r < kTile; ++r) {
+        const uint32_t a = (((uint32_t)code_at(q0, r) << S0) & 0xFFu) | ((((uint32_t)code_at(q1, r) << S1) & 0xFFu) << 8);
+        *reinterpret_cast<uint16_t*>(p.plane0 + (row0 + r) * K + c) = (uint16_t)a;
       }
-      const int64_t off = ((int64_t)t * kTile + row) * K + c;
-      *reinterpret_cast<uint4*>(p.plane0 + off) = make_uint4(a0w[0], a0w[1], a0w[2], a0w[3]);
-      if (planes == 2) {
-        *reinterpret_cast<uint4*>(p.plane1 + off) = make_uint4(a1w[0], a1w[1], a1w[2], a1w[3]);
-        if (nz1) {
-          const int chunk = (int)(c / kChunkK);
-          atomicOr(&s_mask[chunk >> 5], 1u << (chunk & 31));
-        }
+    }
+  } else if (planes == 2) {
+    for (int pr = tid; pr < npairs; pr += kQThreads) {
+      const int64_t c = 2 * (int64_t)pr;
+      const uint4 q0 = *reinterpret_cast<const uint4*>(s_code + 16 * c);
+      const uint4 q1 = *reinterpret_cast<const uint4*>(s_code + 16 * c + 16);
+      // a nonzero code of a two-plane tile has a shift <= 15, so v fits 32 bits
+      const int S0 = min(g - s_fpot[c], 24), S1 = min(g - s_fpot[c + 1], 24);
+      uint32_t nz = 0;
+#pragma unroll
+      for (int r = 0; r < kTile; ++r) {
+        const int v0 = code_at(q0, r) * (1 << S0), v1 = code_at(q1, r) * (1 << S1);
+        const int a00 = (int)(int8_t)(v0 & 0xFF), a01 = (int)(int8_t)(v1 & 0xFF);
+        const int a10 = (v0 - a00) >> 8, a11 = (v1 - a01) >> 8;
+        nz |= (uint32_t)(a10 | a11);
+        *reinterpret_cast<uint16_t*>(p.plane0 + (row0 + r) * K + c) =
+            (uint16_t)(((uint32_t)a00 & 0xFFu) | (((uint32_t)a01 & 0xFFu) << 8));
+        *reinterpret_cast<uint16_t*>(p.plane1 + (row0 + r) * K + c) =
+            (uint16_t)(((uint32_t)a10 & 0xFFu) | (((uint32_t)a11 & 0xFFu) << 8));
+      }
+      // a warp's 32 pairs are 64 aligned channels: one K chunk
+      const uint32_t bal = __ballot_sync(__activemask(), nz != 0);
+      if (bal && nz && (__ffs(bal) - 1) == lane) {
+        const int chunk = (int)(c / kChunkK);
+        atomicOr(&s_mask[chunk >> 5], 1u << (chunk & 31));
       }
     }
   }
@@ -371,15 +345,11 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
     const int64_t k = kb + lane;
     const bool kv = k < k_hi;
     const int f = kv ? s_fpot[k] : 0, b = kv ? s_bits[k] : 0;
-    uint32_t word[4] = {0, 0, 0, 0};
+    uint4 cw = make_uint4(0, 0, 0, 0);
     if (kv) {
-      const uint32_t msk = (1u << b) - 1u;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const uint32_t u = (uint32_t)(int)s_codes[i * cs + k] & msk;  // b-bit two's complement
-#pragma unroll
-        for (int j = 0; j < 4; ++j) word[j] |= ((u >> (2 * j)) & 3u) << (2 * i);
-      }
+      cw = *reinterpret_cast<const uint4*>(s_code + 16 * k);
+      p.fpot[(int64_t)t * K + k] = (int8_t)f;
+      p.bits[(int64_t)t * K + k] = (int8_t)b;
     }
     const uint32_t lt = (1u << lane) - 1u;
     for (int ti = 0; ti < ntags; ++ti) {
@@ -389,20 +359,15 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const QuantParams p
       const uint32_t bal = __ballot_sync(0xffffffffu, has);
       const int base = __shfl_sync(0xffffffffu, off[ti >> 5], ti & 31);
       if (has) {
+        // the field j < b/2 of the b-bit pattern equals that of the 8-bit pattern
         const int j = d >> 1;
-        const uint32_t w = j == 0 ? word[0] : j == 1 ? word[1] : j == 2 ? word[2] : word[3];
         rec[base + __popc(bal & lt)] =
-            make_uint2(w, (uint32_t)k | ((uint32_t)(uint8_t)(int8_t)tag << 16) | ((uint32_t)j << 24));
+            make_uint2(slice_word(cw, j), (uint32_t)k | ((uint32_t)(uint8_t)(int8_t)tag << 16) | ((uint32_t)j << 24));
       }
       if (lane == (ti & 31)) off[ti >> 5] += __popc(bal);
     }
   }
 
-  // per-sub-channel meta and per-tile meta
-  for (int64_t k = tid; k < K; k += kQThreads) {
-    p.fpot[(int64_t)t * K + k] = s_fpot[k];
-    p.bits[(int64_t)t * K + k] = s_bits[k];
-  }
   __syncthreads();  // s_mask complete
   if (tid < p.mask_words) p.mask1[(int64_t)t * p.mask_words + tid] = planes == 2 ? s_mask[tid] : 0u;
   if (tid == 0) {
@@ -416,15 +381,13 @@ int launch_quantize(const QuantParams& p, int in_bf16, void* stream) {
   const int64_t T = p.M / kTile;
   if (T == 0) return 0;
   const size_t smem = quantize_smem_bytes(p.K);
-  cudaError_t e;
+  const int smem_max = (int)quantize_smem_bytes(DSTAR_K_MAX);  // one setting serves every K
+  int e;
   if (in_bf16) {
-    e = cudaFuncSetAttribute(quantize_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
-    if (e != cudaSuccess) return (int)e;
+    if ((e = ensure_max_smem((const void*)quantize_kernel<__nv_bfloat16>, smem_max)) != 0) return e;
     quantize_kernel<__nv_bfloat16><<<(unsigned)T, kQThreads, smem, (cudaStream_t)stream>>>(p);
   } else {
-    e = cudaFuncSetAttribute(quantize_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return (int)e;
+    if ((e = ensure_max_smem((const void*)quantize_kernel<float>, smem_max)) != 0) return e;
     quantize_kernel<float><<<(unsigned)T, kQThreads, smem, (cudaStream_t)stream>>>(p);
   }
   return (int)cudaGetLastError();
