@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--mode", choices=["graph", "eager"], default="graph",
+                    help="graph: each step replays a captured CUDA graph; eager: C-ABI calls per step")
     return ap.parse_args()
 
 
@@ -361,12 +363,44 @@ def run_ours(args, rank, world, local_rank):
         stats.append(dict(k1_bytes=b1, k2_dense=dense, k2_issued=issued, k2_bytes=b2, fallback_tiles=nfall,
                           bits_avg=float(bits.mean()), bit_hist=[float((bits == b).mean()) for b in (2, 4, 6, 8)],
                           planes_hist=[int((planes == p).sum()) for p in (1, 2)] + [int((planes > 2).sum())]))
-    for r in range(args.sets):
-        uses[r] = 0
 
     # timed region
     K = args.steps
-    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(nlayers)] for _ in range(K)]
+    graphs, gev = None, None
+    if args.mode == "graph":
+        # one graph per (input set, parity); each holds the step's launches and
+        # external event-record nodes between them (per-kernel times)
+        from cuda.bindings import runtime as rt
+
+        def ext_event():
+            err, e = rt.cudaEventCreate()
+            assert err == rt.cudaError_t.cudaSuccess
+            return e
+
+        kinds = [(r, par) for par in (0, 1) for r in range(args.sets)]
+        gev = [[[ext_event() for _ in range(3)] for _ in range(nlayers)] for _ in kinds]
+        graphs = []
+        cap_stream = torch.cuda.Stream()
+        for gi, (r, par) in enumerate(kinds):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap_stream):
+                cs = torch.cuda.current_stream()
+                csh = ctypes.c_void_p(cs.cuda_stream)
+                rsh = rt.cudaStream_t(init_value=cs.cuda_stream)
+                for li, lay in enumerate(sets[r]):
+                    rt.cudaEventRecordWithFlags(gev[gi][li][0], rsh, rt.cudaEventRecordExternal)
+                    rc = lay.quantize(L, par, csh)
+                    rt.cudaEventRecordWithFlags(gev[gi][li][1], rsh, rt.cudaEventRecordExternal)
+                    rc |= lay.gemm(L, csh)
+                    rt.cudaEventRecordWithFlags(gev[gi][li][2], rsh, rt.cudaEventRecordExternal)
+                    if rc:
+                        raise RuntimeError(L.dstar_fmdq_last_error().decode())
+            graphs.append(g)
+        for g in graphs:  # warm the graphs (keeps every set's parity alternating)
+            g.replay()
+        torch.cuda.synchronize()
+    evs = None if graphs else \
+        [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(nlayers)] for _ in range(K)]
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
     smi_id = vis.split(",")[local_rank] if vis else str(torch.cuda.current_device())
@@ -377,18 +411,35 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     t_wall0 = time.time()
     ev0.record(stream)
-    for s in range(K):
-        step(s, evs[s])
+    if graphs:
+        for s in range(K):
+            graphs[s % len(graphs)].replay()
+    else:
+        for s in range(K):
+            step(s, evs[s])
     ev1.record(stream)
     torch.cuda.synchronize()
     t_wall1 = time.time()
+    if graphs:  # continue every set's X_t alternation after the replays
+        for s in range(K):
+            gi = s % len(graphs)
+            uses[gi % args.sets] = gi // args.sets + 1
     if dist:
         torch.distributed.barrier()
     time.sleep(0.2)
     clocks.stop()
     ms = ev0.elapsed_time(ev1)
-    k1_ms = [statistics.fmean(evs[s][li][0].elapsed_time(evs[s][li][1]) for s in range(K)) for li in range(nlayers)]
-    k2_ms = [statistics.fmean(evs[s][li][1].elapsed_time(evs[s][li][2]) for s in range(K)) for li in range(nlayers)]
+    if graphs:
+        # the event nodes hold the last replay of each graph: the timed region's last len(graphs) steps
+        def el(a, b):
+            err, v = rt.cudaEventElapsedTime(a, b)
+            assert err == rt.cudaError_t.cudaSuccess
+            return v
+        k1_ms = [statistics.fmean(el(gev[g][li][0], gev[g][li][1]) for g in range(len(graphs))) for li in range(nlayers)]
+        k2_ms = [statistics.fmean(el(gev[g][li][1], gev[g][li][2]) for g in range(len(graphs))) for li in range(nlayers)]
+    else:
+        k1_ms = [statistics.fmean(evs[s][li][0].elapsed_time(evs[s][li][1]) for s in range(K)) for li in range(nlayers)]
+        k2_ms = [statistics.fmean(evs[s][li][1].elapsed_time(evs[s][li][2]) for s in range(K)) for li in range(nlayers)]
     if dist:
         t = torch.tensor([ms], device="cuda")
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
@@ -513,6 +564,8 @@ def run_ours(args, rank, world, local_rank):
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * K,
         "clocks": clocks.summary(t_wall0, t_wall1),
         "kernel_sources": kernel_source_sha(),
+        "timing": ("CUDA-graph replay per step (captured C-ABI calls); per-kernel times from event nodes "
+                   "in the graphs' last replays" if graphs else "eager C-ABI calls with CUDA events per kernel"),
     }
     print(json.dumps(line), flush=True)
 

@@ -384,10 +384,18 @@ __global__ void __launch_bounds__(kGThreads, 1)
 #pragma unroll
         for (int g = 0; g < C::kHalfGroups; ++g)
 #pragma unroll
-          for (int v = 0; v < kVecPerGroup; ++v) {
+          for (int v = 0; v < kVecPerGroup; v += 2) {
             const int64_t n = n_half + g * 32 + v * (16 / (int)sizeof(TOut));
-            ypv[g][v] = (row_ok && n < p.N) ? __ldg(reinterpret_cast<const uint4*>(yp_row + n))
-                                            : make_uint4(0, 0, 0, 0);
+            if (row_ok && n < p.N) {  // N % 16 == 0: a 32-byte pair is whole or absent
+              if (p.vec32) {
+                ld_global_nc_v8(yp_row + n, ypv[g][v], ypv[g][v + 1]);
+              } else {
+                ypv[g][v] = __ldg(reinterpret_cast<const uint4*>(yp_row + n));
+                ypv[g][v + 1] = __ldg(reinterpret_cast<const uint4*>(yp_row + n) + 1);
+              }
+            } else {
+              ypv[g][v] = ypv[g][v + 1] = make_uint4(0, 0, 0, 0);
+            }
           }
 
         uint32_t acc_slot[2];
@@ -407,52 +415,83 @@ __global__ void __launch_bounds__(kGThreads, 1)
         const uint32_t t1a = tmem_base + lane_off + (bi.nplanes == 2 ? acc_slot[1] : acc_slot[0]) * BN + col_half;
         const float* ws_h = ws_t + half * (BN / 2);
 
+        const bool wide_blk = bi.nplanes == 2;  // warp-uniform
+        const bool wide_row = pl == 2;
 #pragma unroll
         for (int g = 0; g < C::kHalfGroups; ++g) {
-          uint32_t d0[32], d1[32];
-          tmem_ld32(t0a + g * 32, d0);
-          if (bi.nplanes == 2) tmem_ld32(t1a + g * 32, d1);
-          tmem_ld_wait();
           const int64_t n0 = n_half + g * 32;
-          if (row_ok && n0 < p.N) {
-            const bool wide = pl == 2;
-            float y[32];
+          const int64_t nv_rem = (p.N - n0) * (int64_t)sizeof(TOut) / 16;  // N % 16 == 0
+          const int nv = nv_rem < kVecPerGroup ? (nv_rem > 0 ? (int)nv_rem : 0) : kVecPerGroup;
+          const float4* wsv = reinterpret_cast<const float4*>(ws_h + g * 32);
+          TOut* yo = reinterpret_cast<TOut*>(p.y_out) + row * p.ld_yo + n0;
+          TOut* yq = reinterpret_cast<TOut*>(p.y_prev) + row * p.ld_yp + n0;
+          constexpr int E = 16 / (int)sizeof(TOut);  // outputs per 16-byte vector
+          uint4 ov[kVecPerGroup];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int64_t acc = wide ? (int64_t)(int32_t)d0[i] + (int64_t)(int32_t)d1[i] * 256
-                                       : (int64_t)(int32_t)d0[i];
-              float ypf;
-              if constexpr (OUT_BF16) {
-                const uint32_t w = reinterpret_cast<const uint32_t*>(ypv[g])[i >> 1];
-                ypf = __uint_as_float((i & 1) ? (w & 0xFFFF0000u) : (w << 16));
-              } else {
-                ypf = __uint_as_float(reinterpret_cast<const uint32_t*>(ypv[g])[i]);
+          for (int h = 0; h < 2; ++h) {  // 16 accumulator columns at a time
+            uint32_t d0[16], d1[16];
+            tmem_ld16(t0a + g * 32 + h * 16, d0);
+            if (wide_blk) tmem_ld16(t1a + g * 32 + h * 16, d1);
+            tmem_ld_wait();
+#pragma unroll
+            for (int vv = 0; vv < kVecPerGroup / 2; ++vv) {
+              const int v = h * (kVecPerGroup / 2) + vv;
+              float y[E];
+#pragma unroll
+              for (int e = 0; e < E; e += 4) {
+                const float4 ws4 = wsv[(v * E + e) >> 2];
+                const float wsa[4] = {ws4.x, ws4.y, ws4.z, ws4.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                  const int i = vv * E + e + u;  // column within this 16-column half
+                  float ypf;
+                  if constexpr (OUT_BF16) {
+                    const uint32_t w = reinterpret_cast<const uint32_t*>(&ypv[g][v])[(e + u) >> 1];
+                    ypf = __uint_as_float(((e + u) & 1) ? (w & 0xFFFF0000u) : (w << 16));
+                  } else {
+                    ypf = __uint_as_float(reinterpret_cast<const uint32_t*>(&ypv[g][v])[e + u]);
+                  }
+                  float a;
+                  if (wide_blk) {
+                    const int64_t acc = (int64_t)(int32_t)d0[i] + (wide_row ? (int64_t)(int32_t)d1[i] * 256 : 0);
+                    a = __ll2float_rn(acc);
+                  } else {
+                    a = __int2float_rn((int32_t)d0[i]);
+                  }
+                  y[e + u] = __fadd_rn(ypf, __fmul_rn(__fmul_rn(a, p2), wsa[u]));
+                }
               }
-              y[i] = epi(acc, wide, p2, ws_h[g * 32 + i], ypf);
-              if (p.debug_acc && n0 + i < p.N) p.debug_acc[row * p.N + n0 + i] = acc;
-            }
-            const int64_t nv_rem = (p.N - n0) * (int64_t)sizeof(TOut) / 16;
-            const int nv = nv_rem < kVecPerGroup ? (int)nv_rem : kVecPerGroup;
-            TOut* yo = reinterpret_cast<TOut*>(p.y_out) + row * p.ld_yo + n0;
-            TOut* yq = reinterpret_cast<TOut*>(p.y_prev) + row * p.ld_yp + n0;
-#pragma unroll
-            for (int v = 0; v < kVecPerGroup; ++v) {
-              uint4 o;
               if constexpr (OUT_BF16) {
                 uint32_t w[4];
 #pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                  const __nv_bfloat162 b2 = __floats2bfloat162_rn(y[v * 8 + 2 * h], y[v * 8 + 2 * h + 1]);
-                  w[h] = *reinterpret_cast<const uint32_t*>(&b2);
+                for (int q = 0; q < 4; ++q) {
+                  const __nv_bfloat162 b2 = __floats2bfloat162_rn(y[2 * q], y[2 * q + 1]);
+                  w[q] = *reinterpret_cast<const uint32_t*>(&b2);
                 }
-                o = make_uint4(w[0], w[1], w[2], w[3]);
+                ov[v] = make_uint4(w[0], w[1], w[2], w[3]);
               } else {
-                o = make_uint4(__float_as_uint(y[4 * v]), __float_as_uint(y[4 * v + 1]),
-                               __float_as_uint(y[4 * v + 2]), __float_as_uint(y[4 * v + 3]));
+                ov[v] = make_uint4(__float_as_uint(y[0]), __float_as_uint(y[1]), __float_as_uint(y[2]),
+                                   __float_as_uint(y[3]));
               }
-              if (v < nv) {
-                reinterpret_cast<uint4*>(yo)[v] = o;
-                if (p.y_distinct) reinterpret_cast<uint4*>(yq)[v] = o;
+            }
+            if (p.debug_acc && row_ok) {
+              for (int i = 0; i < 16 && n0 + h * 16 + i < p.N; ++i)
+                p.debug_acc[row * p.N + n0 + h * 16 + i] =
+                    (int64_t)(int32_t)d0[i] + (wide_blk && wide_row ? (int64_t)(int32_t)d1[i] * 256 : 0);
+            }
+          }
+          if (row_ok) {
+#pragma unroll
+            for (int v = 0; v < kVecPerGroup; v += 2) {
+              if (v < nv) {  // nv is even: 32-byte pairs are whole
+                if (p.vec32) {
+                  st_global_v8(reinterpret_cast<uint4*>(yo) + v, ov[v], ov[v + 1]);
+                  if (p.y_distinct) st_global_v8(reinterpret_cast<uint4*>(yq) + v, ov[v], ov[v + 1]);
+                } else {
+                  reinterpret_cast<uint4*>(yo)[v] = ov[v];
+                  reinterpret_cast<uint4*>(yo)[v + 1] = ov[v + 1];
+                  if (p.y_distinct) reinterpret_cast<uint4*>(yq)[v] = ov[v], reinterpret_cast<uint4*>(yq)[v + 1] = ov[v + 1];
+                }
               }
             }
           }

@@ -174,7 +174,7 @@ T* ws_ptr(const dstar_tile_cfg* c, size_t off) {
 }
 
 int do_quantize(const dstar_mat* x_t, dstar_mat* x_prev, int lb, const dstar_tile_cfg* c, int64_t M, int64_t K,
-                void* stream) {
+                const DevInfo& dev, void* stream) {
   const WsLayout L = ws_layout(M, K);
   QuantParams q{};
   q.x_t = x_t->data;
@@ -196,7 +196,7 @@ int do_quantize(const dstar_mat* x_t, dstar_mat* x_prev, int lb, const dstar_til
   q.record_cap = L.record_cap;
   q.mask_words = L.mask_words;
   q.debug_codes = c->debug_codes;
-  const int e = launch_quantize(q, x_t->dtype == DSTAR_BF16, stream);
+  const int e = launch_quantize(q, x_t->dtype == DSTAR_BF16, dev.sms, stream);
   if (e) return cuda_fail(e, "quantize launch");
   return DSTAR_OK;
 }
@@ -237,6 +237,9 @@ int do_gemm(const dstar_mat* w_q, const float* w_scale, dstar_mat* y_prev, int l
     g.y_out = y_out->data;
     g.ld_yo = y_out->ld;
     g.y_distinct = distinct;
+    const int64_t es = bf16 ? 2 : 4;
+    g.vec32 = ((reinterpret_cast<uintptr_t>(y_prev->data) | reinterpret_cast<uintptr_t>(y_out->data)) & 31u) == 0 &&
+              (y_prev->ld * es) % 32 == 0 && (y_out->ld * es) % 32 == 0;
     g.status = ws_ptr<uint32_t>(c, L.status);
     g.debug_acc = c->debug_acc;
     g.tiles_m = (int)((M + kBlockM - 1) / kBlockM);
@@ -418,7 +421,7 @@ int dstar_fmdq_quantize(const dstar_mat* x_t, dstar_mat* x_prev, float base_scal
   if (M == 0) return ok();
   DevInfo dev;
   if ((r = device_info(&dev)) != DSTAR_OK) return r;
-  if ((r = do_quantize(x_t, x_prev, lb, tile_cfg, M, K, stream)) != DSTAR_OK) return r;
+  if ((r = do_quantize(x_t, x_prev, lb, tile_cfg, M, K, dev, stream)) != DSTAR_OK) return r;
   return ok();
 }
 
@@ -460,7 +463,7 @@ int dstar_fmdq_linear(const dstar_mat* x_t, dstar_mat* x_prev, dstar_mat* y_prev
   if (M == 0) return ok();
   DevInfo dev;
   if ((r = device_info(&dev)) != DSTAR_OK) return r;
-  if ((r = do_quantize(x_t, x_prev, lb, tile_cfg, M, K, stream)) != DSTAR_OK) return r;
+  if ((r = do_quantize(x_t, x_prev, lb, tile_cfg, M, K, dev, stream)) != DSTAR_OK) return r;
   if ((r = do_gemm(w_q, w_scale, y_prev, lb, tile_cfg, y_out, M, K, N, dev, stream)) != DSTAR_OK) return r;
   return ok();
 }

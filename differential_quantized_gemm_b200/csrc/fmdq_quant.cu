@@ -1,21 +1,30 @@
 // K1: the FMDQ quantizer (DSTAR section 3.1 steps 1-4; the paper's QPU,
 // section 4.2 "Design of QPU", stages 1-5).
 //
-// One 256-thread block per 16-token tile.  Phase 1: every thread owns a pair
-// of adjacent channels and walks the 16 tokens of the tile, so a warp reads
-// whole 128-byte row segments of X_t and X_{t-1} and the per-channel max
-// |dX| (stage 1: compare the magnitude bits, sign dropped) stays inside the
-// thread.  PoT (Eq. 3), the bit width (threshold bins, stage 2), FPoT (Eq. 4)
-// and the codes q = rne(dX * s_i) with s_i = base * 2^FPoT (Eq. 5, stage 3)
-// follow per channel; the 16 codes of a channel go to shared memory as one
-// 16-byte column.  Phase 2 knows the tile's finest FPoT (g_ref) and writes
-// (a) the tensor-core operand planes v = q * 2^(g_ref - FPoT), split into int8
-// planes v = A0 + 256 A1, and (b) the encoded stream: one record per 2-bit
-// slice, grouped by slice FPoT ascending then channel ascending (stages 4-5),
-// placed by per-tag counts and an exclusive scan rather than a sort.
+// One 16-token tile is handled by a thread-block cluster of C CTAs (C = 1, 2,
+// 4 or 8, chosen so that small batches still fill every SM); CTA r owns a
+// contiguous range of channels.  Every thread owns pairs of adjacent channels
+// and walks the 16 tokens, so a warp reads whole 128-byte row segments of X_t
+// and X_{t-1} and the per-channel max |dX| (stage 1: compare the magnitude
+// bits, sign dropped) stays inside the thread.  PoT (Eq. 3), the bit width
+// (threshold bins, stage 2), FPoT (Eq. 4) and the codes q = rne(dX s_i) with
+// s_i = base 2^FPoT (Eq. 5, stage 3) follow per channel; a channel's 16 codes
+// go to shared memory as one 16-byte column.
+//
+// The tile's finest FPoT (g_ref), its plane count and the per-tag record
+// counts are combined across the cluster through distributed shared memory.
+// Phase 2 writes (a) the tensor-core operand planes v = q 2^(g_ref - FPoT),
+// split into int8 planes v = A0 + 256 A1, and (b) the encoded stream: one
+// record per 2-bit slice, ordered by slice FPoT ascending then channel
+// ascending (stages 4-5).  A record's position is found by counting, not
+// sorting: warp ballots per tag rank the channels of a 32-channel chunk, and
+// per-tag counts of warps, CTAs and lower tags give the offsets.
+#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 
 #include "fmdq_device.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace fmdq {
 
@@ -23,8 +32,9 @@ namespace {
 
 constexpr int kQThreads = 256;
 constexpr int kQWarps = kQThreads / 32;
-constexpr int kMaxTags = 64;  // tag spread within a tile is at most 6 + kPotMax + 6 < 64
+constexpr int kMaxCluster = 8;
 constexpr int kMaxMaskWords = (DSTAR_K_MAX / kChunkK + 31) / 32;
+constexpr int kTagWin = 8;  // tags ranked per pass (one ballot each)
 
 // Two adjacent channels of one token row.
 template <typename TIn>
@@ -106,51 +116,87 @@ __device__ __forceinline__ int code_at(const uint4 cw, int r) {
   return (int)(int8_t)(w >> (8 * (r & 3)));
 }
 
+// Window slots ti (tag tw + ti, 0 <= ti < 8) that one channel's slices occupy.
+__device__ __forceinline__ uint32_t tag_mask(int f, int b, int tw) {
+  uint32_t m = 0;
+  for (int j = 0; j < (b >> 1); ++j) {  // slice j has tag f - 2j
+    const int ti = f - 2 * j - tw;
+    if (ti >= 0 && ti < kTagWin) m |= 1u << ti;
+  }
+  return m;
+}
+
+// Cluster-wide barrier; a plain block barrier when the cluster is one CTA.
+__device__ __forceinline__ void csync(cg::cluster_group& cluster, int C) {
+  if (C > 1) cluster.sync();
+  else __syncthreads();
+}
+
+struct QSmem {
+  // exchanged across the cluster (read remotely)
+  int fmax, fmin, need, pad;
+  uint32_t mask[kMaxMaskWords];
+  int cta_tot[kTagWin];  // this CTA's record count per tag of the current window
+  // local
+  int warp_a[kQWarps], warp_b[kQWarps];
+  int flags;
+  int base[kTagWin];       // records before this CTA's first record of the tag
+  int warp_cnt[kQWarps][kTagWin];
+};
+
 }  // namespace
 
-size_t quantize_smem_bytes(int64_t K) {
-  size_t b = 16 * (size_t)K + 4 * (size_t)K;  // column-major codes + 4 per-column bytes
+size_t quantize_smem_bytes(int64_t Kc) {
+  size_t b = 20 * (size_t)Kc;  // column-major codes + 4 per-column bytes
   b = (b + 15) & ~(size_t)15;
-  b += sizeof(int) * (64 + 2 * kQWarps * kMaxTags) + sizeof(uint32_t) * kMaxMaskWords;
-  return b;
+  return b + sizeof(QSmem);
+}
+
+int quantize_cluster_size(int64_t M, int64_t K, int num_sms) {
+  const int64_t T = M / kTile;
+  const int64_t units = K / 32;
+  int c = 1;
+  // about 1.5 CTAs per SM when the batch is small, at least 256 channels per CTA
+  while (c < kMaxCluster && 2 * T * c < 3LL * num_sms && units / (2 * c) >= 8) c *= 2;
+  return c;
 }
 
 template <typename TIn>
-__global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParams p) {
+__global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParams p, int C, int64_t kc_max) {
   extern __shared__ __align__(16) uint8_t smem[];
   using PR = Pair<TIn>;
+  cg::cluster_group cluster = cg::this_cluster();
 
   const int64_t K = p.K;
-  const int t = blockIdx.x;
+  const int rank = (int)cluster.block_rank();
+  const int t = (int)(blockIdx.x / C);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t units = K / 32;
+  const int64_t k_lo = 32 * (rank * units / C), k_hi = 32 * ((rank + 1) * units / C);
+  const int64_t Kc = k_hi - k_lo;
 
-  int8_t* s_code = reinterpret_cast<int8_t*>(smem);  // [K][16]: the 16 codes of channel k
-  int8_t* s_fpot = s_code + 16 * K;                   // [K]
-  int8_t* s_bits = s_fpot + K;
-  int8_t* s_qmax = s_bits + K;
-  int8_t* s_qmin = s_qmax + K;
-  int* s_small = reinterpret_cast<int*>(smem + ((20 * K + 15) & ~(int64_t)15));
-  int* s_hist = s_small + 64;                  // [warps][kMaxTags]
-  int* s_off = s_hist + kQWarps * kMaxTags;    // [warps][kMaxTags]
-  uint32_t* s_mask = reinterpret_cast<uint32_t*>(s_off + kQWarps * kMaxTags);
-  // s_small: [0,8) warp max FPoT, [8,16) warp min FPoT, [16,24) warp plane need,
-  //          [24] flags (1 nonfinite, 2 range), [25] g_ref, [26] min FPoT, [27] planes, [28] records
+  int8_t* s_code = reinterpret_cast<int8_t*>(smem);  // [Kc][16]: the 16 codes of local channel k
+  int8_t* s_fpot = s_code + 16 * kc_max;              // [Kc]
+  int8_t* s_bits = s_fpot + kc_max;
+  int8_t* s_qmax = s_bits + kc_max;
+  int8_t* s_qmin = s_qmax + kc_max;
+  QSmem& S = *reinterpret_cast<QSmem*>(smem + ((20 * kc_max + 15) & ~(int64_t)15));
 
-  if (tid < kMaxMaskWords) s_mask[tid] = 0;
-  if (tid == 0) s_small[24] = 0;
+  if (tid < kMaxMaskWords) S.mask[tid] = 0;
+  if (tid == 0) S.flags = 0;
   __syncthreads();
 
   const int lb = p.lb, t0 = p.t0, fb = p.force_bits;
   const float beta = exp2_exact(lb);
   const bool refresh = !(p.flags & DSTAR_FLAG_NO_XPREV_REFRESH);
   const int64_t row0 = (int64_t)t * kTile;
-  const int npairs = (int)(K / 2);
+  const int npairs = (int)(Kc / 2);
   int fmax = -1000, fmin = 1000;
   int flags = 0;
 
   // ---------------------------------------------------------------- phase 1
   for (int pr = tid; pr < npairs; pr += kQThreads) {
-    const int64_t c = 2 * (int64_t)pr;
+    const int64_t lc = 2 * (int64_t)pr, c = k_lo + lc;
     typename PR::Raw rt[kTile], rp[kTile];
 #pragma unroll
     for (int r = 0; r < kTile; ++r) {
@@ -161,43 +207,47 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParam
 #pragma unroll
       for (int r = 0; r < kTile; ++r) PR::store(p.x_prev, (row0 + r) * p.ld_xp + c, rt[r]);
     }
-    float d0[kTile], d1[kTile];
+    // Eq. 1 (one fp32 subtraction per element) and stage 1 on the magnitude bits
     uint32_t m0 = 0, m1 = 0;
 #pragma unroll
     for (int r = 0; r < kTile; ++r) {
-      d0[r] = __fsub_rn(PR::lo(rt[r]), PR::lo(rp[r]));  // Eq. 1, one fp32 subtraction
-      d1[r] = __fsub_rn(PR::hi(rt[r]), PR::hi(rp[r]));
-      m0 = max(m0, __float_as_uint(d0[r]) & 0x7FFFFFFFu);  // stage 1 on the magnitude bits
-      m1 = max(m1, __float_as_uint(d1[r]) & 0x7FFFFFFFu);
+      m0 = max(m0, __float_as_uint(__fsub_rn(PR::lo(rt[r]), PR::lo(rp[r]))) & 0x7FFFFFFFu);
+      m1 = max(m1, __float_as_uint(__fsub_rn(PR::hi(rt[r]), PR::hi(rp[r]))) & 0x7FFFFFFFu);
     }
     const ColParams c0 = col_params(m0, lb, beta, t0, fb, flags);
     const ColParams c1 = col_params(m1, lb, beta, t0, fb, flags);
     uint32_t w0[4] = {0, 0, 0, 0}, w1[4] = {0, 0, 0, 0};
     int qmx0 = -128, qmn0 = 127, qmx1 = -128, qmn1 = 127;
 #pragma unroll
-    for (int r = 0; r < kTile; ++r) {
-      const int q0 = c0.nonfinite ? 0 : __float2int_rn(__fmul_rn(d0[r], c0.scale));  // stage 3
-      const int q1 = c1.nonfinite ? 0 : __float2int_rn(__fmul_rn(d1[r], c1.scale));
+    for (int r = 0; r < kTile; ++r) {  // stage 3 (dX recomputed: the same single subtraction)
+      const float d0 = __fsub_rn(PR::lo(rt[r]), PR::lo(rp[r])), d1 = __fsub_rn(PR::hi(rt[r]), PR::hi(rp[r]));
+      const int q0 = c0.nonfinite ? 0 : __float2int_rn(__fmul_rn(d0, c0.scale));
+      const int q1 = c1.nonfinite ? 0 : __float2int_rn(__fmul_rn(d1, c1.scale));
       w0[r >> 2] |= ((uint32_t)q0 & 0xFFu) << (8 * (r & 3));
       w1[r >> 2] |= ((uint32_t)q1 & 0xFFu) << (8 * (r & 3));
       qmx0 = max(qmx0, q0), qmn0 = min(qmn0, q0);
       qmx1 = max(qmx1, q1), qmn1 = min(qmn1, q1);
-      if (p.debug_codes)
-        *reinterpret_cast<uint16_t*>(p.debug_codes + (row0 + r) * K + c) =
-            (uint16_t)(((uint32_t)q0 & 0xFFu) | (((uint32_t)q1 & 0xFFu) << 8));
     }
-    *reinterpret_cast<uint4*>(s_code + 16 * c) = make_uint4(w0[0], w0[1], w0[2], w0[3]);
-    *reinterpret_cast<uint4*>(s_code + 16 * c + 16) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+    if (p.debug_codes) {
+#pragma unroll
+      for (int r = 0; r < kTile; ++r)
+        *reinterpret_cast<uint16_t*>(p.debug_codes + (row0 + r) * K + c) =
+            (uint16_t)(((w0[r >> 2] >> (8 * (r & 3))) & 0xFFu) | (((w1[r >> 2] >> (8 * (r & 3))) & 0xFFu) << 8));
+    }
+    *reinterpret_cast<uint4*>(s_code + 16 * lc) = make_uint4(w0[0], w0[1], w0[2], w0[3]);
+    *reinterpret_cast<uint4*>(s_code + 16 * lc + 16) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
     auto two = [](int a, int b) { return (uint16_t)(((uint32_t)a & 0xFFu) | (((uint32_t)b & 0xFFu) << 8)); };
-    *reinterpret_cast<uint16_t*>(s_fpot + c) = two(c0.fpot, c1.fpot);
-    *reinterpret_cast<uint16_t*>(s_bits + c) = two(c0.bits, c1.bits);
-    *reinterpret_cast<uint16_t*>(s_qmax + c) = two(qmx0, qmx1);
-    *reinterpret_cast<uint16_t*>(s_qmin + c) = two(qmn0, qmn1);
+    *reinterpret_cast<uint16_t*>(s_fpot + lc) = two(c0.fpot, c1.fpot);
+    *reinterpret_cast<uint16_t*>(s_bits + lc) = two(c0.bits, c1.bits);
+    *reinterpret_cast<uint16_t*>(s_qmax + lc) = two(qmx0, qmx1);
+    *reinterpret_cast<uint16_t*>(s_qmin + lc) = two(qmn0, qmn1);
+    *reinterpret_cast<uint16_t*>(p.fpot + (int64_t)t * K + c) = two(c0.fpot, c1.fpot);
+    *reinterpret_cast<uint16_t*>(p.bits + (int64_t)t * K + c) = two(c0.bits, c1.bits);
     fmax = max(fmax, max(c0.fpot, c1.fpot));
     fmin = min(fmin, min(c0.fpot, c1.fpot));
   }
 
-  // block reductions: finest / coarsest FPoT, flags
+  // CTA reductions, then the cluster's finest / coarsest FPoT
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     fmax = max(fmax, __shfl_xor_sync(0xffffffffu, fmax, o));
@@ -205,52 +255,55 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParam
     flags |= __shfl_xor_sync(0xffffffffu, flags, o);
   }
   if (lane == 0) {
-    s_small[warp] = fmax;
-    s_small[8 + warp] = fmin;
-    if (flags) atomicOr(&s_small[24], flags);
+    S.warp_a[warp] = fmax;
+    S.warp_b[warp] = fmin;
+    if (flags) atomicOr(&S.flags, flags);
   }
   __syncthreads();
   if (tid == 0) {
-    int g = -1000, gm = 1000;
-    for (int w = 0; w < kQWarps; ++w) g = max(g, s_small[w]), gm = min(gm, s_small[8 + w]);
-    s_small[25] = g;
-    s_small[26] = gm;
-    if (s_small[24]) set_status(p.status, (s_small[24] & 1 ? DSTAR_STATUS_NONFINITE : 0u) |
-                                              (s_small[24] & 2 ? DSTAR_STATUS_RANGE : 0u));
+    int a = -1000, b = 1000;
+    for (int w = 0; w < kQWarps; ++w) a = max(a, S.warp_a[w]), b = min(b, S.warp_b[w]);
+    S.fmax = a, S.fmin = b;
+    if (S.flags)
+      set_status(p.status, (S.flags & 1 ? DSTAR_STATUS_NONFINITE : 0u) | (S.flags & 2 ? DSTAR_STATUS_RANGE : 0u));
   }
-  __syncthreads();
-  const int g = s_small[25];
-  const int gmin = s_small[26];
+  csync(cluster, C);
+  int g = -1000, gmin = 1000;
+  for (int q = 0; q < C; ++q) {
+    const QSmem* R = C > 1 ? cluster.map_shared_rank(&S, q) : &S;
+    g = max(g, R->fmax), gmin = min(gmin, R->fmin);
+  }
 
   // planes the tile needs: every v = q 2^(g - FPoT) must fit the split
   int need = 1;
-  for (int64_t k = tid; k < K; k += kQThreads) {
-    const int S = g - s_fpot[k];
-    const int64_t vmax = (int64_t)s_qmax[k] * ((int64_t)1 << S), vmin = (int64_t)s_qmin[k] * ((int64_t)1 << S);
+  for (int64_t k = tid; k < Kc; k += kQThreads) {
+    const int Sh = g - s_fpot[k];
+    const int64_t vmax = (int64_t)s_qmax[k] * ((int64_t)1 << Sh), vmin = (int64_t)s_qmin[k] * ((int64_t)1 << Sh);
     if (vmin < kPlane1Lo || vmax > kPlane1Hi) need = max(need, 2);
     if (vmin < kPlane2Lo || vmax > kPlane2Hi) need = 3;
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) need = max(need, __shfl_xor_sync(0xffffffffu, need, o));
-  if (lane == 0) s_small[16 + warp] = need;
+  if (lane == 0) S.warp_a[warp] = need;
   __syncthreads();
   if (tid == 0) {
     int n = 1;
-    for (int w = 0; w < kQWarps; ++w) n = max(n, s_small[16 + w]);
-    s_small[27] = n;
+    for (int w = 0; w < kQWarps; ++w) n = max(n, S.warp_a[w]);
+    S.need = n;
   }
-  __syncthreads();
-  const int planes = s_small[27];
+  csync(cluster, C);
+  int planes = 1;
+  for (int q = 0; q < C; ++q) planes = max(planes, (C > 1 ? cluster.map_shared_rank(&S, q) : &S)->need);
 
   // ------------------------------------------------- phase 2a: operand planes
   // Same channel-pair mapping: 2-byte stores, a warp writes 64 contiguous bytes per row.
   if (planes == 1) {
     for (int pr = tid; pr < npairs; pr += kQThreads) {
-      const int64_t c = 2 * (int64_t)pr;
-      const uint4 q0 = *reinterpret_cast<const uint4*>(s_code + 16 * c);
-      const uint4 q1 = *reinterpret_cast<const uint4*>(s_code + 16 * c + 16);
+      const int64_t lc = 2 * (int64_t)pr, c = k_lo + lc;
+      const uint4 q0 = *reinterpret_cast<const uint4*>(s_code + 16 * lc);
+      const uint4 q1 = *reinterpret_cast<const uint4*>(s_code + 16 * lc + 16);
       // a nonzero code of a one-plane tile has a shift <= 7; zero codes stay zero
-      const int S0 = min(g - s_fpot[c], 31), S1 = min(g - s_fpot[c + 1], 31);
+      const int S0 = min(g - s_fpot[lc], 31), S1 = min(g - s_fpot[lc + 1], 31);
 #pragma unroll
       for (int r = 0; r < kTile; ++r) {
         const uint32_t a = (((uint32_t)code_at(q0, r) << S0) & 0xFFu) | ((((uint32_t)code_at(q1, r) << S1) & 0xFFu) << 8);
@@ -259,11 +312,11 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParam
     }
   } else if (planes == 2) {
     for (int pr = tid; pr < npairs; pr += kQThreads) {
-      const int64_t c = 2 * (int64_t)pr;
-      const uint4 q0 = *reinterpret_cast<const uint4*>(s_code + 16 * c);
-      const uint4 q1 = *reinterpret_cast<const uint4*>(s_code + 16 * c + 16);
+      const int64_t lc = 2 * (int64_t)pr, c = k_lo + lc;
+      const uint4 q0 = *reinterpret_cast<const uint4*>(s_code + 16 * lc);
+      const uint4 q1 = *reinterpret_cast<const uint4*>(s_code + 16 * lc + 16);
       // a nonzero code of a two-plane tile has a shift <= 15, so v fits 32 bits
-      const int S0 = min(g - s_fpot[c], 24), S1 = min(g - s_fpot[c + 1], 24);
+      const int S0 = min(g - s_fpot[lc], 24), S1 = min(g - s_fpot[lc + 1], 24);
       uint32_t nz = 0;
 #pragma unroll
       for (int r = 0; r < kTile; ++r) {
@@ -276,120 +329,146 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParam
         *reinterpret_cast<uint16_t*>(p.plane1 + (row0 + r) * K + c) =
             (uint16_t)(((uint32_t)a10 & 0xFFu) | (((uint32_t)a11 & 0xFFu) << 8));
       }
-      // a warp's 32 pairs are 64 aligned channels: one K chunk
-      const uint32_t bal = __ballot_sync(__activemask(), nz != 0);
-      if (bal && nz && (__ffs(bal) - 1) == lane) {
+      if (nz) {
         const int chunk = (int)(c / kChunkK);
-        atomicOr(&s_mask[chunk >> 5], 1u << (chunk & 31));
+        atomicOr(&S.mask[chunk >> 5], 1u << (chunk & 31));
       }
     }
   }
 
   // ------------------------------------- phase 2b: FPoT-grouped encoded stream
-  // Slice j of channel k carries tag FPoT(k) - 2j (j < bits/2).  Tags of the
-  // tile lie in [gmin - 6, g]; tag index ti = tag - (gmin - 6).  Each warp owns a
-  // contiguous channel range, so (tag, k) order is (tag, warp, chunk, lane).
+  // Slice j of channel k carries tag FPoT(k) - 2j (j < bits/2).  Tags lie in
+  // [gmin - 6, g] and are handled in windows of 8 consecutive tags.  Each warp
+  // owns a contiguous range of this CTA's channels and walks it 32 channels
+  // at a time (lane = channel); one ballot per tag of the window ranks the
+  // lanes carrying that tag.  The record of (tag, k) lands after: the tile's
+  // records of lower tags, then those of the same tag in lower-ranked CTAs,
+  // lower warps of this CTA, earlier chunks of this warp and lower lanes.
   const int tlo = gmin - 6;
-  const int ntags = g - tlo + 1;  // <= 6 + (g - gmin) + 1 < kMaxTags
-  const int64_t kw = K / kQWarps;  // K % 32 == 0 -> a multiple of 4
-  const int64_t k_lo = warp * kw, k_hi = (warp == kQWarps - 1) ? K : k_lo + kw;
-
-  // pass A: per-warp count of each tag; lane ti % 32 keeps tag ti in cnt[ti / 32]
-  int cnt[2] = {0, 0};
-  for (int64_t kb = k_lo; kb < k_hi; kb += 32) {
-    const int64_t k = kb + lane;
-    const bool kv = k < k_hi;
-    const int f = kv ? s_fpot[k] : 0, b = kv ? s_bits[k] : 0;
-    for (int ti = 0; ti < ntags; ++ti) {
-      const int d = f - (tlo + ti);
-      const bool has = kv && d >= 0 && !(d & 1) && (d >> 1) < (b >> 1);
-      const uint32_t bal = __ballot_sync(0xffffffffu, has);
-      if (lane == (ti & 31)) cnt[ti >> 5] += __popc(bal);
-    }
-  }
-  s_hist[warp * kMaxTags + lane] = cnt[0];
-  s_hist[warp * kMaxTags + 32 + lane] = cnt[1];
-  __syncthreads();
-  // exclusive scan over (tag, warp): warp 0, lane handles tags lane and lane + 32
-  if (warp == 0) {
-    int tot0 = 0, tot1 = 0;
-    for (int w = 0; w < kQWarps; ++w) tot0 += s_hist[w * kMaxTags + lane], tot1 += s_hist[w * kMaxTags + 32 + lane];
-    int inc0 = tot0;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, inc0, o);
-      if (lane >= o) inc0 += y;
-    }
-    const int sum0 = __shfl_sync(0xffffffffu, inc0, 31);
-    int inc1 = tot1;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, inc1, o);
-      if (lane >= o) inc1 += y;
-    }
-    int base0 = inc0 - tot0, base1 = sum0 + inc1 - tot1;
-    for (int w = 0; w < kQWarps; ++w) {
-      const int h0 = s_hist[w * kMaxTags + lane], h1 = s_hist[w * kMaxTags + 32 + lane];
-      s_off[w * kMaxTags + lane] = base0;
-      s_off[w * kMaxTags + 32 + lane] = base1;
-      base0 += h0, base1 += h1;
-    }
-    if (lane == 31) s_small[28] = sum0 + inc1;  // total records of the tile
-  }
-  __syncthreads();
-
-  // pass B: write each record at (tag start) + (rank among earlier channels)
-  int off[2] = {s_off[warp * kMaxTags + lane], s_off[warp * kMaxTags + 32 + lane]};
+  const int ntags = g - tlo + 1;
+  const int64_t kw = ((Kc / 32 + kQWarps - 1) / kQWarps) * 32;  // channels per warp, a multiple of 32
+  const int64_t w_lo = min(Kc, (int64_t)warp * kw), w_hi = min(Kc, w_lo + kw);
+  const uint32_t lt = (1u << lane) - 1u;
   uint2* rec = p.records + (int64_t)t * p.record_cap;
-  for (int64_t kb = k_lo; kb < k_hi; kb += 32) {
-    const int64_t k = kb + lane;
-    const bool kv = k < k_hi;
-    const int f = kv ? s_fpot[k] : 0, b = kv ? s_bits[k] : 0;
-    uint4 cw = make_uint4(0, 0, 0, 0);
-    if (kv) {
-      cw = *reinterpret_cast<const uint4*>(s_code + 16 * k);
-      p.fpot[(int64_t)t * K + k] = (int8_t)f;
-      p.bits[(int64_t)t * K + k] = (int8_t)b;
+  int records_before_window = 0;  // all CTAs, all lower tags (kept by threads tid < kTagWin)
+  for (int wbase = 0; wbase < ntags; wbase += kTagWin) {
+    const int tw = tlo + wbase;  // tag of window slot 0
+    // pass A: this warp's count of each tag of the window
+    int cnt[kTagWin];
+#pragma unroll
+    for (int ti = 0; ti < kTagWin; ++ti) cnt[ti] = 0;
+    for (int64_t kb = w_lo; kb < w_hi; kb += 32) {
+      const int64_t k = kb + lane;
+      const uint32_t m = k < w_hi ? tag_mask(s_fpot[k], s_bits[k], tw) : 0u;
+#pragma unroll
+      for (int ti = 0; ti < kTagWin; ++ti) cnt[ti] += __popc(__ballot_sync(0xffffffffu, (m >> ti) & 1u));
     }
-    const uint32_t lt = (1u << lane) - 1u;
-    for (int ti = 0; ti < ntags; ++ti) {
-      const int tag = tlo + ti;
-      const int d = f - tag;
-      const bool has = kv && d >= 0 && !(d & 1) && (d >> 1) < (b >> 1);
-      const uint32_t bal = __ballot_sync(0xffffffffu, has);
-      const int base = __shfl_sync(0xffffffffu, off[ti >> 5], ti & 31);
-      if (has) {
-        // the field j < b/2 of the b-bit pattern equals that of the 8-bit pattern
-        const int j = d >> 1;
-        rec[base + __popc(bal & lt)] =
-            make_uint2(slice_word(cw, j), (uint32_t)k | ((uint32_t)(uint8_t)(int8_t)tag << 16) | ((uint32_t)j << 24));
+    if (lane == 0) {
+#pragma unroll
+      for (int ti = 0; ti < kTagWin; ++ti) S.warp_cnt[warp][ti] = cnt[ti];
+    }
+    __syncthreads();
+    if (tid < kTagWin) {
+      int tot = 0;
+      for (int w = 0; w < kQWarps; ++w) tot += S.warp_cnt[w][tid];
+      S.cta_tot[tid] = tot;
+    }
+    csync(cluster, C);
+    // window totals of every CTA -> where this CTA's records of each tag start
+    if (tid < kTagWin) {
+      int below = 0, lower_cta = 0, all = 0;
+      for (int q = 0; q < C; ++q) {
+        const QSmem* R = C > 1 ? cluster.map_shared_rank(&S, q) : &S;
+        for (int u = 0; u < kTagWin; ++u) {
+          const int v = R->cta_tot[u];
+          if (u < tid) below += v;
+          if (u == tid && q < rank) lower_cta += v;
+          all += v;
+        }
       }
-      if (lane == (ti & 31)) off[ti >> 5] += __popc(bal);
+      S.base[tid] = records_before_window + below + lower_cta;
+      records_before_window += all;
     }
+    __syncthreads();
+    int off[kTagWin];
+#pragma unroll
+    for (int ti = 0; ti < kTagWin; ++ti) {
+      int o = S.base[ti];
+      for (int w = 0; w < warp; ++w) o += S.warp_cnt[w][ti];
+      off[ti] = o;
+    }
+    // pass B: rank and write
+    for (int64_t kb = w_lo; kb < w_hi; kb += 32) {
+      const int64_t k = kb + lane;
+      const bool kv = k < w_hi;
+      const int f = kv ? s_fpot[k] : 0, b = kv ? s_bits[k] : 0;
+      const uint32_t m = kv ? tag_mask(f, b, tw) : 0u;
+      uint32_t bal[kTagWin];
+#pragma unroll
+      for (int ti = 0; ti < kTagWin; ++ti) bal[ti] = __ballot_sync(0xffffffffu, (m >> ti) & 1u);
+      if (m) {
+        const uint4 cw = *reinterpret_cast<const uint4*>(s_code + 16 * k);
+#pragma unroll
+        for (int ti = 0; ti < kTagWin; ++ti) {
+          if ((m >> ti) & 1u) {
+            // the field j < b/2 of the b-bit pattern equals that of the 8-bit pattern
+            const int j = (f - tw - ti) >> 1;
+            rec[off[ti] + __popc(bal[ti] & lt)] =
+                make_uint2(slice_word(cw, j),
+                           (uint32_t)(k_lo + k) | ((uint32_t)(uint8_t)(int8_t)(tw + ti) << 16) | ((uint32_t)j << 24));
+          }
+        }
+      }
+#pragma unroll
+      for (int ti = 0; ti < kTagWin; ++ti) off[ti] += __popc(bal[ti]);
+    }
+    csync(cluster, C);  // cta_tot and warp_cnt are rewritten by the next window
   }
 
-  __syncthreads();  // s_mask complete
-  if (tid < p.mask_words) p.mask1[(int64_t)t * p.mask_words + tid] = planes == 2 ? s_mask[tid] : 0u;
-  if (tid == 0) {
-    p.g_ref[t] = g;
-    p.planes[t] = planes;
-    p.count[t] = s_small[28];
+  // the tile's meta: rank 0 gathers the cluster's mask words
+  __syncthreads();
+  if (rank == 0) {
+    if (tid < p.mask_words) {
+      uint32_t m = 0;
+      for (int q = 0; q < C; ++q) m |= (C > 1 ? cluster.map_shared_rank(&S, q) : &S)->mask[tid];
+      p.mask1[(int64_t)t * p.mask_words + tid] = planes == 2 ? m : 0u;
+    }
+    if (tid == 0) {
+      p.g_ref[t] = g;
+      p.planes[t] = planes;
+      p.count[t] = records_before_window;
+    }
   }
+  csync(cluster, C);  // no CTA leaves while another may still read its shared memory
 }
 
-int launch_quantize(const QuantParams& p, int in_bf16, void* stream) {
+int launch_quantize(const QuantParams& p, int in_bf16, int num_sms, void* stream) {
   const int64_t T = p.M / kTile;
   if (T == 0) return 0;
-  const size_t smem = quantize_smem_bytes(p.K);
+  const int C = quantize_cluster_size(p.M, p.K, num_sms);
+  const int64_t units = p.K / 32;
+  const int64_t kc_max = 32 * ((units + C - 1) / C);
+  const size_t smem = quantize_smem_bytes(kc_max);
   const int smem_max = (int)quantize_smem_bytes(DSTAR_K_MAX);  // one setting serves every K
-  int e;
-  if (in_bf16) {
-    if ((e = ensure_max_smem((const void*)quantize_kernel<__nv_bfloat16>, smem_max)) != 0) return e;
-    quantize_kernel<__nv_bfloat16><<<(unsigned)T, kQThreads, smem, (cudaStream_t)stream>>>(p);
-  } else {
-    if ((e = ensure_max_smem((const void*)quantize_kernel<float>, smem_max)) != 0) return e;
-    quantize_kernel<float><<<(unsigned)T, kQThreads, smem, (cudaStream_t)stream>>>(p);
-  }
+  const void* fn = in_bf16 ? (const void*)quantize_kernel<__nv_bfloat16> : (const void*)quantize_kernel<float>;
+  int e = ensure_max_smem(fn, smem_max);
+  if (e != 0) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(T * C), 1, 1);
+  cfg.blockDim = dim3(kQThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = (cudaStream_t)stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t ce;
+  if (in_bf16) ce = cudaLaunchKernelEx(&cfg, quantize_kernel<__nv_bfloat16>, p, C, kc_max);
+  else ce = cudaLaunchKernelEx(&cfg, quantize_kernel<float>, p, C, kc_max);
+  if (ce != cudaSuccess) return (int)ce;
   return (int)cudaGetLastError();
 }
 
