@@ -15,16 +15,21 @@
 //   Y_t = Y_{t-1} + ((float)acc * 2^(-lb - g_ref)) * w_scale[n]   (fp32, in this order).
 //
 // Structure (one CTA per SM, persistent over 128 x BN output tiles):
-//   warp 0      TMA producer: A0 chunk (128 x 128 B), W chunk (BN x 128 B) and,
-//               for K chunks where plane 1 is nonzero, the A1 chunk
+//   warp 0      TMA producer: per K chunk, a 128 x 128-byte tile of the operand
+//               plane and a BN x 128-byte tile of W; blocks that need the
+//               second plane run a second K pass over the chunks where it is
+//               nonzero
 //   warp 1      TMEM allocator and MMA issuer (one thread): M=128, N=BN, K=32
-//   warps 2..5  epilogue: tcgen05.ld of their 32 TMEM lanes (= rows), y_prev
-//               loads issued before the accumulator is ready, fp32 epilogue,
-//               bf16/fp32 stores of Y_t to y_out (and y_prev when distinct)
+//   warps 2..9  epilogue, two warps per 32 TMEM lanes (rows), each half of the
+//               columns: TMA-load of its 32 x 32 tiles of y_prev into shared
+//               memory (issued before the accumulator is ready), tcgen05.ld,
+//               fp32 epilogue written in place, TMA-store of Y_t to y_out (and
+//               y_prev when distinct)
 // TMEM holds 512 columns = 512/BN accumulator slots; a one-plane tile takes one
 // slot, a two-plane tile two, so the epilogue of one tile overlaps the MMAs
-// of the next.  Tiles whose planes do not fit in two int8 planes are left to
-// the slice-stream kernel below.  Every wait is bounded (wait_parity).
+// of the next.  Tiles whose operands need more than two int8 planes are
+// computed by the epilogue warps along the slice stream.  Every wait is
+// bounded (wait_parity).
 #include <cuda_bf16.h>
 
 #include "fmdq_device.cuh"
@@ -36,26 +41,30 @@ namespace {
 constexpr int kEpiWarps = 8;                       // two per TMEM lane quarter, each half the columns
 constexpr int kGThreads = 64 + 32 * kEpiWarps;     // producer warp, MMA warp, epilogue warps
 constexpr int kA0Bytes = kBlockM * kChunkK;        // 16 KB
-constexpr int kMaxTileSlots = 64;                  // tiles per CTA whose block info is precomputed
+constexpr int kMaxTileSlots = 32;                  // tiles per CTA whose block info is precomputed
 constexpr int kEpiBarrier = 1;                     // named barrier of the epilogue warps
 
-template <int BN>
+template <int BN, bool OUT_BF16>
 struct GemmCfg {
-  static constexpr int kStages = BN == 256 ? 4 : 6;
+  static constexpr int kStages = BN == 256 ? 3 : (OUT_BF16 ? 5 : 4);
   static constexpr int kWBytes = BN * kChunkK;
   static constexpr int kStageBytes = kA0Bytes + kWBytes;
   static constexpr int kSlots = 512 / BN;
-  static constexpr int kHalfGroups = BN / 64;  // 32-column groups per epilogue warp
-  // small region first, then the 1024-aligned operand buffers
-  static constexpr int kNumBars = 2 * kStages + 1 + 2 * kSlots + 1;
+  static constexpr int kHalfGroups = BN / 64;                        // 32-column groups per epilogue warp
+  static constexpr int kOutBytes = OUT_BF16 ? 2 : 4;
+  static constexpr int kBoxBytes = 32 * 32 * kOutBytes;              // one 32 x 32 tile of Y
+  static constexpr int kYWarpBytes = kHalfGroups * kBoxBytes;        // one epilogue warp's tiles
+  // small region first, then the 1024-aligned buffers
+  static constexpr int kNumBars = 2 * kStages + 2 * kSlots + kEpiWarps + 1;
   static constexpr int kOffBar = 0;
-  static constexpr int kOffMisc = kOffBar + kNumBars * 8;            // tmem base, abort flag
-  static constexpr int kOffWs = kOffMisc + 16;                       // [2][BN] fp32 weight scales
-  static constexpr int kOffInfo = kOffWs + 2 * BN * 4;               // [kMaxTileSlots] block info
+  static constexpr int kOffMisc = (kOffBar + kNumBars * 8 + 15) & ~15;  // tmem base, abort flag
+  static constexpr int kOffWs = kOffMisc + 16;                          // [BN] fp32 weight scales
+  static constexpr int kOffInfo = (kOffWs + BN * 4 + 15) & ~15;         // [kMaxTileSlots] int4 block info
   static constexpr int kSmallBytes = kOffInfo + kMaxTileSlots * 16;
+  static_assert(kOffWs % 16 == 0 && kOffInfo % 16 == 0, "16-byte aligned shared arrays");
   static constexpr int kOffStages = (kSmallBytes + 1023) & ~1023;
-  static constexpr int kOffA1 = kOffStages + kStages * kStageBytes;
-  static constexpr int kBytes = kOffA1 + kA0Bytes + 1024;            // + base alignment slack
+  static constexpr int kOffY = kOffStages + kStages * kStageBytes;
+  static constexpr int kBytes = kOffY + kEpiWarps * kYWarpBytes + 1024;  // + base alignment slack
 };
 
 struct BlockInfo {
@@ -177,29 +186,30 @@ __device__ void slice_stream_column(const uint2* recs, int cnt, const int8_t* bi
 
 }  // namespace
 
-size_t gemm_smem_bytes(int bn) { return bn == 256 ? GemmCfg<256>::kBytes : GemmCfg<128>::kBytes; }
+size_t gemm_smem_bytes(int bn) { return bn == 256 ? GemmCfg<256, true>::kBytes : GemmCfg<128, true>::kBytes; }
 
 template <int BN, bool OUT_BF16>
 __global__ void __launch_bounds__(kGThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CUtensorMap tm_a1,
-                const __grid_constant__ CUtensorMap tm_w, const GemmParams p) {
-  using C = GemmCfg<BN>;
+                const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_yp,
+                const __grid_constant__ CUtensorMap tm_yo, const GemmParams p) {
+  using C = GemmCfg<BN, OUT_BF16>;
   using TOut = typename OutT<OUT_BF16>::T;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* full = bars;                       // [kStages] TMA -> MMA
   uint64_t* empty = full + C::kStages;         // [kStages] MMA -> TMA
-  uint64_t* a1_empty = empty + C::kStages;     // MMA -> TMA (the plane-1 buffer)
-  uint64_t* tm_full = a1_empty + 1;            // [kSlots] MMA -> epilogue
+  uint64_t* tm_full = empty + C::kStages;      // [kSlots] MMA -> epilogue
   uint64_t* tm_empty = tm_full + C::kSlots;    // [kSlots] epilogue -> MMA
-  uint64_t* drain = tm_empty + C::kSlots;      // MMA completion at exit
+  uint64_t* ybar = tm_empty + C::kSlots;       // [kEpiWarps] y_prev tiles landed
+  uint64_t* drain = ybar + kEpiWarps;          // MMA completion at exit
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
   float* s_ws = reinterpret_cast<float*>(smem + C::kOffWs);
   int4* s_info = reinterpret_cast<int4*>(smem + C::kOffInfo);  // {nplanes, any_slice, mask0, mask1}
   uint8_t* stages = smem + C::kOffStages;
-  uint8_t* a1buf = smem + C::kOffA1;
+  uint8_t* ysmem = smem + C::kOffY;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int num_tiles = p.tiles_m * p.tiles_n;
@@ -208,14 +218,16 @@ __global__ void __launch_bounds__(kGThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kStages; ++i) mbar_init(&full[i], 1), mbar_init(&empty[i], 1);
-    mbar_init(a1_empty, 1);
     for (int i = 0; i < C::kSlots; ++i) mbar_init(&tm_full[i], 1), mbar_init(&tm_empty[i], kEpiWarps);
+    for (int i = 0; i < kEpiWarps; ++i) mbar_init(&ybar[i], 1);
     mbar_init(drain, 1);
     *s_abort = 0;
     fence_barrier_init();
     prefetch_tmap(&tm_a0);
     prefetch_tmap(&tm_a1);
     prefetch_tmap(&tm_w);
+    prefetch_tmap(&tm_yp);
+    prefetch_tmap(&tm_yo);
   }
   // block info of this CTA's first kMaxTileSlots tiles, loaded in parallel
   for (int i = threadIdx.x; i < kMaxTileSlots; i += kGThreads) s_info[i] = make_int4(0, 0, 0, 0);
@@ -257,32 +269,26 @@ __global__ void __launch_bounds__(kGThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (elect_one()) {
-      uint32_t it = 0, a1_it = 0;
+      uint32_t it = 0;
       bool ok = true;
       for (int slot = 0; slot < my_tiles && ok; ++slot) {
         const int tile = (int)blockIdx.x + slot * (int)gridDim.x;
         const int rb = tile / p.tiles_n, nb = tile % p.tiles_n;
         const BlockInfo bi = info(slot, rb);
-        if (bi.nplanes == 0) continue;
-        for (int c = 0; c < p.num_chunks; ++c, ++it) {
-          const int s = it % C::kStages;
-          if (!wait_parity(&empty[s], ((it / C::kStages) & 1) ^ 1, s_abort, p.status, kWaitLimitNs)) {
-            ok = false;
-            break;
-          }
-          const bool use1 = chunk_has_plane1(bi, c);
-          if (use1 && !wait_parity(a1_empty, (a1_it & 1) ^ 1, s_abort, p.status, kWaitLimitNs)) {
-            ok = false;  // nothing was loaded into this stage; the MMA side leaves on the abort flag
-            break;
-          }
-          uint8_t* a0 = stages + s * C::kStageBytes;
-          uint8_t* wb = a0 + kA0Bytes;
-          mbar_arrive_expect_tx(&full[s], C::kStageBytes + (use1 ? kA0Bytes : 0));
-          tma_load_2d(a0, &tm_a0, &full[s], c * kChunkK, rb * kBlockM);
-          tma_load_2d(wb, &tm_w, &full[s], c * kChunkK, nb * BN);
-          if (use1) {
-            tma_load_2d(a1buf, &tm_a1, &full[s], c * kChunkK, rb * kBlockM);
-            ++a1_it;
+        for (int pass = 0; pass < bi.nplanes && ok; ++pass) {
+          const CUtensorMap* tm_a = pass == 0 ? &tm_a0 : &tm_a1;
+          for (int c = 0; c < p.num_chunks; ++c) {
+            if (pass == 1 && !chunk_has_plane1(bi, c)) continue;
+            const int s = it % C::kStages;
+            if (!wait_parity(&empty[s], ((it / C::kStages) & 1) ^ 1, s_abort, p.status, kWaitLimitNs)) {
+              ok = false;
+              break;
+            }
+            uint8_t* a = stages + s * C::kStageBytes;
+            mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+            tma_load_2d(a, tm_a, &full[s], c * kChunkK, rb * kBlockM);
+            tma_load_2d(a + kA0Bytes, &tm_w, &full[s], c * kChunkK, nb * BN);
+            ++it;
           }
         }
       }
@@ -295,7 +301,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
     // ----------------------------------------------------------------- MMA
     if (elect_one()) {
       constexpr uint32_t idesc = idesc_i8(BN);
-      uint32_t it = 0, a1_it = 0, slot_it = 0;
+      uint32_t it = 0, slot_it = 0;
       bool ok = true, issued = false;
       for (int slot = 0; slot < my_tiles && ok; ++slot) {
         const int tile = (int)blockIdx.x + slot * (int)gridDim.x;
@@ -310,32 +316,27 @@ __global__ void __launch_bounds__(kGThreads, 1)
         }
         if (!ok) break;
         tc_fence_after();
-        const uint32_t d0 = tmem_base + acc_slot[0] * BN;
-        const uint32_t d1 = tmem_base + (bi.nplanes == 2 ? acc_slot[1] : acc_slot[0]) * BN;
-        bool first1 = true;
-        for (int c = 0; c < p.num_chunks; ++c, ++it) {
-          const int s = it % C::kStages;
-          if (!wait_parity(&full[s], (it / C::kStages) & 1, s_abort, p.status, kWaitLimitNs)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint64_t da = smem_desc_k_sw128(stages + s * C::kStageBytes);
-          const uint64_t dw = smem_desc_k_sw128(stages + s * C::kStageBytes + kA0Bytes);
-#pragma unroll
-          for (int kk = 0; kk < kChunkK / 32; ++kk)
-            mma_i8(d0, da + 2 * kk, dw + 2 * kk, idesc, (c > 0 || kk > 0) ? 1u : 0u);
-          if (chunk_has_plane1(bi, c)) {
-            const uint64_t d_a1 = smem_desc_k_sw128(a1buf);
+        for (int pass = 0; pass < bi.nplanes && ok; ++pass) {
+          const uint32_t d = tmem_base + acc_slot[pass] * BN;
+          bool first = true;
+          for (int c = 0; c < p.num_chunks; ++c) {
+            if (pass == 1 && !chunk_has_plane1(bi, c)) continue;
+            const int s = it % C::kStages;
+            if (!wait_parity(&full[s], (it / C::kStages) & 1, s_abort, p.status, kWaitLimitNs)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t da = smem_desc_k_sw128(stages + s * C::kStageBytes);
+            const uint64_t dw = smem_desc_k_sw128(stages + s * C::kStageBytes + kA0Bytes);
 #pragma unroll
             for (int kk = 0; kk < kChunkK / 32; ++kk)
-              mma_i8(d1, d_a1 + 2 * kk, dw + 2 * kk, idesc, (!first1 || kk > 0) ? 1u : 0u);
-            first1 = false;
-            mma_commit(a1_empty);
-            ++a1_it;
+              mma_i8(d, da + 2 * kk, dw + 2 * kk, idesc, (!first || kk > 0) ? 1u : 0u);
+            first = false;
+            mma_commit(&empty[s]);
+            issued = true;
+            ++it;
           }
-          mma_commit(&empty[s]);
-          issued = true;
         }
         if (!ok) break;
         for (int q = 0; q < bi.nplanes; ++q) mma_commit(&tm_full[acc_slot[q]]);
@@ -353,8 +354,13 @@ __global__ void __launch_bounds__(kGThreads, 1)
     const int etid = threadIdx.x - 64; // 0 .. 32*kEpiWarps-1
     const int quarter = warp & 3;      // TMEM lanes 32*quarter .. +31 are this warp's rows
     const int half = ew >> 2;          // columns [half*BN/2, (half+1)*BN/2)
-    constexpr int kVecPerGroup = 32 * (int)sizeof(TOut) / 16;  // 16-byte vectors per 32 columns
-    uint32_t slot_it = 0;
+    uint8_t* ybuf = ysmem + ew * C::kYWarpBytes;  // this warp's kHalfGroups tiles of 32 x 32
+    constexpr int kChunksPerRow = 32 * C::kOutBytes / 16;  // 16-byte chunks per 32-column row
+    // TMA swizzle of a 32 x 32 tile: 64-byte rows (bf16) use the 64-byte pattern,
+    // 128-byte rows (fp32) the 128-byte one; chunk c of row r sits at chunk c ^ sw(r)
+    auto sw = [](int r) { return OUT_BF16 ? ((r >> 1) & 3) : (r & 7); };
+    uint32_t slot_it = 0, y_it = 0;
+    bool y_pending = false;  // lane 0: a y_prev request whose landing nobody has observed
     int ok = 1;
     // Every epilogue warp runs every iteration and both named barriers of it,
     // also after a timed-out wait (ok == 0), so no warp can be left waiting
@@ -364,39 +370,27 @@ __global__ void __launch_bounds__(kGThreads, 1)
       const int rb = tile / p.tiles_n, nb = tile % p.tiles_n;
       const BlockInfo bi = info(slot, rb);
       const int64_t n_base = (int64_t)nb * BN;
-      // weight scales of the tile's columns, double-buffered by tile parity
-      float* ws_t = s_ws + (slot & 1) * BN;
-      for (int i = etid; i < BN; i += 32 * kEpiWarps) ws_t[i] = (n_base + i < p.N) ? p.w_scale[n_base + i] : 0.f;
+      const int64_t n_half = n_base + half * (BN / 2);
+      const int row0 = rb * kBlockM + quarter * 32;
+      for (int i = etid; i < BN; i += 32 * kEpiWarps) s_ws[i] = (n_base + i < p.N) ? p.w_scale[n_base + i] : 0.f;
       epi_barrier();
 
       if (ok && bi.nplanes > 0) {
-        const int64_t row = (int64_t)rb * kBlockM + quarter * 32 + lane;
+        // this warp's y_prev tiles: the buffer is free once the last tile's stores have read it
+        if (lane == 0) {
+          bulk_wait_read<0>();
+          mbar_arrive_expect_tx(&ybar[ew], C::kYWarpBytes);
+#pragma unroll
+          for (int g = 0; g < C::kHalfGroups; ++g)
+            tma_load_2d(ybuf + g * C::kBoxBytes, &tm_yp, &ybar[ew], (int)(n_half + g * 32), row0);
+          y_pending = true;
+        }
+        const int64_t row = row0 + lane;
         const bool in_range = row < p.M;
         const int t = (int)(row / kTile);
         const int pl = in_range ? p.planes[t] : 3;
         const bool row_ok = in_range && pl <= 2;
         const float p2 = row_ok ? exp2_exact(-p.lb - p.g_ref[t]) : 0.f;
-        const int64_t n_half = n_base + half * (BN / 2);
-        const TOut* yp_row = reinterpret_cast<const TOut*>(p.y_prev) + (row_ok ? row : 0) * p.ld_yp;
-
-        // y_prev of this thread's row and columns, loaded before the accumulator is ready
-        uint4 ypv[C::kHalfGroups][kVecPerGroup];
-#pragma unroll
-        for (int g = 0; g < C::kHalfGroups; ++g)
-#pragma unroll
-          for (int v = 0; v < kVecPerGroup; v += 2) {
-            const int64_t n = n_half + g * 32 + v * (16 / (int)sizeof(TOut));
-            if (row_ok && n < p.N) {  // N % 16 == 0: a 32-byte pair is whole or absent
-              if (p.vec32) {
-                ld_global_nc_v8(yp_row + n, ypv[g][v], ypv[g][v + 1]);
-              } else {
-                ypv[g][v] = __ldg(reinterpret_cast<const uint4*>(yp_row + n));
-                ypv[g][v + 1] = __ldg(reinterpret_cast<const uint4*>(yp_row + n) + 1);
-              }
-            } else {
-              ypv[g][v] = ypv[g][v + 1] = make_uint4(0, 0, 0, 0);
-            }
-          }
 
         uint32_t acc_slot[2];
         for (int q = 0; q < bi.nplanes; ++q) {
@@ -407,119 +401,130 @@ __global__ void __launch_bounds__(kGThreads, 1)
             ok = wait_parity(&tm_full[acc_slot[q]], (si / C::kSlots) & 1, s_abort, p.status, kWaitLimitNs) ? 1 : 0;
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (ok) {
-        tc_fence_after();
-        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-        const uint32_t col_half = half * (BN / 2);
-        const uint32_t t0a = tmem_base + lane_off + acc_slot[0] * BN + col_half;
-        const uint32_t t1a = tmem_base + lane_off + (bi.nplanes == 2 ? acc_slot[1] : acc_slot[0]) * BN + col_half;
-        const float* ws_h = ws_t + half * (BN / 2);
-
-        const bool wide_blk = bi.nplanes == 2;  // warp-uniform
-        const bool wide_row = pl == 2;
-#pragma unroll
-        for (int g = 0; g < C::kHalfGroups; ++g) {
-          const int64_t n0 = n_half + g * 32;
-          const int64_t nv_rem = (p.N - n0) * (int64_t)sizeof(TOut) / 16;  // N % 16 == 0
-          const int nv = nv_rem < kVecPerGroup ? (nv_rem > 0 ? (int)nv_rem : 0) : kVecPerGroup;
-          const float4* wsv = reinterpret_cast<const float4*>(ws_h + g * 32);
-          TOut* yo = reinterpret_cast<TOut*>(p.y_out) + row * p.ld_yo + n0;
-          TOut* yq = reinterpret_cast<TOut*>(p.y_prev) + row * p.ld_yp + n0;
-          constexpr int E = 16 / (int)sizeof(TOut);  // outputs per 16-byte vector
-          uint4 ov[kVecPerGroup];
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {  // 16 accumulator columns at a time
-            uint32_t d0[16], d1[16];
-            tmem_ld16(t0a + g * 32 + h * 16, d0);
-            if (wide_blk) tmem_ld16(t1a + g * 32 + h * 16, d1);
-            tmem_ld_wait();
-#pragma unroll
-            for (int vv = 0; vv < kVecPerGroup / 2; ++vv) {
-              const int v = h * (kVecPerGroup / 2) + vv;
-              float y[E];
-#pragma unroll
-              for (int e = 0; e < E; e += 4) {
-                const float4 ws4 = wsv[(v * E + e) >> 2];
-                const float wsa[4] = {ws4.x, ws4.y, ws4.z, ws4.w};
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                  const int i = vv * E + e + u;  // column within this 16-column half
-                  float ypf;
-                  if constexpr (OUT_BF16) {
-                    const uint32_t w = reinterpret_cast<const uint32_t*>(&ypv[g][v])[(e + u) >> 1];
-                    ypf = __uint_as_float(((e + u) & 1) ? (w & 0xFFFF0000u) : (w << 16));
-                  } else {
-                    ypf = __uint_as_float(reinterpret_cast<const uint32_t*>(&ypv[g][v])[e + u]);
-                  }
-                  float a;
-                  if (wide_blk) {
-                    const int64_t acc = (int64_t)(int32_t)d0[i] + (wide_row ? (int64_t)(int32_t)d1[i] * 256 : 0);
-                    a = __ll2float_rn(acc);
-                  } else {
-                    a = __int2float_rn((int32_t)d0[i]);
-                  }
-                  y[e + u] = __fadd_rn(ypf, __fmul_rn(__fmul_rn(a, p2), wsa[u]));
-                }
-              }
-              if constexpr (OUT_BF16) {
-                uint32_t w[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                  const __nv_bfloat162 b2 = __floats2bfloat162_rn(y[2 * q], y[2 * q + 1]);
-                  w[q] = *reinterpret_cast<const uint32_t*>(&b2);
-                }
-                ov[v] = make_uint4(w[0], w[1], w[2], w[3]);
-              } else {
-                ov[v] = make_uint4(__float_as_uint(y[0]), __float_as_uint(y[1]), __float_as_uint(y[2]),
-                                   __float_as_uint(y[3]));
-              }
-            }
-            if (p.debug_acc && row_ok) {
-              for (int i = 0; i < 16 && n0 + h * 16 + i < p.N; ++i)
-                p.debug_acc[row * p.N + n0 + h * 16 + i] =
-                    (int64_t)(int32_t)d0[i] + (wide_blk && wide_row ? (int64_t)(int32_t)d1[i] * 256 : 0);
-            }
-          }
-          if (row_ok) {
-#pragma unroll
-            for (int v = 0; v < kVecPerGroup; v += 2) {
-              if (v < nv) {  // nv is even: 32-byte pairs are whole
-                if (p.vec32) {
-                  st_global_v8(reinterpret_cast<uint4*>(yo) + v, ov[v], ov[v + 1]);
-                  if (p.y_distinct) st_global_v8(reinterpret_cast<uint4*>(yq) + v, ov[v], ov[v + 1]);
-                } else {
-                  reinterpret_cast<uint4*>(yo)[v] = ov[v];
-                  reinterpret_cast<uint4*>(yo)[v + 1] = ov[v + 1];
-                  if (p.y_distinct) reinterpret_cast<uint4*>(yq)[v] = ov[v], reinterpret_cast<uint4*>(yq)[v + 1] = ov[v + 1];
-                }
-              }
-            }
-          }
+        int yok = 1;
+        if (lane == 0 && ok) {
+          yok = wait_parity(&ybar[ew], y_it & 1, s_abort, p.status, kWaitLimitNs) ? 1 : 0;
+          y_pending = !yok;
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0)
-          for (int q = 0; q < bi.nplanes; ++q) mbar_arrive(&tm_empty[acc_slot[q]]);
-        slot_it += bi.nplanes;
-        }  // ok
+        ++y_it;
+        ok = __shfl_sync(0xffffffffu, ok && yok, 0);
+        if (ok) {
+          // the landed tiles are visible to the lanes that observe the barrier phase
+          mbar_try_wait(&ybar[ew], (y_it - 1) & 1);
+          tc_fence_after();
+          const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+          const uint32_t col_half = half * (BN / 2);
+          const uint32_t t0a = tmem_base + lane_off + acc_slot[0] * BN + col_half;
+          const uint32_t t1a = tmem_base + lane_off + (bi.nplanes == 2 ? acc_slot[1] : acc_slot[0]) * BN + col_half;
+          const float* ws_h = s_ws + half * (BN / 2);
+          const bool wide_blk = bi.nplanes == 2;  // warp-uniform
+          const bool wide_row = pl == 2;
+#pragma unroll 1
+          for (int g = 0; g < C::kHalfGroups; ++g) {
+            uint8_t* box = ybuf + g * C::kBoxBytes + lane * (32 * C::kOutBytes);  // this lane's row
+            const float4* wsv = reinterpret_cast<const float4*>(ws_h + g * 32);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {  // 16 accumulator columns at a time
+              uint32_t d0[16], d1[16];
+              tmem_ld16(t0a + g * 32 + h * 16, d0);
+              if (wide_blk) tmem_ld16(t1a + g * 32 + h * 16, d1);
+              tmem_ld_wait();
+              if (row_ok) {
+                constexpr int E = 16 / C::kOutBytes;  // outputs per 16-byte chunk
+#pragma unroll
+                for (int cc = 0; cc < kChunksPerRow / 2; ++cc) {
+                  const int c = h * (kChunksPerRow / 2) + cc;  // 16-byte chunk of the row
+                  uint4* cp = reinterpret_cast<uint4*>(box + 16 * (c ^ sw(lane)));
+                  const uint4 yv = *cp;
+                  const uint32_t yw[4] = {yv.x, yv.y, yv.z, yv.w};
+                  float y[E];
+#pragma unroll
+                  for (int e = 0; e < E; ++e) {
+                    const int i = cc * E + e;  // column within this 16-column half
+                    const float ws = reinterpret_cast<const float*>(wsv)[h * 16 + i];
+                    float ypf;
+                    if constexpr (OUT_BF16) ypf = __uint_as_float((e & 1) ? (yw[e >> 1] & 0xFFFF0000u) : (yw[e >> 1] << 16));
+                    else ypf = __uint_as_float(yw[e]);
+                    float a;
+                    if (wide_blk) {
+                      const int64_t acc = (int64_t)(int32_t)d0[i] + (wide_row ? (int64_t)(int32_t)d1[i] * 256 : 0);
+                      a = __ll2float_rn(acc);
+                    } else {
+                      a = __int2float_rn((int32_t)d0[i]);
+                    }
+                    y[e] = __fadd_rn(ypf, __fmul_rn(__fmul_rn(a, p2), ws));
+                  }
+                  uint4 o;
+                  if constexpr (OUT_BF16) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                      const __nv_bfloat162 b2 = __floats2bfloat162_rn(y[2 * q], y[2 * q + 1]);
+                      w[q] = *reinterpret_cast<const uint32_t*>(&b2);
+                    }
+                    o = make_uint4(w[0], w[1], w[2], w[3]);
+                  } else {
+                    o = make_uint4(__float_as_uint(y[0]), __float_as_uint(y[1]), __float_as_uint(y[2]),
+                                   __float_as_uint(y[3]));
+                  }
+                  *cp = o;
+                }
+                if (p.debug_acc) {
+                  const int64_t n0 = n_half + g * 32 + h * 16;
+                  for (int i = 0; i < 16 && n0 + i < p.N; ++i)
+                    p.debug_acc[row * p.N + n0 + i] =
+                        (int64_t)(int32_t)d0[i] + (wide_blk && wide_row ? (int64_t)(int32_t)d1[i] * 256 : 0);
+                }
+              }
+            }
+            // the finished 32 x 32 tile goes out through TMA (rows beyond M and
+            // columns beyond N are clipped; rows left to the slice stream carry
+            // their y_prev values unchanged)
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              if (n_half + g * 32 < p.N && row0 < p.M) {  // a store never starts outside the matrix
+                tma_store_2d(&tm_yo, ybuf + g * C::kBoxBytes, (int)(n_half + g * 32), row0);
+                if (p.y_distinct) tma_store_2d(&tm_yp, ybuf + g * C::kBoxBytes, (int)(n_half + g * 32), row0);
+              }
+              bulk_commit();
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0)
+            for (int q = 0; q < bi.nplanes; ++q) mbar_arrive(&tm_empty[acc_slot[q]]);
+          slot_it += bi.nplanes;
+        }
       }
 
       // tiles of this row block whose operands need more than two planes:
-      // the slice stream, one output column per epilogue thread
+      // the slice stream, one output column per epilogue thread, after this
+      // tile's TMA stores have completed
       if (ok && bi.any_slice) {
+        if (lane == 0) bulk_wait<0>();
+        __syncwarp();
+        epi_barrier();
         for (int t = rb * 8; t < min(rb * 8 + 8, T); ++t) {
           if (p.planes[t] <= 2) continue;
           for (int c = etid; c < BN; c += 32 * kEpiWarps) {
             const int64_t n = n_base + c;
             if (n >= p.N) continue;
             slice_stream_column<OUT_BF16>(p.records + (int64_t)t * p.record_cap, p.count[t], p.bits + (int64_t)t * p.K,
-                                          p.g_ref[t], p.w_q + n * p.ld_w, t, n, p.lb, ws_t[c], p.y_prev, p.ld_yp,
+                                          p.g_ref[t], p.w_q + n * p.ld_w, t, n, p.lb, s_ws[c], p.y_prev, p.ld_yp,
                                           p.y_out, p.ld_yo, p.y_distinct, p.debug_acc, p.N);
           }
         }
       }
-      epi_barrier();  // the weight-scale buffer of this parity is free again
+      epi_barrier();  // the weight-scale buffer is free again
     }
+    // nothing of this warp's may still be in flight when the block exits:
+    // y_prev tiles that were requested but not consumed, and the last stores
+    if (lane == 0) {
+      if (y_pending) wait_parity(&ybar[ew], (y_it - 1) & 1, s_abort, p.status, kWaitLimitNs, true);
+      bulk_wait<0>();
+    }
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -567,26 +572,23 @@ __global__ void selftest_wait_kernel(uint32_t* status, uint64_t limit_ns) {
 }
 
 template <int BN, bool BF>
-static int launch_gemm_t(const GemmParams& p, const void* a0, const void* a1, const void* w, int num_sms,
-                         void* stream) {
+static int launch_gemm_t(const GemmParams& p, const CUtensorMap* m, int num_sms, void* stream) {
   const int tiles = p.tiles_m * p.tiles_n;
   const int grid = tiles < num_sms ? tiles : num_sms;
   if (grid == 0) return 0;
-  const int smem = GemmCfg<BN>::kBytes;
+  const int smem = GemmCfg<BN, BF>::kBytes;
   const int e = ensure_max_smem((const void*)gemm_kernel<BN, BF>, smem);
   if (e != 0) return e;
-  gemm_kernel<BN, BF><<<grid, kGThreads, smem, (cudaStream_t)stream>>>(
-      *static_cast<const CUtensorMap*>(a0), *static_cast<const CUtensorMap*>(a1),
-      *static_cast<const CUtensorMap*>(w), p);
+  gemm_kernel<BN, BF><<<grid, kGThreads, smem, (cudaStream_t)stream>>>(m[0], m[1], m[2], m[3], m[4], p);
   return (int)cudaGetLastError();
 }
 
-int launch_gemm(const GemmParams& p, const void* a0, const void* a1, const void* w, int bn, int out_bf16,
-                int num_sms, void* stream) {
-  if (bn == 256) return out_bf16 ? launch_gemm_t<256, true>(p, a0, a1, w, num_sms, stream)
-                                 : launch_gemm_t<256, false>(p, a0, a1, w, num_sms, stream);
-  return out_bf16 ? launch_gemm_t<128, true>(p, a0, a1, w, num_sms, stream)
-                  : launch_gemm_t<128, false>(p, a0, a1, w, num_sms, stream);
+// maps: the A0, A1, W, y_prev and y_out tensor maps (CUtensorMap[5]).
+int launch_gemm(const GemmParams& p, const void* maps, int bn, int out_bf16, int num_sms, void* stream) {
+  const CUtensorMap* m = static_cast<const CUtensorMap*>(maps);
+  if (out_bf16) return bn == 256 ? launch_gemm_t<256, true>(p, m, num_sms, stream)
+                                 : launch_gemm_t<128, true>(p, m, num_sms, stream);
+  return launch_gemm_t<128, false>(p, m, num_sms, stream);  // fp32 outputs use 128-column tiles
 }
 
 int launch_slice_gemm(const SliceParams& p, int out_bf16, int num_sms, void* stream) {

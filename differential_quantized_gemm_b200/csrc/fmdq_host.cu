@@ -88,20 +88,34 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D int8 tensor map: rows x cols with a row pitch of ld bytes, box of
-// box_rows x 128 bytes, 128-byte swizzle, zero fill outside the matrix.
-int make_map_i8(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t ld, int box_rows) {
+// 2-D tensor map of a row-major matrix (rows x cols, row pitch ld elements)
+// with a box of box_cols x box_rows elements; zero fill outside the matrix.
+int make_map(CUtensorMap* map, CUtensorMapDataType dt, int es, const void* base, int64_t rows, int64_t cols,
+             int64_t ld, int box_cols, int box_rows, CUtensorMapSwizzle swz) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(DSTAR_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)ld};
-  const cuuint32_t box[2] = {(cuuint32_t)kChunkK, (cuuint32_t)box_rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)(ld * es)};
+  const cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(DSTAR_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return DSTAR_OK;
+}
+
+// int8 operand: box of box_rows x 128 bytes, 128-byte swizzle (the MMA's K-major layout)
+int make_map_i8(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t ld, int box_rows) {
+  return make_map(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base, rows, cols, ld, kChunkK, box_rows,
+                  CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// Y tiles of the epilogue: 32 x 32 elements; 64-byte rows (bf16) use the
+// 64-byte swizzle, 128-byte rows (fp32) the 128-byte one
+int make_map_y(CUtensorMap* map, const dstar_mat* y) {
+  const bool bf = y->dtype == DSTAR_BF16;
+  return make_map(map, bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, bf ? 2 : 4, y->data,
+                  y->rows, y->cols, y->ld, 32, 32, bf ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -217,12 +231,14 @@ int do_gemm(const dstar_mat* w_q, const float* w_scale, dstar_mat* y_prev, int l
   const bool distinct = y_out->data != y_prev->data;
   const bool slice_all = (c->flags & DSTAR_FLAG_SLICE_PATH) != 0;
   if (!slice_all) {
-    const int bn = choose_bn(M, N, dev.sms);
-    CUtensorMap ma0, ma1, mw;
+    const int bn = bf16 ? choose_bn(M, N, dev.sms) : 128;  // fp32 outputs use 128-column tiles
+    CUtensorMap maps[5];  // A0, A1, W, y_prev, y_out
     int r;
-    if ((r = make_map_i8(&ma0, ws_ptr<void>(c, L.plane0), M, K, K, kBlockM)) != DSTAR_OK) return r;
-    if ((r = make_map_i8(&ma1, ws_ptr<void>(c, L.plane1), M, K, K, kBlockM)) != DSTAR_OK) return r;
-    if ((r = make_map_i8(&mw, w_q->data, N, K, w_q->ld, bn)) != DSTAR_OK) return r;
+    if ((r = make_map_i8(&maps[0], ws_ptr<void>(c, L.plane0), M, K, K, kBlockM)) != DSTAR_OK) return r;
+    if ((r = make_map_i8(&maps[1], ws_ptr<void>(c, L.plane1), M, K, K, kBlockM)) != DSTAR_OK) return r;
+    if ((r = make_map_i8(&maps[2], w_q->data, N, K, w_q->ld, bn)) != DSTAR_OK) return r;
+    if ((r = make_map_y(&maps[3], y_prev)) != DSTAR_OK) return r;
+    if ((r = make_map_y(&maps[4], y_out)) != DSTAR_OK) return r;
     GemmParams g{};
     g.M = M, g.N = N, g.K = K;
     g.lb = lb;
@@ -237,9 +253,6 @@ int do_gemm(const dstar_mat* w_q, const float* w_scale, dstar_mat* y_prev, int l
     g.y_out = y_out->data;
     g.ld_yo = y_out->ld;
     g.y_distinct = distinct;
-    const int64_t es = bf16 ? 2 : 4;
-    g.vec32 = ((reinterpret_cast<uintptr_t>(y_prev->data) | reinterpret_cast<uintptr_t>(y_out->data)) & 31u) == 0 &&
-              (y_prev->ld * es) % 32 == 0 && (y_out->ld * es) % 32 == 0;
     g.status = ws_ptr<uint32_t>(c, L.status);
     g.debug_acc = c->debug_acc;
     g.tiles_m = (int)((M + kBlockM - 1) / kBlockM);
@@ -251,7 +264,7 @@ int do_gemm(const dstar_mat* w_q, const float* w_scale, dstar_mat* y_prev, int l
     g.record_cap = L.record_cap;
     g.count = ws_ptr<const int32_t>(c, L.count);
     g.bits = ws_ptr<const int8_t>(c, L.bits);
-    const int e = launch_gemm(g, &ma0, &ma1, &mw, bn, bf16, dev.sms, stream);
+    const int e = launch_gemm(g, maps, bn, bf16, dev.sms, stream);
     if (e) return cuda_fail(e, "slice-GEMM launch");
     return DSTAR_OK;  // tiles needing the slice stream are handled inside the GEMM kernel
   }

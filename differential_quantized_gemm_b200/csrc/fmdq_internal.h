@@ -57,7 +57,6 @@ struct GemmParams {
   void* y_out;
   int64_t ld_yo;
   int y_distinct;  // y_out is a different buffer: write both
-  int vec32;       // y_prev and y_out rows are 32-byte aligned: 32-byte accesses
   uint32_t* status;
   int64_t* debug_acc;
   int tiles_m, tiles_n, num_chunks;
@@ -101,7 +100,7 @@ WsLayout ws_layout(int64_t M, int64_t K);
 // Launchers (return cudaError_t as int).
 int launch_quantize(const QuantParams& p, int in_bf16, int num_sms, void* stream);
 int quantize_cluster_size(int64_t M, int64_t K, int num_sms);
-int launch_gemm(const GemmParams& p, const void* tmap_a0, const void* tmap_a1, const void* tmap_w, int bn,
+int launch_gemm(const GemmParams& p, const void* maps /* CUtensorMap[5]: A0, A1, W, y_prev, y_out */, int bn,
                 int out_bf16, int num_sms, void* stream);
 int launch_slice_gemm(const SliceParams& p, int out_bf16, int num_sms, void* stream);
 int launch_selftest_wait(uint32_t* status, uint32_t spin_limit, void* stream);
