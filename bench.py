@@ -183,6 +183,11 @@ class Layer:
         return L.dstar_fmdq_slice_gemm(ctypes.byref(self.m_w), self.ws_ptr, ctypes.byref(self.m_y), self.base,
                                        ctypes.byref(self.cfg), ctypes.byref(self.m_y), stream)
 
+    def linear(self, L, parity, stream):
+        return L.dstar_fmdq_linear(ctypes.byref(self.m_x[parity]), ctypes.byref(self.m_xp), ctypes.byref(self.m_y),
+                                   ctypes.byref(self.m_w), self.ws_ptr, self.base, ctypes.byref(self.cfg),
+                                   ctypes.byref(self.m_y), stream)
+
 
 def workload_inputs(cfg, rank):
     from differential_quantized_gemm_b200 import synth
@@ -379,9 +384,18 @@ def run_ours(args, rank, world, local_rank):
 
         kinds = [(r, par) for par in (0, 1) for r in range(args.sets)]
         gev = [[[ext_event() for _ in range(3)] for _ in range(nlayers)] for _ in kinds]
-        graphs = []
+        graphs, prof_graphs = [], []
         cap_stream = torch.cuda.Stream()
         for gi, (r, par) in enumerate(kinds):
+            # the step as a user runs it: one dstar_fmdq_linear call per layer
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap_stream):
+                csh = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+                for lay in sets[r]:
+                    if lay.linear(L, par, csh):
+                        raise RuntimeError(L.dstar_fmdq_last_error().decode())
+            graphs.append(g)
+            # the same step split into its two stages with event nodes between the kernels
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=cap_stream):
                 cs = torch.cuda.current_stream()
@@ -395,7 +409,7 @@ def run_ours(args, rank, world, local_rank):
                     rt.cudaEventRecordWithFlags(gev[gi][li][2], rsh, rt.cudaEventRecordExternal)
                     if rc:
                         raise RuntimeError(L.dstar_fmdq_last_error().decode())
-            graphs.append(g)
+            prof_graphs.append(g)
         for g in graphs:  # warm the graphs (keeps every set's parity alternating)
             g.replay()
         torch.cuda.synchronize()
@@ -420,8 +434,8 @@ def run_ours(args, rank, world, local_rank):
     ev1.record(stream)
     torch.cuda.synchronize()
     t_wall1 = time.time()
-    if graphs:  # continue every set's X_t alternation after the replays
-        for s in range(K):
+    if graphs:  # continue every set's X_t alternation after the replays (both regions)
+        for s in range(K + max(len(graphs), min(K, 1200) // len(graphs) * len(graphs))):
             gi = s % len(graphs)
             uses[gi % args.sets] = gi // args.sets + 1
     if dist:
@@ -430,7 +444,14 @@ def run_ours(args, rank, world, local_rank):
     clocks.stop()
     ms = ev0.elapsed_time(ev1)
     if graphs:
-        # the event nodes hold the last replay of each graph: the timed region's last len(graphs) steps
+        # per-kernel times: a second timed region of the split step, continuing
+        # every set's X_t alternation; the event nodes hold each graph's last replay
+        kp = max(len(graphs), min(K, 1200) // len(graphs) * len(graphs))
+        torch.cuda.synchronize()
+        for s in range(K, K + kp):
+            prof_graphs[s % len(graphs)].replay()
+        torch.cuda.synchronize()
+
         def el(a, b):
             err, v = rt.cudaEventElapsedTime(a, b)
             assert err == rt.cudaError_t.cudaSuccess
@@ -564,8 +585,10 @@ def run_ours(args, rank, world, local_rank):
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * K,
         "clocks": clocks.summary(t_wall0, t_wall1),
         "kernel_sources": kernel_source_sha(),
-        "timing": ("CUDA-graph replay per step (captured C-ABI calls); per-kernel times from event nodes "
-                   "in the graphs' last replays" if graphs else "eager C-ABI calls with CUDA events per kernel"),
+        "timing": ("value: CUDA-graph replay per step of the captured dstar_fmdq_linear calls; per-kernel "
+                   "times: a second timed region of the step split into dstar_fmdq_quantize + "
+                   "dstar_fmdq_slice_gemm with event nodes between the kernels" if graphs
+                   else "eager C-ABI calls with CUDA events per kernel"),
     }
     print(json.dumps(line), flush=True)
 

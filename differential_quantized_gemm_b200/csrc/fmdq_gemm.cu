@@ -184,6 +184,46 @@ __device__ void slice_stream_column(const uint2* recs, int cnt, const int8_t* bi
   }
 }
 
+// One epilogue group: 32 columns of one row (this lane's), in place in its
+// swizzled 32 x 32 shared-memory tile.  acc = d0 (+ 256 d1 for rows of
+// two-plane tiles); y = y_prev + ((float)acc * p2) * w_scale, fp32, no FMA.
+template <bool OUT_BF16, bool WIDE>
+__device__ __forceinline__ void epi_group(uint8_t* row, int swz, const float* ws32, const uint32_t (&d0)[32],
+                                          const uint32_t (&d1)[32], bool wide_row, float p2) {
+  constexpr int kOutBytes = OUT_BF16 ? 2 : 4;
+  constexpr int E = 16 / kOutBytes;              // outputs per 16-byte chunk
+  constexpr int kChunks = 32 * kOutBytes / 16;   // chunks per 32-column row
+#pragma unroll
+  for (int c = 0; c < kChunks; ++c) {
+    uint4* cp = reinterpret_cast<uint4*>(row + 16 * (c ^ swz));
+    const uint4 yv = *cp;
+    const uint32_t yw[4] = {yv.x, yv.y, yv.z, yv.w};
+    float y[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const int i = c * E + e;
+      float ypf;
+      if constexpr (OUT_BF16) ypf = __uint_as_float((e & 1) ? (yw[e >> 1] & 0xFFFF0000u) : (yw[e >> 1] << 16));
+      else ypf = __uint_as_float(yw[e]);
+      float a;
+      if constexpr (WIDE) a = __ll2float_rn((int64_t)(int32_t)d0[i] + (wide_row ? (int64_t)(int32_t)d1[i] * 256 : 0));
+      else a = __int2float_rn((int32_t)d0[i]);
+      y[e] = __fadd_rn(ypf, __fmul_rn(__fmul_rn(a, p2), ws32[i]));
+    }
+    if constexpr (OUT_BF16) {
+      uint32_t w[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const __nv_bfloat162 b2 = __floats2bfloat162_rn(y[2 * q], y[2 * q + 1]);
+        w[q] = *reinterpret_cast<const uint32_t*>(&b2);
+      }
+      *cp = make_uint4(w[0], w[1], w[2], w[3]);
+    } else {
+      *cp = make_uint4(__float_as_uint(y[0]), __float_as_uint(y[1]), __float_as_uint(y[2]), __float_as_uint(y[3]));
+    }
+  }
+}
+
 }  // namespace
 
 size_t gemm_smem_bytes(int bn) { return bn == 256 ? GemmCfg<256, true>::kBytes : GemmCfg<128, true>::kBytes; }
@@ -229,8 +269,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
     prefetch_tmap(&tm_yp);
     prefetch_tmap(&tm_yo);
   }
+  pdl_launch_dependents();
   // block info of this CTA's first kMaxTileSlots tiles, loaded in parallel
   for (int i = threadIdx.x; i < kMaxTileSlots; i += kGThreads) s_info[i] = make_int4(0, 0, 0, 0);
+  pdl_wait();  // the quantizer's outputs (and y_prev, W) are read only after the previous kernel completed
   __syncthreads();
   for (int i = threadIdx.x; i < min(my_tiles, kMaxTileSlots) * 8; i += kGThreads) {
     const int slot = i >> 3, sub = i & 7;
@@ -419,67 +461,9 @@ __global__ void __launch_bounds__(kGThreads, 1)
           const float* ws_h = s_ws + half * (BN / 2);
           const bool wide_blk = bi.nplanes == 2;  // warp-uniform
           const bool wide_row = pl == 2;
-#pragma unroll 1
-          for (int g = 0; g < C::kHalfGroups; ++g) {
-            uint8_t* box = ybuf + g * C::kBoxBytes + lane * (32 * C::kOutBytes);  // this lane's row
-            const float4* wsv = reinterpret_cast<const float4*>(ws_h + g * 32);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {  // 16 accumulator columns at a time
-              uint32_t d0[16], d1[16];
-              tmem_ld16(t0a + g * 32 + h * 16, d0);
-              if (wide_blk) tmem_ld16(t1a + g * 32 + h * 16, d1);
-              tmem_ld_wait();
-              if (row_ok) {
-                constexpr int E = 16 / C::kOutBytes;  // outputs per 16-byte chunk
-#pragma unroll
-                for (int cc = 0; cc < kChunksPerRow / 2; ++cc) {
-                  const int c = h * (kChunksPerRow / 2) + cc;  // 16-byte chunk of the row
-                  uint4* cp = reinterpret_cast<uint4*>(box + 16 * (c ^ sw(lane)));
-                  const uint4 yv = *cp;
-                  const uint32_t yw[4] = {yv.x, yv.y, yv.z, yv.w};
-                  float y[E];
-#pragma unroll
-                  for (int e = 0; e < E; ++e) {
-                    const int i = cc * E + e;  // column within this 16-column half
-                    const float ws = reinterpret_cast<const float*>(wsv)[h * 16 + i];
-                    float ypf;
-                    if constexpr (OUT_BF16) ypf = __uint_as_float((e & 1) ? (yw[e >> 1] & 0xFFFF0000u) : (yw[e >> 1] << 16));
-                    else ypf = __uint_as_float(yw[e]);
-                    float a;
-                    if (wide_blk) {
-                      const int64_t acc = (int64_t)(int32_t)d0[i] + (wide_row ? (int64_t)(int32_t)d1[i] * 256 : 0);
-                      a = __ll2float_rn(acc);
-                    } else {
-                      a = __int2float_rn((int32_t)d0[i]);
-                    }
-                    y[e] = __fadd_rn(ypf, __fmul_rn(__fmul_rn(a, p2), ws));
-                  }
-                  uint4 o;
-                  if constexpr (OUT_BF16) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                      const __nv_bfloat162 b2 = __floats2bfloat162_rn(y[2 * q], y[2 * q + 1]);
-                      w[q] = *reinterpret_cast<const uint32_t*>(&b2);
-                    }
-                    o = make_uint4(w[0], w[1], w[2], w[3]);
-                  } else {
-                    o = make_uint4(__float_as_uint(y[0]), __float_as_uint(y[1]), __float_as_uint(y[2]),
-                                   __float_as_uint(y[3]));
-                  }
-                  *cp = o;
-                }
-                if (p.debug_acc) {
-                  const int64_t n0 = n_half + g * 32 + h * 16;
-                  for (int i = 0; i < 16 && n0 + i < p.N; ++i)
-                    p.debug_acc[row * p.N + n0 + i] =
-                        (int64_t)(int32_t)d0[i] + (wide_blk && wide_row ? (int64_t)(int32_t)d1[i] * 256 : 0);
-                }
-              }
-            }
-            // the finished 32 x 32 tile goes out through TMA (rows beyond M and
-            // columns beyond N are clipped; rows left to the slice stream carry
-            // their y_prev values unchanged)
+          // finished 32 x 32 tiles go out through TMA (rows beyond M and columns
+          // beyond N are clipped; rows left to the slice stream keep y_prev)
+          auto store_group = [&](int g) {
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
@@ -488,6 +472,45 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 if (p.y_distinct) tma_store_2d(&tm_yp, ybuf + g * C::kBoxBytes, (int)(n_half + g * 32), row0);
               }
               bulk_commit();
+            }
+          };
+          auto debug_group = [&](int g, const uint32_t (&d0)[32], const uint32_t (&d1)[32], bool wide) {
+            const int64_t n0 = n_half + g * 32;
+            for (int i = 0; i < 32 && n0 + i < p.N; ++i)
+              p.debug_acc[row * p.N + n0 + i] =
+                  (int64_t)(int32_t)d0[i] + (wide && wide_row ? (int64_t)(int32_t)d1[i] * 256 : 0);
+          };
+          uint8_t* my_row = ybuf + lane * (32 * C::kOutBytes);
+          const int swz = sw(lane);
+          if (!wide_blk) {
+            // one plane: the accumulator of group g+1 is read from TMEM while group g is computed
+            uint32_t dA[32], dB[32];
+            tmem_ld32(t0a, dA);
+            tmem_ld_wait();
+#pragma unroll
+            for (int g = 0; g < C::kHalfGroups; ++g) {
+              uint32_t(&cur)[32] = (g & 1) ? dB : dA;
+              uint32_t(&nxt)[32] = (g & 1) ? dA : dB;
+              if (g + 1 < C::kHalfGroups) tmem_ld32(t0a + (g + 1) * 32, nxt);
+              if (row_ok) {
+                epi_group<OUT_BF16, false>(my_row + g * C::kBoxBytes, swz, ws_h + g * 32, cur, cur, false, p2);
+                if (p.debug_acc) debug_group(g, cur, cur, false);
+              }
+              store_group(g);
+              if (g + 1 < C::kHalfGroups) tmem_ld_wait();
+            }
+          } else {
+#pragma unroll 1
+            for (int g = 0; g < C::kHalfGroups; ++g) {
+              uint32_t d0[32], d1[32];
+              tmem_ld32(t0a + g * 32, d0);
+              tmem_ld32(t1a + g * 32, d1);
+              tmem_ld_wait();
+              if (row_ok) {
+                epi_group<OUT_BF16, true>(my_row + g * C::kBoxBytes, swz, ws_h + g * 32, d0, d1, wide_row, p2);
+                if (p.debug_acc) debug_group(g, d0, d1, true);
+              }
+              store_group(g);
             }
           }
           tc_fence_before();
@@ -579,7 +602,18 @@ static int launch_gemm_t(const GemmParams& p, const CUtensorMap* m, int num_sms,
   const int smem = GemmCfg<BN, BF>::kBytes;
   const int e = ensure_max_smem((const void*)gemm_kernel<BN, BF>, smem);
   if (e != 0) return e;
-  gemm_kernel<BN, BF><<<grid, kGThreads, smem, (cudaStream_t)stream>>>(m[0], m[1], m[2], m[3], m[4], p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid, 1, 1);
+  cfg.blockDim = dim3(kGThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = (cudaStream_t)stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // overlap the launch with the quantizer
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t ce = cudaLaunchKernelEx(&cfg, gemm_kernel<BN, BF>, m[0], m[1], m[2], m[3], m[4], p);
+  if (ce != cudaSuccess) return (int)ce;
   return (int)cudaGetLastError();
 }
 

@@ -96,19 +96,28 @@ __device__ __forceinline__ ColParams col_params(uint32_t mbits, int lb, float be
   return cp;
 }
 
-// The 2-bit field j of the 16 codes of a channel (byte r of word w = token
-// 4w + r), gathered into one word: token i in bits 2i..2i+1.
-__device__ __forceinline__ uint32_t slice_word(const uint4 cw, int j) {
-  const uint32_t ws[4] = {cw.x, cw.y, cw.z, cw.w};
-  uint32_t out = 0;
+// The four 2-bit slice words of a channel from its 16 codes (byte r of code
+// word w = token 4w + r): word j holds field j (bits 2j..2j+1) of every code,
+// token i in bits 2i..2i+1.  Each code word is a 4 x 4 matrix of 2-bit cells
+// (byte i, field j); two delta swaps transpose it to (byte j, field i), and
+// byte permutes gather byte j of the four transposed words.
+__device__ __forceinline__ void slice_words(const uint4 cw, uint32_t (&out)[4]) {
+  uint32_t tw[4] = {cw.x, cw.y, cw.z, cw.w};
 #pragma unroll
   for (int w = 0; w < 4; ++w) {
-    uint32_t x = (ws[w] >> (2 * j)) & 0x03030303u;
-    x = (x | (x >> 6)) & 0x000F000Fu;
-    x = (x | (x >> 12)) & 0xFFu;
-    out |= x << (8 * w);
+    uint32_t x = tw[w], t;
+    t = ((x >> 12) ^ x) & 0x0000F0F0u;  // swap the off-diagonal 2 x 2 blocks of cells
+    x ^= t ^ (t << 12);
+    t = ((x >> 6) ^ x) & 0x00CC00CCu;   // swap the off-diagonal cells inside each block
+    x ^= t ^ (t << 6);
+    tw[w] = x;
   }
-  return out;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t sel = (uint32_t)j | ((uint32_t)(4 + j) << 4);
+    const uint32_t lo = __byte_perm(tw[0], tw[1], sel), hi = __byte_perm(tw[2], tw[3], sel);
+    out[j] = __byte_perm(lo, hi, 0x5410);
+  }
 }
 
 __device__ __forceinline__ int code_at(const uint4 cw, int r) {
@@ -142,6 +151,9 @@ struct QSmem {
   int flags;
   int base[kTagWin];       // records before this CTA's first record of the tag
   int warp_cnt[kQWarps][kTagWin];
+  // copies of the cluster's exchanged values, fetched one remote word per thread
+  int x_fmax[kMaxCluster], x_fmin[kMaxCluster], x_need[kMaxCluster];
+  int x_tot[kMaxCluster][kTagWin];
 };
 
 }  // namespace
@@ -184,6 +196,8 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParam
 
   if (tid < kMaxMaskWords) S.mask[tid] = 0;
   if (tid == 0) S.flags = 0;
+  pdl_launch_dependents();
+  pdl_wait();  // nothing of global memory is touched before the previous kernel completed
   __syncthreads();
 
   const int lb = p.lb, t0 = p.t0, fb = p.force_bits;
@@ -268,11 +282,14 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParam
       set_status(p.status, (S.flags & 1 ? DSTAR_STATUS_NONFINITE : 0u) | (S.flags & 2 ? DSTAR_STATUS_RANGE : 0u));
   }
   csync(cluster, C);
-  int g = -1000, gmin = 1000;
-  for (int q = 0; q < C; ++q) {
-    const QSmem* R = C > 1 ? cluster.map_shared_rank(&S, q) : &S;
-    g = max(g, R->fmax), gmin = min(gmin, R->fmin);
+  if (tid < C) {  // one remote read per thread, all in flight together
+    const QSmem* R = C > 1 ? cluster.map_shared_rank(&S, tid) : &S;
+    S.x_fmax[tid] = R->fmax;
+    S.x_fmin[tid] = R->fmin;
   }
+  __syncthreads();
+  int g = -1000, gmin = 1000;
+  for (int q = 0; q < C; ++q) g = max(g, S.x_fmax[q]), gmin = min(gmin, S.x_fmin[q]);
 
   // planes the tile needs: every v = q 2^(g - FPoT) must fit the split
   int need = 1;
@@ -292,8 +309,10 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParam
     S.need = n;
   }
   csync(cluster, C);
+  if (tid < C) S.x_need[tid] = (C > 1 ? cluster.map_shared_rank(&S, tid) : &S)->need;
+  __syncthreads();
   int planes = 1;
-  for (int q = 0; q < C; ++q) planes = max(planes, (C > 1 ? cluster.map_shared_rank(&S, q) : &S)->need);
+  for (int q = 0; q < C; ++q) planes = max(planes, S.x_need[q]);
 
   // ------------------------------------------------- phase 2a: operand planes
   // Same channel-pair mapping: 2-byte stores, a warp writes 64 contiguous bytes per row.
@@ -357,11 +376,17 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParam
     int cnt[kTagWin];
 #pragma unroll
     for (int ti = 0; ti < kTagWin; ++ti) cnt[ti] = 0;
-    for (int64_t kb = w_lo; kb < w_hi; kb += 32) {
-      const int64_t k = kb + lane;
-      const uint32_t m = k < w_hi ? tag_mask(s_fpot[k], s_bits[k], tw) : 0u;
+    for (int64_t kb = w_lo; kb < w_hi; kb += 4 * 32) {  // four independent chunks per iteration
+      uint32_t m[4];
 #pragma unroll
-      for (int ti = 0; ti < kTagWin; ++ti) cnt[ti] += __popc(__ballot_sync(0xffffffffu, (m >> ti) & 1u));
+      for (int u = 0; u < 4; ++u) {
+        const int64_t k = kb + 32 * u + lane;
+        m[u] = k < w_hi ? tag_mask(s_fpot[k], s_bits[k], tw) : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int ti = 0; ti < kTagWin; ++ti) cnt[ti] += __popc(__ballot_sync(0xffffffffu, (m[u] >> ti) & 1u));
     }
     if (lane == 0) {
 #pragma unroll
@@ -375,12 +400,16 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParam
     }
     csync(cluster, C);
     // window totals of every CTA -> where this CTA's records of each tag start
+    if (tid < C * kTagWin) {
+      const int q = tid / kTagWin, u = tid % kTagWin;
+      S.x_tot[q][u] = (C > 1 ? cluster.map_shared_rank(&S, q) : &S)->cta_tot[u];
+    }
+    __syncthreads();
     if (tid < kTagWin) {
       int below = 0, lower_cta = 0, all = 0;
       for (int q = 0; q < C; ++q) {
-        const QSmem* R = C > 1 ? cluster.map_shared_rank(&S, q) : &S;
         for (int u = 0; u < kTagWin; ++u) {
-          const int v = R->cta_tot[u];
+          const int v = S.x_tot[q][u];
           if (u < tid) below += v;
           if (u == tid && q < rank) lower_cta += v;
           all += v;
@@ -397,30 +426,38 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParam
       for (int w = 0; w < warp; ++w) o += S.warp_cnt[w][ti];
       off[ti] = o;
     }
-    // pass B: rank and write
-    for (int64_t kb = w_lo; kb < w_hi; kb += 32) {
-      const int64_t k = kb + lane;
-      const bool kv = k < w_hi;
-      const int f = kv ? s_fpot[k] : 0, b = kv ? s_bits[k] : 0;
-      const uint32_t m = kv ? tag_mask(f, b, tw) : 0u;
-      uint32_t bal[kTagWin];
+    // pass B: rank and write, two independent chunks per iteration
+    for (int64_t kb = w_lo; kb < w_hi; kb += 2 * 32) {
+      int f[2], b[2];
+      uint32_t m[2], bal[2][kTagWin], words[2][4];
+      int64_t k[2];
 #pragma unroll
-      for (int ti = 0; ti < kTagWin; ++ti) bal[ti] = __ballot_sync(0xffffffffu, (m >> ti) & 1u);
-      if (m) {
-        const uint4 cw = *reinterpret_cast<const uint4*>(s_code + 16 * k);
+      for (int u = 0; u < 2; ++u) {
+        k[u] = kb + 32 * u + lane;
+        const bool kv = k[u] < w_hi;
+        f[u] = kv ? s_fpot[k[u]] : 0, b[u] = kv ? s_bits[k[u]] : 0;
+        m[u] = kv ? tag_mask(f[u], b[u], tw) : 0u;
+        if (m[u]) slice_words(*reinterpret_cast<const uint4*>(s_code + 16 * k[u]), words[u]);
 #pragma unroll
-        for (int ti = 0; ti < kTagWin; ++ti) {
-          if ((m >> ti) & 1u) {
-            // the field j < b/2 of the b-bit pattern equals that of the 8-bit pattern
-            const int j = (f - tw - ti) >> 1;
-            rec[off[ti] + __popc(bal[ti] & lt)] =
-                make_uint2(slice_word(cw, j),
-                           (uint32_t)(k_lo + k) | ((uint32_t)(uint8_t)(int8_t)(tw + ti) << 16) | ((uint32_t)j << 24));
-          }
-        }
+        for (int ti = 0; ti < kTagWin; ++ti) bal[u][ti] = __ballot_sync(0xffffffffu, (m[u] >> ti) & 1u);
       }
 #pragma unroll
-      for (int ti = 0; ti < kTagWin; ++ti) off[ti] += __popc(bal[ti]);
+      for (int u = 0; u < 2; ++u) {
+        if (m[u]) {
+#pragma unroll
+          for (int ti = 0; ti < kTagWin; ++ti) {
+            if ((m[u] >> ti) & 1u) {
+              // the field j < b/2 of the b-bit pattern equals that of the 8-bit pattern
+              const int j = (f[u] - tw - ti) >> 1;
+              const uint32_t w = j == 0 ? words[u][0] : j == 1 ? words[u][1] : j == 2 ? words[u][2] : words[u][3];
+              rec[off[ti] + __popc(bal[u][ti] & lt)] = make_uint2(
+                  w, (uint32_t)(k_lo + k[u]) | ((uint32_t)(uint8_t)(int8_t)(tw + ti) << 16) | ((uint32_t)j << 24));
+            }
+          }
+        }
+#pragma unroll
+        for (int ti = 0; ti < kTagWin; ++ti) off[ti] += __popc(bal[u][ti]);
+      }
     }
     csync(cluster, C);  // cta_tot and warp_cnt are rewritten by the next window
   }
@@ -458,13 +495,15 @@ int launch_quantize(const QuantParams& p, int in_bf16, int num_sms, void* stream
   cfg.blockDim = dim3(kQThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = (cudaStream_t)stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = C;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // overlap the launch with the previous kernel
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   cudaError_t ce;
   if (in_bf16) ce = cudaLaunchKernelEx(&cfg, quantize_kernel<__nv_bfloat16>, p, C, kc_max);
   else ce = cudaLaunchKernelEx(&cfg, quantize_kernel<float>, p, C, kc_max);
