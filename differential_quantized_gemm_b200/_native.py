@@ -28,8 +28,9 @@ K_MAX = 8192
 EXPORTED = [
     "dstar_fmdq_version", "dstar_fmdq_error_string", "dstar_fmdq_last_error", "dstar_fmdq_workspace_size",
     "dstar_fmdq_workspace_layout", "dstar_fmdq_workspace_init", "dstar_fmdq_linear", "dstar_fmdq_quantize",
-    "dstar_fmdq_slice_gemm", "dstar_fmdq_status", "dstar_fmdq_selftest_wait",
+    "dstar_fmdq_slice_gemm", "dstar_fmdq_status", "dstar_fmdq_selftest_wait", "dstar_fmdq_linear_noalloc",
 ]
+NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 class DstarMat(ctypes.Structure):
@@ -78,6 +79,8 @@ def lib():
         L.dstar_fmdq_slice_gemm.argtypes = [MP, P, MP, ctypes.c_float, ctypes.POINTER(TileCfg), MP, P]
         L.dstar_fmdq_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32)]
         L.dstar_fmdq_selftest_wait.argtypes = [P, ctypes.c_uint32, P]
+        L.dstar_fmdq_linear_noalloc.argtypes = [MP, MP, MP, MP, P, ctypes.c_float, ctypes.POINTER(TileCfg), MP, P,
+                                                P]
         for name in EXPORTED[3:]:
             getattr(L, name).restype = ctypes.c_int
         _lib = L
@@ -184,6 +187,25 @@ def linear(x_t, x_prev, y_prev, w_q, w_scale, base_scale: float, ws: Workspace, 
     _check(lib().dstar_fmdq_linear(ctypes.byref(mx), ctypes.byref(mp), ctypes.byref(my), ctypes.byref(mw),
                                    ctypes.c_void_p(w_scale.data_ptr()), base_scale, ctypes.byref(cfg),
                                    ctypes.byref(mo), _stream(stream)))
+    return y_out
+
+
+def linear_noalloc(x_t, x_prev, y_prev, w_q, w_scale, base_scale: float, *, t0: int = 0, force_bits: int = 0,
+                   flags: int = 0, y_out=None, status_out=None, debug_codes=None, debug_acc=None, stream=None):
+    """dstar_fmdq_linear_noalloc: dstar_fmdq_linear with the library's static
+    device scratch in place of a workspace, for callers that cannot allocate.
+    status_out: optional int32/uint32 device tensor of one element that receives
+    this call's status bits.  Returns y_out (y_prev if None)."""
+    if y_out is None:
+        y_out = y_prev
+    cfg = TileCfg(TILE, t0, force_bits, flags, None, 0,
+                  ctypes.c_void_p(debug_codes.data_ptr()) if debug_codes is not None else None,
+                  ctypes.c_void_p(debug_acc.data_ptr()) if debug_acc is not None else None)
+    mx, mp, my, mw, mo = mat(x_t), mat(x_prev), mat(y_prev), mat(w_q), mat(y_out)
+    st = ctypes.c_void_p(status_out.data_ptr()) if status_out is not None else None
+    _check(lib().dstar_fmdq_linear_noalloc(ctypes.byref(mx), ctypes.byref(mp), ctypes.byref(my), ctypes.byref(mw),
+                                           ctypes.c_void_p(w_scale.data_ptr()), base_scale, ctypes.byref(cfg),
+                                           ctypes.byref(mo), st, _stream(stream)))
     return y_out
 
 

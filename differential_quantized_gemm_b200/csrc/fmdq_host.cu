@@ -341,6 +341,9 @@ int ensure_max_smem(const void* func, int bytes) {
   return 0;
 }
 
+int report_error(int code, const char* msg) { return fail(code, "%s", msg); }
+int report_cuda_error(int cuda_error, const char* what) { return cuda_fail(cuda_error, what); }
+
 WsLayout ws_layout(int64_t M, int64_t K) {
   WsLayout L{};
   const int64_t T = M / kTile;

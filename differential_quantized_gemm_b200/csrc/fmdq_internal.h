@@ -111,4 +111,8 @@ size_t quantize_smem_bytes(int64_t Kc);  // shared memory of a CTA owning Kc cha
 int ensure_max_smem(const void* func, int bytes);
 size_t gemm_smem_bytes(int bn);
 
+// Record a one-line reason for dstar_fmdq_last_error() and return `code`.
+int report_error(int code, const char* msg);
+int report_cuda_error(int cuda_error, const char* what);  // returns DSTAR_ERR_CUDA
+
 }  // namespace fmdq

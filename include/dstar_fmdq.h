@@ -20,8 +20,9 @@
  *
  * Conventions for every entry point
  *   - All matrices are row-major in DEVICE memory and owned by the caller; the
- *     library allocates nothing and keeps no global state.  Scratch lives in a
- *     caller-owned device workspace (dstar_fmdq_workspace_size bytes).
+ *     library allocates nothing.  Scratch lives in a caller-owned device
+ *     workspace (dstar_fmdq_workspace_size bytes), except for
+ *     dstar_fmdq_linear_noalloc, which uses a static device array instead.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  All work is enqueued asynchronously on it; nothing synchronises
  *     except dstar_fmdq_status.
@@ -80,6 +81,7 @@ extern "C" {
 #define DSTAR_K_MAX 8192       /* input channels */
 #define DSTAR_BASE_LOG2_MIN (-32)
 #define DSTAR_BASE_LOG2_MAX 32
+#define DSTAR_NOALLOC_SCRATCH_BYTES (64u << 20) /* static scratch of dstar_fmdq_linear_noalloc */
 
 /* A row-major matrix in device memory: element (r, c) is at
  * data + (r * ld + c) * sizeof(element).  ld is in elements. */
@@ -162,6 +164,49 @@ DSTAR_API int dstar_fmdq_workspace_init(void* workspace, size_t bytes, void* str
 DSTAR_API int dstar_fmdq_linear(const dstar_mat* x_t, dstar_mat* x_prev, dstar_mat* y_prev, const dstar_mat* w_q,
                       const float* w_scale, float base_scale, const dstar_tile_cfg* tile_cfg,
                       dstar_mat* y_out, void* stream);
+
+/*
+ * dstar_fmdq_linear for callers that cannot allocate device memory.  The
+ * paper has no counterpart: this is a packaging choice of the library.
+ *
+ * Who needs it: code that runs where device memory belongs to someone else --
+ * a plug-in layer of an inference engine or a custom operator whose host only
+ * hands it input and output buffers, a real-time loop that must not call
+ * cudaMalloc (it can synchronise the device and take milliseconds), or a
+ * framework whose caching allocator must account for every byte.  Such a
+ * caller cannot create the workspace dstar_fmdq_linear asks for.
+ *
+ * Instead the library keeps a static device array of
+ * DSTAR_NOALLOC_SCRATCH_BYTES (64 MiB) in its own image.  Every GPU that loads
+ * the library's device code holds that array until the process exits (with
+ * CUDA's lazy module loading, from this entry point's first call on the
+ * device; with eager loading, from context creation).  The call allocates
+ * nothing: no cudaMalloc, no cudaFree, no allocating library routine.
+ *
+ * Arguments, layouts, shapes and results are those of dstar_fmdq_linear, with
+ * two differences:
+ *   tile_cfg->workspace must be NULL and tile_cfg->workspace_bytes 0
+ *           (INVALID_ARG otherwise); the other fields keep their meaning.
+ *   status_out: NULL, or a 4-byte aligned word in device memory (or host
+ *           memory the device can reach) that receives, in stream order, the
+ *           DSTAR_STATUS_* bits of this call; the array's status word is then
+ *           cleared, so each call reports only its own problems.
+ * Size limit: the call needs dstar_fmdq_workspace_size(M, K) bytes of the
+ * array (about 4.1 * M * K; e.g. M = 2048 tokens with K = 4608 channels fits)
+ * and returns DSTAR_ERR_WORKSPACE, enqueueing nothing, when that exceeds
+ * DSTAR_NOALLOC_SCRATCH_BYTES.
+ * First call on a device: it looks up the array's device address with that
+ * device current and enqueues the clearing of its status word on `stream`.
+ * Make that first call before any stream capture.
+ * Sharing: every call on a device uses the same array, which keeps the
+ * previous call's contents.  Calls that may overlap on the GPU (different
+ * streams without an ordering between them, or several host threads) race on
+ * it and give wrong results: order them, for instance on one stream.
+ */
+DSTAR_API int dstar_fmdq_linear_noalloc(const dstar_mat* x_t, dstar_mat* x_prev, dstar_mat* y_prev,
+                                        const dstar_mat* w_q, const float* w_scale, float base_scale,
+                                        const dstar_tile_cfg* tile_cfg, dstar_mat* y_out, uint32_t* status_out,
+                                        void* stream);
 
 /*
  * First stage alone (section 3.1 steps 1-4, the paper's QPU): dX, max-abs,
