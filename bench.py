@@ -189,6 +189,24 @@ class Layer:
                                    ctypes.byref(self.m_y), stream)
 
 
+def max_over_ranks(value: float, device="cpu") -> float:
+    """The largest of every rank's value (the job's time is its slowest rank's);
+    the value itself in a single-process run."""
+    import torch
+    import torch.distributed as td
+    if not (td.is_available() and td.is_initialized()) or td.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    td.all_reduce(t, op=td.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tops(world: int, ops_per_rank: float, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank does the same work per step (weak
+    scaling), and the step takes the slowest rank's time."""
+    return world * ops_per_rank / (ms_per_step * 1e-3) / 1e12
+
+
 def workload_inputs(cfg, rank):
     from differential_quantized_gemm_b200 import synth
     seed = None if rank == 0 else cfg + 7919 * rank
@@ -461,13 +479,10 @@ def run_ours(args, rank, world, local_rank):
     else:
         k1_ms = [statistics.fmean(evs[s][li][0].elapsed_time(evs[s][li][1]) for s in range(K)) for li in range(nlayers)]
         k2_ms = [statistics.fmean(evs[s][li][1].elapsed_time(evs[s][li][2]) for s in range(K)) for li in range(nlayers)]
-    if dist:
-        t = torch.tensor([ms], device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, "cuda")
     ms_step = ms / K
     dense_step = sum(st["k2_dense"] for st in stats)
-    value = world * dense_step / (ms_step * 1e-3) / 1e12
+    value = job_tops(world, dense_step, ms_step)
 
     # e2e: host buffers, copies inside the timed region
     e2e = None
@@ -510,12 +525,8 @@ def run_ours(args, rank, world, local_rank):
         step_e2e(s)
     e1.record(stream)
     torch.cuda.synchronize()
-    ems = e0.elapsed_time(e1)
-    if dist:
-        t = torch.tensor([ems], device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ems = float(t.item())
-    e2e = {"value": world * dense_step / (ems / ke * 1e-3) / 1e12, "unit": "TOPS", "h2d_bytes_per_step": h2d,
+    ems = max_over_ranks(e0.elapsed_time(e1), "cuda")
+    e2e = {"value": job_tops(world, dense_step, ems / ke), "unit": "TOPS", "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h, "steps": ke, "ms_per_step": ems / ke,
            "path": "pinned host X_t -> device, dstar_fmdq_linear per layer, Y_t -> pinned host"}
 
