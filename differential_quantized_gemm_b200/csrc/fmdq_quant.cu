@@ -34,7 +34,6 @@ constexpr int kQThreads = 256;
 constexpr int kQWarps = kQThreads / 32;
 constexpr int kMaxCluster = 8;
 constexpr int kMaxMaskWords = (DSTAR_K_MAX / kChunkK + 31) / 32;
-constexpr int kTagWin = 8;  // tags ranked per pass (one ballot each)
 
 // Two adjacent channels of one token row.
 template <typename TIn>
@@ -120,19 +119,46 @@ __device__ __forceinline__ void slice_words(const uint4 cw, uint32_t (&out)[4]) 
   }
 }
 
-__device__ __forceinline__ int code_at(const uint4 cw, int r) {
-  const uint32_t w = r < 4 ? cw.x : r < 8 ? cw.y : r < 12 ? cw.z : cw.w;
-  return (int)(int8_t)(w >> (8 * (r & 3)));
+// Shift room of a channel: the largest s with every code q of the channel
+// satisfying lo <= q 2^s <= hi, for the one-plane range [-128, 127] (wide =
+// false) or the two-plane range [-32896, 32639] (wide = true); 99 for a
+// channel whose codes are all zero.  For |q| <= 128 the bounds reduce to bit
+// lengths: q 2^s <= 127 iff bitlen(q) + s <= 7, q 2^s <= 32639 iff
+// bitlen(q) + s <= 15, and -m 2^s >= -128 (resp. -32896) iff
+// bitlen(m - 1) + s <= 7 (resp. 15).
+__device__ __forceinline__ int shift_room(int qmax, int qmin, bool wide) {
+  const int top = wide ? 15 : 7;
+  int r = 99;
+  if (qmax > 0) r = top - (32 - __clz(qmax));
+  if (qmin < 0) r = min(r, top - (32 - __clz(-qmin - 1)));
+  return r;
 }
 
-// Window slots ti (tag tw + ti, 0 <= ti < 8) that one channel's slices occupy.
-__device__ __forceinline__ uint32_t tag_mask(int f, int b, int tw) {
-  uint32_t m = 0;
-  for (int j = 0; j < (b >> 1); ++j) {  // slice j has tag f - 2j
-    const int ti = f - 2 * j - tw;
-    if (ti >= 0 && ti < kTagWin) m |= 1u << ti;
-  }
-  return m;
+// 16-byte slot of local channel c in the code array.  The XOR swizzle inside
+// each 128-byte row keeps three access patterns free of bank conflicts:
+// channel pairs per thread (phase 1), four channels per thread (planes) and one
+// channel per lane (encoded stream).
+__device__ __forceinline__ int code_slot(int c) { return c ^ ((c >> 3) & 7); }
+
+// Window slots (tag - tw, 0..31) of the slices of a channel with FPoT f and
+// width b: slice j has tag f - 2j, j < b/2, so the slots are lo, lo + 2, ..,
+// lo + b - 2 with lo = f - b + 2 - tw.
+__device__ __forceinline__ uint32_t tag_mask32(int f, int b, int tw) {
+  const uint32_t pat = 0x55u & ((1u << b) - 1u);
+  const int lo = f - b + 2 - tw;
+  if (lo >= 32 || lo < -8) return 0u;
+  return (uint32_t)(((uint64_t)pat << (lo + 32)) >> 32);
+}
+
+// Rows 4R..4R+3 of four channels (word R of each channel's 16 codes, one byte
+// per row) -> four row words of four channels each.
+__device__ __forceinline__ void transpose4(uint32_t a, uint32_t b, uint32_t c, uint32_t d, uint32_t (&row)[4]) {
+  const uint32_t t0 = __byte_perm(a, b, 0x5140), t1 = __byte_perm(c, d, 0x5140);
+  const uint32_t t2 = __byte_perm(a, b, 0x7362), t3 = __byte_perm(c, d, 0x7362);
+  row[0] = __byte_perm(t0, t1, 0x5410);
+  row[1] = __byte_perm(t0, t1, 0x7632);
+  row[2] = __byte_perm(t2, t3, 0x5410);
+  row[3] = __byte_perm(t2, t3, 0x7632);
 }
 
 // Cluster-wide barrier; a plain block barrier when the cluster is one CTA.
@@ -140,26 +166,32 @@ __device__ __forceinline__ void csync(cg::cluster_group& cluster, int C) {
   if (C > 1) cluster.sync();
   else __syncthreads();
 }
+// The two halves of a cluster barrier, for work that may overlap it.
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+
+constexpr int kTagWin = 32;  // tags handled per pass of the encoded stream
+constexpr uint32_t kFull = 0xffffffffu;
 
 struct QSmem {
-  // exchanged across the cluster (read remotely)
-  int fmax, fmin, need, pad;
+  // read by the other CTAs of the cluster
+  int xv[4];  // finest FPoT, coarsest FPoT, min(FPoT + one-plane room), min(FPoT + two-plane room)
   uint32_t mask[kMaxMaskWords];
   int cta_tot[kTagWin];  // this CTA's record count per tag of the current window
   // local
-  int warp_a[kQWarps], warp_b[kQWarps];
   int flags;
-  int base[kTagWin];       // records before this CTA's first record of the tag
+  int total;
+  int red[4][kQWarps];
   int warp_cnt[kQWarps][kTagWin];
-  // copies of the cluster's exchanged values, fetched one remote word per thread
-  int x_fmax[kMaxCluster], x_fmin[kMaxCluster], x_need[kMaxCluster];
+  int base[kTagWin];  // first record of this CTA per tag of the window
+  int x[kMaxCluster][4];
   int x_tot[kMaxCluster][kTagWin];
 };
 
 }  // namespace
 
 size_t quantize_smem_bytes(int64_t Kc) {
-  size_t b = 20 * (size_t)Kc;  // column-major codes + 4 per-column bytes
+  size_t b = 18 * (size_t)Kc;  // codes (16 per channel), FPoT and width
   b = (b + 15) & ~(size_t)15;
   return b + sizeof(QSmem);
 }
@@ -185,14 +217,12 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParam
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t units = K / 32;
   const int64_t k_lo = 32 * (rank * units / C), k_hi = 32 * ((rank + 1) * units / C);
-  const int64_t Kc = k_hi - k_lo;
+  const int Kc = (int)(k_hi - k_lo);
 
-  int8_t* s_code = reinterpret_cast<int8_t*>(smem);  // [Kc][16]: the 16 codes of local channel k
+  int8_t* s_code = reinterpret_cast<int8_t*>(smem);  // 16-byte slots: the 16 codes of a local channel
   int8_t* s_fpot = s_code + 16 * kc_max;              // [Kc]
-  int8_t* s_bits = s_fpot + kc_max;
-  int8_t* s_qmax = s_bits + kc_max;
-  int8_t* s_qmin = s_qmax + kc_max;
-  QSmem& S = *reinterpret_cast<QSmem*>(smem + ((20 * kc_max + 15) & ~(int64_t)15));
+  int8_t* s_bits = s_fpot + kc_max;                   // [Kc]
+  QSmem& S = *reinterpret_cast<QSmem*>(smem + ((18 * kc_max + 15) & ~(int64_t)15));
 
   if (tid < kMaxMaskWords) S.mask[tid] = 0;
   if (tid == 0) S.flags = 0;
@@ -204,13 +234,14 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParam
   const float beta = exp2_exact(lb);
   const bool refresh = !(p.flags & DSTAR_FLAG_NO_XPREV_REFRESH);
   const int64_t row0 = (int64_t)t * kTile;
-  const int npairs = (int)(Kc / 2);
-  int fmax = -1000, fmin = 1000;
+  const int npairs = Kc / 2;
+  int fmax = -1000, fmin = 1000, a1 = 1000, a2 = 1000;
   int flags = 0;
 
   // ---------------------------------------------------------------- phase 1
   for (int pr = tid; pr < npairs; pr += kQThreads) {
-    const int64_t lc = 2 * (int64_t)pr, c = k_lo + lc;
+    const int lc = 2 * pr;
+    const int64_t c = k_lo + lc;
     typename PR::Raw rt[kTile], rp[kTile];
 #pragma unroll
     for (int r = 0; r < kTile; ++r) {
@@ -231,7 +262,7 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParam
     const ColParams c0 = col_params(m0, lb, beta, t0, fb, flags);
     const ColParams c1 = col_params(m1, lb, beta, t0, fb, flags);
     uint32_t w0[4] = {0, 0, 0, 0}, w1[4] = {0, 0, 0, 0};
-    int qmx0 = -128, qmn0 = 127, qmx1 = -128, qmn1 = 127;
+    int qmx0 = 0, qmn0 = 0, qmx1 = 0, qmn1 = 0;
 #pragma unroll
     for (int r = 0; r < kTile; ++r) {  // stage 3 (dX recomputed: the same single subtraction)
       const float d0 = __fsub_rn(PR::lo(rt[r]), PR::lo(rp[r])), d1 = __fsub_rn(PR::hi(rt[r]), PR::hi(rp[r]));
@@ -248,108 +279,121 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParam
         *reinterpret_cast<uint16_t*>(p.debug_codes + (row0 + r) * K + c) =
             (uint16_t)(((w0[r >> 2] >> (8 * (r & 3))) & 0xFFu) | (((w1[r >> 2] >> (8 * (r & 3))) & 0xFFu) << 8));
     }
-    *reinterpret_cast<uint4*>(s_code + 16 * lc) = make_uint4(w0[0], w0[1], w0[2], w0[3]);
-    *reinterpret_cast<uint4*>(s_code + 16 * lc + 16) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+    *reinterpret_cast<uint4*>(s_code + 16 * code_slot(lc)) = make_uint4(w0[0], w0[1], w0[2], w0[3]);
+    *reinterpret_cast<uint4*>(s_code + 16 * code_slot(lc + 1)) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
     auto two = [](int a, int b) { return (uint16_t)(((uint32_t)a & 0xFFu) | (((uint32_t)b & 0xFFu) << 8)); };
     *reinterpret_cast<uint16_t*>(s_fpot + lc) = two(c0.fpot, c1.fpot);
     *reinterpret_cast<uint16_t*>(s_bits + lc) = two(c0.bits, c1.bits);
-    *reinterpret_cast<uint16_t*>(s_qmax + lc) = two(qmx0, qmx1);
-    *reinterpret_cast<uint16_t*>(s_qmin + lc) = two(qmn0, qmn1);
     *reinterpret_cast<uint16_t*>(p.fpot + (int64_t)t * K + c) = two(c0.fpot, c1.fpot);
     *reinterpret_cast<uint16_t*>(p.bits + (int64_t)t * K + c) = two(c0.bits, c1.bits);
     fmax = max(fmax, max(c0.fpot, c1.fpot));
     fmin = min(fmin, min(c0.fpot, c1.fpot));
+    a1 = min(a1, min(c0.fpot + shift_room(qmx0, qmn0, false), c1.fpot + shift_room(qmx1, qmn1, false)));
+    a2 = min(a2, min(c0.fpot + shift_room(qmx0, qmn0, true), c1.fpot + shift_room(qmx1, qmn1, true)));
   }
 
-  // CTA reductions, then the cluster's finest / coarsest FPoT
+  // CTA reductions, then one exchange across the cluster
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
-    fmax = max(fmax, __shfl_xor_sync(0xffffffffu, fmax, o));
-    fmin = min(fmin, __shfl_xor_sync(0xffffffffu, fmin, o));
-    flags |= __shfl_xor_sync(0xffffffffu, flags, o);
+    fmax = max(fmax, __shfl_xor_sync(kFull, fmax, o));
+    fmin = min(fmin, __shfl_xor_sync(kFull, fmin, o));
+    a1 = min(a1, __shfl_xor_sync(kFull, a1, o));
+    a2 = min(a2, __shfl_xor_sync(kFull, a2, o));
+    flags |= __shfl_xor_sync(kFull, flags, o);
   }
   if (lane == 0) {
-    S.warp_a[warp] = fmax;
-    S.warp_b[warp] = fmin;
+    S.red[0][warp] = fmax, S.red[1][warp] = fmin, S.red[2][warp] = a1, S.red[3][warp] = a2;
     if (flags) atomicOr(&S.flags, flags);
   }
   __syncthreads();
-  if (tid == 0) {
-    int a = -1000, b = 1000;
-    for (int w = 0; w < kQWarps; ++w) a = max(a, S.warp_a[w]), b = min(b, S.warp_b[w]);
-    S.fmax = a, S.fmin = b;
-    if (S.flags)
+  if (tid < 4) {
+    int v = S.red[tid][0];
+    for (int w = 1; w < kQWarps; ++w) v = tid == 0 ? max(v, S.red[tid][w]) : min(v, S.red[tid][w]);
+    S.xv[tid] = v;
+    if (tid == 0 && S.flags)
       set_status(p.status, (S.flags & 1 ? DSTAR_STATUS_NONFINITE : 0u) | (S.flags & 2 ? DSTAR_STATUS_RANGE : 0u));
   }
   csync(cluster, C);
-  if (tid < C) {  // one remote read per thread, all in flight together
-    const QSmem* R = C > 1 ? cluster.map_shared_rank(&S, tid) : &S;
-    S.x_fmax[tid] = R->fmax;
-    S.x_fmin[tid] = R->fmin;
+  if (tid < 4 * C) {  // one remote read per thread, all in flight together
+    const int q = tid >> 2, u = tid & 3;
+    S.x[q][u] = (C > 1 ? cluster.map_shared_rank(&S, q) : &S)->xv[u];
   }
   __syncthreads();
-  int g = -1000, gmin = 1000;
-  for (int q = 0; q < C; ++q) g = max(g, S.x_fmax[q]), gmin = min(gmin, S.x_fmin[q]);
-
-  // planes the tile needs: every v = q 2^(g - FPoT) must fit the split
-  int need = 1;
-  for (int64_t k = tid; k < Kc; k += kQThreads) {
-    const int Sh = g - s_fpot[k];
-    const int64_t vmax = (int64_t)s_qmax[k] * ((int64_t)1 << Sh), vmin = (int64_t)s_qmin[k] * ((int64_t)1 << Sh);
-    if (vmin < kPlane1Lo || vmax > kPlane1Hi) need = max(need, 2);
-    if (vmin < kPlane2Lo || vmax > kPlane2Hi) need = 3;
+  int g = -1000, gmin = 1000, A1 = 1000, A2 = 1000;
+  for (int q = 0; q < C; ++q) {
+    g = max(g, S.x[q][0]), gmin = min(gmin, S.x[q][1]);
+    A1 = min(A1, S.x[q][2]), A2 = min(A2, S.x[q][3]);
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) need = max(need, __shfl_xor_sync(0xffffffffu, need, o));
-  if (lane == 0) S.warp_a[warp] = need;
-  __syncthreads();
-  if (tid == 0) {
-    int n = 1;
-    for (int w = 0; w < kQWarps; ++w) n = max(n, S.warp_a[w]);
-    S.need = n;
-  }
-  csync(cluster, C);
-  if (tid < C) S.x_need[tid] = (C > 1 ? cluster.map_shared_rank(&S, tid) : &S)->need;
-  __syncthreads();
-  int planes = 1;
-  for (int q = 0; q < C; ++q) planes = max(planes, S.x_need[q]);
+  // every v = q 2^(g - FPoT) must fit the split: g - FPoT <= room for each channel
+  const int planes = g <= A1 ? 1 : g <= A2 ? 2 : 3;
 
   // ------------------------------------------------- phase 2a: operand planes
-  // Same channel-pair mapping: 2-byte stores, a warp writes 64 contiguous bytes per row.
+  // Four channels per thread: their 16-code columns, shifted, are transposed
+  // into 4-byte row words; a warp writes 128 contiguous bytes per row.
   if (planes == 1) {
-    for (int pr = tid; pr < npairs; pr += kQThreads) {
-      const int64_t lc = 2 * (int64_t)pr, c = k_lo + lc;
-      const uint4 q0 = *reinterpret_cast<const uint4*>(s_code + 16 * lc);
-      const uint4 q1 = *reinterpret_cast<const uint4*>(s_code + 16 * lc + 16);
-      // a nonzero code of a one-plane tile has a shift <= 7; zero codes stay zero
-      const int S0 = min(g - s_fpot[lc], 31), S1 = min(g - s_fpot[lc + 1], 31);
+    for (int qd = tid; qd < Kc / 4; qd += kQThreads) {
+      const int lc = 4 * qd;
+      const uint32_t f4 = *reinterpret_cast<const uint32_t*>(s_fpot + lc);
+      uint32_t col[4][4];
 #pragma unroll
-      for (int r = 0; r < kTile; ++r) {
-        const uint32_t a = (((uint32_t)code_at(q0, r) << S0) & 0xFFu) | ((((uint32_t)code_at(q1, r) << S1) & 0xFFu) << 8);
-        *reinterpret_cast<uint16_t*>(p.plane0 + (row0 + r) * K + c) = (uint16_t)a;
+      for (int i = 0; i < 4; ++i) {
+        const uint4 v = *reinterpret_cast<const uint4*>(s_code + 16 * code_slot(lc + i));
+        // nonzero codes of a one-plane tile have a shift <= 7; zero codes stay zero
+        const int sh = min(g - (int)(int8_t)(f4 >> (8 * i)), 7);
+        const uint32_t keep = ((0xFFu << sh) & 0xFFu) * 0x01010101u;  // drops bits carried into the next byte
+        col[i][0] = (v.x << sh) & keep, col[i][1] = (v.y << sh) & keep;
+        col[i][2] = (v.z << sh) & keep, col[i][3] = (v.w << sh) & keep;
+      }
+      int8_t* dst = p.plane0 + row0 * K + k_lo + lc;
+#pragma unroll
+      for (int R = 0; R < 4; ++R) {
+        uint32_t row[4];
+        transpose4(col[0][R], col[1][R], col[2][R], col[3][R], row);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) *reinterpret_cast<uint32_t*>(dst + (4 * R + i) * K) = row[i];
       }
     }
   } else if (planes == 2) {
-    for (int pr = tid; pr < npairs; pr += kQThreads) {
-      const int64_t lc = 2 * (int64_t)pr, c = k_lo + lc;
-      const uint4 q0 = *reinterpret_cast<const uint4*>(s_code + 16 * lc);
-      const uint4 q1 = *reinterpret_cast<const uint4*>(s_code + 16 * lc + 16);
-      // a nonzero code of a two-plane tile has a shift <= 15, so v fits 32 bits
-      const int S0 = min(g - s_fpot[lc], 24), S1 = min(g - s_fpot[lc + 1], 24);
+    for (int qd = tid; qd < Kc / 4; qd += kQThreads) {
+      const int lc = 4 * qd;
+      uint32_t c0w[4][4], c1w[4][4];
       uint32_t nz = 0;
 #pragma unroll
-      for (int r = 0; r < kTile; ++r) {
-        const int v0 = code_at(q0, r) * (1 << S0), v1 = code_at(q1, r) * (1 << S1);
-        const int a00 = (int)(int8_t)(v0 & 0xFF), a01 = (int)(int8_t)(v1 & 0xFF);
-        const int a10 = (v0 - a00) >> 8, a11 = (v1 - a01) >> 8;
-        nz |= (uint32_t)(a10 | a11);
-        *reinterpret_cast<uint16_t*>(p.plane0 + (row0 + r) * K + c) =
-            (uint16_t)(((uint32_t)a00 & 0xFFu) | (((uint32_t)a01 & 0xFFu) << 8));
-        *reinterpret_cast<uint16_t*>(p.plane1 + (row0 + r) * K + c) =
-            (uint16_t)(((uint32_t)a10 & 0xFFu) | (((uint32_t)a11 & 0xFFu) << 8));
+      for (int i = 0; i < 4; ++i) {
+        const uint4 v = *reinterpret_cast<const uint4*>(s_code + 16 * code_slot(lc + i));
+        const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+        // nonzero codes of a two-plane tile have a shift <= 15, so q 2^shift fits 32 bits
+        const int sh = min(g - (int)s_fpot[lc + i], 24);
+#pragma unroll
+        for (int R = 0; R < 4; ++R) {
+          uint32_t lo = 0, hi = 0;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int val = (int)(int8_t)(vw[R] >> (8 * e)) * (1 << sh);
+            const int p0 = (int)(int8_t)(val & 0xFF);
+            const int p1 = (val - p0) >> 8;
+            nz |= (uint32_t)p1;
+            lo |= ((uint32_t)p0 & 0xFFu) << (8 * e);
+            hi |= ((uint32_t)p1 & 0xFFu) << (8 * e);
+          }
+          c0w[i][R] = lo, c1w[i][R] = hi;
+        }
+      }
+      int8_t* d0 = p.plane0 + row0 * K + k_lo + lc;
+      int8_t* d1 = p.plane1 + row0 * K + k_lo + lc;
+#pragma unroll
+      for (int R = 0; R < 4; ++R) {
+        uint32_t r0[4], r1[4];
+        transpose4(c0w[0][R], c0w[1][R], c0w[2][R], c0w[3][R], r0);
+        transpose4(c1w[0][R], c1w[1][R], c1w[2][R], c1w[3][R], r1);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          *reinterpret_cast<uint32_t*>(d0 + (4 * R + i) * K) = r0[i];
+          *reinterpret_cast<uint32_t*>(d1 + (4 * R + i) * K) = r1[i];
+        }
       }
       if (nz) {
-        const int chunk = (int)(c / kChunkK);
+        const int chunk = (int)((k_lo + lc) / kChunkK);
         atomicOr(&S.mask[chunk >> 5], 1u << (chunk & 31));
       }
     }
@@ -357,126 +401,115 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParam
 
   // ------------------------------------- phase 2b: FPoT-grouped encoded stream
   // Slice j of channel k carries tag FPoT(k) - 2j (j < bits/2).  Tags lie in
-  // [gmin - 6, g] and are handled in windows of 8 consecutive tags.  Each warp
-  // owns a contiguous range of this CTA's channels and walks it 32 channels
-  // at a time (lane = channel); one ballot per tag of the window ranks the
-  // lanes carrying that tag.  The record of (tag, k) lands after: the tile's
-  // records of lower tags, then those of the same tag in lower-ranked CTAs,
-  // lower warps of this CTA, earlier chunks of this warp and lower lanes.
+  // [gmin - 6, g] and are handled in windows of 32 consecutive tags (one
+  // window unless the tile's FPoT spread exceeds 25).  Each warp owns a
+  // contiguous run of 32-channel chunks (lane = channel) and visits, per
+  // chunk, only the tags present in it; one ballot ranks the lanes carrying a
+  // tag.  Lane u of a warp keeps the running offset of window tag u.  The
+  // record of (tag, k) lands after the tile's records of lower tags, then those
+  // of the same tag in lower-ranked CTAs, lower warps of this CTA, earlier
+  // chunks of this warp and lower lanes.
   const int tlo = gmin - 6;
-  const int ntags = g - tlo + 1;
-  const int64_t kw = ((Kc / 32 + kQWarps - 1) / kQWarps) * 32;  // channels per warp, a multiple of 32
-  const int64_t w_lo = min(Kc, (int64_t)warp * kw), w_hi = min(Kc, w_lo + kw);
+  const int nchunks = Kc / 32;
+  const int ch_lo = warp * nchunks / kQWarps, ch_hi = (warp + 1) * nchunks / kQWarps;
   const uint32_t lt = (1u << lane) - 1u;
   uint2* rec = p.records + (int64_t)t * p.record_cap;
-  int records_before_window = 0;  // all CTAs, all lower tags (kept by threads tid < kTagWin)
-  for (int wbase = 0; wbase < ntags; wbase += kTagWin) {
-    const int tw = tlo + wbase;  // tag of window slot 0
-    // pass A: this warp's count of each tag of the window
-    int cnt[kTagWin];
-#pragma unroll
-    for (int ti = 0; ti < kTagWin; ++ti) cnt[ti] = 0;
-    for (int64_t kb = w_lo; kb < w_hi; kb += 4 * 32) {  // four independent chunks per iteration
-      uint32_t m[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int64_t k = kb + 32 * u + lane;
-        m[u] = k < w_hi ? tag_mask(s_fpot[k], s_bits[k], tw) : 0u;
+  int total = 0;  // records of lower windows, all CTAs (kept by warp 0)
+  bool first = true;
+  for (int tw = tlo; tw <= g; tw += kTagWin) {
+    if (!first) {
+      __syncthreads();             // every warp is done with the previous window's counts and bases
+      if (C > 1) cluster_wait();   // and every CTA with its remote reads of them
+    }
+    first = false;
+    // pass A: this warp's count of every tag of the window (lane u: tag tw + u)
+    int cnt = 0;
+    for (int ch = ch_lo; ch < ch_hi; ++ch) {
+      const int c = 32 * ch + lane;
+      const uint32_t m = tag_mask32(s_fpot[c], s_bits[c], tw);
+      uint32_t any = __reduce_or_sync(kFull, m);
+      while (any) {
+        const int ti = __ffs(any) - 1;
+        any &= any - 1u;
+        const int n = __popc(__ballot_sync(kFull, (m >> ti) & 1u));
+        if (lane == ti) cnt += n;
       }
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-#pragma unroll
-        for (int ti = 0; ti < kTagWin; ++ti) cnt[ti] += __popc(__ballot_sync(0xffffffffu, (m[u] >> ti) & 1u));
     }
-    if (lane == 0) {
-#pragma unroll
-      for (int ti = 0; ti < kTagWin; ++ti) S.warp_cnt[warp][ti] = cnt[ti];
-    }
+    S.warp_cnt[warp][lane] = cnt;
     __syncthreads();
     if (tid < kTagWin) {
-      int tot = 0;
-      for (int w = 0; w < kQWarps; ++w) tot += S.warp_cnt[w][tid];
-      S.cta_tot[tid] = tot;
+      int s = 0;
+#pragma unroll
+      for (int w = 0; w < kQWarps; ++w) s += S.warp_cnt[w][tid];
+      S.cta_tot[tid] = s;
     }
     csync(cluster, C);
-    // window totals of every CTA -> where this CTA's records of each tag start
-    if (tid < C * kTagWin) {
+    if (tid < kTagWin * C) {  // every CTA's window totals, one remote word per thread
       const int q = tid / kTagWin, u = tid % kTagWin;
       S.x_tot[q][u] = (C > 1 ? cluster.map_shared_rank(&S, q) : &S)->cta_tot[u];
     }
-    __syncthreads();
-    if (tid < kTagWin) {
-      int below = 0, lower_cta = 0, all = 0;
-      for (int q = 0; q < C; ++q) {
-        for (int u = 0; u < kTagWin; ++u) {
-          const int v = S.x_tot[q][u];
-          if (u < tid) below += v;
-          if (u == tid && q < rank) lower_cta += v;
-          all += v;
-        }
-      }
-      S.base[tid] = records_before_window + below + lower_cta;
-      records_before_window += all;
-    }
-    __syncthreads();
-    int off[kTagWin];
-#pragma unroll
-    for (int ti = 0; ti < kTagWin; ++ti) {
-      int o = S.base[ti];
-      for (int w = 0; w < warp; ++w) o += S.warp_cnt[w][ti];
-      off[ti] = o;
-    }
-    // pass B: rank and write, two independent chunks per iteration
-    for (int64_t kb = w_lo; kb < w_hi; kb += 2 * 32) {
-      int f[2], b[2];
-      uint32_t m[2], bal[2][kTagWin], words[2][4];
-      int64_t k[2];
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        k[u] = kb + 32 * u + lane;
-        const bool kv = k[u] < w_hi;
-        f[u] = kv ? s_fpot[k[u]] : 0, b[u] = kv ? s_bits[k[u]] : 0;
-        m[u] = kv ? tag_mask(f[u], b[u], tw) : 0u;
-        if (m[u]) slice_words(*reinterpret_cast<const uint4*>(s_code + 16 * k[u]), words[u]);
-#pragma unroll
-        for (int ti = 0; ti < kTagWin; ++ti) bal[u][ti] = __ballot_sync(0xffffffffu, (m[u] >> ti) & 1u);
-      }
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        if (m[u]) {
-#pragma unroll
-          for (int ti = 0; ti < kTagWin; ++ti) {
-            if ((m[u] >> ti) & 1u) {
-              // the field j < b/2 of the b-bit pattern equals that of the 8-bit pattern
-              const int j = (f[u] - tw - ti) >> 1;
-              const uint32_t w = j == 0 ? words[u][0] : j == 1 ? words[u][1] : j == 2 ? words[u][2] : words[u][3];
-              rec[off[ti] + __popc(bal[u][ti] & lt)] = make_uint2(
-                  w, (uint32_t)(k_lo + k[u]) | ((uint32_t)(uint8_t)(int8_t)(tw + ti) << 16) | ((uint32_t)j << 24));
-            }
-          }
-        }
-#pragma unroll
-        for (int ti = 0; ti < kTagWin; ++ti) off[ti] += __popc(bal[u][ti]);
-      }
-    }
-    csync(cluster, C);  // cta_tot and warp_cnt are rewritten by the next window
-  }
-
-  // the tile's meta: rank 0 gathers the cluster's mask words
-  __syncthreads();
-  if (rank == 0) {
-    if (tid < p.mask_words) {
+    if (tw == tlo && rank == 0 && tid >= 32 * (kQWarps - 1) && tid - 32 * (kQWarps - 1) < p.mask_words) {
+      // the tile's plane-1 chunk mask (every CTA finished its planes before the barrier)
+      const int wd = tid - 32 * (kQWarps - 1);
       uint32_t m = 0;
-      for (int q = 0; q < C; ++q) m |= (C > 1 ? cluster.map_shared_rank(&S, q) : &S)->mask[tid];
-      p.mask1[(int64_t)t * p.mask_words + tid] = planes == 2 ? m : 0u;
+      for (int q = 0; q < C; ++q) m |= (C > 1 ? cluster.map_shared_rank(&S, q) : &S)->mask[wd];
+      p.mask1[(int64_t)t * p.mask_words + wd] = planes == 2 ? m : 0u;
     }
-    if (tid == 0) {
-      p.g_ref[t] = g;
-      p.planes[t] = planes;
-      p.count[t] = records_before_window;
+    __syncthreads();
+    if (C > 1) cluster_arrive();  // remote reads of this window done; waited for before reuse or exit
+    if (warp == 0) {
+      int all = 0, lower = 0;
+      for (int q = 0; q < C; ++q) {
+        const int v = S.x_tot[q][lane];
+        all += v;
+        if (q < rank) lower += v;
+      }
+      int incl = all;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += n;
+      }
+      S.base[lane] = total + incl - all + lower;
+      total += __shfl_sync(kFull, incl, 31);
+    }
+    __syncthreads();
+    int off = S.base[lane];
+    for (int w = 0; w < warp; ++w) off += S.warp_cnt[w][lane];
+    // pass B: rank and write
+    for (int ch = ch_lo; ch < ch_hi; ++ch) {
+      const int c = 32 * ch + lane;
+      const int f = s_fpot[c], b = s_bits[c];
+      const uint32_t m = tag_mask32(f, b, tw);
+      uint32_t any = __reduce_or_sync(kFull, m);
+      if (!any) continue;
+      uint32_t words[4];
+      slice_words(*reinterpret_cast<const uint4*>(s_code + 16 * code_slot(c)), words);
+      const uint32_t meta_k = (uint32_t)(k_lo + c);
+      while (any) {
+        const int ti = __ffs(any) - 1;
+        any &= any - 1u;
+        const uint32_t bal = __ballot_sync(kFull, (m >> ti) & 1u);
+        const int base = __shfl_sync(kFull, off, ti);
+        if ((m >> ti) & 1u) {
+          // the field j < b/2 of the b-bit pattern equals that of the 8-bit pattern
+          const int j = (f - tw - ti) >> 1;
+          const uint32_t w = j == 0 ? words[0] : j == 1 ? words[1] : j == 2 ? words[2] : words[3];
+          rec[base + __popc(bal & lt)] =
+              make_uint2(w, meta_k | ((uint32_t)(uint8_t)(int8_t)(tw + ti) << 16) | ((uint32_t)j << 24));
+        }
+        if (lane == ti) off += __popc(bal);
+      }
     }
   }
-  csync(cluster, C);  // no CTA leaves while another may still read its shared memory
+  if (rank == 0 && tid == 0) {
+    p.g_ref[t] = g;
+    p.planes[t] = planes;
+  }
+  if (warp == 0 && lane == 0) S.total = total;
+  __syncthreads();
+  if (rank == 0 && tid == 0) p.count[t] = S.total;
+  if (C > 1) cluster_wait();  // no CTA leaves while another may still read its shared memory
 }
 
 int launch_quantize(const QuantParams& p, int in_bf16, int num_sms, void* stream) {
