@@ -122,6 +122,32 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Pull [p, p + bytes) into L2 (a hint; p 16-byte aligned, bytes a multiple of 16).
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
+               : "memory");
+}
+
+// This CTA's share (CTA `part` of `parts`) of an L2 prefetch of a row-major
+// region, issued by one thread in pieces of at most 32 KB.
+__device__ __forceinline__ void prefetch_region_share(const L2Region& r, int part, int parts) {
+  if (!r.base || r.rows <= 0 || r.row_bytes <= 0) return;
+  constexpr int64_t kPiece = 32768;
+  if (r.ld_bytes == r.row_bytes) {  // one contiguous range
+    const int64_t total = r.rows * r.row_bytes;
+    const int64_t per = ((total + parts - 1) / parts + 15) & ~(int64_t)15;
+    const int64_t lo = (int64_t)part * per, hi = lo + per < total ? lo + per : total;
+    for (int64_t o = lo; o < hi; o += kPiece)
+      prefetch_l2_bulk(r.base + o, (uint32_t)(hi - o < kPiece ? hi - o : kPiece));
+  } else {  // row by row
+    const int64_t lo = r.rows * part / parts, hi = r.rows * (part + 1) / parts;
+    for (int64_t row = lo; row < hi; ++row)
+      for (int64_t o = 0; o < r.row_bytes; o += kPiece)
+        prefetch_l2_bulk(r.base + row * r.ld_bytes + o,
+                         (uint32_t)(r.row_bytes - o < kPiece ? r.row_bytes - o : kPiece));
+  }
+}
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

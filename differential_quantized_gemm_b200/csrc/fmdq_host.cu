@@ -188,7 +188,7 @@ T* ws_ptr(const dstar_tile_cfg* c, size_t off) {
 }
 
 int do_quantize(const dstar_mat* x_t, dstar_mat* x_prev, int lb, const dstar_tile_cfg* c, int64_t M, int64_t K,
-                const DevInfo& dev, void* stream) {
+                const DevInfo& dev, void* stream, const dstar_mat* pf_w = nullptr, const dstar_mat* pf_y = nullptr) {
   const WsLayout L = ws_layout(M, K);
   QuantParams q{};
   q.x_t = x_t->data;
@@ -210,6 +210,14 @@ int do_quantize(const dstar_mat* x_t, dstar_mat* x_prev, int lb, const dstar_til
   q.record_cap = L.record_cap;
   q.mask_words = L.mask_words;
   q.debug_codes = c->debug_codes;
+  const dstar_mat* pf[2] = {pf_w, pf_y};
+  for (int i = 0; i < 2; ++i) {
+    if (pf[i] && pf[i]->data && pf[i]->rows > 0 && pf[i]->cols > 0) {
+      const int64_t es = (int64_t)elem_size(pf[i]->dtype);
+      q.prefetch[i] = L2Region{static_cast<const uint8_t*>(pf[i]->data), pf[i]->rows, pf[i]->cols * es,
+                               pf[i]->ld * es};
+    }
+  }
   const int e = launch_quantize(q, x_t->dtype == DSTAR_BF16, dev.sms, stream);
   if (e) return cuda_fail(e, "quantize launch");
   return DSTAR_OK;
@@ -479,7 +487,9 @@ int dstar_fmdq_linear(const dstar_mat* x_t, dstar_mat* x_prev, dstar_mat* y_prev
   if (M == 0) return ok();
   DevInfo dev;
   if ((r = device_info(&dev)) != DSTAR_OK) return r;
-  if ((r = do_quantize(x_t, x_prev, lb, tile_cfg, M, K, dev, stream)) != DSTAR_OK) return r;
+  if ((r = do_quantize(x_t, x_prev, lb, tile_cfg, M, K, dev, stream, N > 0 ? w_q : nullptr,
+                       N > 0 ? y_prev : nullptr)) != DSTAR_OK)
+    return r;
   if ((r = do_gemm(w_q, w_scale, y_prev, lb, tile_cfg, y_out, M, K, N, dev, stream)) != DSTAR_OK) return r;
   return ok();
 }

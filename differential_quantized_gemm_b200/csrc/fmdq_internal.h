@@ -21,6 +21,13 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded waits give up after
 constexpr int64_t kPlane1Lo = -128, kPlane1Hi = 127;
 constexpr int64_t kPlane2Lo = -128 * 257, kPlane2Hi = 127 * 257;
 
+// A row-major region to pull into L2 ahead of its reader: rows of row_bytes,
+// ld_bytes apart (both multiples of 16, base 16-byte aligned).
+struct L2Region {
+  const uint8_t* base;
+  int64_t rows, row_bytes, ld_bytes;
+};
+
 struct QuantParams {
   const void* x_t;
   void* x_prev;
@@ -41,6 +48,9 @@ struct QuantParams {
   int64_t record_cap;
   int64_t mask_words;
   int8_t* debug_codes;
+  // operands of the GEMM that follows in the same call (weights, cached
+  // output): prefetched into L2 once the quantizer no longer streams HBM
+  L2Region prefetch[2];
 };
 
 struct GemmParams {

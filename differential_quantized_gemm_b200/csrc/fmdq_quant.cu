@@ -171,6 +171,8 @@ __device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
 
 constexpr int kTagWin = 32;  // tags handled per pass of the encoded stream
+constexpr int kUA = 4;       // chunks per round of ballots when counting
+constexpr int kUB = 4;       // chunks per round of ballots when writing
 constexpr uint32_t kFull = 0xffffffffu;
 
 struct QSmem {
@@ -326,6 +328,11 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParam
   }
   // every v = q 2^(g - FPoT) must fit the split: g - FPoT <= room for each channel
   const int planes = g <= A1 ? 1 : g <= A2 ? 2 : 3;
+  // HBM is idle from here on: pull the next GEMM's operands into L2
+  if (tid == 0) {
+    prefetch_region_share(p.prefetch[0], (int)blockIdx.x, (int)gridDim.x);
+    prefetch_region_share(p.prefetch[1], (int)blockIdx.x, (int)gridDim.x);
+  }
 
   // ------------------------------------------------- phase 2a: operand planes
   // Four channels per thread: their 16-code columns, shifted, are transposed
@@ -422,16 +429,24 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParam
       if (C > 1) cluster_wait();   // and every CTA with its remote reads of them
     }
     first = false;
-    // pass A: this warp's count of every tag of the window (lane u: tag tw + u)
+    // pass A: this warp's count of every tag of the window (lane u: tag tw + u);
+    // kUA chunks share each round of ballots
     int cnt = 0;
-    for (int ch = ch_lo; ch < ch_hi; ++ch) {
-      const int c = 32 * ch + lane;
-      const uint32_t m = tag_mask32(s_fpot[c], s_bits[c], tw);
-      uint32_t any = __reduce_or_sync(kFull, m);
+    for (int ch0 = ch_lo; ch0 < ch_hi; ch0 += kUA) {
+      uint32_t m[kUA], un = 0;
+#pragma unroll
+      for (int u = 0; u < kUA; ++u) {
+        const int c = 32 * (ch0 + u) + lane;
+        m[u] = ch0 + u < ch_hi ? tag_mask32(s_fpot[c], s_bits[c], tw) : 0u;
+        un |= m[u];
+      }
+      uint32_t any = __reduce_or_sync(kFull, un);
       while (any) {
         const int ti = __ffs(any) - 1;
         any &= any - 1u;
-        const int n = __popc(__ballot_sync(kFull, (m >> ti) & 1u));
+        int n = 0;
+#pragma unroll
+        for (int u = 0; u < kUA; ++u) n += __popc(__ballot_sync(kFull, (m[u] >> ti) & 1u));
         if (lane == ti) cnt += n;
       }
     }
@@ -476,29 +491,42 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParam
     __syncthreads();
     int off = S.base[lane];
     for (int w = 0; w < warp; ++w) off += S.warp_cnt[w][lane];
-    // pass B: rank and write
-    for (int ch = ch_lo; ch < ch_hi; ++ch) {
-      const int c = 32 * ch + lane;
-      const int f = s_fpot[c], b = s_bits[c];
-      const uint32_t m = tag_mask32(f, b, tw);
-      uint32_t any = __reduce_or_sync(kFull, m);
-      if (!any) continue;
-      uint32_t words[4];
-      slice_words(*reinterpret_cast<const uint4*>(s_code + 16 * code_slot(c)), words);
-      const uint32_t meta_k = (uint32_t)(k_lo + c);
+    // pass B: rank and write; kUB chunks share each round, chunk u's records of
+    // a tag before chunk u + 1's
+    for (int ch0 = ch_lo; ch0 < ch_hi; ch0 += kUB) {
+      uint32_t m[kUB], words[kUB][4], un = 0;
+      int f[kUB];
+#pragma unroll
+      for (int u = 0; u < kUB; ++u) {
+        const int c = 32 * (ch0 + u) + lane;
+        const bool valid = ch0 + u < ch_hi;
+        f[u] = valid ? s_fpot[c] : 0;
+        m[u] = valid ? tag_mask32(f[u], s_bits[c], tw) : 0u;
+        un |= m[u];
+        if (valid) slice_words(*reinterpret_cast<const uint4*>(s_code + 16 * code_slot(c)), words[u]);
+        else words[u][0] = words[u][1] = words[u][2] = words[u][3] = 0u;
+      }
+      uint32_t any = __reduce_or_sync(kFull, un);
       while (any) {
         const int ti = __ffs(any) - 1;
         any &= any - 1u;
-        const uint32_t bal = __ballot_sync(kFull, (m >> ti) & 1u);
-        const int base = __shfl_sync(kFull, off, ti);
-        if ((m >> ti) & 1u) {
-          // the field j < b/2 of the b-bit pattern equals that of the 8-bit pattern
-          const int j = (f - tw - ti) >> 1;
-          const uint32_t w = j == 0 ? words[0] : j == 1 ? words[1] : j == 2 ? words[2] : words[3];
-          rec[base + __popc(bal & lt)] =
-              make_uint2(w, meta_k | ((uint32_t)(uint8_t)(int8_t)(tw + ti) << 16) | ((uint32_t)j << 24));
+        uint32_t bal[kUB];
+#pragma unroll
+        for (int u = 0; u < kUB; ++u) bal[u] = __ballot_sync(kFull, (m[u] >> ti) & 1u);
+        int base = __shfl_sync(kFull, off, ti);
+        const uint32_t meta_t = (uint32_t)(uint8_t)(int8_t)(tw + ti) << 16;
+#pragma unroll
+        for (int u = 0; u < kUB; ++u) {
+          if ((m[u] >> ti) & 1u) {
+            // the field j < b/2 of the b-bit pattern equals that of the 8-bit pattern
+            const int j = (f[u] - tw - ti) >> 1;
+            const uint32_t w = j == 0 ? words[u][0] : j == 1 ? words[u][1] : j == 2 ? words[u][2] : words[u][3];
+            rec[base + __popc(bal[u] & lt)] =
+                make_uint2(w, (uint32_t)(k_lo + 32 * (ch0 + u) + lane) | meta_t | ((uint32_t)j << 24));
+          }
+          base += __popc(bal[u]);
         }
-        if (lane == ti) off += __popc(bal);
+        if (lane == ti) off = base;
       }
     }
   }
