@@ -55,7 +55,7 @@ struct GemmCfg {
   static constexpr int kBoxBytes = 32 * 32 * kOutBytes;              // one 32 x 32 tile of Y
   static constexpr int kYWarpBytes = kHalfGroups * kBoxBytes;        // one epilogue warp's tiles
   // small region first, then the 1024-aligned buffers
-  static constexpr int kNumBars = 2 * kStages + 2 * kSlots + kEpiWarps + 1;
+  static constexpr int kNumBars = 2 * kStages + 2 * kSlots + kEpiWarps + 2;
   static constexpr int kOffBar = 0;
   static constexpr int kOffMisc = (kOffBar + kNumBars * 8 + 15) & ~15;  // tmem base, abort flag
   static constexpr int kOffWs = kOffMisc + 16;                          // [BN] fp32 weight scales
@@ -68,7 +68,7 @@ struct GemmCfg {
 };
 
 struct BlockInfo {
-  int nplanes;  // 0: no tile of the row block uses the tensor cores; 1 or 2 planes
+  int nplanes;  // 1 or 2 operand planes (plane 0 is computed even when every tile takes the slice stream)
   int any_slice;  // some tile of the row block goes through the slice stream
   uint32_t mask[2];
 };
@@ -91,7 +91,7 @@ __device__ __forceinline__ BlockInfo block_info_global(const GemmParams& p, int 
     }
     for (int w = 0; w < (int)p.mask_words && w < 2; ++w) bi.mask[w] |= p.mask1[(int64_t)t * p.mask_words + w];
   }
-  bi.nplanes = !any ? 0 : (np == 2 && (bi.mask[0] | bi.mask[1])) ? 2 : 1;
+  bi.nplanes = (any && np == 2 && (bi.mask[0] | bi.mask[1])) ? 2 : 1;
   return bi;
 }
 
@@ -244,6 +244,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
   uint64_t* tm_empty = tm_full + C::kSlots;    // [kSlots] epilogue -> MMA
   uint64_t* ybar = tm_empty + C::kSlots;       // [kEpiWarps] y_prev tiles landed
   uint64_t* drain = ybar + kEpiWarps;          // MMA completion at exit
+  uint64_t* info_bar = drain + 1;              // block info in shared memory
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
   float* s_ws = reinterpret_cast<float*>(smem + C::kOffWs);
@@ -261,6 +262,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
     for (int i = 0; i < C::kSlots; ++i) mbar_init(&tm_full[i], 1), mbar_init(&tm_empty[i], kEpiWarps);
     for (int i = 0; i < kEpiWarps; ++i) mbar_init(&ybar[i], 1);
     mbar_init(drain, 1);
+    mbar_init(info_bar, 1);
     *s_abort = 0;
     fence_barrier_init();
     prefetch_tmap(&tm_a0);
@@ -269,24 +271,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
     prefetch_tmap(&tm_yp);
     prefetch_tmap(&tm_yo);
   }
-  pdl_launch_dependents();
-  // block info of this CTA's first kMaxTileSlots tiles, loaded in parallel
+  // set-up that does not touch memory written by the previous kernel
   for (int i = threadIdx.x; i < kMaxTileSlots; i += kGThreads) s_info[i] = make_int4(0, 0, 0, 0);
-  pdl_wait();  // the quantizer's outputs (and y_prev, W) are read only after the previous kernel completed
-  __syncthreads();
-  for (int i = threadIdx.x; i < min(my_tiles, kMaxTileSlots) * 8; i += kGThreads) {
-    const int slot = i >> 3, sub = i & 7;
-    const int rb = ((int)blockIdx.x + slot * (int)gridDim.x) / p.tiles_n;
-    const int t = rb * 8 + sub;
-    if (t < T) {
-      const int pl = p.planes[t];
-      int* e = reinterpret_cast<int*>(&s_info[slot]);
-      if (pl <= 2) atomicMax(&e[0], pl);
-      else atomicOr(&e[1], 1);
-      if (p.mask_words > 0) atomicOr(reinterpret_cast<unsigned*>(&e[2]), p.mask1[(int64_t)t * p.mask_words]);
-      if (p.mask_words > 1) atomicOr(reinterpret_cast<unsigned*>(&e[3]), p.mask1[(int64_t)t * p.mask_words + 1]);
-    }
-  }
   if (warp == 1) {
     tmem_alloc(s_tmem, 512);
     tmem_relinquish();
@@ -295,6 +281,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
+  pdl_launch_dependents();
 
   auto info = [&](int slot, int rb) -> BlockInfo {
     if (slot < kMaxTileSlots) {
@@ -302,7 +289,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
       BlockInfo bi;
       bi.mask[0] = (uint32_t)e.z, bi.mask[1] = (uint32_t)e.w;
       bi.any_slice = e.y;
-      bi.nplanes = e.x == 0 ? 0 : (e.x == 2 && (e.z | e.w)) ? 2 : 1;
+      bi.nplanes = (e.x == 2 && (e.z | e.w)) ? 2 : 1;
       return bi;
     }
     return block_info_global(p, rb);
@@ -313,20 +300,44 @@ __global__ void __launch_bounds__(kGThreads, 1)
     if (elect_one()) {
       uint32_t it = 0;
       bool ok = true;
+      // The weights do not depend on the previous kernel: the W tiles of the
+      // first stages are requested before waiting for it.
+      uint32_t pre = 0;
+      if (my_tiles > 0) {
+        const int nb0 = (int)blockIdx.x % p.tiles_n;
+        pre = (uint32_t)min(C::kStages, p.num_chunks);
+        for (uint32_t c = 0; c < pre; ++c) {
+          mbar_arrive_expect_tx(&full[c], C::kStageBytes);
+          tma_load_2d(stages + c * C::kStageBytes + kA0Bytes, &tm_w, &full[c], (int)c * kChunkK, nb0 * BN);
+        }
+      }
+      pdl_wait();  // the operand planes are the previous kernel's output
+      bool have_info = false;
       for (int slot = 0; slot < my_tiles && ok; ++slot) {
         const int tile = (int)blockIdx.x + slot * (int)gridDim.x;
         const int rb = tile / p.tiles_n, nb = tile % p.tiles_n;
-        const BlockInfo bi = info(slot, rb);
-        for (int pass = 0; pass < bi.nplanes && ok; ++pass) {
+        for (int pass = 0; pass < 2 && ok; ++pass) {
+          BlockInfo bi{};
+          if (pass == 1) {  // plane 1 only where the block needs it
+            if (!have_info && !(ok = wait_parity(info_bar, 0, s_abort, p.status, kWaitLimitNs))) break;
+            have_info = true;
+            bi = info(slot, rb);
+            if (bi.nplanes < 2) break;
+          }
           const CUtensorMap* tm_a = pass == 0 ? &tm_a0 : &tm_a1;
           for (int c = 0; c < p.num_chunks; ++c) {
             if (pass == 1 && !chunk_has_plane1(bi, c)) continue;
             const int s = it % C::kStages;
+            uint8_t* a = stages + s * C::kStageBytes;
+            if (it < pre) {  // the stage's W tile is already on its way
+              tma_load_2d(a, tm_a, &full[s], c * kChunkK, rb * kBlockM);
+              ++it;
+              continue;
+            }
             if (!wait_parity(&empty[s], ((it / C::kStages) & 1) ^ 1, s_abort, p.status, kWaitLimitNs)) {
               ok = false;
               break;
             }
-            uint8_t* a = stages + s * C::kStageBytes;
             mbar_arrive_expect_tx(&full[s], C::kStageBytes);
             tma_load_2d(a, tm_a, &full[s], c * kChunkK, rb * kBlockM);
             tma_load_2d(a + kA0Bytes, &tm_w, &full[s], c * kChunkK, nb * BN);
@@ -342,24 +353,32 @@ __global__ void __launch_bounds__(kGThreads, 1)
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
     if (elect_one()) {
+      pdl_wait();  // block info beyond the shared-memory table is read from global memory
       constexpr uint32_t idesc = idesc_i8(BN);
       uint32_t it = 0, slot_it = 0;
-      bool ok = true, issued = false;
+      bool ok = true, issued = false, have_info = false;
       for (int slot = 0; slot < my_tiles && ok; ++slot) {
         const int tile = (int)blockIdx.x + slot * (int)gridDim.x;
-        const BlockInfo bi = info(slot, tile / p.tiles_n);
-        if (bi.nplanes == 0) continue;
-        // acquire accumulator slots
-        uint32_t acc_slot[2];
-        for (int q = 0; q < bi.nplanes && ok; ++q) {
-          const uint32_t si = slot_it + q;
-          acc_slot[q] = si % C::kSlots;
-          ok = wait_parity(&tm_empty[acc_slot[q]], ((si / C::kSlots) & 1) ^ 1, s_abort, p.status, kWaitLimitNs);
-        }
-        if (!ok) break;
-        tc_fence_after();
-        for (int pass = 0; pass < bi.nplanes && ok; ++pass) {
-          const uint32_t d = tmem_base + acc_slot[pass] * BN;
+        const int rb = tile / p.tiles_n;
+        uint32_t acc0 = 0, acc1 = 0;
+        int np = 1;
+        for (int pass = 0; pass < 2 && ok; ++pass) {
+          BlockInfo bi{};
+          if (pass == 1) {
+            if (!have_info && !(ok = wait_parity(info_bar, 0, s_abort, p.status, kWaitLimitNs))) break;
+            have_info = true;
+            bi = info(slot, rb);
+            if (bi.nplanes < 2) break;
+            np = 2;
+          }
+          // the pass's accumulator slot
+          const uint32_t si = slot_it + pass;
+          const uint32_t acc = si % C::kSlots;
+          (pass == 0 ? acc0 : acc1) = acc;
+          if (!(ok = wait_parity(&tm_empty[acc], ((si / C::kSlots) & 1) ^ 1, s_abort, p.status, kWaitLimitNs)))
+            break;
+          tc_fence_after();
+          const uint32_t d = tmem_base + acc * BN;
           bool first = true;
           for (int c = 0; c < p.num_chunks; ++c) {
             if (pass == 1 && !chunk_has_plane1(bi, c)) continue;
@@ -381,8 +400,9 @@ __global__ void __launch_bounds__(kGThreads, 1)
           }
         }
         if (!ok) break;
-        for (int q = 0; q < bi.nplanes; ++q) mma_commit(&tm_full[acc_slot[q]]);
-        slot_it += bi.nplanes;
+        mma_commit(&tm_full[acc0]);
+        if (np == 2) mma_commit(&tm_full[acc1]);
+        slot_it += np;
       }
       // drain: all MMAs this thread issued complete before TMEM and SMEM go away
       if (issued) {
@@ -404,6 +424,24 @@ __global__ void __launch_bounds__(kGThreads, 1)
     uint32_t slot_it = 0, y_it = 0;
     bool y_pending = false;  // lane 0: a y_prev request whose landing nobody has observed
     int ok = 1;
+    pdl_wait();  // the quantizer's outputs and the cached output are read from here on
+    // block info of this CTA's first kMaxTileSlots tiles, loaded in parallel,
+    // then published to the producer and MMA threads
+    for (int i = etid; i < min(my_tiles, kMaxTileSlots) * 8; i += 32 * kEpiWarps) {
+      const int slot = i >> 3, sub = i & 7;
+      const int rb = ((int)blockIdx.x + slot * (int)gridDim.x) / p.tiles_n;
+      const int t = rb * 8 + sub;
+      if (t < T) {
+        const int pl = p.planes[t];
+        int* e = reinterpret_cast<int*>(&s_info[slot]);
+        if (pl <= 2) atomicMax(&e[0], pl);
+        else atomicOr(&e[1], 1);
+        if (p.mask_words > 0) atomicOr(reinterpret_cast<unsigned*>(&e[2]), p.mask1[(int64_t)t * p.mask_words]);
+        if (p.mask_words > 1) atomicOr(reinterpret_cast<unsigned*>(&e[3]), p.mask1[(int64_t)t * p.mask_words + 1]);
+      }
+    }
+    epi_barrier();
+    if (etid == 0) mbar_arrive(info_bar);
     // Every epilogue warp runs every iteration and both named barriers of it,
     // also after a timed-out wait (ok == 0), so no warp can be left waiting
     // at a barrier that another warp skipped.
@@ -417,7 +455,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
       for (int i = etid; i < BN; i += 32 * kEpiWarps) s_ws[i] = (n_base + i < p.N) ? p.w_scale[n_base + i] : 0.f;
       epi_barrier();
 
-      if (ok && bi.nplanes > 0) {
+      if (ok) {
         // this warp's y_prev tiles: the buffer is free once the last tile's stores have read it
         if (lane == 0) {
           bulk_wait_read<0>();
