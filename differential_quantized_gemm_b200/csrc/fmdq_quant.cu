@@ -170,9 +170,8 @@ __device__ __forceinline__ void csync(cg::cluster_group& cluster, int C) {
 __device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
 
-constexpr int kTagWin = 32;  // tags handled per pass of the encoded stream
+constexpr int kTagWin = 16;  // tags handled per pass of the encoded stream
 constexpr int kUA = 4;       // chunks per round of ballots when counting
-constexpr int kUB = 4;       // chunks per round of ballots when writing
 constexpr uint32_t kFull = 0xffffffffu;
 
 struct QSmem {
@@ -185,7 +184,8 @@ struct QSmem {
   int total;
   int red[4][kQWarps];
   int warp_cnt[kQWarps][kTagWin];
-  int base[kTagWin];  // first record of this CTA per tag of the window
+  int base[kTagWin];              // first record of this CTA per tag of the window
+  int wbase[kQWarps][kTagWin];    // first record of each warp per tag of the window
   int x[kMaxCluster][4];
   int x_tot[kMaxCluster][kTagWin];
 };
@@ -193,7 +193,8 @@ struct QSmem {
 }  // namespace
 
 size_t quantize_smem_bytes(int64_t Kc) {
-  size_t b = 18 * (size_t)Kc;  // codes (16 per channel), FPoT and width
+  // codes (16 per channel), FPoT and width, rank table (kTagWin 8-byte entries per 32 channels)
+  size_t b = 18 * (size_t)Kc + (size_t)Kc / 32 * kTagWin * 8;
   b = (b + 15) & ~(size_t)15;
   return b + sizeof(QSmem);
 }
@@ -224,7 +225,11 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParam
   int8_t* s_code = reinterpret_cast<int8_t*>(smem);  // 16-byte slots: the 16 codes of a local channel
   int8_t* s_fpot = s_code + 16 * kc_max;              // [Kc]
   int8_t* s_bits = s_fpot + kc_max;                   // [Kc]
-  QSmem& S = *reinterpret_cast<QSmem*>(smem + ((18 * kc_max + 15) & ~(int64_t)15));
+  // [Kc / 32][kTagWin]: per 32-channel chunk and window tag, the ballot of the
+  // lanes carrying the tag and the warp's records of the tag in earlier chunks
+  uint2* s_tab = reinterpret_cast<uint2*>(s_bits + kc_max);
+  const int64_t tab_bytes = kc_max / 32 * kTagWin * 8;
+  QSmem& S = *reinterpret_cast<QSmem*>(smem + ((18 * kc_max + tab_bytes + 15) & ~(int64_t)15));
 
   if (tid < kMaxMaskWords) S.mask[tid] = 0;
   if (tid == 0) S.flags = 0;
@@ -408,14 +413,15 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParam
 
   // ------------------------------------- phase 2b: FPoT-grouped encoded stream
   // Slice j of channel k carries tag FPoT(k) - 2j (j < bits/2).  Tags lie in
-  // [gmin - 6, g] and are handled in windows of 32 consecutive tags (one
-  // window unless the tile's FPoT spread exceeds 25).  Each warp owns a
-  // contiguous run of 32-channel chunks (lane = channel) and visits, per
-  // chunk, only the tags present in it; one ballot ranks the lanes carrying a
-  // tag.  Lane u of a warp keeps the running offset of window tag u.  The
-  // record of (tag, k) lands after the tile's records of lower tags, then those
-  // of the same tag in lower-ranked CTAs, lower warps of this CTA, earlier
-  // chunks of this warp and lower lanes.
+  // [gmin - 6, g] and are handled in windows of 16 consecutive tags (one
+  // window unless the tile's FPoT spread exceeds 9).  Each warp owns a
+  // contiguous run of 32-channel chunks (lane = channel).  The record of
+  // (tag, k) lands after the tile's records of lower tags, then those of the
+  // same tag in lower-ranked CTAs, lower warps of this CTA, earlier chunks of
+  // this warp and lower lanes of its chunk.  Pass A counts, and keeps per
+  // (chunk, tag) the ballot of the lanes carrying the tag with the warp's
+  // count of the tag before the chunk; pass B then places every record by
+  // itself: that count plus the set lanes below it in the ballot.
   const int tlo = gmin - 6;
   const int nchunks = Kc / 32;
   const int ch_lo = warp * nchunks / kQWarps, ch_hi = (warp + 1) * nchunks / kQWarps;
@@ -437,20 +443,24 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParam
 #pragma unroll
       for (int u = 0; u < kUA; ++u) {
         const int c = 32 * (ch0 + u) + lane;
-        m[u] = ch0 + u < ch_hi ? tag_mask32(s_fpot[c], s_bits[c], tw) : 0u;
+        m[u] = ch0 + u < ch_hi ? tag_mask32(s_fpot[c], s_bits[c], tw) & ((1u << kTagWin) - 1u) : 0u;
         un |= m[u];
       }
       uint32_t any = __reduce_or_sync(kFull, un);
       while (any) {
         const int ti = __ffs(any) - 1;
         any &= any - 1u;
-        int n = 0;
 #pragma unroll
-        for (int u = 0; u < kUA; ++u) n += __popc(__ballot_sync(kFull, (m[u] >> ti) & 1u));
-        if (lane == ti) cnt += n;
+        for (int u = 0; u < kUA; ++u) {
+          const uint32_t bal = __ballot_sync(kFull, (m[u] >> ti) & 1u);
+          if (lane == ti && ch0 + u < ch_hi) {
+            s_tab[(ch0 + u) * kTagWin + ti] = make_uint2(bal, (uint32_t)cnt);
+            cnt += __popc(bal);
+          }
+        }
       }
     }
-    S.warp_cnt[warp][lane] = cnt;
+    if (lane < kTagWin) S.warp_cnt[warp][lane] = cnt;
     __syncthreads();
     if (tid < kTagWin) {
       int s = 0;
@@ -474,7 +484,7 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParam
     if (C > 1) cluster_arrive();  // remote reads of this window done; waited for before reuse or exit
     if (warp == 0) {
       int all = 0, lower = 0;
-      for (int q = 0; q < C; ++q) {
+      for (int q = 0; q < C && lane < kTagWin; ++q) {
         const int v = S.x_tot[q][lane];
         all += v;
         if (q < rank) lower += v;
@@ -485,48 +495,35 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParam
         const int n = __shfl_up_sync(kFull, incl, o);
         if (lane >= o) incl += n;
       }
-      S.base[lane] = total + incl - all + lower;
+      if (lane < kTagWin) S.base[lane] = total + incl - all + lower;
       total += __shfl_sync(kFull, incl, 31);
     }
     __syncthreads();
-    int off = S.base[lane];
-    for (int w = 0; w < warp; ++w) off += S.warp_cnt[w][lane];
-    // pass B: rank and write; kUB chunks share each round, chunk u's records of
-    // a tag before chunk u + 1's
-    for (int ch0 = ch_lo; ch0 < ch_hi; ch0 += kUB) {
-      uint32_t m[kUB], words[kUB][4], un = 0;
-      int f[kUB];
+    if (lane < kTagWin) {
+      int o = S.base[lane];
+      for (int w = 0; w < warp; ++w) o += S.warp_cnt[w][lane];
+      S.wbase[warp][lane] = o;
+    }
+    __syncwarp();
+    // pass B: every lane writes its channel's records of the window
+    const int* wb = S.wbase[warp];
+#pragma unroll 2
+    for (int ch = ch_lo; ch < ch_hi; ++ch) {
+      const int c = 32 * ch + lane;
+      const int f = s_fpot[c], b = s_bits[c];
+      uint32_t words[4];
+      slice_words(*reinterpret_cast<const uint4*>(s_code + 16 * code_slot(c)), words);
+      const uint2* row = s_tab + ch * kTagWin;
+      const uint32_t meta_k = (uint32_t)(k_lo + c);
 #pragma unroll
-      for (int u = 0; u < kUB; ++u) {
-        const int c = 32 * (ch0 + u) + lane;
-        const bool valid = ch0 + u < ch_hi;
-        f[u] = valid ? s_fpot[c] : 0;
-        m[u] = valid ? tag_mask32(f[u], s_bits[c], tw) : 0u;
-        un |= m[u];
-        if (valid) slice_words(*reinterpret_cast<const uint4*>(s_code + 16 * code_slot(c)), words[u]);
-        else words[u][0] = words[u][1] = words[u][2] = words[u][3] = 0u;
-      }
-      uint32_t any = __reduce_or_sync(kFull, un);
-      while (any) {
-        const int ti = __ffs(any) - 1;
-        any &= any - 1u;
-        uint32_t bal[kUB];
-#pragma unroll
-        for (int u = 0; u < kUB; ++u) bal[u] = __ballot_sync(kFull, (m[u] >> ti) & 1u);
-        int base = __shfl_sync(kFull, off, ti);
-        const uint32_t meta_t = (uint32_t)(uint8_t)(int8_t)(tw + ti) << 16;
-#pragma unroll
-        for (int u = 0; u < kUB; ++u) {
-          if ((m[u] >> ti) & 1u) {
-            // the field j < b/2 of the b-bit pattern equals that of the 8-bit pattern
-            const int j = (f[u] - tw - ti) >> 1;
-            const uint32_t w = j == 0 ? words[u][0] : j == 1 ? words[u][1] : j == 2 ? words[u][2] : words[u][3];
-            rec[base + __popc(bal[u] & lt)] =
-                make_uint2(w, (uint32_t)(k_lo + 32 * (ch0 + u) + lane) | meta_t | ((uint32_t)j << 24));
-          }
-          base += __popc(bal[u]);
+      for (int j = 0; j < 4; ++j) {
+        const int ti = f - 2 * j - tw;  // window slot of slice j
+        if (2 * j < b && ti >= 0 && ti < kTagWin) {
+          const uint2 e = row[ti];
+          // the field j < b/2 of the b-bit pattern equals that of the 8-bit pattern
+          rec[wb[ti] + (int)e.y + __popc(e.x & lt)] =
+              make_uint2(words[j], meta_k | ((uint32_t)(uint8_t)(int8_t)(tw + ti) << 16) | ((uint32_t)j << 24));
         }
-        if (lane == ti) off = base;
       }
     }
   }
