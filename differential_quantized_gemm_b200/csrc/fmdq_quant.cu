@@ -119,19 +119,13 @@ __device__ __forceinline__ void slice_words(const uint4 cw, uint32_t (&out)[4]) 
   }
 }
 
-// Shift room of a channel: the largest s with every code q of the channel
-// satisfying lo <= q 2^s <= hi, for the one-plane range [-128, 127] (wide =
-// false) or the two-plane range [-32896, 32639] (wide = true); 99 for a
-// channel whose codes are all zero.  For |q| <= 128 the bounds reduce to bit
-// lengths: q 2^s <= 127 iff bitlen(q) + s <= 7, q 2^s <= 32639 iff
-// bitlen(q) + s <= 15, and -m 2^s >= -128 (resp. -32896) iff
-// bitlen(m - 1) + s <= 7 (resp. 15).
-__device__ __forceinline__ int shift_room(int qmax, int qmin, bool wide) {
-  const int top = wide ? 15 : 7;
-  int r = 99;
-  if (qmax > 0) r = top - (32 - __clz(qmax));
-  if (qmin < 0) r = min(r, top - (32 - __clz(-qmin - 1)));
-  return r;
+// Shift room of a channel whose codes satisfy |q| <= qa: an s with every
+// q 2^s inside the one-plane range [-128, 127] (wide = false) or the
+// two-plane range [-32896, 32639] (wide = true); 99 when qa is 0.  For
+// 0 < qa <= 128, |q| 2^s <= 127 holds when bitlen(qa) + s <= 7 and
+// |q| 2^s <= 32639 when bitlen(qa) + s <= 15 (the negative bounds are looser).
+__device__ __forceinline__ int shift_room(int qa, bool wide) {
+  return qa > 0 ? (wide ? 15 : 7) - (32 - __clz(qa)) : 99;
 }
 
 // 16-byte slot of local channel c in the code array.  The XOR swizzle inside
@@ -148,6 +142,20 @@ __device__ __forceinline__ uint32_t tag_mask32(int f, int b, int tw) {
   const int lo = f - b + 2 - tw;
   if (lo >= 32 || lo < -8) return 0u;
   return (uint32_t)(((uint64_t)pat << (lo + 32)) >> 32);
+}
+
+// Transpose of a 32 x 32 bit matrix held one row per lane: afterwards lane c
+// holds column c (its bit l is bit c of lane l's row).  Five exchange steps
+// swap the off-diagonal blocks of halving size.
+__device__ __forceinline__ uint32_t warp_bit_transpose(uint32_t x, int lane) {
+#pragma unroll
+  for (int s = 16; s >= 1; s >>= 1) {
+    const uint32_t lo = s == 16 ? 0x0000FFFFu : s == 8 ? 0x00FF00FFu : s == 4 ? 0x0F0F0F0Fu : s == 2 ? 0x33333333u
+                                                                                                    : 0x55555555u;
+    const uint32_t y = __shfl_xor_sync(0xffffffffu, x, s);
+    x = (lane & s) ? ((x & ~lo) | ((y & ~lo) >> s)) : ((x & lo) | ((y & lo) << s));
+  }
+  return x;
 }
 
 // Rows 4R..4R+3 of four channels (word R of each channel's 16 codes, one byte
@@ -259,27 +267,36 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParam
 #pragma unroll
       for (int r = 0; r < kTile; ++r) PR::store(p.x_prev, (row0 + r) * p.ld_xp + c, rt[r]);
     }
-    // Eq. 1 (one fp32 subtraction per element) and stage 1 on the magnitude bits
+    // Eq. 1 (one fp32 subtraction per element, kept) and stage 1 on the magnitude bits
+    float d0[kTile], d1[kTile];
     uint32_t m0 = 0, m1 = 0;
 #pragma unroll
     for (int r = 0; r < kTile; ++r) {
-      m0 = max(m0, __float_as_uint(__fsub_rn(PR::lo(rt[r]), PR::lo(rp[r]))) & 0x7FFFFFFFu);
-      m1 = max(m1, __float_as_uint(__fsub_rn(PR::hi(rt[r]), PR::hi(rp[r]))) & 0x7FFFFFFFu);
+      d0[r] = __fsub_rn(PR::lo(rt[r]), PR::lo(rp[r]));
+      d1[r] = __fsub_rn(PR::hi(rt[r]), PR::hi(rp[r]));
+      m0 = max(m0, __float_as_uint(d0[r]) & 0x7FFFFFFFu);
+      m1 = max(m1, __float_as_uint(d1[r]) & 0x7FFFFFFFu);
     }
     const ColParams c0 = col_params(m0, lb, beta, t0, fb, flags);
     const ColParams c1 = col_params(m1, lb, beta, t0, fb, flags);
-    uint32_t w0[4] = {0, 0, 0, 0}, w1[4] = {0, 0, 0, 0};
-    int qmx0 = 0, qmn0 = 0, qmx1 = 0, qmn1 = 0;
+    // stage 3; a non-finite sub-channel has scale 0, and its NaN products convert to 0
+    const float s0 = c0.nonfinite ? 0.f : c0.scale, s1 = c1.nonfinite ? 0.f : c1.scale;
+    uint32_t w0[4], w1[4];
 #pragma unroll
-    for (int r = 0; r < kTile; ++r) {  // stage 3 (dX recomputed: the same single subtraction)
-      const float d0 = __fsub_rn(PR::lo(rt[r]), PR::lo(rp[r])), d1 = __fsub_rn(PR::hi(rt[r]), PR::hi(rp[r]));
-      const int q0 = c0.nonfinite ? 0 : __float2int_rn(__fmul_rn(d0, c0.scale));
-      const int q1 = c1.nonfinite ? 0 : __float2int_rn(__fmul_rn(d1, c1.scale));
-      w0[r >> 2] |= ((uint32_t)q0 & 0xFFu) << (8 * (r & 3));
-      w1[r >> 2] |= ((uint32_t)q1 & 0xFFu) << (8 * (r & 3));
-      qmx0 = max(qmx0, q0), qmn0 = min(qmn0, q0);
-      qmx1 = max(qmx1, q1), qmn1 = min(qmn1, q1);
+    for (int R = 0; R < 4; ++R) {
+      int a[4], b[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        a[e] = __float2int_rn(__fmul_rn(d0[4 * R + e], s0));
+        b[e] = __float2int_rn(__fmul_rn(d1[4 * R + e], s1));
+      }
+      // low bytes of four codes, token 4R + e in byte e
+      w0[R] = __byte_perm(__byte_perm(a[0], a[1], 0x0040), __byte_perm(a[2], a[3], 0x0040), 0x5410);
+      w1[R] = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
     }
+    // largest |code| of each channel: rne(M_i s_i) bounds every |rne(dX s_i)|
+    const int qa0 = c0.nonfinite ? 0 : __float2int_rn(__fmul_rn(__uint_as_float(m0), s0));
+    const int qa1 = c1.nonfinite ? 0 : __float2int_rn(__fmul_rn(__uint_as_float(m1), s1));
     if (p.debug_codes) {
 #pragma unroll
       for (int r = 0; r < kTile; ++r)
@@ -295,8 +312,8 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParam
     *reinterpret_cast<uint16_t*>(p.bits + (int64_t)t * K + c) = two(c0.bits, c1.bits);
     fmax = max(fmax, max(c0.fpot, c1.fpot));
     fmin = min(fmin, min(c0.fpot, c1.fpot));
-    a1 = min(a1, min(c0.fpot + shift_room(qmx0, qmn0, false), c1.fpot + shift_room(qmx1, qmn1, false)));
-    a2 = min(a2, min(c0.fpot + shift_room(qmx0, qmn0, true), c1.fpot + shift_room(qmx1, qmn1, true)));
+    a1 = min(a1, min(c0.fpot + shift_room(qa0, false), c1.fpot + shift_room(qa1, false)));
+    a2 = min(a2, min(c0.fpot + shift_room(qa0, true), c1.fpot + shift_room(qa1, true)));
   }
 
   // CTA reductions, then one exchange across the cluster
@@ -435,28 +452,24 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParam
       if (C > 1) cluster_wait();   // and every CTA with its remote reads of them
     }
     first = false;
-    // pass A: this warp's count of every tag of the window (lane u: tag tw + u);
-    // kUA chunks share each round of ballots
+    // pass A: per chunk, the lane ballot of every window tag is a column of the
+    // bit matrix whose rows are the lanes' tag masks, so one warp transpose
+    // gives them all (lane u: tag tw + u); lane u also keeps this warp's count
+    // of its tag so far
     int cnt = 0;
     for (int ch0 = ch_lo; ch0 < ch_hi; ch0 += kUA) {
-      uint32_t m[kUA], un = 0;
+      uint32_t col[kUA];
 #pragma unroll
       for (int u = 0; u < kUA; ++u) {
         const int c = 32 * (ch0 + u) + lane;
-        m[u] = ch0 + u < ch_hi ? tag_mask32(s_fpot[c], s_bits[c], tw) & ((1u << kTagWin) - 1u) : 0u;
-        un |= m[u];
+        const uint32_t m = ch0 + u < ch_hi ? tag_mask32(s_fpot[c], s_bits[c], tw) & ((1u << kTagWin) - 1u) : 0u;
+        col[u] = warp_bit_transpose(m, lane);
       }
-      uint32_t any = __reduce_or_sync(kFull, un);
-      while (any) {
-        const int ti = __ffs(any) - 1;
-        any &= any - 1u;
 #pragma unroll
-        for (int u = 0; u < kUA; ++u) {
-          const uint32_t bal = __ballot_sync(kFull, (m[u] >> ti) & 1u);
-          if (lane == ti && ch0 + u < ch_hi) {
-            s_tab[(ch0 + u) * kTagWin + ti] = make_uint2(bal, (uint32_t)cnt);
-            cnt += __popc(bal);
-          }
+      for (int u = 0; u < kUA; ++u) {
+        if (ch0 + u < ch_hi && lane < kTagWin) {
+          s_tab[(ch0 + u) * kTagWin + lane] = make_uint2(col[u], (uint32_t)cnt);
+          cnt += __popc(col[u]);
         }
       }
     }
