@@ -207,6 +207,15 @@ def job_tops(world: int, ops_per_rank: float, ms_per_step: float) -> float:
     return world * ops_per_rank / (ms_per_step * 1e-3) / 1e12
 
 
+def workload_config(cfg, inputs, world):
+    """The `config` of the JSON line: the workload, the same for both arms."""
+    from differential_quantized_gemm_b200 import synth
+    return {"workload": synth.CONFIG_NAMES[cfg],
+            "layers": [f"{i.spec.name} M={i.spec.M} K={i.spec.K} N={i.spec.N}" for i in inputs],
+            "base_scale": f"2^{inputs[0].spec.lb}", "tile_tokens": 16,
+            "parallelism": f"{world} replica(s), one batch per GPU, no collective"}
+
+
 def workload_inputs(cfg, rank):
     from differential_quantized_gemm_b200 import synth
     seed = None if rank == 0 else cfg + 7919 * rank
@@ -246,32 +255,62 @@ def algorithmic_k2(spec, ws_sections, out_bytes=2):
 
 # ------------------------------------------------------------ oracle timing
 
-def oracle_sample_time(inputs, seconds: float, steps_hint: int | None = None):
-    """Time the CPU oracle on whole tiles of each layer until about `seconds`
-    of CPU work; returns (ops, elapsed, description, threads)."""
+def oracle_step(inputs, nt: int, frac: float) -> float:
+    """One oracle pass over the first nt token tiles of every layer and the
+    first `frac` of its output channels (quantize, int64 accumulation, fp32
+    epilogue); returns the dense-equivalent ops it covered."""
     import numpy as np
     import oracle
 
-    def run(nt):
-        ops = 0.0
-        t0 = time.perf_counter()
-        for inp in inputs:
-            s = inp.spec
-            rows = slice(0, 16 * nt)
-            q = oracle.quantize(inp.as_f32("x_t")[rows], inp.as_f32("x_prev")[rows], s.lb, s.t0, s.force_bits)
-            acc = oracle.acc_direct(q, inp.w_q)
-            oracle.epilogue_f32(acc, q.g_ref, s.lb, inp.w_scale, inp.as_f32("y_prev")[rows], s.dtype == "bf16")
-            ops += 2.0 * 16 * nt * s.N * s.K
-        return ops, time.perf_counter() - t0
+    ops = 0.0
+    for inp in inputs:
+        s = inp.spec
+        rows = slice(0, 16 * nt)
+        ncols = s.N if frac >= 1.0 else max(16, int(s.N * frac) // 16 * 16)
+        q = oracle.quantize(inp.as_f32("x_t")[rows], inp.as_f32("x_prev")[rows], s.lb, s.t0, s.force_bits)
+        acc = oracle.acc_direct(q, np.ascontiguousarray(inp.w_q[:ncols]))
+        oracle.epilogue_f32(acc, q.g_ref, s.lb, np.ascontiguousarray(inp.w_scale[:ncols]),
+                            np.ascontiguousarray(inp.as_f32("y_prev")[rows, :ncols]), s.dtype == "bf16")
+        ops += 2.0 * 16 * nt * ncols * s.K
+    return ops
 
-    run(1)  # load and warm
-    ops, el = run(1)
+
+def oracle_calibrate(inputs, per_step: float):
+    """A step size of about per_step seconds that keeps every oracle thread
+    busy: at least one token tile per thread, then more tiles, or a fraction
+    of the output channels when even that is too long."""
+    import oracle
+
+    threads = oracle.n_threads()
     T = min(inp.spec.M // 16 for inp in inputs)
-    nt = int(max(1, min(T, seconds / max(el, 1e-6))))
-    ops, el = run(nt)
-    desc = (f"{nt} of {T} token tiles (first {16 * nt} tokens) of every layer: quantize, direct int64 "
+    nt = min(T, threads)
+    oracle_step(inputs, nt, 1.0)  # load and warm
+    t0 = time.perf_counter()
+    oracle_step(inputs, nt, 1.0)
+    el = time.perf_counter() - t0
+    if el <= per_step:
+        return max(nt, min(T, int(nt * per_step / el))), 1.0, min(threads, nt), T
+    return nt, max(per_step / el, 1e-3), min(threads, nt), T
+
+
+def oracle_sample_time(inputs, seconds: float):
+    """Time the CPU oracle on the whole workload (every token tile of every
+    layer), repeated until about `seconds`; returns (ops, elapsed,
+    description, threads used)."""
+    import oracle
+
+    T = min(inp.spec.M // 16 for inp in inputs)
+    oracle_step(inputs, min(T, oracle.n_threads()), 1.0)  # load and warm
+    ops = el = 0.0
+    reps = 0
+    while reps == 0 or (el < seconds and reps < 100):
+        t0 = time.perf_counter()
+        ops += oracle_step(inputs, T, 1.0)
+        el += time.perf_counter() - t0
+        reps += 1
+    desc = (f"the whole workload ({T} token tiles of every layer) {reps} time(s): quantize, direct int64 "
             f"accumulation, fp32 epilogue")
-    return ops, el, desc, oracle.n_threads(), nt
+    return ops, el, desc, min(oracle.n_threads(), T)
 
 
 # ----------------------------------------------------------------- arms
@@ -280,43 +319,16 @@ def run_reference(args, rank, world):
     """The oracle as the reference arm: rank 0 times it on the host cores."""
     if rank != 0:
         return
-    import numpy as np
     inputs = workload_inputs(args.config, 0)
     budget = 150.0  # seconds for warmup + steps
     per_step = budget / max(1, args.steps + args.warmup)
-    import oracle
-    threads = oracle.n_threads()
-    T = min(inp.spec.M // 16 for inp in inputs)
-
-    def step(nt, frac):
-        ops = 0.0
-        for inp in inputs:
-            s = inp.spec
-            rows = slice(0, 16 * nt)
-            ncols = max(16, int(s.N * frac) // 16 * 16)
-            q = oracle.quantize(inp.as_f32("x_t")[rows], inp.as_f32("x_prev")[rows], s.lb, s.t0, s.force_bits)
-            acc = oracle.acc_direct(q, np.ascontiguousarray(inp.w_q[:ncols]))
-            oracle.epilogue_f32(acc, q.g_ref, s.lb, np.ascontiguousarray(inp.w_scale[:ncols]),
-                                np.ascontiguousarray(inp.as_f32("y_prev")[rows, :ncols]), s.dtype == "bf16")
-            ops += 2.0 * 16 * nt * ncols * s.K
-        return ops
-
-    # size one step's sample from a one-tile probe: whole tiles while they fit,
-    # else a column subset of one tile
-    step(1, 1.0)
-    t0 = time.perf_counter()
-    step(1, 1.0)
-    el1 = time.perf_counter() - t0
-    if el1 <= per_step:
-        nt, frac = max(1, min(T, int(per_step / el1))), 1.0
-    else:
-        nt, frac = 1, max(per_step / el1, 1e-3)
+    nt, frac, threads, T = oracle_calibrate(inputs, per_step)
     for _ in range(args.warmup):
-        step(nt, frac)
+        oracle_step(inputs, nt, frac)
     t0 = time.perf_counter()
     ops = 0.0
     for _ in range(args.steps):
-        ops += step(nt, frac)
+        ops += oracle_step(inputs, nt, frac)
     el = time.perf_counter() - t0
     val = ops / el / 1e12
     sample = (f"{nt} of {T} token tiles x {frac:.3f} of the output channels of every layer per step "
@@ -326,7 +338,7 @@ def run_reference(args, rank, world):
         "impl": "reference", "metric": METRIC, "value": val, "unit": "TOPS", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64", "data": "synthetic",
-        "config": {"workload": synth.CONFIG_NAMES[args.config]},
+        "config": workload_config(args.config, inputs, world),
         "cpu_baseline": {"value": val, "unit": "TOPS", "cores": threads, "kind": "oracle", "sample": sample},
         "e2e": {"value": val, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -571,7 +583,7 @@ def run_ours(args, rank, world, local_rank):
 
     cpu = None
     if not args.no_cpu_baseline:
-        ops, el, desc, threads, _ = oracle_sample_time(inputs, args.cpu_seconds)
+        ops, el, desc, threads = oracle_sample_time(inputs, args.cpu_seconds)
         cpu = {"value": ops / el / 1e12, "unit": "TOPS", "cores": threads, "kind": "oracle", "sample": desc,
                "seconds": el}
 
@@ -582,12 +594,9 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "int8", "data": "synthetic",
-        "config": {"workload": synth.CONFIG_NAMES[args.config],
-                   "layers": [f"{i.spec.name} M={i.spec.M} K={i.spec.K} N={i.spec.N}" for i in inputs],
-                   "base_scale": f"2^{inputs[0].spec.lb}", "tile_tokens": 16,
-                   "l2": f"inputs rotate over {args.sets} buffer sets of {set_mb:.0f} MB each "
-                         f"({args.sets * set_mb:.0f} MB > 126 MB L2); no flush needed",
-                   "parallelism": f"{world} replica(s), one batch per GPU, no collective"},
+        "config": dict(workload_config(args.config, inputs, world),
+                       l2=f"inputs rotate over {args.sets} buffer sets of {set_mb:.0f} MB each "
+                          f"({args.sets * set_mb:.0f} MB > 126 MB L2); no flush needed"),
         "roofline": roofline,
         "kernels": kernels,
         "quantizer_GBps": [k["achieved"] for k in kern if k["kernel"] == "quantize"],
