@@ -211,8 +211,9 @@ int quantize_cluster_size(int64_t M, int64_t K, int num_sms) {
   const int64_t T = M / kTile;
   const int64_t units = K / 32;
   int c = 1;
-  // about 1.5 CTAs per SM when the batch is small, at least 256 channels per CTA
-  while (c < kMaxCluster && 2 * T * c < 3LL * num_sms && units / (2 * c) >= 8) c *= 2;
+  // about 1.5 CTAs per SM when the batch is small, at least 1024 channels per
+  // CTA (below that the cluster exchanges cost more than the split gains)
+  while (c < kMaxCluster && 2 * T * c < 3LL * num_sms && units / (2 * c) >= 32) c *= 2;
   return c;
 }
 
