@@ -58,8 +58,8 @@ struct GemmCfg {
   static constexpr int kNumBars = 2 * kStages + 2 * kSlots + kEpiWarps + 2;
   static constexpr int kOffBar = 0;
   static constexpr int kOffMisc = (kOffBar + kNumBars * 8 + 15) & ~15;  // tmem base, abort flag
-  static constexpr int kOffWs = kOffMisc + 16;                          // [BN] fp32 weight scales
-  static constexpr int kOffInfo = (kOffWs + BN * 4 + 15) & ~15;         // [kMaxTileSlots] int4 block info
+  static constexpr int kOffWs = kOffMisc + 16;                          // [2][BN] fp32 weight scales
+  static constexpr int kOffInfo = (kOffWs + 2 * BN * 4 + 15) & ~15;         // [kMaxTileSlots] int4 block info
   static constexpr int kSmallBytes = kOffInfo + kMaxTileSlots * 16;
   static_assert(kOffWs % 16 == 0 && kOffInfo % 16 == 0, "16-byte aligned shared arrays");
   static constexpr int kOffStages = (kSmallBytes + 1023) & ~1023;
@@ -193,11 +193,18 @@ __device__ __forceinline__ void epi_group(uint8_t* row, int swz, const float* ws
   constexpr int kOutBytes = OUT_BF16 ? 2 : 4;
   constexpr int E = 16 / kOutBytes;              // outputs per 16-byte chunk
   constexpr int kChunks = 32 * kOutBytes / 16;   // chunks per 32-column row
+  const float4* ws4 = reinterpret_cast<const float4*>(ws32);  // 16-byte aligned
 #pragma unroll
   for (int c = 0; c < kChunks; ++c) {
     uint4* cp = reinterpret_cast<uint4*>(row + 16 * (c ^ swz));
     const uint4 yv = *cp;
     const uint32_t yw[4] = {yv.x, yv.y, yv.z, yv.w};
+    float wsv[E];
+#pragma unroll
+    for (int h = 0; h < E / 4; ++h) {
+      const float4 w = ws4[c * (E / 4) + h];
+      wsv[4 * h] = w.x, wsv[4 * h + 1] = w.y, wsv[4 * h + 2] = w.z, wsv[4 * h + 3] = w.w;
+    }
     float y[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) {
@@ -208,7 +215,7 @@ __device__ __forceinline__ void epi_group(uint8_t* row, int swz, const float* ws
       float a;
       if constexpr (WIDE) a = __ll2float_rn((int64_t)(int32_t)d0[i] + (wide_row ? (int64_t)(int32_t)d1[i] * 256 : 0));
       else a = __int2float_rn((int32_t)d0[i]);
-      y[e] = __fadd_rn(ypf, __fmul_rn(__fmul_rn(a, p2), ws32[i]));
+      y[e] = __fadd_rn(ypf, __fmul_rn(__fmul_rn(a, p2), wsv[e]));
     }
     if constexpr (OUT_BF16) {
       uint32_t w[4];
@@ -417,20 +424,49 @@ __global__ void __launch_bounds__(kGThreads, 1)
     const int quarter = warp & 3;      // TMEM lanes 32*quarter .. +31 are this warp's rows
     const int half = ew >> 2;          // columns [half*BN/2, (half+1)*BN/2)
     uint8_t* ybuf = ysmem + ew * C::kYWarpBytes;  // this warp's kHalfGroups tiles of 32 x 32
-    constexpr int kChunksPerRow = 32 * C::kOutBytes / 16;  // 16-byte chunks per 32-column row
+    static_assert(BN <= 32 * kEpiWarps, "one weight scale per epilogue thread and tile");
+    static_assert(C::kHalfGroups % 2 == 0, "groups are processed in pairs");
     // TMA swizzle of a 32 x 32 tile: 64-byte rows (bf16) use the 64-byte pattern,
     // 128-byte rows (fp32) the 128-byte one; chunk c of row r sits at chunk c ^ sw(r)
     auto sw = [](int r) { return OUT_BF16 ? ((r >> 1) & 3) : (r & 7); };
-    uint32_t slot_it = 0, y_it = 0;
-    bool y_pending = false;  // lane 0: a y_prev request whose landing nobody has observed
+    auto tile_rb = [&](int s) { return ((int)blockIdx.x + s * (int)gridDim.x) / p.tiles_n; };
+    auto tile_nb = [&](int s) { return ((int)blockIdx.x + s * (int)gridDim.x) % p.tiles_n; };
+    // Everything a tile needs besides its accumulator is requested one tile
+    // ahead: its y_prev boxes (each as soon as the previous tile's store has
+    // read the box), its weight scales (shared memory, double-buffered) and
+    // this lane's row data.
+    auto weight_scale = [&](int s) -> float {
+      const int64_t n = (int64_t)tile_nb(s) * BN + etid;
+      return (etid < BN && n < p.N) ? p.w_scale[n] : 0.f;
+    };
+    auto row_planes = [&](int s, int& pl, int& gref) {
+      const int64_t row = (int64_t)tile_rb(s) * kBlockM + quarter * 32 + lane;
+      pl = 3, gref = 0;
+      if (row < p.M) pl = p.planes[row / kTile], gref = p.g_ref[row / kTile];
+    };
+    auto load_y_box = [&](int s, int box) {  // lane 0
+      if (box == 0) mbar_arrive_expect_tx(&ybar[ew], C::kYWarpBytes);
+      tma_load_2d(ybuf + box * C::kBoxBytes, &tm_yp, &ybar[ew], tile_nb(s) * BN + half * (BN / 2) + box * 32,
+                  tile_rb(s) * kBlockM + quarter * 32);
+    };
+    uint32_t slot_it = 0;
+    uint32_t y_issued = 0, y_seen = 0;  // batches of y_prev boxes requested (lane 0) / observed landed
     int ok = 1;
     pdl_wait();  // the quantizer's outputs and the cached output are read from here on
+    if (lane == 0 && my_tiles > 0) {
+      for (int g = 0; g < C::kHalfGroups; ++g) load_y_box(0, g);
+      ++y_issued;
+    }
+    int pl_cur = 3, gref_cur = 0;
+    if (my_tiles > 0) {
+      row_planes(0, pl_cur, gref_cur);
+      if (etid < BN) s_ws[etid] = weight_scale(0);
+    }
     // block info of this CTA's first kMaxTileSlots tiles, loaded in parallel,
     // then published to the producer and MMA threads
     for (int i = etid; i < min(my_tiles, kMaxTileSlots) * 8; i += 32 * kEpiWarps) {
       const int slot = i >> 3, sub = i & 7;
-      const int rb = ((int)blockIdx.x + slot * (int)gridDim.x) / p.tiles_n;
-      const int t = rb * 8 + sub;
+      const int t = tile_rb(slot) * 8 + sub;
       if (t < T) {
         const int pl = p.planes[t];
         int* e = reinterpret_cast<int*>(&s_info[slot]);
@@ -442,35 +478,29 @@ __global__ void __launch_bounds__(kGThreads, 1)
     }
     epi_barrier();
     if (etid == 0) mbar_arrive(info_bar);
-    // Every epilogue warp runs every iteration and both named barriers of it,
+    // Every epilogue warp runs every iteration and the named barrier of it,
     // also after a timed-out wait (ok == 0), so no warp can be left waiting
     // at a barrier that another warp skipped.
     for (int slot = 0; slot < my_tiles; ++slot) {
-      const int tile = (int)blockIdx.x + slot * (int)gridDim.x;
-      const int rb = tile / p.tiles_n, nb = tile % p.tiles_n;
+      const int rb = tile_rb(slot), nb = tile_nb(slot);
+      const bool has_next = slot + 1 < my_tiles;
       const BlockInfo bi = info(slot, rb);
       const int64_t n_base = (int64_t)nb * BN;
       const int64_t n_half = n_base + half * (BN / 2);
       const int row0 = rb * kBlockM + quarter * 32;
-      for (int i = etid; i < BN; i += 32 * kEpiWarps) s_ws[i] = (n_base + i < p.N) ? p.w_scale[n_base + i] : 0.f;
-      epi_barrier();
+      const float* ws_tile = s_ws + (slot & 1) * BN;
+      float ws_next = 0.f;
+      int pl_next = 3, gref_next = 0;
+      if (has_next) {
+        ws_next = weight_scale(slot + 1);
+        row_planes(slot + 1, pl_next, gref_next);
+      }
 
       if (ok) {
-        // this warp's y_prev tiles: the buffer is free once the last tile's stores have read it
-        if (lane == 0) {
-          bulk_wait_read<0>();
-          mbar_arrive_expect_tx(&ybar[ew], C::kYWarpBytes);
-#pragma unroll
-          for (int g = 0; g < C::kHalfGroups; ++g)
-            tma_load_2d(ybuf + g * C::kBoxBytes, &tm_yp, &ybar[ew], (int)(n_half + g * 32), row0);
-          y_pending = true;
-        }
         const int64_t row = row0 + lane;
-        const bool in_range = row < p.M;
-        const int t = (int)(row / kTile);
-        const int pl = in_range ? p.planes[t] : 3;
-        const bool row_ok = in_range && pl <= 2;
-        const float p2 = row_ok ? exp2_exact(-p.lb - p.g_ref[t]) : 0.f;
+        const int pl = pl_cur;
+        const bool row_ok = row < p.M && pl <= 2;
+        const float p2 = row_ok ? exp2_exact(-p.lb - gref_cur) : 0.f;
 
         uint32_t acc_slot[2];
         for (int q = 0; q < bi.nplanes; ++q) {
@@ -481,26 +511,24 @@ __global__ void __launch_bounds__(kGThreads, 1)
             ok = wait_parity(&tm_full[acc_slot[q]], (si / C::kSlots) & 1, s_abort, p.status, kWaitLimitNs) ? 1 : 0;
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
-        int yok = 1;
-        if (lane == 0 && ok) {
-          yok = wait_parity(&ybar[ew], y_it & 1, s_abort, p.status, kWaitLimitNs) ? 1 : 0;
-          y_pending = !yok;
-        }
-        ++y_it;
-        ok = __shfl_sync(0xffffffffu, ok && yok, 0);
+        if (lane == 0 && ok) ok = wait_parity(&ybar[ew], y_seen & 1, s_abort, p.status, kWaitLimitNs) ? 1 : 0;
+        ok = __shfl_sync(0xffffffffu, ok, 0);
         if (ok) {
           // the landed tiles are visible to the lanes that observe the barrier phase
-          mbar_try_wait(&ybar[ew], (y_it - 1) & 1);
+          mbar_try_wait(&ybar[ew], y_seen & 1);
+          ++y_seen;
           tc_fence_after();
           const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
           const uint32_t col_half = half * (BN / 2);
           const uint32_t t0a = tmem_base + lane_off + acc_slot[0] * BN + col_half;
           const uint32_t t1a = tmem_base + lane_off + (bi.nplanes == 2 ? acc_slot[1] : acc_slot[0]) * BN + col_half;
-          const float* ws_h = s_ws + half * (BN / 2);
+          const float* ws_h = ws_tile + half * (BN / 2);
           const bool wide_blk = bi.nplanes == 2;  // warp-uniform
           const bool wide_row = pl == 2;
-          // finished 32 x 32 tiles go out through TMA (rows beyond M and columns
-          // beyond N are clipped; rows left to the slice stream keep y_prev)
+          // Finished 32 x 32 tiles go out through TMA (rows beyond M and columns
+          // beyond N are clipped; rows left to the slice stream keep y_prev).
+          // Once a store has read its box, the next tile's y_prev box is
+          // requested into it.
           auto store_group = [&](int g) {
             fence_proxy_async_smem();
             __syncwarp();
@@ -510,6 +538,15 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 if (p.y_distinct) tma_store_2d(&tm_yp, ybuf + g * C::kBoxBytes, (int)(n_half + g * 32), row0);
               }
               bulk_commit();
+              if (has_next && g > 0) {
+                bulk_wait_read<1>();
+                load_y_box(slot + 1, g - 1);
+              }
+              if (has_next && g == C::kHalfGroups - 1) {
+                bulk_wait_read<0>();
+                load_y_box(slot + 1, g);
+                ++y_issued;
+              }
             }
           };
           auto debug_group = [&](int g, const uint32_t (&d0)[32], const uint32_t (&d1)[32], bool wide) {
@@ -520,22 +557,27 @@ __global__ void __launch_bounds__(kGThreads, 1)
           };
           uint8_t* my_row = ybuf + lane * (32 * C::kOutBytes);
           const int swz = sw(lane);
+          auto one_plane_group = [&](int g, const uint32_t (&d)[32]) {
+            if (row_ok) {
+              epi_group<OUT_BF16, false>(my_row + g * C::kBoxBytes, swz, ws_h + g * 32, d, d, false, p2);
+              if (p.debug_acc) debug_group(g, d, d, false);
+            }
+            store_group(g);
+          };
           if (!wide_blk) {
-            // one plane: the accumulator of group g+1 is read from TMEM while group g is computed
+            // one plane: groups in pairs, the accumulator of the next group is
+            // read from TMEM while the current one is computed
             uint32_t dA[32], dB[32];
             tmem_ld32(t0a, dA);
-            tmem_ld_wait();
-#pragma unroll
-            for (int g = 0; g < C::kHalfGroups; ++g) {
-              uint32_t(&cur)[32] = (g & 1) ? dB : dA;
-              uint32_t(&nxt)[32] = (g & 1) ? dA : dB;
-              if (g + 1 < C::kHalfGroups) tmem_ld32(t0a + (g + 1) * 32, nxt);
-              if (row_ok) {
-                epi_group<OUT_BF16, false>(my_row + g * C::kBoxBytes, swz, ws_h + g * 32, cur, cur, false, p2);
-                if (p.debug_acc) debug_group(g, cur, cur, false);
-              }
-              store_group(g);
-              if (g + 1 < C::kHalfGroups) tmem_ld_wait();
+            tmem_ld_wait(dA);
+#pragma unroll 1
+            for (int g = 0; g < C::kHalfGroups; g += 2) {
+              tmem_ld32(t0a + (g + 1) * 32, dB);
+              one_plane_group(g, dA);
+              tmem_ld_wait(dB);
+              if (g + 2 < C::kHalfGroups) tmem_ld32(t0a + (g + 2) * 32, dA);
+              one_plane_group(g + 1, dB);
+              if (g + 2 < C::kHalfGroups) tmem_ld_wait(dA);
             }
           } else {
 #pragma unroll 1
@@ -543,7 +585,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
               uint32_t d0[32], d1[32];
               tmem_ld32(t0a + g * 32, d0);
               tmem_ld32(t1a + g * 32, d1);
-              tmem_ld_wait();
+              tmem_ld_wait(d0);
+              tmem_ld_wait(d1);
               if (row_ok) {
                 epi_group<OUT_BF16, true>(my_row + g * C::kBoxBytes, swz, ws_h + g * 32, d0, d1, wide_row, p2);
                 if (p.debug_acc) debug_group(g, d0, d1, true);
@@ -572,17 +615,22 @@ __global__ void __launch_bounds__(kGThreads, 1)
             const int64_t n = n_base + c;
             if (n >= p.N) continue;
             slice_stream_column<OUT_BF16>(p.records + (int64_t)t * p.record_cap, p.count[t], p.bits + (int64_t)t * p.K,
-                                          p.g_ref[t], p.w_q + n * p.ld_w, t, n, p.lb, s_ws[c], p.y_prev, p.ld_yp,
+                                          p.g_ref[t], p.w_q + n * p.ld_w, t, n, p.lb, ws_tile[c], p.y_prev, p.ld_yp,
                                           p.y_out, p.ld_yo, p.y_distinct, p.debug_acc, p.N);
           }
         }
       }
-      epi_barrier();  // the weight-scale buffer is free again
+      // the next tile's weight scales go to the other buffer, whose readers
+      // finished before the previous iteration's barrier
+      if (has_next && etid < BN) s_ws[((slot + 1) & 1) * BN + etid] = ws_next;
+      pl_cur = pl_next, gref_cur = gref_next;
+      epi_barrier();
     }
     // nothing of this warp's may still be in flight when the block exits:
-    // y_prev tiles that were requested but not consumed, and the last stores
+    // y_prev boxes that were requested but not observed, and the last stores
+    y_issued = __shfl_sync(0xffffffffu, y_issued, 0);
     if (lane == 0) {
-      if (y_pending) wait_parity(&ybar[ew], (y_it - 1) & 1, s_abort, p.status, kWaitLimitNs, true);
+      if (y_issued > y_seen) wait_parity(&ybar[ew], (y_issued - 1) & 1, s_abort, p.status, kWaitLimitNs, true);
       bulk_wait<0>();
     }
     __syncwarp();
