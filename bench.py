@@ -46,6 +46,9 @@ def parse():
     ap.add_argument("--config", type=int, default=2, help="workload (2: DiT-XL/2 FFN pair)")
     ap.add_argument("--sets", type=int, default=3, help="rotating input sets (together larger than L2)")
     ap.add_argument("--e2e-steps", type=int, default=300)
+    ap.add_argument("--xprev", choices=["swap", "copy"], default="copy",
+                    help="swap: X_t and X_{t-1} stay resident and trade buffers each step (no refresh copy); "
+                         "copy: the quantizer copies X_t into one x_prev cache")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
@@ -150,8 +153,9 @@ class ClockSampler:
 class Layer:
     """Device buffers and prebuilt C-ABI arguments of one layer in one input set."""
 
-    def __init__(self, inp, torch, nat):
+    def __init__(self, inp, torch, nat, swap):
         spec = inp.spec
+        self.swap = swap
         self.spec = spec
         dev = "cuda"
 
@@ -161,22 +165,26 @@ class Layer:
 
         self.x_a = bf(inp.x_t)           # X at even uses
         self.x_b = bf(inp.x_prev)        # X at odd uses
-        self.x_prev = self.x_b.clone()   # cache
+        self.x_prev = None if swap else self.x_b.clone()  # cache (copy mode)
         self.y_prev = bf(inp.y_prev)     # cache, updated in place
         self.w_q = torch.from_numpy(inp.w_q).to(dev)
         self.w_scale = torch.from_numpy(inp.w_scale).to(dev)
         self.ws = nat.Workspace(spec.M, spec.K)
         self.base = 2.0 ** spec.lb
-        self.cfg = nat.TileCfg(16, spec.t0, spec.force_bits, 0, ctypes.c_void_p(self.ws.ptr), self.ws.nbytes,
-                               None, None)
+        self.cfg = nat.TileCfg(16, spec.t0, spec.force_bits, nat.FLAG_NO_XPREV_REFRESH if swap else 0,
+                               ctypes.c_void_p(self.ws.ptr), self.ws.nbytes, None, None)
         self.m_x = [nat.mat(self.x_a), nat.mat(self.x_b)]
-        self.m_xp = nat.mat(self.x_prev)
+        self.m_xp = None if swap else nat.mat(self.x_prev)
         self.m_y = nat.mat(self.y_prev)
         self.m_w = nat.mat(self.w_q)
         self.ws_ptr = ctypes.c_void_p(self.w_scale.data_ptr())
 
+    def xp(self, parity):
+        """X_{t-1}: the other buffer (swap), or the cache (copy)."""
+        return self.m_x[1 - parity] if self.swap else self.m_xp
+
     def quantize(self, L, parity, stream):
-        return L.dstar_fmdq_quantize(ctypes.byref(self.m_x[parity]), ctypes.byref(self.m_xp), self.base,
+        return L.dstar_fmdq_quantize(ctypes.byref(self.m_x[parity]), ctypes.byref(self.xp(parity)), self.base,
                                      ctypes.byref(self.cfg), stream)
 
     def gemm(self, L, stream):
@@ -184,7 +192,7 @@ class Layer:
                                        ctypes.byref(self.cfg), ctypes.byref(self.m_y), stream)
 
     def linear(self, L, parity, stream):
-        return L.dstar_fmdq_linear(ctypes.byref(self.m_x[parity]), ctypes.byref(self.m_xp), ctypes.byref(self.m_y),
+        return L.dstar_fmdq_linear(ctypes.byref(self.m_x[parity]), ctypes.byref(self.xp(parity)), ctypes.byref(self.m_y),
                                    ctypes.byref(self.m_w), self.ws_ptr, self.base, ctypes.byref(self.cfg),
                                    ctypes.byref(self.m_y), stream)
 
@@ -207,12 +215,19 @@ def job_tops(world: int, ops_per_rank: float, ms_per_step: float) -> float:
     return world * ops_per_rank / (ms_per_step * 1e-3) / 1e12
 
 
-def workload_config(cfg, inputs, world):
+XPREV_DESC = {
+    "swap": "X_t and X_{t-1} resident in two buffers that trade roles each step (DSTAR_FLAG_NO_XPREV_REFRESH)",
+    "copy": "one x_prev cache per layer, refreshed with X_t by the quantizer",
+}
+
+
+def workload_config(cfg, inputs, world, xprev="copy"):
     """The `config` of the JSON line: the workload, the same for both arms."""
     from differential_quantized_gemm_b200 import synth
     return {"workload": synth.CONFIG_NAMES[cfg],
             "layers": [f"{i.spec.name} M={i.spec.M} K={i.spec.K} N={i.spec.N}" for i in inputs],
             "base_scale": f"2^{inputs[0].spec.lb}", "tile_tokens": 16,
+            "x_prev": XPREV_DESC[xprev],
             "parallelism": f"{world} replica(s), one batch per GPU, no collective"}
 
 
@@ -222,16 +237,17 @@ def workload_inputs(cfg, rank):
     return [synth.make_layer(cfg, li, seed=seed) for li in range(len(synth.config_layers(cfg)))]
 
 
-def algorithmic_k1_bytes(spec, ws_sections, in_bytes=2):
+def algorithmic_k1_bytes(spec, ws_sections, in_bytes=2, refresh=True):
     """Bytes K1 must move for one launch: read X_t and X_{t-1}, write X_t into
-    the cache, write plane 0 (and plane 1 for two-plane tiles), the encoded
-    stream (8 bytes per slice record) and the per-sub-channel FPoT and width."""
+    the cache (only when it refreshes one), write plane 0 (and plane 1 for
+    two-plane tiles), the encoded stream (8 bytes per slice record) and the
+    per-sub-channel FPoT and width."""
     import numpy as np
     M, K = spec.M, spec.K
     count = ws_sections["count"].cpu().numpy().astype(np.int64)
     planes = ws_sections["planes"].cpu().numpy()
     rows2 = int((planes == 2).sum()) * 16
-    return (3 * M * K * in_bytes + M * K + rows2 * K + int(count.sum()) * 8 + 2 * (M // 16) * K)
+    return ((3 if refresh else 2) * M * K * in_bytes + M * K + rows2 * K + int(count.sum()) * 8 + 2 * (M // 16) * K)
 
 
 def algorithmic_k2(spec, ws_sections, out_bytes=2):
@@ -338,7 +354,7 @@ def run_reference(args, rank, world):
         "impl": "reference", "metric": METRIC, "value": val, "unit": "TOPS", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64", "data": "synthetic",
-        "config": workload_config(args.config, inputs, world),
+        "config": workload_config(args.config, inputs, world, args.xprev),
         "cpu_baseline": {"value": val, "unit": "TOPS", "cores": threads, "kind": "oracle", "sample": sample},
         "e2e": {"value": val, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -362,7 +378,8 @@ def run_ours(args, rank, world, local_rank):
     dist = world > 1
 
     inputs = workload_inputs(args.config, rank)
-    sets = [[Layer(inp, torch, nat) for inp in inputs] for _ in range(args.sets)]
+    swap = args.xprev == "swap"
+    sets = [[Layer(inp, torch, nat, swap) for inp in inputs] for _ in range(args.sets)]
     nlayers = len(inputs)
     stream = torch.cuda.current_stream()
     sh = ctypes.c_void_p(stream.cuda_stream)
@@ -391,7 +408,7 @@ def run_ours(args, rank, world, local_rank):
     stats = []
     for lay in sets[0]:
         sec = lay.ws.sections(lay.spec.M, lay.spec.K)
-        b1 = algorithmic_k1_bytes(lay.spec, sec)
+        b1 = algorithmic_k1_bytes(lay.spec, sec, refresh=not swap)
         dense, issued, b2, nfall = algorithmic_k2(lay.spec, sec)
         bits = sec["bits"].cpu().numpy()
         planes = sec["planes"].cpu().numpy()
@@ -520,18 +537,21 @@ def run_ours(args, rank, world, local_rank):
             host_x[r][li][1].copy_(lay.x_b.cpu())
     h2d = sum(lay.x_a.numel() * lay.x_a.element_size() for lay in sets[0])
     d2h = sum(lay.y_prev.numel() * lay.y_prev.element_size() for lay in sets[0])
-    # device landing buffers for the copied inputs
-    land = [[torch.empty_like(lay.x_a) for lay in st] for st in sets]
-    land_m = [[nat.mat(t) for t in row] for row in land]
+    # device landing buffers for the copied inputs: one per parity in swap
+    # mode (the buffer of the other parity holds X_{t-1}), else one
+    land = [[[lay.x_a.clone(), lay.x_b.clone()] if swap else [torch.empty_like(lay.x_a)] for lay in st]
+            for st in sets]
+    land_m = [[[nat.mat(t) for t in bufs] for bufs in row] for row in land]
 
     def step_e2e(s):
         r = s % args.sets
         parity = uses[r] & 1
         uses[r] += 1
         for li, lay in enumerate(sets[r]):
-            land[r][li].copy_(host_x[r][li][parity], non_blocking=True)
-            mp = lay.m_xp
-            rc = L.dstar_fmdq_linear(ctypes.byref(land_m[r][li]), ctypes.byref(mp), ctypes.byref(lay.m_y),
+            slot = parity if swap else 0
+            land[r][li][slot].copy_(host_x[r][li][parity], non_blocking=True)
+            mp = land_m[r][li][1 - parity] if swap else lay.m_xp
+            rc = L.dstar_fmdq_linear(ctypes.byref(land_m[r][li][slot]), ctypes.byref(mp), ctypes.byref(lay.m_y),
                                      ctypes.byref(lay.m_w), lay.ws_ptr, lay.base, ctypes.byref(lay.cfg),
                                      ctypes.byref(lay.m_y), sh)
             if rc:
@@ -600,13 +620,14 @@ def run_ours(args, rank, world, local_rank):
                "seconds": el}
 
     set_mb = sum(t.numel() * t.element_size() for lay in sets[0]
-                 for t in (lay.x_a, lay.x_b, lay.x_prev, lay.y_prev, lay.w_q, lay.w_scale, lay.ws.buf)) / 1e6
+                 for t in (lay.x_a, lay.x_b, lay.x_prev, lay.y_prev, lay.w_q, lay.w_scale, lay.ws.buf)
+                 if t is not None) / 1e6
     launches_per_step = 2 * nlayers  # quantizer and slice GEMM (slice-stream tiles run inside it) per layer
     line = {
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "int8", "data": "synthetic",
-        "config": dict(workload_config(args.config, inputs, world),
+        "config": dict(workload_config(args.config, inputs, world, args.xprev),
                        l2=f"inputs rotate over {args.sets} buffer sets of {set_mb:.0f} MB each "
                           f"({args.sets * set_mb:.0f} MB > 126 MB L2); no flush needed"),
         "roofline": roofline,
