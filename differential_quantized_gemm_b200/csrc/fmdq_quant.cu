@@ -255,14 +255,30 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParam
   int flags = 0;
 
   // ---------------------------------------------------------------- phase 1
+  // bf16 inputs: the row words of a thread's next channel pair are requested
+  // before its current pair is processed, so two pairs' loads are in flight
+  // per thread (fp32 inputs would not fit the registers twice).
+  constexpr bool kAhead = sizeof(typename PR::Raw) == 4;
+  typename PR::Raw nt[kTile], np[kTile];
+  auto load_pair = [&](int pr, typename PR::Raw (&a)[kTile], typename PR::Raw (&b)[kTile]) {
+    const int64_t c = k_lo + 2 * pr;
+#pragma unroll
+    for (int r = 0; r < kTile; ++r) {
+      a[r] = PR::load(p.x_t, (row0 + r) * p.ld_xt + c);
+      b[r] = PR::load(p.x_prev, (row0 + r) * p.ld_xp + c);
+    }
+  };
+  if (kAhead && tid < npairs) load_pair(tid, nt, np);
   for (int pr = tid; pr < npairs; pr += kQThreads) {
     const int lc = 2 * pr;
     const int64_t c = k_lo + lc;
     typename PR::Raw rt[kTile], rp[kTile];
+    if constexpr (kAhead) {
 #pragma unroll
-    for (int r = 0; r < kTile; ++r) {
-      rt[r] = PR::load(p.x_t, (row0 + r) * p.ld_xt + c);
-      rp[r] = PR::load(p.x_prev, (row0 + r) * p.ld_xp + c);
+      for (int r = 0; r < kTile; ++r) rt[r] = nt[r], rp[r] = np[r];
+      if (pr + kQThreads < npairs) load_pair(pr + kQThreads, nt, np);
+    } else {
+      load_pair(pr, rt, rp);
     }
     if (refresh) {
 #pragma unroll
