@@ -50,6 +50,25 @@ def test_no_xprev_refresh_flag():
     assert np.array_equal(after, inp.x_prev)
 
 
+def test_swapped_xprev_buffers_equal_refreshed_cache():
+    """Two resident X buffers that trade roles each step (no refresh) give the
+    same Y sequence, bit for bit, as one x_prev cache refreshed by the call."""
+    inp = synth.make_layer(2, 1, M=256)
+    base = 2.0 ** inp.spec.lb
+    a, b = to_dev(inp), to_dev(inp)
+    ws_a, ws_b = nat.Workspace(inp.spec.M, inp.spec.K), nat.Workspace(inp.spec.M, inp.spec.K)
+    xs = [a["x_t"], a["x_prev"].clone()]        # X at even / odd steps
+    cache = a["x_prev"]                          # refreshed cache, holds X of the odd steps at first
+    for s in range(4):
+        nat.linear(xs[s & 1], cache, a["y_prev"], a["w_q"], a["w_scale"], base, ws_a)
+        nat.linear(xs[s & 1], xs[1 - (s & 1)], b["y_prev"], b["w_q"], b["w_scale"], base, ws_b,
+                   flags=nat.FLAG_NO_XPREV_REFRESH)
+        torch.cuda.synchronize()
+        assert torch.equal(a["y_prev"], b["y_prev"]), s
+        assert torch.equal(cache, xs[s & 1])
+    assert not nat.status(ws_a) and not nat.status(ws_b)
+
+
 def test_stationary_input_keeps_output_bit_exact():
     inp = synth.make_layer(3, 2, M=256)
     inp.x_t = inp.x_prev.copy()
