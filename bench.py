@@ -412,7 +412,10 @@ def run_ours(args, rank, world, local_rank):
         dense, issued, b2, nfall = algorithmic_k2(lay.spec, sec)
         bits = sec["bits"].cpu().numpy()
         planes = sec["planes"].cpu().numpy()
+        # the paper's unit of MPU work: one 2-bit slice of 16 tokens against one weight
+        slice_macs = 16 * int(sec["count"].cpu().numpy().astype(np.int64).sum()) * lay.spec.N
         stats.append(dict(k1_bytes=b1, k2_dense=dense, k2_issued=issued, k2_bytes=b2, fallback_tiles=nfall,
+                          slice_macs=slice_macs,
                           bits_avg=float(bits.mean()), bit_hist=[float((bits == b).mean()) for b in (2, 4, 6, 8)],
                           planes_hist=[int((planes == p).sum()) for p in (1, 2)] + [int((planes > 2).sum())]))
 
@@ -658,8 +661,10 @@ def run_ours(args, rank, world, local_rank):
         "roofline": roofline,
         "kernels": kernels,
         "quantizer_GBps": [k["achieved"] for k in kern if k["kernel"] == "quantize"],
+        "quantizer_frac_of_8TBs_spec": [k["achieved"] / 8000.0 for k in kern if k["kernel"] == "quantize"],
         "workload_stats": [{k: v for k, v in s.items() if k in ("bits_avg", "bit_hist", "planes_hist",
-                                                              "fallback_tiles")} for s in stats],
+                                                              "fallback_tiles", "slice_macs")} for s in stats],
+        "slice_macs_per_s": sum(s["slice_macs"] for s in stats) / (ms_step * 1e-3),
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * K,
         "clocks": clocks.summary(t_wall0, t_wall1),
         "kernel_sources": kernel_source_sha(),

@@ -179,7 +179,7 @@ __device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
 
 constexpr int kTagWin = 16;  // tags handled per pass of the encoded stream
-constexpr int kUA = 2;       // chunks per round of ballots when counting
+constexpr int kUA = 1;       // chunks per round of ballots when counting
 constexpr uint32_t kFull = 0xffffffffu;
 
 struct QSmem {
