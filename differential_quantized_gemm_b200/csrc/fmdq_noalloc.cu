@@ -4,8 +4,12 @@
 // dstar_fmdq_linear, which it calls with the array as the workspace.
 //
 // In host code the name of a __device__ array only stands for it: the address
-// a kernel needs comes from cudaGetSymbolAddress, fetched here once per device
-// with that device current and cached.
+// a kernel needs comes from cudaGetSymbolAddress, looked up on every call with
+// the caller's device current (cheap once the module is loaded).  A device
+// reset or a new primary context loads the module again, possibly at another
+// address and with stale contents, so the one-time clearing of the status word
+// is keyed to the context's unique ID, never to the device number.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdio>
@@ -21,29 +25,59 @@ static __device__ __align__(256) uint8_t g_noalloc_scratch[DSTAR_NOALLOC_SCRATCH
 namespace fmdq {
 namespace {
 
-constexpr int kMaxDevices = 64;
+// IDs of the contexts whose copy of the array has had its status word cleared
+// (a small ring; re-clearing after an eviction is harmless).
+constexpr int kMaxContexts = 64;
 std::mutex g_scratch_mu;
-void* g_scratch_addr[kMaxDevices] = {};  // device address of the array, per device ordinal
+unsigned long long g_cleared[kMaxContexts] = {};
+int g_ncleared = 0, g_next = 0;
 
-// Device address of the scratch on the current device.  The first call on a
-// device looks it up and enqueues the clearing of the status word on `stream`
-// (the only part of the workspace that must start at zero).
-int scratch_address(void** out, cudaStream_t stream) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return report_cuda_error(e, "cudaGetDevice");
-  if (dev < 0 || dev >= kMaxDevices)
-    return report_error(DSTAR_ERR_UNSUPPORTED, "device ordinal out of range for the static scratch");
-  std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Unique ID (for the life of the process) of the calling thread's current context.
+int current_context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) return report_cuda_error(e, "cudaGetSymbolAddress of the static scratch");
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  if (!get_current || !get_id) return report_error(DSTAR_ERR_CUDA, "cuCtxGetCurrent/cuCtxGetId are not available");
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return report_error(DSTAR_ERR_CUDA, "no current CUDA context");
+  if (get_id(ctx, id) != CUDA_SUCCESS) return report_error(DSTAR_ERR_CUDA, "cuCtxGetId failed");
+  return DSTAR_OK;
+}
+
+// Device address of the scratch in the current context.  The first call in a
+// context enqueues the clearing of the status word on `stream` (the only part
+// of the workspace that must start at zero).
+int scratch_address(void** out, cudaStream_t stream) {
+  void* p = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);  // makes the primary context current if needed
+  if (e != cudaSuccess) return report_cuda_error(e, "cudaGetSymbolAddress of the static scratch");
+  unsigned long long id = 0;
+  int r = current_context_id(&id);
+  if (r != DSTAR_OK) return r;
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  bool cleared = false;
+  for (int i = 0; i < g_ncleared && !cleared; ++i) cleared = g_cleared[i] == id;
+  if (!cleared) {
     e = cudaMemsetAsync(p, 0, 256, stream);
     if (e != cudaSuccess) return report_cuda_error(e, "clearing the static scratch's status word");
-    g_scratch_addr[dev] = p;
+    g_cleared[g_next] = id;
+    g_next = (g_next + 1) % kMaxContexts;
+    if (g_ncleared < kMaxContexts) ++g_ncleared;
   }
-  *out = g_scratch_addr[dev];
+  *out = p;
   return DSTAR_OK;
 }
 

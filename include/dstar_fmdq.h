@@ -35,6 +35,18 @@
  *     outputs of the calls since the last read are unspecified.
  *   - The entry points are reentrant; two calls that share a workspace must be
  *     ordered on the device (same stream, or events).
+ *
+ * Interface choices
+ *   - The status word lives in the caller's workspace, so the library keeps no
+ *     global state (no per-stream or per-device table to create, look up or
+ *     free): dstar_fmdq_status takes the workspace whose calls it reports.
+ *   - The workspace size depends on M and K only: every section is per token
+ *     or per (token tile, channel); N and the quantizer settings do not change
+ *     it, so dstar_fmdq_workspace_size takes neither.
+ *   - Debug output is requested by passing device buffers (debug_codes,
+ *     debug_acc), not by a flag; the bounded device wait is exercised by its
+ *     own entry point, dstar_fmdq_selftest_wait, so no flag of the production
+ *     call can make a wait run out.
  */
 #ifndef DSTAR_FMDQ_H
 #define DSTAR_FMDQ_H
@@ -195,9 +207,10 @@ DSTAR_API int dstar_fmdq_linear(const dstar_mat* x_t, dstar_mat* x_prev, dstar_m
  * array (about 4.1 * M * K; e.g. M = 2048 tokens with K = 4608 channels fits)
  * and returns DSTAR_ERR_WORKSPACE, enqueueing nothing, when that exceeds
  * DSTAR_NOALLOC_SCRATCH_BYTES.
- * First call on a device: it looks up the array's device address with that
- * device current and enqueues the clearing of its status word on `stream`.
- * Make that first call before any stream capture.
+ * Set-up: every call looks up the array's device address with the caller's
+ * device current.  The first call in a CUDA context (the first on a device,
+ * and again after a device reset) also enqueues the clearing of the array's
+ * status word on `stream`.  Make that first call before any stream capture.
  * Sharing: every call on a device uses the same array, which keeps the
  * previous call's contents.  Calls that may overlap on the GPU (different
  * streams without an ordering between them, or several host threads) race on

@@ -59,6 +59,37 @@ def run_gpu(inp: synth.LayerInputs, t0=None, force_bits=None, flags=0, y_distinc
     return res
 
 
+def run_gpu_bench_launch(inp: synth.LayerInputs):
+    """The call exactly as the benchmark times it: dstar_fmdq_linear captured in
+    a CUDA graph and replayed, y_out = y_prev (in place), x_prev refreshed, no
+    debug buffers.  Returns Y_t, the refreshed caches and the workspace's
+    integer sections."""
+    spec = inp.spec
+    d = to_dev(inp)
+    ws = nat.Workspace(spec.M, spec.K)
+    x_t_live = d["x_t"].clone()  # the graph reads this buffer; the inputs are copied into it before replay
+    x_prev_live = torch.empty_like(d["x_prev"])
+    y_live = torch.empty_like(d["y_prev"])
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    with torch.cuda.graph(g, stream=side):
+        nat.linear(x_t_live, x_prev_live, y_live, d["w_q"], d["w_scale"], 2.0 ** spec.lb, ws, t0=spec.t0,
+                   force_bits=spec.force_bits)
+    x_prev_live.copy_(d["x_prev"])
+    y_live.copy_(d["y_prev"])
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    st = nat.status(ws)
+    sec = ws.sections(spec.M, spec.K)
+    res = dict(status=st, y=dev_to_f32(y_live), x_prev_after=x_prev_live,
+               fpot=sec["fpot"].cpu().numpy(), bits=sec["bits"].cpu().numpy(), g_ref=sec["g_ref"].cpu().numpy(),
+               count=sec["count"].cpu().numpy(), planes=sec["planes"].cpu().numpy(),
+               records=sec["records"].cpu().numpy().view(np.uint32))
+    del g
+    return res
+
+
 def run_oracle(inp: synth.LayerInputs, t0=None, force_bits=None, tiles=None, y_prev_f32=None):
     spec = inp.spec
     q = oracle.quantize(inp.as_f32("x_t"), inp.as_f32("x_prev"), spec.lb, spec.t0 if t0 is None else t0,
@@ -76,7 +107,9 @@ def tile_rows(T, tiles):
 
 
 def assert_quant_parity(g, q):
-    assert np.array_equal(g["codes"], q.codes), "codes differ"
+    """Every integer output of the quantizer; the codes only when they were dumped."""
+    if "codes" in g:
+        assert np.array_equal(g["codes"], q.codes), "codes differ"
     assert np.array_equal(g["bits"], q.bits), "bit widths differ"
     assert np.array_equal(g["fpot"], q.fpot), "FPoT differs"
     assert np.array_equal(g["g_ref"], q.g_ref), "g_ref differs"

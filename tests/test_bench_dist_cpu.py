@@ -4,7 +4,9 @@ The batch split needs no data exchange: each rank runs its own batch of the
 same workload, and the only collectives are the barrier around the timed region
 and the max of the ranks' times.  These tests run two processes and check
 that reduction, the whole-job throughput formula, the per-rank inputs (same
-shapes, different draws) and that the reference arm does nothing off rank 0.
+shapes, different draws), that the reference arm does nothing off rank 0, and
+that splitting one batch by token tiles across two ranks reproduces the whole
+batch's accumulators and Y_t bit for bit (the oracle on each half).
 """
 import os
 import socket
@@ -49,8 +51,21 @@ def _worker(rank, world, port, out):
                 steps = 1
                 warmup = 3
             ref = bench.run_reference(A(), rank, world)
+        # the batch split itself: each rank runs the oracle on its own whole
+        # 16-token tiles of one batch; together they must give the whole
+        # batch's Y_t (rows of Y depend only on the same rows of dX)
+        import oracle
+        from differential_quantized_gemm_b200 import synth
+        whole = synth.make_layer(2, 0, M=256)
+        T = whole.spec.M // 16
+        lo, hi = 16 * (T * rank // world), 16 * (T * (rank + 1) // world)
+        rows = slice(lo, hi)
+        _, acc, y = oracle.linear(whole.as_f32("x_t")[rows], whole.as_f32("x_prev")[rows],
+                                  whole.as_f32("y_prev")[rows], whole.w_q, whole.w_scale, whole.spec.lb)
+        parts = [None] * world
+        td.all_gather_object(parts, (lo, hi, acc, y))
         td.barrier()
-        out[rank] = (t, gathered, ref)
+        out[rank] = (t, gathered, ref, parts if rank == 0 else None)
     finally:
         td.destroy_process_group()
 
@@ -70,11 +85,21 @@ def test_two_gloo_ranks():
         res = dict(out)
     assert codes == [0, 0], codes
     for r in range(world):
-        t, gathered, ref = res[r]
+        t, gathered, ref, _ = res[r]
         assert t == pytest.approx(2.5)
         assert gathered[0][:3] == gathered[1][:3]
         assert gathered[0][3] != gathered[1][3]
         assert ref is None
+    # the shards, stacked in rank order, are the whole batch's result bit for bit
+    import oracle
+    from differential_quantized_gemm_b200 import synth
+    parts = res[0][3]
+    whole = synth.make_layer(2, 0, M=256)
+    _, acc, y = oracle.linear(whole.as_f32("x_t"), whole.as_f32("x_prev"), whole.as_f32("y_prev"), whole.w_q,
+                              whole.w_scale, whole.spec.lb)
+    assert [p[0] for p in parts] == [0, 128] and [p[1] for p in parts] == [128, 256]
+    assert np.array_equal(np.concatenate([p[2] for p in parts]), acc)
+    assert np.array_equal(np.concatenate([p[3] for p in parts]), y)
 
 
 def test_job_throughput_is_weak_scaling():

@@ -1,8 +1,10 @@
 """GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
 five synthetic workloads, at sizes the oracle finishes in seconds (several
-128-row blocks plus a ragged tail) and at the full sizes in the launch
-configuration the benchmark times (y_out = y_prev, x_prev refreshed), with
-accumulators and Y_t compared on sampled token tiles there.
+128-row blocks plus a ragged tail) and at the full sizes, compared in full:
+every code, bit width, FPoT, g_ref, record and int64 accumulator of every
+tile, and Y_t element by element, both with the debug dumps and in the
+launch the benchmark times (graph replay, y_out = y_prev, x_prev refreshed,
+no debug buffers).
 """
 import numpy as np
 import pytest
@@ -11,7 +13,8 @@ import torch
 import oracle
 from differential_quantized_gemm_b200 import synth
 
-from gpu_helpers import assert_quant_parity, assert_y_close, full_parity, run_gpu, run_oracle, tile_rows
+from gpu_helpers import (assert_quant_parity, assert_y_close, full_parity, run_gpu, run_gpu_bench_launch,
+                         run_oracle)
 
 pytestmark = pytest.mark.gpu
 
@@ -47,57 +50,84 @@ def test_small_parity(cfg, layer):
     assert exact > 0.999
 
 
-@pytest.mark.parametrize("cfg,layer", [(2, 0), (2, 1), (3, 0), (3, 1), (3, 2), (3, 3), (4, 0), (4, 1)],
-                         ids=lambda v: str(v))
-def test_full_size_sampled(cfg, layer):
-    """Full-size workload in the benchmark's launch configuration; every integer
-    stage compared in full, accumulators and Y_t on sampled tiles."""
+FULL_CASES = [(2, 0), (2, 1), (3, 0), (3, 1), (3, 2), (3, 3), (4, 0), (4, 1)]
+
+
+@pytest.mark.parametrize("cfg,layer", FULL_CASES, ids=lambda v: str(v))
+def test_full_size_compared_in_full(cfg, layer):
+    """Full-size workload, compared in full against one oracle run:
+    (a) the benchmark's own launch (graph replay, Y in place, x_prev refreshed,
+        no debug buffers): Y_t element by element and every integer section;
+    (b) the same call with the debug dumps: every code and every int64
+        accumulator of every tile."""
     inp = synth.make_layer(cfg, layer)
-    T = inp.spec.M // 16
-    rng = np.random.default_rng(cfg * 10 + layer)
-    tiles = np.unique(np.concatenate([[0, T - 1, T // 2], rng.choice(T, 13, replace=False)]))
+    q, acc, y = run_oracle(inp)
+    b = run_gpu_bench_launch(inp)
+    assert b["status"] == 0
+    assert_quant_parity(b, q)
+    assert_y_close(b["y"], y)
+    xp = b["x_prev_after"].cpu().view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(xp, inp.x_t), "x_prev refresh"
     g = run_gpu(inp)
-    q, acc, y = run_oracle(inp, tiles=tiles)
     assert g["status"] == 0
     assert_quant_parity(g, q)
-    rows = tile_rows(T, tiles)
-    assert np.array_equal(g["acc"][rows], acc[rows])
-    assert_y_close(g["y"][rows], y[rows])
+    assert np.array_equal(g["acc"], acc), "accumulators differ"
+    assert np.array_equal(g["y"], b["y"]), "debug dumps changed Y_t"
     assert (g["planes"] <= 2).any()
 
 
-def test_sweep_chain_with_caches():
-    """Timestep sweep: consecutive steps with caches carried on both sides
-    independently (the oracle chains its own outputs)."""
-    M = 512
+def _chain_parity(chain):
+    """Consecutive calls of one layer with caches carried on both sides
+    independently (the oracle chains its own outputs); everything compared."""
+    d = ws = yo = None
+    for inp in chain.steps():
+        if d is None:
+            g = run_gpu(inp)
+            d, ws = g["dev"], g["ws"]
+        else:  # the device caches carry over: only X_t changes
+            d["x_t"] = torch.from_numpy(inp.x_t).view(torch.bfloat16).cuda()
+            g = run_gpu(inp, dev_bufs=d, ws=ws)
+        q, acc, y = run_oracle(inp, y_prev_f32=yo)
+        assert g["status"] == 0
+        assert_quant_parity(g, q)
+        assert np.array_equal(g["acc"], acc), "accumulators differ"
+        assert_y_close(g["y"], y)
+        yo = y
+    return g, q
+
+
+def test_sweep_chain_small():
     for layer in (0, 1):
-        chain = synth.sweep_chain(layer, steps=[0, 1, 2, 24, 25, 49], M=M)
-        spec = chain.spec
-        d = None
-        yo = None
-        for inp in chain.steps():
-            if d is None:
-                g = run_gpu(inp)
-                d = g["dev"]
-                ws = g["ws"]
-            else:
-                # the device caches carry over: only X_t changes
-                d["x_t"] = torch.from_numpy(inp.x_t).view(torch.bfloat16).cuda()
-                g = run_gpu(inp, dev_bufs=d, ws=ws)
-            q, acc, y = run_oracle(inp, y_prev_f32=yo)
-            assert g["status"] == 0
-            assert_quant_parity(g, q)
-            assert np.array_equal(g["acc"], acc)
-            assert_y_close(g["y"], y)
-            yo = y
-        assert spec.K in (1152, 4608)
+        _chain_parity(synth.sweep_chain(layer, steps=[0, 1, 2, 24, 25, 49], M=512))
+
+
+# first and last layer of the 28-layer stack, both projections of each
+SWEEP_LAYERS = [(0, "l0_up"), (1, "l0_down"), (54, "l27_up"), (55, "l27_down")]
+
+
+@pytest.mark.parametrize("layer", [li for li, _ in SWEEP_LAYERS], ids=[n for _, n in SWEEP_LAYERS])
+def test_sweep_full_size(layer):
+    """The timestep sweep at its full size (8192 tokens): steps 0, 1, 24, 25
+    and 49 of the U-shaped schedule in a row, caches carried."""
+    _chain_parity(synth.sweep_chain(layer, steps=[0, 1, 24, 25, 49], M=8192))
 
 
 @pytest.mark.parametrize("force", [2, 8])
-def test_forced_extremes(force):
+def test_forced_extremes_small(force):
     inp = synth.make_layer(5, 0, step=10, force_bits=force, M=SMALL_M)
     g, q, acc, y, _ = full_parity(inp)
     assert (g["bits"] == force).all()
+
+
+@pytest.mark.parametrize("force", [2, 8])
+@pytest.mark.parametrize("layer", [0, 1], ids=["up", "down"])
+def test_forced_extremes_full_size(force, layer):
+    """The all-2-bit and all-8-bit runs of the sweep at 8192 tokens, compared in full."""
+    inp = synth.make_layer(5, layer, step=10, force_bits=force)
+    g, q, acc, y, _ = full_parity(inp)
+    assert (g["bits"] == force).all()
+    if force == 8:
+        assert (g["planes"] > 1).any(), "8-bit tiles should need more than one operand plane"
 
 
 def test_adversarial_uses_slice_stream_for_wide_tiles():

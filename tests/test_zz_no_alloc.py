@@ -6,10 +6,11 @@ static device array of the library instead of a caller-made workspace.
 
 The GPU test calls it through the C ABI twice in a row, with the caches
 carried from one call to the next, and checks each result against
-dstar_fmdq_linear with a workspace on separate copies of the same buffers,
-within the tolerance of the other parity tests.  It must pass in a fresh
-process (the first call sets up the array's device address) and after the
-other tests.  This file is named so that pytest collects it last.
+dstar_fmdq_linear with a workspace on separate copies of the same buffers:
+both run the same kernels, so Y_t must agree bit for bit.  It must pass in a
+fresh process (the first call in a context clears the array's status word)
+and after the other tests.  This file is named so that pytest collects it
+last.
 """
 from __future__ import annotations
 
@@ -75,6 +76,9 @@ def test_noalloc_matches_workspace_path_on_two_calls_in_a_row():
         y_r, y_a = dev_to_f32(y_ref), dev_to_f32(y_alt)
         assert np.isfinite(y_a).all()
         assert np.abs(y_r).max() > 0, "the reference output is all zero: the comparison would be empty"
+        # the same kernels on the same inputs: Y_t must agree bit for bit;
+        # assert_y_close runs first only for the error summary it prints
         assert_y_close(y_a, y_r)
+        assert torch.equal(y_alt, y_ref), f"call {call}: Y_t differs from the workspace path"
         # the caches the next call reads: X_{t-1} refreshed the same way
         assert torch.equal(alt["x_prev"], ref["x_prev"]), f"call {call}: x_prev refresh differs"
