@@ -3,9 +3,12 @@
 
 One step = one pass of the whole hot path over one batch: for every layer of
 the workload, the quantizer (K1) and the slice GEMM with its fused epilogue
-(K2, plus the slice-stream kernel for tiles that need it), through the C ABI.
-Default workload: the DiT-XL/2 256px FFN pair, batch 8 x 256 tokens,
-1152 -> 4608 -> 1152, bf16 activations, int8 weights.
+(K2), through the C ABI.  Headline workload: the Latte-like video DiT FFN,
+batch 4 x 16 frames x 256 tokens = 16384 tokens, 1152 -> 4608 -> 1152, bf16
+activations, int8 weights (the largest of the five workloads; it fits one
+GPU).  On one GPU the same line also carries the DiT-XL/2 256px FFN pair, the
+PixArt 1024px layer and the 28-layer x 50-step timestep sweep with its forced
+all-2-bit and all-8-bit runs (`per_config`, `sweep`).
 
 Metric: dense-equivalent int8 TOPS, sum over layers of 2*M*N*K per step / step
 time, with the quantizer's HBM GB/s and the slice GEMM's tensor throughput as
@@ -35,17 +38,25 @@ sys.path.insert(0, ROOT)
 METRIC = "FMDQ linear dense-equiv TOPS & % int8 tensor peak; quantizer GB/s vs HBM"
 INT8_PER_BF16 = 2.0  # nominal dense int8 : bf16 tensor throughput on B200 (4.5 : 2.25 PFLOP/s)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+HEADLINE_CONFIG = 4
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=4000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", type=int, default=2, help="workload (2: DiT-XL/2 FFN pair)")
+    ap.add_argument("--config", type=int, default=HEADLINE_CONFIG,
+                    help="headline workload (4: Latte video FFN; 2: DiT-XL/2 FFN pair; 3: PixArt layer)")
+    ap.add_argument("--extra-configs", default="2,3",
+                    help="further workloads measured on one GPU and reported under per_config ('' for none)")
+    ap.add_argument("--extra-steps", type=int, default=1200, help="timed steps of each extra workload")
+    ap.add_argument("--sweep-steps", type=int, default=50,
+                    help="steps of the 28-layer timestep sweep on one GPU (0 to skip)")
+    ap.add_argument("--extreme-reps", type=int, default=5, help="timed steps of each forced-width sweep run")
     ap.add_argument("--sets", type=int, default=3, help="rotating input sets (together larger than L2)")
-    ap.add_argument("--e2e-steps", type=int, default=300)
+    ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--xprev", choices=["swap", "copy"], default="copy",
                     help="swap: X_t and X_{t-1} stay resident and trade buffers each step (no refresh copy); "
                          "copy: the quantizer copies X_t into one x_prev cache")
@@ -54,7 +65,7 @@ def parse():
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--mode", choices=["graph", "eager"], default="graph",
                     help="graph: each step replays a captured CUDA graph; eager: C-ABI calls per step")
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
 # ----------------------------------------------------------------- peaks
@@ -77,7 +88,7 @@ def kernel_source_sha():
 
 def load_traffic():
     """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel sources (else None)."""
+    on the current kernel sources (else {})."""
     p = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     if not os.path.exists(p):
         return {}
@@ -93,6 +104,16 @@ def load_traffic():
             except ValueError:
                 pass
     return out if sha == kernel_source_sha() else {}
+
+
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.lower().startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
 # -------------------------------------------------------------- clocks
@@ -178,6 +199,10 @@ class Layer:
         self.m_y = nat.mat(self.y_prev)
         self.m_w = nat.mat(self.w_q)
         self.ws_ptr = ctypes.c_void_p(self.w_scale.data_ptr())
+
+    def tensors(self):
+        return [t for t in (self.x_a, self.x_b, self.x_prev, self.y_prev, self.w_q, self.w_scale, self.ws.buf)
+                if t is not None]
 
     def xp(self, parity):
         """X_{t-1}: the other buffer (swap), or the cache (copy)."""
@@ -269,12 +294,51 @@ def algorithmic_k2(spec, ws_sections, out_bytes=2):
     return dense_ops, issued, bytes_, int((planes > 2).sum())
 
 
+def kernel_rows(inputs, stats, k1_ms, k2_ms, peaks):
+    """Per launch: time, achieved rate and fraction of the bound that applies
+    (HBM for the quantizer; for the slice GEMM the larger of tensor and HBM
+    time at the measured peaks)."""
+    hbm = peaks["hbm_gbs"]
+    i8 = peaks["bf16_tflops"] * INT8_PER_BF16
+    kern = []
+    for li, stt in enumerate(stats):
+        name = inputs[li].spec.name
+        kern.append(dict(kernel="quantize", layer=name, ms=k1_ms[li], bound="hbm",
+                         achieved=stt["k1_bytes"] / (k1_ms[li] * 1e-3) / 1e9, peak=hbm, unit="GB/s",
+                         algorithmic=stt["k1_bytes"]))
+        if stt["k2_issued"] / (i8 * 1e12) >= stt["k2_bytes"] / (hbm * 1e9):
+            kern.append(dict(kernel="slice_gemm", layer=name, ms=k2_ms[li], bound="tensor",
+                             achieved=stt["k2_dense"] / (k2_ms[li] * 1e-3) / 1e12, peak=i8, unit="TOPS",
+                             algorithmic=stt["k2_dense"]))
+        else:
+            kern.append(dict(kernel="slice_gemm", layer=name, ms=k2_ms[li], bound="hbm",
+                             achieved=stt["k2_bytes"] / (k2_ms[li] * 1e-3) / 1e9, peak=hbm, unit="GB/s",
+                             algorithmic=stt["k2_bytes"]))
+    for k in kern:
+        k["frac"] = k["achieved"] / k["peak"]
+    return kern
+
+
+def roofline_of(kern, peak_src):
+    dom = max(kern, key=lambda k: k["ms"])
+    traffic = load_traffic().get(f"{dom['kernel']}.{dom['layer']}.dram_bytes")
+    return {"bound": dom["bound"], "achieved": dom["achieved"], "peak": dom["peak"], "unit": dom["unit"],
+            "frac": dom["frac"], "traffic": traffic, "kernel": f"{dom['kernel']} ({dom['layer']})",
+            "peak_source": (f"{peak_src} hbm_gbs" if dom["bound"] == "hbm" else
+                            f"{peak_src} bf16_tflops x {INT8_PER_BF16} (nominal int8:bf16)")}
+
+
+def rounded(kern):
+    return [{k: (round(v, 4) if isinstance(v, float) else v) for k, v in kk.items()} for kk in kern]
+
+
 # ------------------------------------------------------------ oracle timing
 
-def oracle_step(inputs, nt: int, frac: float) -> float:
+def oracle_step(inputs, nt: int, frac: float, stage_s=None) -> float:
     """One oracle pass over the first nt token tiles of every layer and the
     first `frac` of its output channels (quantize, int64 accumulation, fp32
-    epilogue); returns the dense-equivalent ops it covered."""
+    epilogue); returns the dense-equivalent ops it covered and adds each
+    stage's seconds to stage_s."""
     import numpy as np
     import oracle
 
@@ -283,10 +347,21 @@ def oracle_step(inputs, nt: int, frac: float) -> float:
         s = inp.spec
         rows = slice(0, 16 * nt)
         ncols = s.N if frac >= 1.0 else max(16, int(s.N * frac) // 16 * 16)
-        q = oracle.quantize(inp.as_f32("x_t")[rows], inp.as_f32("x_prev")[rows], s.lb, s.t0, s.force_bits)
-        acc = oracle.acc_direct(q, np.ascontiguousarray(inp.w_q[:ncols]))
-        oracle.epilogue_f32(acc, q.g_ref, s.lb, np.ascontiguousarray(inp.w_scale[:ncols]),
-                            np.ascontiguousarray(inp.as_f32("y_prev")[rows, :ncols]), s.dtype == "bf16")
+        xt, xp = inp.as_f32("x_t")[rows], inp.as_f32("x_prev")[rows]
+        w = np.ascontiguousarray(inp.w_q[:ncols])
+        ws = np.ascontiguousarray(inp.w_scale[:ncols])
+        yp = np.ascontiguousarray(inp.as_f32("y_prev")[rows, :ncols])
+        t0 = time.perf_counter()
+        q = oracle.quantize(xt, xp, s.lb, s.t0, s.force_bits)
+        t1 = time.perf_counter()
+        acc = oracle.acc_direct(q, w)
+        t2 = time.perf_counter()
+        oracle.epilogue_f32(acc, q.g_ref, s.lb, ws, yp, s.dtype == "bf16")
+        t3 = time.perf_counter()
+        if stage_s is not None:
+            stage_s["quantize"] += t1 - t0
+            stage_s["gemm"] += t2 - t1
+            stage_s["epilogue"] += t3 - t2
         ops += 2.0 * 16 * nt * ncols * s.K
     return ops
 
@@ -309,24 +384,42 @@ def oracle_calibrate(inputs, per_step: float):
     return nt, max(per_step / el, 1e-3), min(threads, nt), T
 
 
-def oracle_sample_time(inputs, seconds: float):
-    """Time the CPU oracle on the whole workload (every token tile of every
-    layer), repeated until about `seconds`; returns (ops, elapsed,
-    description, threads used)."""
+def oracle_baseline(inputs, seconds: float):
+    """The CPU oracle as it stands on the host cores: (a) all threads, on the
+    first token tiles of every layer, as many as take about `seconds` (the
+    whole workload when it fits), timed per stage; (b) one thread on a small
+    sample.  Returns the cpu_baseline entry of the JSON line."""
     import oracle
 
     T = min(inp.spec.M // 16 for inp in inputs)
-    oracle_step(inputs, min(T, oracle.n_threads()), 1.0)  # load and warm
-    ops = el = 0.0
-    reps = 0
-    while reps == 0 or (el < seconds and reps < 100):
+    threads = oracle.n_threads()
+    oracle_step(inputs, min(T, threads), 1.0)  # load and warm
+    t0 = time.perf_counter()
+    oracle_step(inputs, min(T, threads), 1.0)
+    probe = time.perf_counter() - t0
+    nt = max(min(T, threads), min(T, int(min(T, threads) * seconds / max(probe, 1e-6))))
+    stages = {"quantize": 0.0, "gemm": 0.0, "epilogue": 0.0}
+    t0 = time.perf_counter()
+    ops = oracle_step(inputs, nt, 1.0, stages)
+    el = time.perf_counter() - t0
+    # one thread: a few token tiles of every layer
+    nt1 = max(1, min(T, 4))
+    stages1 = {"quantize": 0.0, "gemm": 0.0, "epilogue": 0.0}
+    oracle.set_threads(1)
+    try:
         t0 = time.perf_counter()
-        ops += oracle_step(inputs, T, 1.0)
-        el += time.perf_counter() - t0
-        reps += 1
-    desc = (f"the whole workload ({T} token tiles of every layer) {reps} time(s): quantize, direct int64 "
-            f"accumulation, fp32 epilogue")
-    return ops, el, desc, min(oracle.n_threads(), T)
+        ops1 = oracle_step(inputs, nt1, 1.0, stages1)
+        el1 = time.perf_counter() - t0
+    finally:
+        oracle.set_threads(threads)
+    sample = (f"{'the whole workload' if nt == T else f'the first {nt} of {T} token tiles of every layer'} "
+              f"(quantize, direct int64 accumulation, fp32 epilogue) once, {threads} threads")
+    return {"value": ops / el / 1e12, "unit": "TOPS", "cores": min(threads, nt), "kind": "oracle",
+            "sample": sample, "seconds": el, "cpu_model": cpu_model(), "nproc": os.cpu_count(),
+            "stages_s": {k: round(v, 4) for k, v in stages.items()},
+            "single_thread": {"value": ops1 / el1 / 1e12, "unit": "TOPS", "cores": 1, "seconds": el1,
+                              "sample": f"the first {nt1} token tiles of every layer",
+                              "stages_s": {k: round(v, 4) for k, v in stages1.items()}}}
 
 
 # ----------------------------------------------------------------- arms
@@ -349,25 +442,415 @@ def run_reference(args, rank, world):
     val = ops / el / 1e12
     sample = (f"{nt} of {T} token tiles x {frac:.3f} of the output channels of every layer per step "
               f"(oracle: quantize, int64 accumulation, fp32 epilogue)")
-    from differential_quantized_gemm_b200 import synth
     line = {
         "impl": "reference", "metric": METRIC, "value": val, "unit": "TOPS", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64", "data": "synthetic",
         "config": workload_config(args.config, inputs, world, args.xprev),
-        "cpu_baseline": {"value": val, "unit": "TOPS", "cores": threads, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": val, "unit": "TOPS", "cores": threads, "kind": "oracle", "sample": sample,
+                         "cpu_model": cpu_model()},
         "e2e": {"value": val, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
 
+class ConfigBench:
+    """One workload on this GPU: rotating input sets, CUDA graphs of the step
+    (one dstar_fmdq_linear call per layer) and of the same step split into its
+    two stages with event nodes between the kernels."""
+
+    def __init__(self, cfg, args, rank, torch, nat, L):
+        import numpy as np
+        self.cfg, self.args, self.torch, self.nat, self.L = cfg, args, torch, nat, L
+        self.inputs = workload_inputs(cfg, rank)
+        self.swap = args.xprev == "swap"
+        self.nsets = args.sets
+        self.sets = [[Layer(inp, torch, nat, self.swap) for inp in self.inputs] for _ in range(self.nsets)]
+        self.nlayers = len(self.inputs)
+        self.stream = torch.cuda.current_stream()
+        self.sh = ctypes.c_void_p(self.stream.cuda_stream)
+        self.uses = [0] * self.nsets
+        self.graphs = self.prof_graphs = self.cycle = self.gev = None
+        self.np = np
+
+    def set_mb(self):
+        return sum(t.numel() * t.element_size() for lay in self.sets[0] for t in lay.tensors()) / 1e6
+
+    def step(self, s):
+        r = s % self.nsets
+        parity = self.uses[r] & 1
+        self.uses[r] += 1
+        for lay in self.sets[r]:
+            if lay.linear(self.L, parity, self.sh):
+                raise RuntimeError(self.L.dstar_fmdq_last_error().decode())
+
+    def warm_and_stats(self, warmup):
+        """Untimed warm-up steps, then the workload statistics of one call per layer."""
+        np = self.np
+        for s in range(max(warmup, 3)):
+            self.step(s)
+        self.torch.cuda.synchronize()
+        stats = []
+        for lay in self.sets[0]:
+            sec = lay.ws.sections(lay.spec.M, lay.spec.K)
+            b1 = algorithmic_k1_bytes(lay.spec, sec, refresh=not self.swap)
+            dense, issued, b2, nfall = algorithmic_k2(lay.spec, sec)
+            bits = sec["bits"].cpu().numpy()
+            planes = sec["planes"].cpu().numpy()
+            # the paper's unit of MPU work: one 2-bit slice of 16 tokens against one weight
+            slice_macs = 16 * int(sec["count"].cpu().numpy().astype(np.int64).sum()) * lay.spec.N
+            stats.append(dict(k1_bytes=b1, k2_dense=dense, k2_issued=issued, k2_bytes=b2, fallback_tiles=nfall,
+                              slice_macs=slice_macs, bits_avg=float(bits.mean()),
+                              bit_hist=[float((bits == b).mean()) for b in (2, 4, 6, 8)],
+                              planes_hist=[int((planes == p).sum()) for p in (1, 2)] + [int((planes > 2).sum())]))
+        self.stats = stats
+        return stats
+
+    def capture(self):
+        """Graphs: per (set, parity) the step and its split form, and one graph
+        holding a whole cycle of steps (every set with both X_t)."""
+        torch, L = self.torch, self.L
+        from cuda.bindings import runtime as rt
+        self.rt = rt
+
+        def ext_event():
+            err, e = rt.cudaEventCreate()
+            assert err == rt.cudaError_t.cudaSuccess
+            return e
+
+        kinds = [(r, par) for par in (0, 1) for r in range(self.nsets)]
+        self.gev = [[[ext_event() for _ in range(3)] for _ in range(self.nlayers)] for _ in kinds]
+        self.graphs, self.prof_graphs = [], []
+        cap_stream = torch.cuda.Stream()
+        for gi, (r, par) in enumerate(kinds):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap_stream):
+                csh = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+                for lay in self.sets[r]:
+                    if lay.linear(L, par, csh):
+                        raise RuntimeError(L.dstar_fmdq_last_error().decode())
+            self.graphs.append(g)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap_stream):
+                cs = torch.cuda.current_stream()
+                csh = ctypes.c_void_p(cs.cuda_stream)
+                rsh = rt.cudaStream_t(init_value=cs.cuda_stream)
+                for li, lay in enumerate(self.sets[r]):
+                    rt.cudaEventRecordWithFlags(self.gev[gi][li][0], rsh, rt.cudaEventRecordExternal)
+                    rc = lay.quantize(L, par, csh)
+                    rt.cudaEventRecordWithFlags(self.gev[gi][li][1], rsh, rt.cudaEventRecordExternal)
+                    rc |= lay.gemm(L, csh)
+                    rt.cudaEventRecordWithFlags(self.gev[gi][li][2], rsh, rt.cudaEventRecordExternal)
+                    if rc:
+                        raise RuntimeError(L.dstar_fmdq_last_error().decode())
+            self.prof_graphs.append(g)
+        self.cycle = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.cycle, stream=cap_stream):
+            csh = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+            for r, par in kinds:
+                for lay in self.sets[r]:
+                    if lay.linear(L, par, csh):
+                        raise RuntimeError(L.dstar_fmdq_last_error().decode())
+        for g in self.graphs:  # warm the graphs (keeps every set's parity alternating)
+            g.replay()
+        self.cycle.replay()
+        torch.cuda.synchronize()
+
+    def replay(self, K):
+        """K steps: whole cycles, then the first steps of one."""
+        n = len(self.graphs)
+        for _ in range(K // n):
+            self.cycle.replay()
+        for s in range(K % n):
+            self.graphs[s].replay()
+
+    def split_times(self, K):
+        """Mean per-kernel times from replays of the split step (event nodes)."""
+        torch, rt = self.torch, self.rt
+        n = len(self.graphs)
+        kp = max(n, min(K, 1200) // n * n)
+        torch.cuda.synchronize()
+        for s in range(kp):
+            self.prof_graphs[s % n].replay()
+        torch.cuda.synchronize()
+
+        def el(a, b):
+            err, v = rt.cudaEventElapsedTime(a, b)
+            assert err == rt.cudaError_t.cudaSuccess
+            return v
+        k1 = [statistics.fmean(el(self.gev[g][li][0], self.gev[g][li][1]) for g in range(n))
+              for li in range(self.nlayers)]
+        k2 = [statistics.fmean(el(self.gev[g][li][1], self.gev[g][li][2]) for g in range(n))
+              for li in range(self.nlayers)]
+        return k1, k2
+
+    def timed(self, K, dist=False, clocks_id=None, clocks_on=True):
+        """Device time of K steps (CUDA events, barrier + synchronize around)."""
+        torch = self.torch
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        clocks = ClockSampler(clocks_id, clocks_on) if clocks_id is not None else None
+        if clocks is not None:
+            time.sleep(0.3)
+        if dist:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        t_wall0 = time.time()
+        ev0.record(self.stream)
+        if self.graphs:
+            self.replay(K)
+        else:
+            for s in range(K):
+                self.step(s)
+        ev1.record(self.stream)
+        torch.cuda.synchronize()
+        t_wall1 = time.time()
+        if dist:
+            torch.distributed.barrier()
+        clock_summary = None
+        if clocks is not None:
+            time.sleep(0.2)
+            clocks.stop()
+            clock_summary = clocks.summary(t_wall0, t_wall1)
+        return ev0.elapsed_time(ev1), clock_summary
+
+    def e2e(self, steps, world, dense_step):
+        """The same metric through the public API with host buffers: per step
+        X_t of every layer copied in from pinned host memory, the calls, Y_t
+        of every layer copied back.  Copies run on their own streams; a set's
+        landing buffers are rewritten only after that set's previous compute
+        finished, and its Y cache updated only after that set's previous
+        read-back finished."""
+        torch, L, nat = self.torch, self.L, self.nat
+        sets, swap, stream, sh = self.sets, self.swap, self.stream, self.sh
+        host_x = [[[torch.empty_like(lay.x_a, device="cpu").pin_memory() for _ in range(2)] for lay in st]
+                  for st in sets]
+        host_y = [[torch.empty_like(lay.y_prev, device="cpu").pin_memory() for lay in st] for st in sets]
+        for r, st in enumerate(sets):
+            for li, lay in enumerate(st):
+                host_x[r][li][0].copy_(lay.x_a.cpu())
+                host_x[r][li][1].copy_(lay.x_b.cpu())
+        h2d = sum(lay.x_a.numel() * lay.x_a.element_size() for lay in sets[0])
+        d2h = sum(lay.y_prev.numel() * lay.y_prev.element_size() for lay in sets[0])
+        # device landing buffers: one per parity in swap mode (the other
+        # parity's buffer holds X_{t-1}), else one
+        land = [[[lay.x_a.clone(), lay.x_b.clone()] if swap else [torch.empty_like(lay.x_a)] for lay in st]
+                for st in sets]
+        land_m = [[[nat.mat(t) for t in bufs] for bufs in row] for row in land]
+        h2d_s, d2h_s = torch.cuda.Stream(), torch.cuda.Stream()
+        last_c = [None] * self.nsets  # per set: its last compute, its last read-back
+        last_d = [None] * self.nsets
+
+        def step_e2e(s):
+            r = s % self.nsets
+            parity = self.uses[r] & 1
+            self.uses[r] += 1
+            slot = parity if swap else 0
+            if last_c[r] is not None:
+                h2d_s.wait_event(last_c[r])
+            with torch.cuda.stream(h2d_s):
+                for li in range(len(sets[r])):
+                    land[r][li][slot].copy_(host_x[r][li][parity], non_blocking=True)
+            ev_h = torch.cuda.Event()
+            ev_h.record(h2d_s)
+            stream.wait_event(ev_h)
+            if last_d[r] is not None:
+                stream.wait_event(last_d[r])
+            for li, lay in enumerate(sets[r]):
+                mp = land_m[r][li][1 - parity] if swap else lay.m_xp
+                rc = L.dstar_fmdq_linear(ctypes.byref(land_m[r][li][slot]), ctypes.byref(mp), ctypes.byref(lay.m_y),
+                                         ctypes.byref(lay.m_w), lay.ws_ptr, lay.base, ctypes.byref(lay.cfg),
+                                         ctypes.byref(lay.m_y), sh)
+                if rc:
+                    raise RuntimeError(L.dstar_fmdq_last_error().decode())
+            ev_c = torch.cuda.Event()
+            ev_c.record(stream)
+            last_c[r] = ev_c
+            d2h_s.wait_event(ev_c)
+            with torch.cuda.stream(d2h_s):
+                for li, lay in enumerate(sets[r]):
+                    host_y[r][li].copy_(lay.y_prev, non_blocking=True)
+            ev_d = torch.cuda.Event()
+            ev_d.record(d2h_s)
+            last_d[r] = ev_d
+
+        for s in range(3):
+            step_e2e(s)
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(h2d_s)
+        for s in range(steps):
+            step_e2e(s)
+        stream.wait_stream(h2d_s)
+        stream.wait_stream(d2h_s)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ems = max_over_ranks(e0.elapsed_time(e1), "cuda")
+        return {"value": job_tops(world, dense_step, ems / steps), "unit": "TOPS", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": ems / steps,
+                "path": "pinned host X_t -> device, dstar_fmdq_linear per layer, Y_t -> pinned host; copies on "
+                        "their own streams overlap the neighbouring steps' compute"}
+
+    def status(self):
+        st = 0
+        for row in self.sets:
+            for lay in row:
+                st |= self.nat.status(lay.ws)
+        return st
+
+    def close(self):
+        self.graphs = self.prof_graphs = self.cycle = None
+        self.sets = None
+        self.torch.cuda.synchronize()
+        self.torch.cuda.empty_cache()
+
+
+def measure_extra(cfg, args, torch, nat, L, peaks, peak_src):
+    """A further workload on this GPU: step time, per-kernel times, roofline
+    and workload statistics (no e2e, no clocks)."""
+    from differential_quantized_gemm_b200 import synth
+    cb = ConfigBench(cfg, args, 0, torch, nat, L)
+    stats = cb.warm_and_stats(args.warmup)
+    cb.capture()
+    ms, _ = cb.timed(args.extra_steps)
+    k1, k2 = cb.split_times(args.extra_steps)
+    st = cb.status()
+    if st:
+        raise RuntimeError(f"device status {st} after workload {cfg}")
+    dense = sum(s["k2_dense"] for s in stats)
+    kern = kernel_rows(cb.inputs, stats, k1, k2, peaks)
+    out = {"workload": synth.CONFIG_NAMES[cfg], "value": job_tops(1, dense, ms / args.extra_steps), "unit": "TOPS",
+           "ms_per_step": ms / args.extra_steps, "steps": args.extra_steps,
+           "layers": [f"{i.spec.name} M={i.spec.M} K={i.spec.K} N={i.spec.N}" for i in cb.inputs],
+           "roofline": roofline_of(kern, peak_src), "kernels": rounded(kern),
+           "workload_stats": [{k: v for k, v in s.items() if k in ("bits_avg", "bit_hist", "planes_hist",
+                                                                 "fallback_tiles", "slice_macs")} for s in stats]}
+    cb.close()
+    return out
+
+
+def measure_sweep(args, torch, nat, L):
+    """The 28-layer DiT-XL stack over the timestep sweep: 50 steps with every
+    layer's caches carried from step to step (X_t = X_{t-1} + sigma_t N(0, 1),
+    sigma_t U-shaped), then the forced all-2-bit and all-8-bit runs at
+    sigma 0.03.  Before each step (untimed) the new X_t of all 56 calls is
+    drawn on the device from a seeded generator; the step itself (56
+    dstar_fmdq_linear calls replayed from one CUDA graph) is timed with events."""
+    from differential_quantized_gemm_b200 import synth
+    specs = synth.config_layers(5)
+    nl = len(specs)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(5)
+    xs, xn, ys, wq, wsc, wss, cfgs = [], [], [], [], [], [], {0: [], 2: [], 8: []}
+    for li, sp in enumerate(specs):
+        w, sc = synth.layer_weights(5, li)
+        wq.append(torch.from_numpy(w).cuda())
+        wsc.append(torch.from_numpy(sc).cuda())
+        x0 = torch.randn(sp.M, sp.K, generator=gen, device="cuda").to(torch.bfloat16)
+        xs.append(x0)                         # x_prev cache, refreshed by the quantizer
+        xn.append(torch.empty_like(x0))      # X_t of the step
+        # step-0 dense initialisation of the cached output (not timed): Y = X W_deq
+        wdeq = wq[-1].float().t() * wsc[-1][None, :]
+        ys.append((x0.float() @ wdeq).to(torch.bfloat16))
+        ws = nat.Workspace(sp.M, sp.K)
+        wss.append(ws)
+        for fb in cfgs:
+            cfgs[fb].append(nat.TileCfg(16, sp.t0, fb, 0, ctypes.c_void_p(ws.ptr), ws.nbytes, None, None))
+    m_xn = [nat.mat(t) for t in xn]
+    m_xs = [nat.mat(t) for t in xs]
+    m_y = [nat.mat(t) for t in ys]
+    m_w = [nat.mat(t) for t in wq]
+    base = 2.0 ** specs[0].lb
+    zbuf = torch.empty(max(sp.M * sp.K for sp in specs), device="cuda")
+
+    def draw(sigma):
+        for li, sp in enumerate(specs):
+            z = zbuf[:sp.M * sp.K].view(sp.M, sp.K)
+            torch.randn(sp.M, sp.K, generator=gen, out=z)
+            xn[li].copy_((xs[li].float() + sigma * z).to(torch.bfloat16))
+
+    graphs = {}
+    cap = torch.cuda.Stream()
+    for fb in cfgs:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            csh = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+            for li in range(nl):
+                rc = L.dstar_fmdq_linear(ctypes.byref(m_xn[li]), ctypes.byref(m_xs[li]), ctypes.byref(m_y[li]),
+                                         ctypes.byref(m_w[li]), ctypes.c_void_p(wsc[li].data_ptr()), base,
+                                         ctypes.byref(cfgs[fb][li]), ctypes.byref(m_y[li]), csh)
+                if rc:
+                    raise RuntimeError(L.dstar_fmdq_last_error().decode())
+        graphs[fb] = g
+    dense_step = sum(2.0 * sp.M * sp.N * sp.K for sp in specs)
+    stream = torch.cuda.current_stream()
+
+    def layer_stats():
+        bits_sum = torch.zeros((), dtype=torch.float64, device="cuda")
+        n = 0
+        ph = torch.zeros(3, dtype=torch.int64, device="cuda")
+        for li, sp in enumerate(specs):
+            sec = wss[li].sections(sp.M, sp.K)
+            bits_sum += sec["bits"].double().sum()
+            n += sec["bits"].numel()
+            pl = sec["planes"].long()
+            ph += torch.stack([(pl == 1).sum(), (pl == 2).sum(), (pl > 2).sum()])
+        return bits_sum, n, ph
+
+    def run(fb, sigma_of, nsteps):
+        ms, bits, planes = [], [], []
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nsteps)]
+        pend = []
+        for t in range(nsteps):
+            draw(sigma_of(t))
+            ev[t][0].record(stream)
+            graphs[fb].replay()
+            ev[t][1].record(stream)
+            pend.append(layer_stats())
+        torch.cuda.synchronize()
+        for t in range(nsteps):
+            ms.append(ev[t][0].elapsed_time(ev[t][1]))
+            bsum, n, ph = pend[t]
+            bits.append(float(bsum.item()) / n)
+            planes.append([int(v) for v in ph.cpu()])
+        return ms, bits, planes
+
+    draw(synth.sweep_sigma(0))  # warm the graphs on a throw-away step of each kind (caches advance)
+    for fb in cfgs:
+        graphs[fb].replay()
+    torch.cuda.synchronize()
+    steps = args.sweep_steps
+    ms, bits, planes = run(0, synth.sweep_sigma, steps)
+    out = {"workload": synth.CONFIG_NAMES[5], "layers": nl, "M": specs[0].M, "steps": steps,
+           "timing": "each step: 56 dstar_fmdq_linear calls replayed from one CUDA graph, CUDA events around "
+                     "it; the step's X_t are drawn on the device before it (untimed)",
+           "ms_per_step": [round(v, 4) for v in ms], "ms_per_step_mean": statistics.fmean(ms),
+           "value": dense_step / (statistics.fmean(ms) * 1e-3) / 1e12, "unit": "TOPS",
+           "bits_avg_per_step": [round(b, 3) for b in bits],
+           "planes_hist_per_step": planes, "fallback_tiles_total": int(sum(p[2] for p in planes))}
+    for fb, key in ((2, "forced_2bit"), (8, "forced_8bit")):
+        ms_f, bits_f, planes_f = run(fb, lambda t: 0.03, args.extreme_reps)
+        out[key] = {"ms_per_step_mean": statistics.fmean(ms_f),
+                    "value": dense_step / (statistics.fmean(ms_f) * 1e-3) / 1e12, "unit": "TOPS",
+                    "bits_avg": bits_f[-1], "planes_hist": planes_f[-1], "fallback_tiles": planes_f[-1][2],
+                    "vs_adaptive_mean_step": statistics.fmean(ms_f) / statistics.fmean(ms), "reps": args.extreme_reps}
+    st = 0
+    for ws in wss:
+        st |= nat.status(ws)
+    if st:
+        raise RuntimeError(f"device status {st} after the sweep")
+    del graphs
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args, rank, world, local_rank):
-    import numpy as np
     import torch
 
     from differential_quantized_gemm_b200 import _native as nat
     from differential_quantized_gemm_b200 import build as cuda_build
-    from differential_quantized_gemm_b200 import synth
 
     if rank == 0:
         cuda_build.build()
@@ -376,281 +859,66 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     L = nat.lib()
     dist = world > 1
+    peaks, peak_src = load_peaks()
 
-    inputs = workload_inputs(args.config, rank)
-    swap = args.xprev == "swap"
-    sets = [[Layer(inp, torch, nat, swap) for inp in inputs] for _ in range(args.sets)]
-    nlayers = len(inputs)
-    stream = torch.cuda.current_stream()
-    sh = ctypes.c_void_p(stream.cuda_stream)
-    uses = [0] * args.sets
-
-    def step(s, evs=None):
-        r = s % args.sets
-        parity = uses[r] & 1
-        uses[r] += 1
-        for li, lay in enumerate(sets[r]):
-            if evs is not None:
-                evs[li][0].record(stream)
-            rc = lay.quantize(L, parity, sh)
-            if evs is not None:
-                evs[li][1].record(stream)
-            rc |= lay.gemm(L, sh)
-            if evs is not None:
-                evs[li][2].record(stream)
-            if rc:
-                raise RuntimeError(L.dstar_fmdq_last_error().decode())
-
-    # warm-up (untimed) and the workload statistics of one call per layer
-    for s in range(max(args.warmup, 3)):
-        step(s)
-    torch.cuda.synchronize()
-    stats = []
-    for lay in sets[0]:
-        sec = lay.ws.sections(lay.spec.M, lay.spec.K)
-        b1 = algorithmic_k1_bytes(lay.spec, sec, refresh=not swap)
-        dense, issued, b2, nfall = algorithmic_k2(lay.spec, sec)
-        bits = sec["bits"].cpu().numpy()
-        planes = sec["planes"].cpu().numpy()
-        # the paper's unit of MPU work: one 2-bit slice of 16 tokens against one weight
-        slice_macs = 16 * int(sec["count"].cpu().numpy().astype(np.int64).sum()) * lay.spec.N
-        stats.append(dict(k1_bytes=b1, k2_dense=dense, k2_issued=issued, k2_bytes=b2, fallback_tiles=nfall,
-                          slice_macs=slice_macs,
-                          bits_avg=float(bits.mean()), bit_hist=[float((bits == b).mean()) for b in (2, 4, 6, 8)],
-                          planes_hist=[int((planes == p).sum()) for p in (1, 2)] + [int((planes > 2).sum())]))
-
-    # timed region
+    cb = ConfigBench(args.config, args, rank, torch, nat, L)
+    stats = cb.warm_and_stats(args.warmup)
     K = args.steps
-    graphs, gev = None, None
     if args.mode == "graph":
-        # one graph per (input set, parity); each holds the step's launches and
-        # external event-record nodes between them (per-kernel times)
-        from cuda.bindings import runtime as rt
-
-        def ext_event():
-            err, e = rt.cudaEventCreate()
-            assert err == rt.cudaError_t.cudaSuccess
-            return e
-
-        kinds = [(r, par) for par in (0, 1) for r in range(args.sets)]
-        gev = [[[ext_event() for _ in range(3)] for _ in range(nlayers)] for _ in kinds]
-        graphs, prof_graphs = [], []
-        cap_stream = torch.cuda.Stream()
-        for gi, (r, par) in enumerate(kinds):
-            # the step as a user runs it: one dstar_fmdq_linear call per layer
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=cap_stream):
-                csh = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-                for lay in sets[r]:
-                    if lay.linear(L, par, csh):
-                        raise RuntimeError(L.dstar_fmdq_last_error().decode())
-            graphs.append(g)
-            # the same step split into its two stages with event nodes between the kernels
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=cap_stream):
-                cs = torch.cuda.current_stream()
-                csh = ctypes.c_void_p(cs.cuda_stream)
-                rsh = rt.cudaStream_t(init_value=cs.cuda_stream)
-                for li, lay in enumerate(sets[r]):
-                    rt.cudaEventRecordWithFlags(gev[gi][li][0], rsh, rt.cudaEventRecordExternal)
-                    rc = lay.quantize(L, par, csh)
-                    rt.cudaEventRecordWithFlags(gev[gi][li][1], rsh, rt.cudaEventRecordExternal)
-                    rc |= lay.gemm(L, csh)
-                    rt.cudaEventRecordWithFlags(gev[gi][li][2], rsh, rt.cudaEventRecordExternal)
-                    if rc:
-                        raise RuntimeError(L.dstar_fmdq_last_error().decode())
-            prof_graphs.append(g)
-        # the whole cycle of steps in one graph: a replay launches it once, so
-        # consecutive steps follow each other without a graph launch between them
-        cycle = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(cycle, stream=cap_stream):
-            csh = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-            for r, par in kinds:
-                for lay in sets[r]:
-                    if lay.linear(L, par, csh):
-                        raise RuntimeError(L.dstar_fmdq_last_error().decode())
-        for g in graphs:  # warm the graphs (keeps every set's parity alternating)
-            g.replay()
-        cycle.replay()
-        torch.cuda.synchronize()
-    evs = None if graphs else \
-        [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(nlayers)] for _ in range(K)]
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        cb.capture()
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
     smi_id = vis.split(",")[local_rank] if vis else str(torch.cuda.current_device())
-    clocks = ClockSampler(smi_id, not args.no_clocks)
-    time.sleep(0.3)
-    if dist:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    t_wall0 = time.time()
-    ev0.record(stream)
-    if graphs:  # step s runs graph s % len(graphs): whole cycles, then the first steps of one
-        for _ in range(K // len(graphs)):
-            cycle.replay()
-        for s in range(K % len(graphs)):
-            graphs[s].replay()
-    else:
+    ms, clocks = cb.timed(K, dist, smi_id, not args.no_clocks)
+    if cb.graphs:
+        k1_ms, k2_ms = cb.split_times(K)
+    else:  # eager: one more pass with events around each stage
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(cb.nlayers)]
+        k1_ms, k2_ms = [0.0] * cb.nlayers, [0.0] * cb.nlayers
         for s in range(K):
-            step(s, evs[s])
-    ev1.record(stream)
-    torch.cuda.synchronize()
-    t_wall1 = time.time()
-    if graphs:  # continue every set's X_t alternation after the replays (both regions)
-        for s in range(K + max(len(graphs), min(K, 1200) // len(graphs) * len(graphs))):
-            gi = s % len(graphs)
-            uses[gi % args.sets] = gi // args.sets + 1
-    if dist:
-        torch.distributed.barrier()
-    time.sleep(0.2)
-    clocks.stop()
-    ms = ev0.elapsed_time(ev1)
-    if graphs:
-        # per-kernel times: a second timed region of the split step, continuing
-        # every set's X_t alternation; the event nodes hold each graph's last replay
-        kp = max(len(graphs), min(K, 1200) // len(graphs) * len(graphs))
-        torch.cuda.synchronize()
-        for s in range(K, K + kp):
-            prof_graphs[s % len(graphs)].replay()
-        torch.cuda.synchronize()
-
-        def el(a, b):
-            err, v = rt.cudaEventElapsedTime(a, b)
-            assert err == rt.cudaError_t.cudaSuccess
-            return v
-        k1_ms = [statistics.fmean(el(gev[g][li][0], gev[g][li][1]) for g in range(len(graphs))) for li in range(nlayers)]
-        k2_ms = [statistics.fmean(el(gev[g][li][1], gev[g][li][2]) for g in range(len(graphs))) for li in range(nlayers)]
-    else:
-        k1_ms = [statistics.fmean(evs[s][li][0].elapsed_time(evs[s][li][1]) for s in range(K)) for li in range(nlayers)]
-        k2_ms = [statistics.fmean(evs[s][li][1].elapsed_time(evs[s][li][2]) for s in range(K)) for li in range(nlayers)]
+            r = s % cb.nsets
+            parity = cb.uses[r] & 1
+            cb.uses[r] += 1
+            for li, lay in enumerate(cb.sets[r]):
+                evs[li][0].record(cb.stream)
+                lay.quantize(L, parity, cb.sh)
+                evs[li][1].record(cb.stream)
+                lay.gemm(L, cb.sh)
+                evs[li][2].record(cb.stream)
+            torch.cuda.synchronize()
+            for li in range(cb.nlayers):
+                k1_ms[li] += evs[li][0].elapsed_time(evs[li][1]) / K
+                k2_ms[li] += evs[li][1].elapsed_time(evs[li][2]) / K
     ms = max_over_ranks(ms, "cuda")
     ms_step = ms / K
     dense_step = sum(st["k2_dense"] for st in stats)
     value = job_tops(world, dense_step, ms_step)
-
-    # e2e: host buffers, copies inside the timed region
-    e2e = None
-    ke = min(args.e2e_steps, K)
-    host_x = [[[torch.empty_like(lay.x_a, device="cpu").pin_memory() for _ in range(2)] for lay in st]
-              for st in sets]
-    host_y = [[torch.empty_like(lay.y_prev, device="cpu").pin_memory() for lay in st] for st in sets]
-    for r, st in enumerate(sets):
-        for li, lay in enumerate(st):
-            host_x[r][li][0].copy_(lay.x_a.cpu())
-            host_x[r][li][1].copy_(lay.x_b.cpu())
-    h2d = sum(lay.x_a.numel() * lay.x_a.element_size() for lay in sets[0])
-    d2h = sum(lay.y_prev.numel() * lay.y_prev.element_size() for lay in sets[0])
-    # device landing buffers for the copied inputs: one per parity in swap
-    # mode (the buffer of the other parity holds X_{t-1}), else one
-    land = [[[lay.x_a.clone(), lay.x_b.clone()] if swap else [torch.empty_like(lay.x_a)] for lay in st]
-            for st in sets]
-    land_m = [[[nat.mat(t) for t in bufs] for bufs in row] for row in land]
-
-    # Three streams: host->device copies, the compute (the library's calls) and
-    # device->host copies, so one step's copies overlap its neighbours' compute.
-    # A step's landing buffers are rewritten only after the set's previous step
-    # has computed, and its Y cache is updated only after the set's previous
-    # read-back has finished.
-    h2d_s, d2h_s = torch.cuda.Stream(), torch.cuda.Stream()
-    n_ev = ke + 3
-    ev_h, ev_c, ev_d = ([torch.cuda.Event() for _ in range(n_ev)] for _ in range(3))
-
-    def step_e2e(s, i):
-        r = s % args.sets
-        parity = uses[r] & 1
-        uses[r] += 1
-        slot = parity if swap else 0
-        if i >= args.sets:
-            h2d_s.wait_event(ev_c[i - args.sets])
-        with torch.cuda.stream(h2d_s):
-            for li in range(len(sets[r])):
-                land[r][li][slot].copy_(host_x[r][li][parity], non_blocking=True)
-        ev_h[i].record(h2d_s)
-        stream.wait_event(ev_h[i])
-        if i >= args.sets:
-            stream.wait_event(ev_d[i - args.sets])
-        for li, lay in enumerate(sets[r]):
-            mp = land_m[r][li][1 - parity] if swap else lay.m_xp
-            rc = L.dstar_fmdq_linear(ctypes.byref(land_m[r][li][slot]), ctypes.byref(mp), ctypes.byref(lay.m_y),
-                                     ctypes.byref(lay.m_w), lay.ws_ptr, lay.base, ctypes.byref(lay.cfg),
-                                     ctypes.byref(lay.m_y), sh)
-            if rc:
-                raise RuntimeError(L.dstar_fmdq_last_error().decode())
-        ev_c[i].record(stream)
-        d2h_s.wait_event(ev_c[i])
-        with torch.cuda.stream(d2h_s):
-            for li, lay in enumerate(sets[r]):
-                host_y[r][li].copy_(lay.y_prev, non_blocking=True)
-        ev_d[i].record(d2h_s)
-
-    for s in range(3):
-        step_e2e(s, s)
-    if dist:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(h2d_s)
-    for s in range(ke):
-        step_e2e(s, 3 + s)
-    stream.wait_stream(h2d_s)
-    stream.wait_stream(d2h_s)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    ems = max_over_ranks(e0.elapsed_time(e1), "cuda")
-    e2e = {"value": job_tops(world, dense_step, ems / ke), "unit": "TOPS", "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h, "steps": ke, "ms_per_step": ems / ke,
-           "path": "pinned host X_t -> device, dstar_fmdq_linear per layer, Y_t -> pinned host; copies on "
-                   "their own streams overlap the neighbouring steps' compute"}
-
-    st = nat.status(sets[0][0].ws)
-    for row in sets:
-        for lay in row:
-            st |= nat.status(lay.ws)
+    e2e = cb.e2e(min(args.e2e_steps, K), world, dense_step)
+    st = cb.status()
     if st:
         raise RuntimeError(f"device status {st} after the benchmark")
+    inputs = cb.inputs
+    set_mb = cb.set_mb()
+    cb.close()
+
+    # further workloads, on one GPU only (every rank would have to run them alike)
+    per_config, sweep = [], None
+    if world == 1:
+        for c in [int(x) for x in args.extra_configs.split(",") if x.strip()]:
+            if c != args.config:
+                per_config.append(measure_extra(c, args, torch, nat, L, peaks, peak_src))
+        if args.sweep_steps > 0:
+            sweep = measure_sweep(args, torch, nat, L)
 
     if rank != 0:
         return
 
-    # roofline of the dominant kernel, from the live event times
-    peaks, peak_src = load_peaks()
-    hbm = peaks["hbm_gbs"]
-    i8_burst = peaks["bf16_tflops"] * INT8_PER_BF16
-    kern = []
-    for li, stt in enumerate(stats):
-        kern.append(dict(kernel="quantize", layer=inputs[li].spec.name, ms=k1_ms[li], bound="hbm",
-                         achieved=stt["k1_bytes"] / (k1_ms[li] * 1e-3) / 1e9, peak=hbm, unit="GB/s",
-                         algorithmic=stt["k1_bytes"]))
-        t_tc = stt["k2_issued"] / (i8_burst * 1e12)
-        t_hbm = stt["k2_bytes"] / (hbm * 1e9)
-        if t_tc >= t_hbm:
-            kern.append(dict(kernel="slice_gemm", layer=inputs[li].spec.name, ms=k2_ms[li], bound="tensor",
-                             achieved=stt["k2_dense"] / (k2_ms[li] * 1e-3) / 1e12, peak=i8_burst, unit="TOPS",
-                             algorithmic=stt["k2_dense"]))
-        else:
-            kern.append(dict(kernel="slice_gemm", layer=inputs[li].spec.name, ms=k2_ms[li], bound="hbm",
-                             achieved=stt["k2_bytes"] / (k2_ms[li] * 1e-3) / 1e9, peak=hbm, unit="GB/s",
-                             algorithmic=stt["k2_bytes"]))
-    for k in kern:
-        k["frac"] = k["achieved"] / k["peak"]
-    dom = max(kern, key=lambda k: k["ms"])
-    traffic = load_traffic().get(f"{dom['kernel']}.{dom['layer']}.dram_bytes")
-    roofline = {"bound": dom["bound"], "achieved": dom["achieved"], "peak": dom["peak"], "unit": dom["unit"],
-                "frac": dom["frac"], "traffic": traffic, "kernel": f"{dom['kernel']} ({dom['layer']})",
-                "peak_source": (f"{peak_src} hbm_gbs" if dom["bound"] == "hbm" else
-                                f"{peak_src} bf16_tflops x {INT8_PER_BF16} (nominal int8:bf16)")}
-    kernels = [{k: (round(v, 4) if isinstance(v, float) else v) for k, v in kk.items()} for kk in kern]
-
+    kern = kernel_rows(inputs, stats, k1_ms, k2_ms, peaks)
+    roofline = roofline_of(kern, peak_src)
     cpu = None
     if not args.no_cpu_baseline:
-        ops, el, desc, threads = oracle_sample_time(inputs, args.cpu_seconds)
-        cpu = {"value": ops / el / 1e12, "unit": "TOPS", "cores": threads, "kind": "oracle", "sample": desc,
-               "seconds": el}
+        cpu = oracle_baseline(inputs, args.cpu_seconds)
 
-    set_mb = sum(t.numel() * t.element_size() for lay in sets[0]
-                 for t in (lay.x_a, lay.x_b, lay.x_prev, lay.y_prev, lay.w_q, lay.w_scale, lay.ws.buf)
-                 if t is not None) / 1e6
-    launches_per_step = 2 * nlayers  # quantizer and slice GEMM (slice-stream tiles run inside it) per layer
+    nlayers = len(inputs)
     line = {
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -659,20 +927,21 @@ def run_ours(args, rank, world, local_rank):
                        l2=f"inputs rotate over {args.sets} buffer sets of {set_mb:.0f} MB each "
                           f"({args.sets * set_mb:.0f} MB > 126 MB L2); no flush needed"),
         "roofline": roofline,
-        "kernels": kernels,
+        "kernels": rounded(kern),
         "quantizer_GBps": [k["achieved"] for k in kern if k["kernel"] == "quantize"],
         "quantizer_frac_of_8TBs_spec": [k["achieved"] / 8000.0 for k in kern if k["kernel"] == "quantize"],
         "workload_stats": [{k: v for k, v in s.items() if k in ("bits_avg", "bit_hist", "planes_hist",
                                                               "fallback_tiles", "slice_macs")} for s in stats],
         "slice_macs_per_s": sum(s["slice_macs"] for s in stats) / (ms_step * 1e-3),
-        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * K,
-        "clocks": clocks.summary(t_wall0, t_wall1),
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * nlayers * K,
+        "clocks": clocks,
+        "per_config": per_config, "sweep": sweep,
         "kernel_sources": kernel_source_sha(),
         "timing": ("value: CUDA-graph replays of the captured dstar_fmdq_linear calls, one graph per cycle of "
                    f"{2 * args.sets} steps (every input set with both X_t); per-kernel times: a second timed "
                    "region of the step split into dstar_fmdq_quantize + dstar_fmdq_slice_gemm with event nodes "
-                   "between the kernels" if graphs
-                   else "eager C-ABI calls with CUDA events per kernel"),
+                   "between the kernels" if args.mode == "graph"
+                   else "eager C-ABI calls; per-kernel times from events around each stage"),
     }
     print(json.dumps(line), flush=True)
 

@@ -116,6 +116,13 @@ def _weights(rng, K, N):
     return w_q, w_scale
 
 
+def layer_weights(cfg: int, layer: int, seed: int | None = None) -> tuple[np.ndarray, np.ndarray]:
+    """The int8 weights and per-output-channel scales make_layer draws for
+    (cfg, layer), without drawing the activations."""
+    spec = config_layers(cfg)[layer]
+    return _weights(_rng(cfg if seed is None else seed, layer, 101), spec.K, spec.N)
+
+
 def _dx(cfg: int, spec: LayerSpec, rng, sigma: float | None) -> np.ndarray:
     M, K = spec.M, spec.K
     if cfg == 1:

@@ -59,6 +59,9 @@ def _load():
         lib.fmdq_orc_slice_digit.argtypes = [ctypes.c_uint32, ci, ci]
         lib.fmdq_orc_slice_digit.restype = ci
         lib.fmdq_orc_pot_max.restype = ci
+        lib.fmdq_orc_set_threads.argtypes = [ci]
+        lib.fmdq_orc_set_threads.restype = None
+        lib.fmdq_orc_max_threads.restype = ci
         _lib = lib
     return _lib
 
@@ -194,4 +197,10 @@ def linear(x_t, x_prev, y_prev, w_q, w_scale, lb, t0=0, force_bits=0, out_bf16=T
 
 
 def n_threads() -> int:
-    return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    """Threads the oracle's loops use now."""
+    return int(_load().fmdq_orc_max_threads())
+
+
+def set_threads(n: int) -> None:
+    """Run the oracle's loops on n threads (timing only; results do not change)."""
+    _load().fmdq_orc_set_threads(int(n))

@@ -352,3 +352,9 @@ void fmdq_orc_f32_to_bf16(const float* f, int64_t n, uint16_t* h) {
 }
 
 int fmdq_orc_pot_max(void) { return ORC_POT_MAX; }
+
+/* Thread count of the OpenMP loops above (for timing at 1 thread and at all
+ * cores); it changes no result. */
+#include <omp.h>
+void fmdq_orc_set_threads(int n) { omp_set_num_threads(n > 0 ? n : 1); }
+int fmdq_orc_max_threads(void) { return omp_get_max_threads(); }

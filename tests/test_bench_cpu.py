@@ -57,3 +57,23 @@ def test_workload_config_names_the_xprev_mode():
 
 def test_job_throughput_counts_every_rank():
     assert bench.job_tops(4, 1e12, 1.0) == 4 * bench.job_tops(1, 1e12, 1.0)
+
+
+def test_oracle_baseline_reports_stages_threads_and_cpu():
+    """The CPU baseline: all threads with a per-stage split, one thread on a
+    small sample, and the CPU model."""
+    inputs = bench.workload_inputs(1, 0)
+    cpu = bench.oracle_baseline(inputs, 0.2)
+    assert cpu["kind"] == "oracle" and cpu["value"] > 0 and cpu["cores"] >= 1
+    assert set(cpu["stages_s"]) == {"quantize", "gemm", "epilogue"}
+    assert cpu["single_thread"]["cores"] == 1 and cpu["single_thread"]["value"] > 0
+    assert isinstance(cpu["cpu_model"], str) and cpu["cpu_model"]
+    import oracle
+    assert oracle.n_threads() == os.cpu_count() or oracle.n_threads() >= 1  # restored after the 1-thread run
+
+
+def test_bench_defaults_to_the_largest_workload():
+    args = bench.parse([])
+    assert args.config == 4 and args.steps > 0 and args.warmup >= 3
+    from differential_quantized_gemm_b200 import synth
+    assert max(s.M for s in synth.config_layers(args.config)) == 16384
