@@ -19,6 +19,11 @@ Parity status of each function (what pins it, see tests/test_oracle_pins.py):
   acc_direct    -- equality with a numpy int64 matmul of the shifted codes.
   epilogue_f32  -- bounded against epilogue_f64 and against the dense fp64
                    product within the quantization error bound.
+  quantize_dyn  -- (dynamic base) base equal to a brute-force minimum of the
+                   nonzero M_i; PoT against exact rational comparisons; equal
+                   to the static quantizer when the minimum is a power of two;
+                   the error bound on tiny shapes.
+  epilogue_dyn_f32 -- equal to epilogue_f32 when the base is a power of two.
 """
 from __future__ import annotations
 
@@ -59,6 +64,10 @@ def _load():
         lib.fmdq_orc_slice_digit.argtypes = [ctypes.c_uint32, ci, ci]
         lib.fmdq_orc_slice_digit.restype = ci
         lib.fmdq_orc_pot_max.restype = ci
+        lib.fmdq_orc_quantize_dyn.argtypes = [P, P, i64, i64, ci, ci, ci] + [P] * 12
+        lib.fmdq_orc_quantize_dyn.restype = ci
+        lib.fmdq_orc_epilogue_dyn_f32.argtypes = [i64, i64, P, P, ctypes.c_float, P, P, ci, P]
+        lib.fmdq_orc_epilogue_dyn_f32.restype = None
         lib.fmdq_orc_set_threads.argtypes = [ci]
         lib.fmdq_orc_set_threads.restype = None
         lib.fmdq_orc_max_threads.restype = ci
@@ -127,6 +136,48 @@ def quantize(x_t: np.ndarray, x_prev: np.ndarray, lb: int, t0: int = 0, force_bi
         _p(x_t), _p(x_prev), M, K, lb, t0, force_bits, _p(q.codes), _p(q.bits), _p(q.fpot), _p(q.pot),
         _p(q.g_ref), _p(q.count), _p(q.rec_word), _p(q.rec_k), _p(q.rec_tag), _p(q.rec_j), _p(q.shift))
     return q
+
+
+def quantize_dyn(x_t: np.ndarray, x_prev: np.ndarray, thr_lb: int, t0: int = 0,
+                 force_bits: int = 0) -> Quantized:
+    """Steps 1-4 with the dynamic base (FMDQ-DYN): base = the minimum nonzero
+    M_i of the call (first pass), widths from the predefined thresholds
+    Thr_N = 2^(thr_lb + t0 + 2N); `fpot` holds FPoT relative to the base and
+    `base` the base itself (fp32)."""
+    x_t = np.ascontiguousarray(x_t, np.float32)
+    x_prev = np.ascontiguousarray(x_prev, np.float32)
+    M, K = x_t.shape
+    assert x_prev.shape == (M, K) and M % TILE == 0
+    q = Quantized(M, K)
+    base = np.zeros(1, np.float32)
+    q.status = _load().fmdq_orc_quantize_dyn(
+        _p(x_t), _p(x_prev), M, K, thr_lb, t0, force_bits, _p(base), _p(q.codes), _p(q.bits), _p(q.fpot),
+        _p(q.pot), _p(q.g_ref), _p(q.count), _p(q.rec_word), _p(q.rec_k), _p(q.rec_tag), _p(q.rec_j),
+        _p(q.shift))
+    q.base = float(base[0])
+    return q
+
+
+def epilogue_dyn_f32(acc: np.ndarray, g_ref: np.ndarray, base: float, w_scale: np.ndarray, y_prev: np.ndarray,
+                     out_bf16: bool) -> np.ndarray:
+    """Y_t = Y_{t-1} + acc * 2^-g_ref * base * w_scale in the fixed fp32 order (dynamic base)."""
+    acc = np.ascontiguousarray(acc, np.int64)
+    M, N = acc.shape
+    w_scale = np.ascontiguousarray(w_scale, np.float32)
+    y_prev = np.ascontiguousarray(y_prev, np.float32)
+    g_ref = np.ascontiguousarray(g_ref, np.int32)
+    out = np.zeros((M, N), np.float32)
+    _load().fmdq_orc_epilogue_dyn_f32(M, N, _p(acc), _p(g_ref), float(np.float32(base)), _p(w_scale), _p(y_prev),
+                                      int(out_bf16), _p(out))
+    return out
+
+
+def linear_dyn(x_t, x_prev, y_prev, w_q, w_scale, thr_lb, t0=0, force_bits=0, out_bf16=True):
+    """The whole differential linear with the dynamic base: (Quantized, acc, y_out)."""
+    q = quantize_dyn(x_t, x_prev, thr_lb, t0, force_bits)
+    acc = acc_direct(q, w_q)
+    y = epilogue_dyn_f32(acc, q.g_ref, q.base, w_scale, y_prev, out_bf16)
+    return q, acc, y
 
 
 def _mask(T, tiles):

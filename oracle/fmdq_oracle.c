@@ -217,6 +217,187 @@ int fmdq_orc_quantize(const float* x_t, const float* x_prev, int64_t M, int64_t 
   return status;
 }
 
+/* ------------------------------------------------- dynamic base (FMDQ-DYN) */
+
+/*
+ * Steps 2-4 for one tile whose codes, widths and FPoTs are known: b/2 slices
+ * per sub-channel (slice j carries FPoT - 2j), reordered by (FPoT, channel)
+ * ascending, shift counts.  The same rules as in fmdq_orc_quantize.
+ */
+static void encode_tile(int64_t t, int64_t K, const int8_t* codes, const int8_t* bits,
+                        const int8_t* fpot, int32_t* count, uint32_t* rec_word, uint16_t* rec_k,
+                        int8_t* rec_tag, uint8_t* rec_j, int8_t* shift) {
+  const int64_t cap = 4 * K;
+  typedef struct {
+    int tag;
+    int k;
+    int j;
+    uint32_t word;
+  } rec_t;
+  rec_t* recs = (rec_t*)malloc((size_t)cap * sizeof(rec_t));
+  int64_t nrec = 0;
+  for (int64_t k = 0; k < K; ++k) {
+    int b = bits[t * K + k];
+    for (int j = 0; j < b / 2; ++j) {
+      uint32_t word = 0;
+      for (int i = 0; i < ORC_TILE; ++i) {
+        uint32_t u = (uint32_t)(int32_t)codes[(t * ORC_TILE + i) * K + k] & ((1u << b) - 1u);
+        word |= ((u >> (2 * j)) & 3u) << (2 * i);
+      }
+      recs[nrec].tag = fpot[t * K + k] - 2 * j;
+      recs[nrec].k = (int)k;
+      recs[nrec].j = j;
+      recs[nrec].word = word;
+      ++nrec;
+    }
+  }
+  for (int64_t a = 1; a < nrec; ++a) {
+    rec_t key = recs[a];
+    int64_t c = a - 1;
+    while (c >= 0 && (recs[c].tag > key.tag || (recs[c].tag == key.tag && recs[c].k > key.k))) {
+      recs[c + 1] = recs[c];
+      --c;
+    }
+    recs[c + 1] = key;
+  }
+  for (int64_t r = 0; r < nrec; ++r) {
+    rec_word[t * cap + r] = recs[r].word;
+    rec_k[t * cap + r] = (uint16_t)recs[r].k;
+    rec_tag[t * cap + r] = (int8_t)recs[r].tag;
+    rec_j[t * cap + r] = (uint8_t)recs[r].j;
+    shift[t * cap + r] = (int8_t)(r == 0 ? 0 : recs[r].tag - recs[r - 1].tag);
+  }
+  count[t] = (int32_t)nrec;
+  free(recs);
+}
+
+/*
+ * Step 1 with the dynamic base of Eqs. 2-3 (section 3.1: the base is the
+ * minimum of M_i over all sub-channels, found by a first pass over the data;
+ * the paper's DS-FMDQ-DYN variant of section 5.2, Table 2).  Readings:
+ *   - the minimum is taken over the sub-channels with a nonzero, finite M_i
+ *     (a zero M_i would make Eq. 3 undefined); with none, every code is 0
+ *     and base is reported as 1;
+ *   - the bit width still comes from the predefined thresholds,
+ *     M_i <= Thr_N = 2^(thr_lb + t0 + 2N) (Thr_0 = 2^(thr_lb + t0));
+ *   - PoT_i = ceil(log2(M_i / base)) exactly: the smallest P >= 0 with
+ *     M_i <= base * 2^P (both sides exact in double);
+ *   - the base is not a power of two, so the relative FPoT b - 2 - PoT is
+ *     stored (the absolute one of Eq. 4 differs from it by -2 log2(base),
+ *     the same for every sub-channel) and the code is
+ *     q = rne(fl32(dX / base) * 2^(b - 2 - PoT)): one IEEE fp32 division,
+ *     then an exact power-of-two scaling;
+ *   - the dequantized value of a code is q * 2^-(FPoT) * base.
+ * Outputs as fmdq_orc_quantize (fpot holds the relative FPoT), plus *base_out.
+ */
+int fmdq_orc_quantize_dyn(const float* x_t, const float* x_prev, int64_t M, int64_t K, int thr_lb,
+                          int t0, int force_bits, float* base_out, int8_t* codes, int8_t* bits,
+                          int8_t* fpot, int16_t* pot, int32_t* g_ref, int32_t* count,
+                          uint32_t* rec_word, uint16_t* rec_k, int8_t* rec_tag, uint8_t* rec_j,
+                          int8_t* shift) {
+  const int64_t T = M / ORC_TILE;
+  int status = 0;
+
+  /* Pass 1: M_i of every sub-channel, and their minimum over nonzero finite ones. */
+  float base = 0.0f;
+  int have = 0;
+  for (int64_t t = 0; t < T; ++t) {
+    for (int64_t k = 0; k < K; ++k) {
+      float Mi = 0.0f;
+      int nonfinite = 0;
+      for (int i = 0; i < ORC_TILE; ++i) {
+        int64_t m = t * ORC_TILE + i;
+        float a = fabsf(x_t[m * K + k] - x_prev[m * K + k]);
+        if (!isfinite(a)) nonfinite = 1;
+        else if (a > Mi) Mi = a;
+      }
+      if (nonfinite || Mi == 0.0f) continue;
+      if (!have || Mi < base) base = Mi;
+      have = 1;
+    }
+  }
+  if (!have) base = 1.0f;
+  *base_out = base;
+
+  /* Pass 2: per sub-channel width, PoT, FPoT and codes; then steps 2-4. */
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : status)
+  for (int64_t t = 0; t < T; ++t) {
+    int gmax = -1000;
+    for (int64_t k = 0; k < K; ++k) {
+      float dx[ORC_TILE];
+      float Mi = 0.0f;
+      int nonfinite = 0;
+      for (int i = 0; i < ORC_TILE; ++i) {
+        int64_t m = t * ORC_TILE + i;
+        dx[i] = x_t[m * K + k] - x_prev[m * K + k];
+        float a = fabsf(dx[i]);
+        if (!isfinite(a)) nonfinite = 1;
+        else if (a > Mi) Mi = a;
+      }
+      if (nonfinite) {
+        status |= ORC_ST_NONFINITE;
+        Mi = 0.0f;
+        for (int i = 0; i < ORC_TILE; ++i) dx[i] = 0.0f;
+      }
+      /* Eq. 3 with the dynamic base: the smallest P >= 0 with M_i <= base * 2^P. */
+      int PoT = 0;
+      if (Mi > 0.0f)
+        while ((double)Mi > ldexp((double)base, PoT) && PoT <= ORC_POT_MAX) ++PoT;
+      if (PoT > ORC_POT_MAX) {
+        status |= ORC_ST_RANGE;
+        PoT = ORC_POT_MAX;
+      }
+      /* width by binning M_i against the predefined thresholds Thr_N */
+      int b;
+      if (force_bits) b = force_bits;
+      else if ((double)Mi <= ldexp(1.0, thr_lb + t0)) b = 2;
+      else if ((double)Mi <= ldexp(1.0, thr_lb + t0 + 2)) b = 4;
+      else if ((double)Mi <= ldexp(1.0, thr_lb + t0 + 4)) b = 6;
+      else b = 8;
+      int FPoT = (b - 2) - PoT; /* relative to the base: PCeil = 2^(b-2) */
+      for (int i = 0; i < ORC_TILE; ++i) {
+        volatile float u = dx[i] / base;              /* IEEE fp32 division */
+        double v = (double)u * ldexp(1.0, b - 2 - PoT); /* exact power-of-two scaling */
+        int32_t q = (int32_t)nearbyint(v);             /* ties to even */
+        if (abs(q) > (1 << (b - 2))) status |= ORC_ST_RANGE;
+        codes[(t * ORC_TILE + i) * K + k] = (int8_t)q;
+      }
+      bits[t * K + k] = (int8_t)b;
+      fpot[t * K + k] = (int8_t)FPoT;
+      pot[t * K + k] = (int16_t)PoT;
+      if (FPoT > gmax) gmax = FPoT;
+    }
+    g_ref[t] = gmax;
+    encode_tile(t, K, codes, bits, fpot, count, rec_word, rec_k, rec_tag, rec_j, shift);
+  }
+  return status;
+}
+
+/*
+ * Epilogue of the dynamic-base variant: the code unit is base * 2^-FPoT, so
+ *   a = (float)acc;  a = a * 2^(-g_ref) (exact);  a = a * base;  a = a * w_scale[n];
+ *   y = y_prev + a;  bf16 outputs round y to nearest-even.  No FMA.
+ */
+void fmdq_orc_epilogue_dyn_f32(int64_t M, int64_t N, const int64_t* acc, const int32_t* g_ref,
+                               float base, const float* w_scale, const float* y_prev, int out_bf16,
+                               float* y_out) {
+#pragma omp parallel for schedule(static)
+  for (int64_t m = 0; m < M; ++m) {
+    int64_t t = m / ORC_TILE;
+    float p2 = (float)ldexp(1.0, -g_ref[t]);
+    for (int64_t n = 0; n < N; ++n) {
+      volatile float a = (float)acc[m * N + n];
+      a = a * p2;
+      a = a * base;
+      a = a * w_scale[n];
+      volatile float y = y_prev[m * N + n] + a;
+      float r = y;
+      if (out_bf16) r = bf16_bits_to_float(float_to_bf16_bits(y));
+      y_out[m * N + n] = r;
+    }
+  }
+}
+
 /* Signed value of the 2-bit field of slice j of a b-bit code: the top slice
  * (j == b/2 - 1) carries the sign of the two's-complement pattern. */
 static int slice_digit(uint32_t field, int j, int b) {
