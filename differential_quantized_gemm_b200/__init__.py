@@ -9,7 +9,7 @@ The computation lives in the CUDA library built from csrc/ (C ABI in
 include/dstar_fmdq.h); this package is its Python binding.
 """
 from ._native import (  # noqa: F401
-    BF16, F32, FLAG_NO_XPREV_REFRESH, FLAG_SLICE_PATH, I8, POT_MAX, STATUS_NONFINITE, STATUS_RANGE,
+    BF16, F32, FLAG_DYNAMIC_BASE, FLAG_NO_XPREV_REFRESH, FLAG_SLICE_PATH, I8, POT_MAX, STATUS_NONFINITE, STATUS_RANGE,
     STATUS_TIMEOUT, TILE, DstarError, Workspace, lib, linear, quantize, selftest_wait, slice_gemm, status,
     version, workspace_layout, workspace_size,
 )

@@ -21,6 +21,7 @@ STATUS_NONFINITE, STATUS_RANGE, STATUS_TIMEOUT = 1, 2, 4
 F32, BF16, I8 = 0, 1, 2
 FLAG_NO_XPREV_REFRESH = 1
 FLAG_SLICE_PATH = 2
+FLAG_DYNAMIC_BASE = 4
 TILE = 16
 POT_MAX = 32
 K_MAX = 8192
@@ -47,7 +48,7 @@ class TileCfg(ctypes.Structure):
 class WsLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in ("total", "status", "plane0", "plane1", "fpot", "bits", "g_ref",
                                                "planes", "count", "mask1", "records")] + \
-               [("mask_words", ctypes.c_int64), ("record_cap", ctypes.c_int64)]
+               [("mask_words", ctypes.c_int64), ("record_cap", ctypes.c_int64), ("dyn_base", ctypes.c_size_t)]
 
 
 class DstarError(RuntimeError):
@@ -168,6 +169,7 @@ class Workspace:
             "count": view(L.count, T, torch.int32),
             "mask1": view(L.mask1, T * L.mask_words, torch.int32).view(T, L.mask_words),
             "records": view(L.records, T * L.record_cap * 2, torch.int32).view(T, L.record_cap, 2),
+            "dyn_base": view(L.dyn_base, 1, torch.float32),
         }
 
 

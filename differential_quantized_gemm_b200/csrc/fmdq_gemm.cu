@@ -116,10 +116,19 @@ struct OutT<false> {
   using T = float;
 };
 
-// y = y_prev + ((float)acc * p2) * ws  -- fp32, no contraction
-__device__ __forceinline__ float epi(int64_t acc, bool wide, float p2, float ws, float yp) {
+// y = y_prev + (((float)acc * p2) * beta) * ws  -- fp32, no contraction.  beta is
+// the dynamic base, or exactly 1 with the static base (whose scale is in p2).
+__device__ __forceinline__ float epi(int64_t acc, bool wide, float p2, float beta, float ws, float yp) {
   const float a = wide ? __ll2float_rn(acc) : __int2float_rn((int)acc);
-  return __fadd_rn(yp, __fmul_rn(__fmul_rn(a, p2), ws));
+  return __fadd_rn(yp, __fmul_rn(__fmul_rn(__fmul_rn(a, p2), beta), ws));
+}
+
+// The dynamic base written by the quantizer's first pass (1 when no M_i was
+// nonzero), or 1 with the static base.
+__device__ __forceinline__ float dyn_beta(const uint32_t* dyn_base) {
+  if (!dyn_base) return 1.f;
+  const uint32_t b = *dyn_base;
+  return b == 0xFFFFFFFFu ? 1.f : __uint_as_float(b);
 }
 
 template <bool OUT_BF16>
@@ -141,7 +150,7 @@ __device__ __forceinline__ void store_y(void* base, int64_t off, float y) {
 // units of the last FPoT and are shifted to g_ref.
 template <bool OUT_BF16>
 __device__ void slice_stream_column(const uint2* recs, int cnt, const int8_t* bits_row, int g_ref,
-                                    const int8_t* w_row, int64_t t, int64_t n, int lb, float ws,
+                                    const int8_t* w_row, int64_t t, int64_t n, int lb, float beta, float ws,
                                     void* y_prev, int64_t ld_yp, void* y_out, int64_t ld_yo, int y_distinct,
                                     int64_t* debug_acc, int64_t N) {
   int64_t acc[kTile];
@@ -177,7 +186,7 @@ __device__ void slice_stream_column(const uint2* recs, int cnt, const int8_t* bi
 #pragma unroll
   for (int i = 0; i < kTile; ++i) {
     const int64_t row = t * kTile + i;
-    const float y = epi(acc[i], true, p2, ws, load_y<OUT_BF16>(y_prev, row * ld_yp + n));
+    const float y = epi(acc[i], true, p2, beta, ws, load_y<OUT_BF16>(y_prev, row * ld_yp + n));
     store_y<OUT_BF16>(y_out, row * ld_yo + n, y);
     if (y_distinct) store_y<OUT_BF16>(y_prev, row * ld_yp + n, y);
     if (debug_acc) debug_acc[row * N + n] = acc[i];
@@ -186,10 +195,10 @@ __device__ void slice_stream_column(const uint2* recs, int cnt, const int8_t* bi
 
 // One epilogue group: 32 columns of one row (this lane's), in place in its
 // swizzled 32 x 32 shared-memory tile.  acc = d0 (+ 256 d1 for rows of
-// two-plane tiles); y = y_prev + ((float)acc * p2) * w_scale, fp32, no FMA.
+// two-plane tiles); y = y_prev + (((float)acc * p2) * beta) * w_scale, fp32, no FMA.
 template <bool OUT_BF16, bool WIDE>
 __device__ __forceinline__ void epi_group(uint8_t* row, int swz, const float* ws32, const uint32_t (&d0)[32],
-                                          const uint32_t (&d1)[32], bool wide_row, float p2) {
+                                          const uint32_t (&d1)[32], bool wide_row, float p2, float beta) {
   constexpr int kOutBytes = OUT_BF16 ? 2 : 4;
   constexpr int E = 16 / kOutBytes;              // outputs per 16-byte chunk
   constexpr int kChunks = 32 * kOutBytes / 16;   // chunks per 32-column row
@@ -215,7 +224,7 @@ __device__ __forceinline__ void epi_group(uint8_t* row, int swz, const float* ws
       float a;
       if constexpr (WIDE) a = __ll2float_rn((int64_t)(int32_t)d0[i] + (wide_row ? (int64_t)(int32_t)d1[i] * 256 : 0));
       else a = __int2float_rn((int32_t)d0[i]);
-      y[e] = __fadd_rn(ypf, __fmul_rn(__fmul_rn(a, p2), wsv[e]));
+      y[e] = __fadd_rn(ypf, __fmul_rn(__fmul_rn(__fmul_rn(a, p2), beta), wsv[e]));
     }
     if constexpr (OUT_BF16) {
       uint32_t w[4];
@@ -453,6 +462,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
     uint32_t y_issued = 0, y_seen = 0;  // batches of y_prev boxes requested (lane 0) / observed landed
     int ok = 1;
     pdl_wait();  // the quantizer's outputs and the cached output are read from here on
+    const float beta = dyn_beta(p.dyn_base);
     if (lane == 0 && my_tiles > 0) {
       for (int g = 0; g < C::kHalfGroups; ++g) load_y_box(0, g);
       ++y_issued;
@@ -559,7 +569,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
           const int swz = sw(lane);
           auto one_plane_group = [&](int g, const uint32_t (&d)[32]) {
             if (row_ok) {
-              epi_group<OUT_BF16, false>(my_row + g * C::kBoxBytes, swz, ws_h + g * 32, d, d, false, p2);
+              epi_group<OUT_BF16, false>(my_row + g * C::kBoxBytes, swz, ws_h + g * 32, d, d, false, p2, beta);
               if (p.debug_acc) debug_group(g, d, d, false);
             }
             store_group(g);
@@ -588,7 +598,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
               tmem_ld_wait(d0);
               tmem_ld_wait(d1);
               if (row_ok) {
-                epi_group<OUT_BF16, true>(my_row + g * C::kBoxBytes, swz, ws_h + g * 32, d0, d1, wide_row, p2);
+                epi_group<OUT_BF16, true>(my_row + g * C::kBoxBytes, swz, ws_h + g * 32, d0, d1, wide_row, p2, beta);
                 if (p.debug_acc) debug_group(g, d0, d1, true);
               }
               store_group(g);
@@ -615,7 +625,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
             const int64_t n = n_base + c;
             if (n >= p.N) continue;
             slice_stream_column<OUT_BF16>(p.records + (int64_t)t * p.record_cap, p.count[t], p.bits + (int64_t)t * p.K,
-                                          p.g_ref[t], p.w_q + n * p.ld_w, t, n, p.lb, ws_tile[c], p.y_prev, p.ld_yp,
+                                          p.g_ref[t], p.w_q + n * p.ld_w, t, n, p.lb, beta, ws_tile[c], p.y_prev, p.ld_yp,
                                           p.y_out, p.ld_yo, p.y_distinct, p.debug_acc, p.N);
           }
         }
@@ -656,13 +666,14 @@ template <bool OUT_BF16>
 __global__ void __launch_bounds__(256) slice_gemm_kernel(const SliceParams p) {
   const int64_t T = p.M / kTile;
   const int64_t nblk = (p.N + 255) / 256;
+  const float beta = dyn_beta(p.dyn_base);
   for (int64_t item = blockIdx.x; item < T * nblk; item += gridDim.x) {
     const int64_t t = item / nblk;
     const int64_t n = (item % nblk) * 256 + threadIdx.x;
     if (!p.all_tiles && p.planes[t] <= 2) continue;
     if (n >= p.N) continue;
     slice_stream_column<OUT_BF16>(p.records + t * p.record_cap, p.count[t], p.bits + t * p.K, p.g_ref[t],
-                                  p.w_q + n * p.ld_w, t, n, p.lb, p.w_scale[n], p.y_prev, p.ld_yp, p.y_out, p.ld_yo,
+                                  p.w_q + n * p.ld_w, t, n, p.lb, beta, p.w_scale[n], p.y_prev, p.ld_yp, p.y_out, p.ld_yo,
                                   p.y_distinct, p.debug_acc, p.N);
   }
 }

@@ -163,7 +163,7 @@ int check_cfg(const dstar_tile_cfg* c, int64_t M, int64_t K) {
   if (c->force_bits != 0 && c->force_bits != 2 && c->force_bits != 4 && c->force_bits != 6 && c->force_bits != 8)
     return fail(DSTAR_ERR_INVALID_ARG, "force_bits must be 0, 2, 4, 6 or 8");
   if (c->thr0_log2 < -100 || c->thr0_log2 > 100) return fail(DSTAR_ERR_INVALID_ARG, "thr0_log2 out of [-100, 100]");
-  if (c->flags & ~(DSTAR_FLAG_NO_XPREV_REFRESH | DSTAR_FLAG_SLICE_PATH))
+  if (c->flags & ~(DSTAR_FLAG_NO_XPREV_REFRESH | DSTAR_FLAG_SLICE_PATH | DSTAR_FLAG_DYNAMIC_BASE))
     return fail(DSTAR_ERR_INVALID_ARG, "unknown flag bits 0x%x", c->flags);
   const WsLayout L = ws_layout(M, K);
   if (!c->workspace) return fail(DSTAR_ERR_WORKSPACE, "workspace is NULL");
@@ -210,6 +210,17 @@ int do_quantize(const dstar_mat* x_t, dstar_mat* x_prev, int lb, const dstar_til
   q.record_cap = L.record_cap;
   q.mask_words = L.mask_words;
   q.debug_codes = c->debug_codes;
+  q.dyn_base = nullptr;
+  const bool in_bf16 = x_t->dtype == DSTAR_BF16;
+  if (c->flags & DSTAR_FLAG_DYNAMIC_BASE) {
+    // first pass: base = min of the nonzero M_i (atomic minimum from all ones)
+    q.dyn_base = ws_ptr<uint32_t>(c, L.dyn_base);
+    cudaError_t ce = cudaMemsetAsync(q.dyn_base, 0xFF, sizeof(uint32_t), (cudaStream_t)stream);
+    if (ce != cudaSuccess) return cuda_fail(ce, "clearing the dynamic base");
+    const int e = launch_base_min(x_t->data, x_prev->data, x_t->ld, x_prev->ld, M, K, in_bf16, q.dyn_base, dev.sms,
+                                  stream);
+    if (e) return cuda_fail(e, "dynamic-base launch");
+  }
   const dstar_mat* pf[2] = {pf_w, pf_y};
   for (int i = 0; i < 2; ++i) {
     if (pf[i] && pf[i]->data && pf[i]->rows > 0 && pf[i]->cols > 0) {
@@ -218,7 +229,7 @@ int do_quantize(const dstar_mat* x_t, dstar_mat* x_prev, int lb, const dstar_til
                                pf[i]->ld * es};
     }
   }
-  const int e = launch_quantize(q, x_t->dtype == DSTAR_BF16, dev.sms, stream);
+  const int e = launch_quantize(q, in_bf16, dev.sms, stream);
   if (e) return cuda_fail(e, "quantize launch");
   return DSTAR_OK;
 }
@@ -238,6 +249,10 @@ int do_gemm(const dstar_mat* w_q, const float* w_scale, dstar_mat* y_prev, int l
   const bool bf16 = y_prev->dtype == DSTAR_BF16;
   const bool distinct = y_out->data != y_prev->data;
   const bool slice_all = (c->flags & DSTAR_FLAG_SLICE_PATH) != 0;
+  // with the dynamic base the FPoTs are relative to it: no 2^lb in the epilogue
+  const bool dyn = (c->flags & DSTAR_FLAG_DYNAMIC_BASE) != 0;
+  const uint32_t* dyn_base = dyn ? ws_ptr<const uint32_t>(c, L.dyn_base) : nullptr;
+  if (dyn) lb = 0;
   if (!slice_all) {
     const int bn = bf16 ? choose_bn(M, N, dev.sms) : 128;  // fp32 outputs use 128-column tiles
     CUtensorMap maps[5];  // A0, A1, W, y_prev, y_out
@@ -263,6 +278,7 @@ int do_gemm(const dstar_mat* w_q, const float* w_scale, dstar_mat* y_prev, int l
     g.y_distinct = distinct;
     g.status = ws_ptr<uint32_t>(c, L.status);
     g.debug_acc = c->debug_acc;
+    g.dyn_base = dyn_base;
     g.tiles_m = (int)((M + kBlockM - 1) / kBlockM);
     g.tiles_n = (int)((N + bn - 1) / bn);
     g.num_chunks = (int)((K + kChunkK - 1) / kChunkK);
@@ -295,6 +311,7 @@ int do_gemm(const dstar_mat* w_q, const float* w_scale, dstar_mat* y_prev, int l
   s.y_distinct = distinct;
   s.all_tiles = 1;
   s.debug_acc = c->debug_acc;
+  s.dyn_base = dyn_base;
   const int e = launch_slice_gemm(s, bf16, dev.sms, stream);
   if (e) return cuda_fail(e, "slice-stream launch");
   return DSTAR_OK;
@@ -360,6 +377,7 @@ WsLayout ws_layout(int64_t M, int64_t K) {
   L.record_cap = 4 * K;
   size_t o = 0;
   L.status = o, o = align256(o + 256);
+  L.dyn_base = L.status + 16;
   L.plane0 = o, o = align256(o + (size_t)(M * K));
   L.plane1 = o, o = align256(o + (size_t)(M * K));
   L.fpot = o, o = align256(o + (size_t)(T * K));
@@ -418,6 +436,7 @@ int dstar_fmdq_workspace_layout(int64_t M, int64_t K, dstar_fmdq_ws_layout* out)
   out->records = L.records;
   out->mask_words = L.mask_words;
   out->record_cap = L.record_cap;
+  out->dyn_base = L.dyn_base;
   return ok();
 }
 

@@ -48,6 +48,9 @@ struct QuantParams {
   int64_t record_cap;
   int64_t mask_words;
   int8_t* debug_codes;
+  // dynamic base (DSTAR_FLAG_DYNAMIC_BASE): the fp32 bits of min M_i written
+  // by the first pass (all ones when none is nonzero); nullptr = static base
+  uint32_t* dyn_base;
   // operands of the GEMM that follows in the same call (weights, cached
   // output): prefetched into L2 once the quantizer no longer streams HBM
   L2Region prefetch[2];
@@ -69,6 +72,7 @@ struct GemmParams {
   int y_distinct;  // y_out is a different buffer: write both
   uint32_t* status;
   int64_t* debug_acc;
+  const uint32_t* dyn_base;  // dynamic base word (nullptr = static base, whose scale is in lb)
   int tiles_m, tiles_n, num_chunks;
   // encoded stream, for tiles whose operands need more than two planes
   const int8_t* w_q;
@@ -98,17 +102,23 @@ struct SliceParams {
   int y_distinct;
   int all_tiles;  // 1: every tile; 0: only tiles that need more than two planes
   int64_t* debug_acc;
+  const uint32_t* dyn_base;
 };
 
 // Workspace sections (byte offsets from the workspace base).
 struct WsLayout {
   size_t total, status, plane0, plane1, fpot, bits, g_ref, planes, count, mask1, records;
   int64_t mask_words, record_cap;
+  size_t dyn_base;  // inside the 256-byte header that starts with the status word
 };
 WsLayout ws_layout(int64_t M, int64_t K);
 
 // Launchers (return cudaError_t as int).
 int launch_quantize(const QuantParams& p, int in_bf16, int num_sms, void* stream);
+// First pass of the dynamic base: atomic minimum of the nonzero finite M_i
+// into *out (which the caller set to all ones).
+int launch_base_min(const void* x_t, const void* x_prev, int64_t ld_xt, int64_t ld_xp, int64_t M, int64_t K,
+                    int in_bf16, uint32_t* out, int num_sms, void* stream);
 int quantize_cluster_size(int64_t M, int64_t K, int num_sms);
 int launch_gemm(const GemmParams& p, const void* maps /* CUtensorMap[5]: A0, A1, W, y_prev, y_out */, int bn,
                 int out_bf16, int num_sms, void* stream);

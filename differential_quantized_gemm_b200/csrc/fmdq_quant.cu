@@ -95,6 +95,49 @@ __device__ __forceinline__ ColParams col_params(uint32_t mbits, int lb, float be
   return cp;
 }
 
+// Normalised form of a positive finite float: value = (sig / 2^23) * 2^exp
+// with sig in [2^23, 2^24); subnormals are normalised too.
+__device__ __forceinline__ int norm_float(uint32_t bits, uint32_t& sig) {
+  const int e = (int)(bits >> 23);
+  const uint32_t m = bits & 0x7FFFFFu;
+  if (e == 0) {
+    const int sh = __clz(m) - 8;
+    sig = m << sh;
+    return -126 - sh;
+  }
+  sig = m | 0x800000u;
+  return e - 127;
+}
+
+// Per-channel parameters with the dynamic base (FMDQ-DYN): PoT =
+// ceil(log2(M_i / base)) exactly, from the normalised exponents and
+// significands; the width from the predefined thresholds M_i <= 2^(thr + 2N)
+// (thr = lb + t0), i.e. ceil(log2 M_i) <= thr + 2N; FPoT relative to the base.
+// The code scale is 2^(b-2-PoT), applied to fl32(dX / base).
+__device__ __forceinline__ ColParams col_params_dyn(uint32_t mbits, uint32_t bbits, int thr, int fb, int& flags) {
+  ColParams cp;
+  cp.nonfinite = mbits >= 0x7F800000u;
+  int P = 0, b;
+  if (cp.nonfinite) flags |= 1;
+  if (!cp.nonfinite && mbits != 0u) {
+    uint32_t sm, sb;
+    const int em = norm_float(mbits, sm), eb = norm_float(bbits, sb);
+    P = max(em - eb + (sm > sb ? 1 : 0), 0);
+    if (P > kPotMax) {
+      P = kPotMax;
+      flags |= 2;
+    }
+    const int pabs = em + (sm > 0x800000u ? 1 : 0);  // ceil(log2 M_i)
+    b = pabs <= thr ? 2 : pabs <= thr + 2 ? 4 : pabs <= thr + 4 ? 6 : 8;
+  } else {
+    b = 2;  // M_i = 0 lies below every threshold
+  }
+  cp.bits = fb ? fb : b;
+  cp.fpot = cp.bits - 2 - P;
+  cp.scale = exp2_exact(cp.bits - 2 - P);
+  return cp;
+}
+
 // The four 2-bit slice words of a channel from its 16 codes (byte r of code
 // word w = token 4w + r): word j holds field j (bits 2j..2j+1) of every code,
 // token i in bits 2i..2i+1.  Each code word is a 4 x 4 matrix of 2-bit cells
@@ -217,7 +260,7 @@ int quantize_cluster_size(int64_t M, int64_t K, int num_sms) {
   return c;
 }
 
-template <typename TIn>
+template <typename TIn, bool DYN>
 __global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParams p, int C, int64_t kc_max) {
   extern __shared__ __align__(16) uint8_t smem[];
   using PR = Pair<TIn>;
@@ -248,6 +291,13 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParam
 
   const int lb = p.lb, t0 = p.t0, fb = p.force_bits;
   const float beta = exp2_exact(lb);
+  // dynamic base: written by the first pass; all ones when no M_i was nonzero
+  uint32_t dbits = 0x3F800000u;
+  if constexpr (DYN) {
+    dbits = *p.dyn_base;
+    if (dbits == 0xFFFFFFFFu) dbits = 0x3F800000u;
+  }
+  const float dbase = __uint_as_float(dbits);
   const bool refresh = !(p.flags & DSTAR_FLAG_NO_XPREV_REFRESH);
   const int64_t row0 = (int64_t)t * kTile;
   const int npairs = Kc / 2;
@@ -294,10 +344,22 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParam
       m0 = max(m0, __float_as_uint(d0[r]) & 0x7FFFFFFFu);
       m1 = max(m1, __float_as_uint(d1[r]) & 0x7FFFFFFFu);
     }
-    const ColParams c0 = col_params(m0, lb, beta, t0, fb, flags);
-    const ColParams c1 = col_params(m1, lb, beta, t0, fb, flags);
+    ColParams c0, c1;
+    if constexpr (DYN) {
+      c0 = col_params_dyn(m0, dbits, lb + t0, fb, flags);
+      c1 = col_params_dyn(m1, dbits, lb + t0, fb, flags);
+    } else {
+      c0 = col_params(m0, lb, beta, t0, fb, flags);
+      c1 = col_params(m1, lb, beta, t0, fb, flags);
+    }
     // stage 3; a non-finite sub-channel has scale 0, and its NaN products convert to 0
     const float s0 = c0.nonfinite ? 0.f : c0.scale, s1 = c1.nonfinite ? 0.f : c1.scale;
+    if constexpr (DYN) {  // dX / base first (one IEEE division), then the power-of-two scale
+#pragma unroll
+      for (int r = 0; r < kTile; ++r) d0[r] = __fdiv_rn(d0[r], dbase), d1[r] = __fdiv_rn(d1[r], dbase);
+      m0 = __float_as_uint(__fdiv_rn(__uint_as_float(m0), dbase));
+      m1 = __float_as_uint(__fdiv_rn(__uint_as_float(m1), dbase));
+    }
     uint32_t w0[4], w1[4];
 #pragma unroll
     for (int R = 0; R < 4; ++R) {
@@ -575,7 +637,10 @@ int launch_quantize(const QuantParams& p, int in_bf16, int num_sms, void* stream
   const int64_t kc_max = 32 * ((units + C - 1) / C);
   const size_t smem = quantize_smem_bytes(kc_max);
   const int smem_max = (int)quantize_smem_bytes(DSTAR_K_MAX);  // one setting serves every K
-  const void* fn = in_bf16 ? (const void*)quantize_kernel<__nv_bfloat16> : (const void*)quantize_kernel<float>;
+  const bool dyn = p.dyn_base != nullptr;
+  const void* fn = in_bf16 ? (dyn ? (const void*)quantize_kernel<__nv_bfloat16, true>
+                                  : (const void*)quantize_kernel<__nv_bfloat16, false>)
+                           : (dyn ? (const void*)quantize_kernel<float, true> : (const void*)quantize_kernel<float, false>);
   int e = ensure_max_smem(fn, smem_max);
   if (e != 0) return e;
   cudaLaunchConfig_t cfg = {};
@@ -593,8 +658,89 @@ int launch_quantize(const QuantParams& p, int in_bf16, int num_sms, void* stream
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   cudaError_t ce;
-  if (in_bf16) ce = cudaLaunchKernelEx(&cfg, quantize_kernel<__nv_bfloat16>, p, C, kc_max);
-  else ce = cudaLaunchKernelEx(&cfg, quantize_kernel<float>, p, C, kc_max);
+  if (in_bf16) ce = dyn ? cudaLaunchKernelEx(&cfg, quantize_kernel<__nv_bfloat16, true>, p, C, kc_max)
+                        : cudaLaunchKernelEx(&cfg, quantize_kernel<__nv_bfloat16, false>, p, C, kc_max);
+  else ce = dyn ? cudaLaunchKernelEx(&cfg, quantize_kernel<float, true>, p, C, kc_max)
+                : cudaLaunchKernelEx(&cfg, quantize_kernel<float, false>, p, C, kc_max);
+  if (ce != cudaSuccess) return (int)ce;
+  return (int)cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// First pass of the dynamic base (section 3.1: the base is the minimum of M_i
+// over all sub-channels, which needs a pass over the data before any
+// sub-channel can be quantized).  Each thread owns 16 bytes of channels (8
+// bf16 or 4 fp32) of one 16-token tile, reads its 16 rows of X_t and X_{t-1},
+// forms |dX| with the same fp32 subtraction as the quantizer and keeps the
+// per-channel maxima; the smallest nonzero finite one of the warp goes to an
+// atomic minimum on the fp32 bits (positive floats order like their bits).
+// ---------------------------------------------------------------------------
+template <typename TIn>
+__global__ void __launch_bounds__(256) base_min_kernel(const TIn* __restrict__ x_t, const TIn* __restrict__ x_prev,
+                                                       int64_t ld_xt, int64_t ld_xp, int64_t M, int64_t K,
+                                                       uint32_t* out) {
+  constexpr int E = 16 / sizeof(TIn);  // channels per thread
+  const int64_t groups = K / E, T = M / kTile;
+  uint32_t best = 0xFFFFFFFFu;
+  pdl_launch_dependents();
+  pdl_wait();
+  for (int64_t item = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; item < T * groups;
+       item += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = item / groups, c = (item % groups) * E;
+    uint32_t mx[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) mx[e] = 0;
+#pragma unroll 8
+    for (int r = 0; r < kTile; ++r) {
+      const int64_t row = t * kTile + r;
+      const uint4 a = *reinterpret_cast<const uint4*>(x_t + row * ld_xt + c);
+      const uint4 b = *reinterpret_cast<const uint4*>(x_prev + row * ld_xp + c);
+      const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        float xa, xb;
+        if constexpr (sizeof(TIn) == 2) {
+          xa = __uint_as_float((e & 1) ? (aw[e >> 1] & 0xFFFF0000u) : (aw[e >> 1] << 16));
+          xb = __uint_as_float((e & 1) ? (bw[e >> 1] & 0xFFFF0000u) : (bw[e >> 1] << 16));
+        } else {
+          xa = __uint_as_float(aw[e]);
+          xb = __uint_as_float(bw[e]);
+        }
+        const uint32_t m = __float_as_uint(__fsub_rn(xa, xb)) & 0x7FFFFFFFu;
+        mx[e] = max(mx[e], m);  // NaN bits sort above infinity: the channel reads as non-finite
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < E; ++e)
+      if (mx[e] != 0u && mx[e] < 0x7F800000u) best = min(best, mx[e]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) best = min(best, __shfl_xor_sync(0xffffffffu, best, o));
+  if ((threadIdx.x & 31) == 0 && best != 0xFFFFFFFFu) atomicMin(out, best);
+}
+
+int launch_base_min(const void* x_t, const void* x_prev, int64_t ld_xt, int64_t ld_xp, int64_t M, int64_t K,
+                    int in_bf16, uint32_t* out, int num_sms, void* stream) {
+  const int64_t items = (M / kTile) * (K / (in_bf16 ? 8 : 4));
+  if (items == 0) return 0;
+  const int64_t want = (items + 255) / 256;
+  const int grid = (int)(want < 8LL * num_sms ? want : 8LL * num_sms);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid, 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.stream = (cudaStream_t)stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t ce;
+  if (in_bf16)
+    ce = cudaLaunchKernelEx(&cfg, base_min_kernel<__nv_bfloat16>, static_cast<const __nv_bfloat16*>(x_t),
+                            static_cast<const __nv_bfloat16*>(x_prev), ld_xt, ld_xp, M, K, out);
+  else
+    ce = cudaLaunchKernelEx(&cfg, base_min_kernel<float>, static_cast<const float*>(x_t),
+                            static_cast<const float*>(x_prev), ld_xt, ld_xp, M, K, out);
   if (ce != cudaSuccess) return (int)ce;
   return (int)cudaGetLastError();
 }

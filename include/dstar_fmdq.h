@@ -58,7 +58,7 @@
 extern "C" {
 #endif
 
-#define DSTAR_FMDQ_VERSION 1
+#define DSTAR_FMDQ_VERSION 2
 
 #if defined(__GNUC__)
 #define DSTAR_API __attribute__((visibility("default")))
@@ -86,6 +86,7 @@ extern "C" {
 /* tile_cfg.flags */
 #define DSTAR_FLAG_NO_XPREV_REFRESH 1u /* leave x_prev untouched (caller swaps buffers) */
 #define DSTAR_FLAG_SLICE_PATH 2u       /* compute every tile with the slice-stream kernel */
+#define DSTAR_FLAG_DYNAMIC_BASE 4u     /* FMDQ-DYN: base = min M_i of the call (see dstar_fmdq_linear) */
 
 /* limits of this implementation */
 #define DSTAR_TILE_TOKENS 16   /* tokens per sub-channel (the only supported tile) */
@@ -132,7 +133,9 @@ typedef struct {
  *   planes  int32 [T]      tensor-core operand planes the tile needs
  *   plane0/plane1 int8 [M x K]  shift-folded operands of the tensor-core GEMM
  *   mask1   uint32 [T x mask_words]  K-chunks (128 wide) where plane 1 is nonzero
- * T = M / 16. */
+ *   dyn_base fp32 word  the base found by the last DSTAR_FLAG_DYNAMIC_BASE call
+ * T = M / 16.  With DSTAR_FLAG_DYNAMIC_BASE, fpot holds FPoT relative to the
+ * dynamic base (b - 2 - PoT) and the records carry those tags. */
 typedef struct {
   size_t total;
   size_t status;
@@ -143,6 +146,8 @@ typedef struct {
   size_t records;
   int64_t mask_words;
   int64_t record_cap;
+  size_t dyn_base; /* fp32 word: the dynamic base of the last DSTAR_FLAG_DYNAMIC_BASE call
+                      (all bits set when no sub-channel had a nonzero M_i) */
 } dstar_fmdq_ws_layout;
 
 /* Workspace bytes needed by calls with M tokens and K input channels.
@@ -165,7 +170,15 @@ DSTAR_API int dstar_fmdq_workspace_init(void* workspace, size_t bytes, void* str
  *   w_q     [N x K] I8 in [-127, 127]: weights, W_deq[k][n] = w_q[n][k] * w_scale[n]
  *   w_scale [N] fp32 device array: per-output-channel weight scale
  *   base_scale: the static base of Eq. 3 (section 3.1 "predefined static base");
- *           an exact power of two 2^lb, lb in [DSTAR_BASE_LOG2_MIN, DSTAR_BASE_LOG2_MAX]
+ *           an exact power of two 2^lb, lb in [DSTAR_BASE_LOG2_MIN, DSTAR_BASE_LOG2_MAX].
+ *           With DSTAR_FLAG_DYNAMIC_BASE (FMDQ-DYN, the paper's dynamic-base
+ *           reference of section 5.2) a first pass over X_t and X_{t-1} finds
+ *           base = the minimum of M_i over the sub-channels with a nonzero,
+ *           finite M_i, and Eqs. 2-5 use it: PoT = ceil(log2(M_i / base)),
+ *           codes q = rne(fl32(dX / base) * 2^(b-2-PoT)), FPoT relative to the
+ *           base (b - 2 - PoT), Y_t = Y_{t-1} + acc * 2^-g_ref * base * w_scale.
+ *           base_scale then only sets the predefined thresholds,
+ *           Thr_N = base_scale * 2^(t0 + 2N) compared with M_i.
  *   tile_cfg: quantizer settings and workspace (see dstar_tile_cfg)
  *   y_out   [M x N] same dtype as y_prev: receives Y_t; may be y_prev itself
  *           (same pointer and ld) or a disjoint buffer, never a partial overlap

@@ -152,3 +152,27 @@ def full_parity(inp, tiles=None, flags=0, y_distinct=False, t0=None, force_bits=
     assert np.array_equal(g["acc"][rows], acc[rows]), "accumulators differ"
     exact = assert_y_close(g["y"][rows], y[rows])
     return g, q, acc, y, exact
+
+
+def run_oracle_dyn(inp: synth.LayerInputs, y_prev_f32=None):
+    """The oracle with the dynamic base; the call's base_scale (2^lb) sets the thresholds."""
+    spec = inp.spec
+    q = oracle.quantize_dyn(inp.as_f32("x_t"), inp.as_f32("x_prev"), spec.lb, spec.t0, spec.force_bits)
+    acc = oracle.acc_direct(q, inp.w_q)
+    yp = inp.as_f32("y_prev") if y_prev_f32 is None else y_prev_f32
+    y = oracle.epilogue_dyn_f32(acc, q.g_ref, q.base, inp.w_scale, yp, spec.dtype == "bf16")
+    return q, acc, y
+
+
+def dyn_parity(inp, debug=True):
+    """Dynamic base: GPU (DSTAR_FLAG_DYNAMIC_BASE) against the oracle, everything compared."""
+    g = run_gpu(inp, flags=nat.FLAG_DYNAMIC_BASE, debug=debug)
+    q, acc, y = run_oracle_dyn(inp)
+    assert g["status"] == 0, g["status"]
+    base = float(g["ws"].sections(inp.spec.M, inp.spec.K)["dyn_base"].cpu()[0])
+    assert base == q.base, (base, q.base)
+    assert_quant_parity(g, q)
+    if debug:
+        assert np.array_equal(g["acc"], acc), "accumulators differ"
+    exact = assert_y_close(g["y"], y)
+    return g, q, acc, y, exact

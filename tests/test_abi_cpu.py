@@ -42,7 +42,7 @@ def test_every_declared_symbol_is_exported(L):
 
 
 def test_version_and_strings(L):
-    assert nat.version() == 1
+    assert nat.version() == 2
     assert L.dstar_fmdq_error_string(-1) == b"invalid argument"
     assert L.dstar_fmdq_error_string(0) == b"ok"
 
@@ -58,6 +58,8 @@ def test_workspace_layout_consistent(L):
                 lay.mask1, lay.records]
         assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
         assert lay.plane1 - lay.plane0 >= M * K and lay.records + T * 4 * K * 8 <= lay.total
+        # the dynamic base word sits in the header, after the status word
+        assert lay.status + 4 <= lay.dyn_base and lay.dyn_base + 4 <= lay.plane0 and lay.dyn_base % 4 == 0
 
 
 def _fake_mat(rows, cols, dtype, ptr=0x100000, ld=None):
