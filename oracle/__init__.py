@@ -24,6 +24,9 @@ Parity status of each function (what pins it, see tests/test_oracle_pins.py):
                    to the static quantizer when the minimum is a power of two;
                    the error bound on tiny shapes.
   epilogue_dyn_f32 -- equal to epilogue_f32 when the base is a power of two.
+  gelu          -- GELU(0) = 0, GELU(1) = Phi(1), GELU(y) - GELU(-y) = y,
+                   against Python's math.erf element by element.
+  ffn_gelu      -- composition of the pinned pieces above.
 """
 from __future__ import annotations
 
@@ -68,6 +71,8 @@ def _load():
         lib.fmdq_orc_quantize_dyn.restype = ci
         lib.fmdq_orc_epilogue_dyn_f32.argtypes = [i64, i64, P, P, ctypes.c_float, P, P, ci, P]
         lib.fmdq_orc_epilogue_dyn_f32.restype = None
+        lib.fmdq_orc_gelu.argtypes = [P, i64, ci, P]
+        lib.fmdq_orc_gelu.restype = None
         lib.fmdq_orc_set_threads.argtypes = [ci]
         lib.fmdq_orc_set_threads.restype = None
         lib.fmdq_orc_max_threads.restype = ci
@@ -245,6 +250,25 @@ def linear(x_t, x_prev, y_prev, w_q, w_scale, lb, t0=0, force_bits=0, out_bf16=T
     acc = acc_direct(q, w_q, tiles) if path == "direct" else acc_slices(q, w_q, tiles)
     y = epilogue_f32(acc, q.g_ref, lb, w_scale, y_prev, out_bf16, tiles)
     return q, acc, y
+
+
+def gelu(y: np.ndarray, out_bf16: bool) -> np.ndarray:
+    """GELU(y) = y * Phi(y) in fp64, rounded to fp32 (then bf16 when out_bf16)."""
+    y = np.ascontiguousarray(y, np.float32)
+    out = np.empty_like(y)
+    _load().fmdq_orc_gelu(_p(y), y.size, int(out_bf16), _p(out))
+    return out
+
+
+def ffn_gelu(x_t, x_prev, y1_prev, w1, w1_scale, h_prev, y2_prev, w2, w2_scale, lb, t0=0, force_bits=0,
+             out_bf16=True):
+    """The chained FFN pair with the GELU between the layers (section 4.3):
+    layer 1 on (X_t, X_{t-1}), H_t = GELU(Y1_t), layer 2 on (H_t, H_{t-1}).
+    Returns (q1, acc1, y1, h, q2, acc2, y2)."""
+    q1, acc1, y1 = linear(x_t, x_prev, y1_prev, w1, w1_scale, lb, t0, force_bits, out_bf16)
+    h = gelu(y1, out_bf16)
+    q2, acc2, y2 = linear(h, h_prev, y2_prev, w2, w2_scale, lb, t0, force_bits, out_bf16)
+    return q1, acc1, y1, h, q2, acc2, y2
 
 
 def n_threads() -> int:
