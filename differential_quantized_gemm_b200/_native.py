@@ -30,6 +30,7 @@ EXPORTED = [
     "dstar_fmdq_version", "dstar_fmdq_error_string", "dstar_fmdq_last_error", "dstar_fmdq_workspace_size",
     "dstar_fmdq_workspace_layout", "dstar_fmdq_workspace_init", "dstar_fmdq_linear", "dstar_fmdq_quantize",
     "dstar_fmdq_slice_gemm", "dstar_fmdq_status", "dstar_fmdq_selftest_wait", "dstar_fmdq_linear_noalloc",
+    "dstar_fmdq_ffn_gelu",
 ]
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -82,6 +83,8 @@ def lib():
         L.dstar_fmdq_selftest_wait.argtypes = [P, ctypes.c_uint32, P]
         L.dstar_fmdq_linear_noalloc.argtypes = [MP, MP, MP, MP, P, ctypes.c_float, ctypes.POINTER(TileCfg), MP, P,
                                                 P]
+        L.dstar_fmdq_ffn_gelu.argtypes = [MP, MP, MP, MP, P, MP, MP, MP, MP, P, ctypes.c_float,
+                                          ctypes.POINTER(TileCfg), ctypes.POINTER(TileCfg), P]
         for name in EXPORTED[3:]:
             getattr(L, name).restype = ctypes.c_int
         _lib = L
@@ -209,6 +212,21 @@ def linear_noalloc(x_t, x_prev, y_prev, w_q, w_scale, base_scale: float, *, t0: 
                                            ctypes.c_void_p(w_scale.data_ptr()), base_scale, ctypes.byref(cfg),
                                            ctypes.byref(mo), st, _stream(stream)))
     return y_out
+
+
+def ffn_gelu(x_t, x_prev, y1_prev, w1, w1_scale, h_t, h_prev, y2_prev, w2, w2_scale, base_scale: float,
+             ws1: Workspace, ws2: Workspace, *, t0: int = 0, force_bits: int = 0, flags1: int = 0, flags2: int = 0,
+             debug1=(None, None), debug2=(None, None), stream=None):
+    """dstar_fmdq_ffn_gelu: layer 1, H_t = GELU(Y1_t) from its epilogue, layer 2 on
+    (H_t, H_{t-1}); y1_prev, y2_prev updated in place, h_t written, h_prev
+    refreshed.  debugN = (codes, acc) device buffers of layer N, or None."""
+    c1 = _cfg(ws1, t0, force_bits, flags1, *debug1)
+    c2 = _cfg(ws2, t0, force_bits, flags2, *debug2)
+    m = [mat(t) for t in (x_t, x_prev, y1_prev, w1, h_t, h_prev, y2_prev, w2)]
+    _check(lib().dstar_fmdq_ffn_gelu(*(ctypes.byref(v) for v in m[:4]), ctypes.c_void_p(w1_scale.data_ptr()),
+                                     *(ctypes.byref(v) for v in m[4:]), ctypes.c_void_p(w2_scale.data_ptr()),
+                                     base_scale, ctypes.byref(c1), ctypes.byref(c2), _stream(stream)))
+    return y2_prev
 
 
 def quantize(x_t, x_prev, base_scale: float, ws: Workspace, *, t0: int = 0, force_bits: int = 0, flags: int = 0,

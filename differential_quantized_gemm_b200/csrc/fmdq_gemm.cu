@@ -143,6 +143,21 @@ __device__ __forceinline__ void store_y(void* base, int64_t off, float y) {
   else static_cast<float*>(base)[off] = y;
 }
 
+// GELU(y) = y Phi(y) = 0.5 y (1 + erf(y / sqrt 2)), the activation between
+// the two layers of a DiT feed-forward block (section 4.3 "Operator
+// Mapping"), in fp32 with CUDA's erff.
+__device__ __forceinline__ float gelu(float y) {
+  return __fmul_rn(__fmul_rn(0.5f, y), __fadd_rn(1.f, erff(__fmul_rn(y, 0.70710678118654752f))));
+}
+
+// The stored Y_t as a float (bf16 outputs are rounded first), so that the
+// activation is a function of the cached output alone.
+template <bool OUT_BF16>
+__device__ __forceinline__ float stored_value(float y) {
+  if constexpr (OUT_BF16) return __bfloat162float(__float2bfloat16_rn(y));
+  else return y;
+}
+
 // The paper's accumulation order literally, for one 16-token tile and one
 // output column n: walk the tile's encoded stream in (FPoT, channel) order;
 // when the FPoT changes, shift the 16 running sums left by the difference,
@@ -152,7 +167,7 @@ template <bool OUT_BF16>
 __device__ void slice_stream_column(const uint2* recs, int cnt, const int8_t* bits_row, int g_ref,
                                     const int8_t* w_row, int64_t t, int64_t n, int lb, float beta, float ws,
                                     void* y_prev, int64_t ld_yp, void* y_out, int64_t ld_yo, int y_distinct,
-                                    int64_t* debug_acc, int64_t N) {
+                                    int64_t* debug_acc, int64_t N, void* h_out, int64_t ld_h) {
   int64_t acc[kTile];
 #pragma unroll
   for (int i = 0; i < kTile; ++i) acc[i] = 0;
@@ -189,6 +204,7 @@ __device__ void slice_stream_column(const uint2* recs, int cnt, const int8_t* bi
     const float y = epi(acc[i], true, p2, beta, ws, load_y<OUT_BF16>(y_prev, row * ld_yp + n));
     store_y<OUT_BF16>(y_out, row * ld_yo + n, y);
     if (y_distinct) store_y<OUT_BF16>(y_prev, row * ld_yp + n, y);
+    if (h_out) store_y<OUT_BF16>(h_out, row * ld_h + n, gelu(stored_value<OUT_BF16>(y)));
     if (debug_acc) debug_acc[row * N + n] = acc[i];
   }
 }
@@ -196,9 +212,13 @@ __device__ void slice_stream_column(const uint2* recs, int cnt, const int8_t* bi
 // One epilogue group: 32 columns of one row (this lane's), in place in its
 // swizzled 32 x 32 shared-memory tile.  acc = d0 (+ 256 d1 for rows of
 // two-plane tiles); y = y_prev + (((float)acc * p2) * beta) * w_scale, fp32, no FMA.
-template <bool OUT_BF16, bool WIDE>
+// With GELU, the activation of the stored values also goes to hrow (this
+// lane's row of the activation output at the group's first column, global
+// memory), 16 bytes per chunk, for the first hchunks chunks (columns < N).
+template <bool OUT_BF16, bool WIDE, bool GELU>
 __device__ __forceinline__ void epi_group(uint8_t* row, int swz, const float* ws32, const uint32_t (&d0)[32],
-                                          const uint32_t (&d1)[32], bool wide_row, float p2, float beta) {
+                                          const uint32_t (&d1)[32], bool wide_row, float p2, float beta,
+                                          uint8_t* hrow, int hchunks) {
   constexpr int kOutBytes = OUT_BF16 ? 2 : 4;
   constexpr int E = 16 / kOutBytes;              // outputs per 16-byte chunk
   constexpr int kChunks = 32 * kOutBytes / 16;   // chunks per 32-column row
@@ -234,8 +254,27 @@ __device__ __forceinline__ void epi_group(uint8_t* row, int swz, const float* ws
         w[q] = *reinterpret_cast<const uint32_t*>(&b2);
       }
       *cp = make_uint4(w[0], w[1], w[2], w[3]);
+      if constexpr (GELU) {
+        if (c < hchunks) {
+          uint32_t h[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162*>(&w[q]);
+            const __nv_bfloat162 g2 =
+                __floats2bfloat162_rn(gelu(__bfloat162float(b2.x)), gelu(__bfloat162float(b2.y)));
+            h[q] = *reinterpret_cast<const uint32_t*>(&g2);
+          }
+          *reinterpret_cast<uint4*>(hrow + 16 * c) = make_uint4(h[0], h[1], h[2], h[3]);
+        }
+      }
     } else {
       *cp = make_uint4(__float_as_uint(y[0]), __float_as_uint(y[1]), __float_as_uint(y[2]), __float_as_uint(y[3]));
+      if constexpr (GELU) {
+        if (c < hchunks)
+          *reinterpret_cast<uint4*>(hrow + 16 * c) = make_uint4(
+              __float_as_uint(gelu(y[0])), __float_as_uint(gelu(y[1])), __float_as_uint(gelu(y[2])),
+              __float_as_uint(gelu(y[3])));
+      }
     }
   }
 }
@@ -244,7 +283,7 @@ __device__ __forceinline__ void epi_group(uint8_t* row, int swz, const float* ws
 
 size_t gemm_smem_bytes(int bn) { return bn == 256 ? GemmCfg<256, true>::kBytes : GemmCfg<128, true>::kBytes; }
 
-template <int BN, bool OUT_BF16>
+template <int BN, bool OUT_BF16, bool GELU>
 __global__ void __launch_bounds__(kGThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CUtensorMap tm_a1,
                 const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_yp,
@@ -567,9 +606,22 @@ __global__ void __launch_bounds__(kGThreads, 1)
           };
           uint8_t* my_row = ybuf + lane * (32 * C::kOutBytes);
           const int swz = sw(lane);
+          // this lane's row of the activation output at group g (GELU only)
+          auto h_row = [&](int g, int& hch) -> uint8_t* {
+            hch = 0;
+            if constexpr (!GELU) return nullptr;
+            constexpr int E = 16 / C::kOutBytes;
+            const int64_t n0 = n_half + g * 32, left = p.N - n0;
+            if (left <= 0) return nullptr;
+            hch = left >= 32 ? 32 / E : (int)(left / E);
+            return static_cast<uint8_t*>(p.h_out) + (row * p.ld_h + n0) * C::kOutBytes;
+          };
           auto one_plane_group = [&](int g, const uint32_t (&d)[32]) {
             if (row_ok) {
-              epi_group<OUT_BF16, false>(my_row + g * C::kBoxBytes, swz, ws_h + g * 32, d, d, false, p2, beta);
+              int hch;
+              uint8_t* hr = h_row(g, hch);
+              epi_group<OUT_BF16, false, GELU>(my_row + g * C::kBoxBytes, swz, ws_h + g * 32, d, d, false, p2, beta,
+                                               hr, hch);
               if (p.debug_acc) debug_group(g, d, d, false);
             }
             store_group(g);
@@ -598,7 +650,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
               tmem_ld_wait(d0);
               tmem_ld_wait(d1);
               if (row_ok) {
-                epi_group<OUT_BF16, true>(my_row + g * C::kBoxBytes, swz, ws_h + g * 32, d0, d1, wide_row, p2, beta);
+                int hch;
+                uint8_t* hr = h_row(g, hch);
+                epi_group<OUT_BF16, true, GELU>(my_row + g * C::kBoxBytes, swz, ws_h + g * 32, d0, d1, wide_row, p2,
+                                                beta, hr, hch);
                 if (p.debug_acc) debug_group(g, d0, d1, true);
               }
               store_group(g);
@@ -626,7 +681,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
             if (n >= p.N) continue;
             slice_stream_column<OUT_BF16>(p.records + (int64_t)t * p.record_cap, p.count[t], p.bits + (int64_t)t * p.K,
                                           p.g_ref[t], p.w_q + n * p.ld_w, t, n, p.lb, beta, ws_tile[c], p.y_prev, p.ld_yp,
-                                          p.y_out, p.ld_yo, p.y_distinct, p.debug_acc, p.N);
+                                          p.y_out, p.ld_yo, p.y_distinct, p.debug_acc, p.N, p.h_out, p.ld_h);
           }
         }
       }
@@ -674,7 +729,7 @@ __global__ void __launch_bounds__(256) slice_gemm_kernel(const SliceParams p) {
     if (n >= p.N) continue;
     slice_stream_column<OUT_BF16>(p.records + t * p.record_cap, p.count[t], p.bits + t * p.K, p.g_ref[t],
                                   p.w_q + n * p.ld_w, t, n, p.lb, beta, p.w_scale[n], p.y_prev, p.ld_yp, p.y_out, p.ld_yo,
-                                  p.y_distinct, p.debug_acc, p.N);
+                                  p.y_distinct, p.debug_acc, p.N, p.h_out, p.ld_h);
   }
 }
 
@@ -691,13 +746,13 @@ __global__ void selftest_wait_kernel(uint32_t* status, uint64_t limit_ns) {
   }
 }
 
-template <int BN, bool BF>
+template <int BN, bool BF, bool GELU>
 static int launch_gemm_t(const GemmParams& p, const CUtensorMap* m, int num_sms, void* stream) {
   const int tiles = p.tiles_m * p.tiles_n;
   const int grid = tiles < num_sms ? tiles : num_sms;
   if (grid == 0) return 0;
   const int smem = GemmCfg<BN, BF>::kBytes;
-  const int e = ensure_max_smem((const void*)gemm_kernel<BN, BF>, smem);
+  const int e = ensure_max_smem((const void*)gemm_kernel<BN, BF, GELU>, smem);
   if (e != 0) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid, 1, 1);
@@ -709,17 +764,23 @@ static int launch_gemm_t(const GemmParams& p, const CUtensorMap* m, int num_sms,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t ce = cudaLaunchKernelEx(&cfg, gemm_kernel<BN, BF>, m[0], m[1], m[2], m[3], m[4], p);
+  const cudaError_t ce = cudaLaunchKernelEx(&cfg, gemm_kernel<BN, BF, GELU>, m[0], m[1], m[2], m[3], m[4], p);
   if (ce != cudaSuccess) return (int)ce;
   return (int)cudaGetLastError();
 }
 
 // maps: the A0, A1, W, y_prev and y_out tensor maps (CUtensorMap[5]).
+template <bool GELU>
+static int launch_gemm_g(const GemmParams& p, const CUtensorMap* m, int bn, int out_bf16, int num_sms, void* stream) {
+  if (out_bf16) return bn == 256 ? launch_gemm_t<256, true, GELU>(p, m, num_sms, stream)
+                                 : launch_gemm_t<128, true, GELU>(p, m, num_sms, stream);
+  return launch_gemm_t<128, false, GELU>(p, m, num_sms, stream);  // fp32 outputs use 128-column tiles
+}
+
 int launch_gemm(const GemmParams& p, const void* maps, int bn, int out_bf16, int num_sms, void* stream) {
   const CUtensorMap* m = static_cast<const CUtensorMap*>(maps);
-  if (out_bf16) return bn == 256 ? launch_gemm_t<256, true>(p, m, num_sms, stream)
-                                 : launch_gemm_t<128, true>(p, m, num_sms, stream);
-  return launch_gemm_t<128, false>(p, m, num_sms, stream);  // fp32 outputs use 128-column tiles
+  return p.h_out ? launch_gemm_g<true>(p, m, bn, out_bf16, num_sms, stream)
+                 : launch_gemm_g<false>(p, m, bn, out_bf16, num_sms, stream);
 }
 
 int launch_slice_gemm(const SliceParams& p, int out_bf16, int num_sms, void* stream) {

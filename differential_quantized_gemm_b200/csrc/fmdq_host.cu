@@ -243,7 +243,8 @@ int choose_bn(int64_t M, int64_t N, int sms) {
 }
 
 int do_gemm(const dstar_mat* w_q, const float* w_scale, dstar_mat* y_prev, int lb, const dstar_tile_cfg* c,
-            dstar_mat* y_out, int64_t M, int64_t K, int64_t N, const DevInfo& dev, void* stream) {
+            dstar_mat* y_out, int64_t M, int64_t K, int64_t N, const DevInfo& dev, void* stream,
+            dstar_mat* h_out = nullptr) {
   if (N == 0 || M == 0) return DSTAR_OK;
   const WsLayout L = ws_layout(M, K);
   const bool bf16 = y_prev->dtype == DSTAR_BF16;
@@ -279,6 +280,8 @@ int do_gemm(const dstar_mat* w_q, const float* w_scale, dstar_mat* y_prev, int l
     g.status = ws_ptr<uint32_t>(c, L.status);
     g.debug_acc = c->debug_acc;
     g.dyn_base = dyn_base;
+    g.h_out = h_out ? h_out->data : nullptr;
+    g.ld_h = h_out ? h_out->ld : 0;
     g.tiles_m = (int)((M + kBlockM - 1) / kBlockM);
     g.tiles_n = (int)((N + bn - 1) / bn);
     g.num_chunks = (int)((K + kChunkK - 1) / kChunkK);
@@ -312,6 +315,8 @@ int do_gemm(const dstar_mat* w_q, const float* w_scale, dstar_mat* y_prev, int l
   s.all_tiles = 1;
   s.debug_acc = c->debug_acc;
   s.dyn_base = dyn_base;
+  s.h_out = h_out ? h_out->data : nullptr;
+  s.ld_h = h_out ? h_out->ld : 0;
   const int e = launch_slice_gemm(s, bf16, dev.sms, stream);
   if (e) return cuda_fail(e, "slice-stream launch");
   return DSTAR_OK;
@@ -510,6 +515,54 @@ int dstar_fmdq_linear(const dstar_mat* x_t, dstar_mat* x_prev, dstar_mat* y_prev
                        N > 0 ? y_prev : nullptr)) != DSTAR_OK)
     return r;
   if ((r = do_gemm(w_q, w_scale, y_prev, lb, tile_cfg, y_out, M, K, N, dev, stream)) != DSTAR_OK) return r;
+  return ok();
+}
+
+int dstar_fmdq_ffn_gelu(const dstar_mat* x_t, dstar_mat* x_prev, dstar_mat* y1_prev, const dstar_mat* w1,
+                        const float* w1_scale, dstar_mat* h_t, dstar_mat* h_prev, dstar_mat* y2_prev,
+                        const dstar_mat* w2, const float* w2_scale, float base_scale, const dstar_tile_cfg* cfg1,
+                        const dstar_tile_cfg* cfg2, void* stream) {
+  int r;
+  if (!x_t || !x_prev || !w1 || !w2 || !h_t || !h_prev || !y1_prev || !y2_prev)
+    return fail(DSTAR_ERR_INVALID_ARG, "a matrix argument is NULL");
+  const int64_t M = x_t->rows, K1 = x_t->cols, N1 = w1->rows;
+  // layer 1: X (M x K1) -> Y1 (M x N1); its GELU output H is layer 2's input (K2 = N1)
+  if ((r = check_mk(M, K1)) != DSTAR_OK) return r;
+  if ((r = check_mat(x_t, "x_t", M, K1, true)) != DSTAR_OK) return r;
+  if ((r = check_mat(x_prev, "x_prev", M, K1, true)) != DSTAR_OK) return r;
+  if (x_t->dtype != x_prev->dtype) return fail(DSTAR_ERR_INVALID_ARG, "x_t and x_prev must share a dtype");
+  if (!(x_t->data == x_prev->data && x_t->ld == x_prev->ld) && overlap(x_t, x_prev))
+    return fail(DSTAR_ERR_INVALID_ARG, "x_t partially overlaps x_prev");
+  int64_t n1 = 0, n2 = 0;
+  if ((r = check_gemm_args(w1, w1_scale, y1_prev, y1_prev, M, K1, &n1)) != DSTAR_OK) return r;
+  if (N1 <= 0 || N1 % 32 != 0 || N1 > DSTAR_K_MAX)
+    return fail(DSTAR_ERR_INVALID_ARG, "N1=%lld (layer 2's K) must be a positive multiple of 32 up to %d",
+                (long long)N1, DSTAR_K_MAX);
+  if ((r = check_mat(h_t, "h_t", M, N1, true)) != DSTAR_OK) return r;
+  if ((r = check_mat(h_prev, "h_prev", M, N1, true)) != DSTAR_OK) return r;
+  if (h_t->dtype != y1_prev->dtype || h_prev->dtype != y1_prev->dtype)
+    return fail(DSTAR_ERR_INVALID_ARG, "h_t and h_prev must have y1_prev's dtype");
+  if (overlap(h_t, h_prev) || overlap(h_t, y1_prev) || overlap(h_prev, y1_prev))
+    return fail(DSTAR_ERR_INVALID_ARG, "h_t, h_prev and y1_prev must be disjoint");
+  if ((r = check_gemm_args(w2, w2_scale, y2_prev, y2_prev, M, N1, &n2)) != DSTAR_OK) return r;
+  if (overlap(y2_prev, h_t) || overlap(y2_prev, h_prev) || overlap(y2_prev, y1_prev))
+    return fail(DSTAR_ERR_INVALID_ARG, "y2_prev overlaps another buffer of the pair");
+  int lb = 0;
+  if ((r = base_log2(base_scale, &lb)) != DSTAR_OK) return r;
+  if ((r = check_cfg(cfg1, M, K1)) != DSTAR_OK) return r;
+  if ((r = check_cfg(cfg2, M, N1)) != DSTAR_OK) return r;
+  if (cfg1->workspace == cfg2->workspace) return fail(DSTAR_ERR_WORKSPACE, "the two layers need two workspaces");
+  if (M == 0) return ok();
+  DevInfo dev;
+  if ((r = device_info(&dev)) != DSTAR_OK) return r;
+  // layer 1, its epilogue also writing H_t = GELU(Y1_t)
+  if ((r = do_quantize(x_t, x_prev, lb, cfg1, M, K1, dev, stream, w1, y1_prev)) != DSTAR_OK) return r;
+  if ((r = do_gemm(w1, w1_scale, y1_prev, lb, cfg1, y1_prev, M, K1, N1, dev, stream, h_t)) != DSTAR_OK) return r;
+  // layer 2 on the differential H_t - H_{t-1}
+  if ((r = do_quantize(h_t, h_prev, lb, cfg2, M, N1, dev, stream, n2 > 0 ? w2 : nullptr,
+                       n2 > 0 ? y2_prev : nullptr)) != DSTAR_OK)
+    return r;
+  if ((r = do_gemm(w2, w2_scale, y2_prev, lb, cfg2, y2_prev, M, N1, n2, dev, stream)) != DSTAR_OK) return r;
   return ok();
 }
 

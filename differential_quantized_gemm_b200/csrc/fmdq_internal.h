@@ -73,6 +73,8 @@ struct GemmParams {
   uint32_t* status;
   int64_t* debug_acc;
   const uint32_t* dyn_base;  // dynamic base word (nullptr = static base, whose scale is in lb)
+  void* h_out;               // GELU(Y_t) output, same dtype as y (nullptr = none)
+  int64_t ld_h;
   int tiles_m, tiles_n, num_chunks;
   // encoded stream, for tiles whose operands need more than two planes
   const int8_t* w_q;
@@ -103,6 +105,8 @@ struct SliceParams {
   int all_tiles;  // 1: every tile; 0: only tiles that need more than two planes
   int64_t* debug_acc;
   const uint32_t* dyn_base;
+  void* h_out;  // GELU(Y_t) output (nullptr = none)
+  int64_t ld_h;
 };
 
 // Workspace sections (byte offsets from the workspace base).

@@ -191,6 +191,33 @@ DSTAR_API int dstar_fmdq_linear(const dstar_mat* x_t, dstar_mat* x_prev, dstar_m
                       dstar_mat* y_out, void* stream);
 
 /*
+ * The chained feed-forward pair of a DiT block with the GELU fused into the
+ * first layer's epilogue (section 4.3 "Operator Mapping": the reverse
+ * differential and the GELU activation are fused with the linear layer):
+ *   Y1_t = Y1_{t-1} + FMDQ(X_t - X_{t-1}) W1        (layer 1, cache y1_prev)
+ *   H_t  = GELU(Y1_t) = Y1_t Phi(Y1_t)                written by layer 1's epilogue
+ *   Y2_t = Y2_{t-1} + FMDQ(H_t - H_{t-1}) W2        (layer 2, cache y2_prev)
+ *   x_t, x_prev   [M x K1]: as in dstar_fmdq_linear (x_prev refreshed unless
+ *                 cfg1 has DSTAR_FLAG_NO_XPREV_REFRESH)
+ *   y1_prev       [M x N1] F32/BF16: layer 1's cache, updated in place to Y1_t
+ *   w1 [N1 x K1] I8, w1_scale [N1]
+ *   h_t           [M x N1], y1_prev's dtype: receives H_t (GELU of the stored
+ *                 Y1_t value, fp32 erf form, rounded to the dtype)
+ *   h_prev        [M x N1]: H_{t-1}; refreshed to H_t unless cfg2 has
+ *                 DSTAR_FLAG_NO_XPREV_REFRESH (then the caller swaps h_t, h_prev)
+ *   y2_prev       [M x N2] F32/BF16: layer 2's cache, updated in place to Y2_t
+ *   w2 [N2 x N1] I8, w2_scale [N2]
+ *   cfg1, cfg2    each layer's settings and its own workspace, sized for
+ *                 (M, K1) and (M, N1)
+ * N1 must be a positive multiple of 32 (it is layer 2's K); h_t, h_prev,
+ * y1_prev and y2_prev must not overlap.  Errors as dstar_fmdq_linear.
+ */
+DSTAR_API int dstar_fmdq_ffn_gelu(const dstar_mat* x_t, dstar_mat* x_prev, dstar_mat* y1_prev, const dstar_mat* w1,
+                                  const float* w1_scale, dstar_mat* h_t, dstar_mat* h_prev, dstar_mat* y2_prev,
+                                  const dstar_mat* w2, const float* w2_scale, float base_scale,
+                                  const dstar_tile_cfg* cfg1, const dstar_tile_cfg* cfg2, void* stream);
+
+/*
  * dstar_fmdq_linear for callers that cannot allocate device memory.  The
  * paper has no counterpart: this is a packaging choice of the library.
  *
