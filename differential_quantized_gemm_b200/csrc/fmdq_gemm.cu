@@ -143,11 +143,12 @@ __device__ __forceinline__ void store_y(void* base, int64_t off, float y) {
   else static_cast<float*>(base)[off] = y;
 }
 
-// GELU(y) = y Phi(y) = 0.5 y (1 + erf(y / sqrt 2)), the activation between
-// the two layers of a DiT feed-forward block (section 4.3 "Operator
-// Mapping"), in fp32 with CUDA's erff.
+// GELU(y) = y Phi(y) = 0.5 y erfc(-y / sqrt 2), the activation between the
+// two layers of a DiT feed-forward block (section 4.3 "Operator Mapping"),
+// in fp32 with CUDA's erfcf (the erfc form keeps its relative accuracy in
+// the negative tail, where 1 + erf cancels).
 __device__ __forceinline__ float gelu(float y) {
-  return __fmul_rn(__fmul_rn(0.5f, y), __fadd_rn(1.f, erff(__fmul_rn(y, 0.70710678118654752f))));
+  return __fmul_rn(__fmul_rn(0.5f, y), erfcf(__fmul_rn(y, -0.70710678118654752f)));
 }
 
 // The stored Y_t as a float (bf16 outputs are rounded first), so that the

@@ -202,7 +202,7 @@ DSTAR_API int dstar_fmdq_linear(const dstar_mat* x_t, dstar_mat* x_prev, dstar_m
  *   y1_prev       [M x N1] F32/BF16: layer 1's cache, updated in place to Y1_t
  *   w1 [N1 x K1] I8, w1_scale [N1]
  *   h_t           [M x N1], y1_prev's dtype: receives H_t (GELU of the stored
- *                 Y1_t value, fp32 erf form, rounded to the dtype)
+ *                 Y1_t value, 0.5 y erfc(-y / sqrt 2) in fp32, rounded to the dtype)
  *   h_prev        [M x N1]: H_{t-1}; refreshed to H_t unless cfg2 has
  *                 DSTAR_FLAG_NO_XPREV_REFRESH (then the caller swaps h_t, h_prev)
  *   y2_prev       [M x N2] F32/BF16: layer 2's cache, updated in place to Y2_t

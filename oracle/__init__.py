@@ -25,7 +25,8 @@ Parity status of each function (what pins it, see tests/test_oracle_pins.py):
                    the error bound on tiny shapes.
   epilogue_dyn_f32 -- equal to epilogue_f32 when the base is a power of two.
   gelu          -- GELU(0) = 0, GELU(1) = Phi(1), GELU(y) - GELU(-y) = y,
-                   against Python's math.erf element by element.
+                   against Python's math.erfc element by element, and
+                   against math.erf away from the negative tail.
   ffn_gelu      -- composition of the pinned pieces above.
 """
 from __future__ import annotations
@@ -253,7 +254,7 @@ def linear(x_t, x_prev, y_prev, w_q, w_scale, lb, t0=0, force_bits=0, out_bf16=T
 
 
 def gelu(y: np.ndarray, out_bf16: bool) -> np.ndarray:
-    """GELU(y) = y * Phi(y) in fp64, rounded to fp32 (then bf16 when out_bf16)."""
+    """GELU(y) = y * Phi(y) = 0.5 y erfc(-y / sqrt 2) in fp64, rounded to fp32 (then bf16 when out_bf16)."""
     y = np.ascontiguousarray(y, np.float32)
     out = np.empty_like(y)
     _load().fmdq_orc_gelu(_p(y), y.size, int(out_bf16), _p(out))

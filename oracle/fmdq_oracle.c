@@ -530,15 +530,17 @@ void fmdq_orc_epilogue_f64(int64_t M, int64_t N, const int64_t* acc, const int32
  * GELU between the two linear layers of a DiT feed-forward block (section
  * 4.3, "Operator Mapping": the activation is fused with the first layer's
  * output).  The pages name GELU without a variant; this is its definition,
- * GELU(y) = y * Phi(y) = 0.5 y (1 + erf(y / sqrt 2)), evaluated in fp64 on
- * the layer's cached output value y (fp32, or bf16 widened exactly) and
- * rounded to fp32, then to bf16 (RNE) when out_bf16 is set.
+ * GELU(y) = y * Phi(y), with the normal CDF written Phi(y) = erfc(-y / sqrt 2) / 2
+ * (the same function as (1 + erf(y / sqrt 2)) / 2, without the cancellation
+ * of 1 + erf in the negative tail), evaluated in fp64 on the layer's cached
+ * output value y (fp32, or bf16 widened exactly) and rounded to fp32, then
+ * to bf16 (RNE) when out_bf16 is set.
  */
 void fmdq_orc_gelu(const float* y, int64_t n, int out_bf16, float* out) {
 #pragma omp parallel for schedule(static)
   for (int64_t i = 0; i < n; ++i) {
     double v = (double)y[i];
-    double g = 0.5 * v * (1.0 + erf(v / sqrt(2.0)));
+    double g = 0.5 * v * erfc(-v / sqrt(2.0));
     float r = (float)g;
     if (out_bf16) r = bf16_bits_to_float(float_to_bf16_bits(r));
     out[i] = r;

@@ -12,7 +12,7 @@ from differential_quantized_gemm_b200 import synth
 
 
 def _gelu_math(v: float) -> float:
-    return 0.5 * v * (1.0 + math.erf(v / math.sqrt(2.0)))
+    return 0.5 * v * math.erfc(-v / math.sqrt(2.0))
 
 
 def test_closed_form_values(orc):
@@ -33,13 +33,19 @@ def test_odd_part_identity():
     assert (err <= 2.0 ** -23 * (np.abs(gp) + np.abs(gm)) + 1e-30).all()
 
 
-def test_against_math_erf_elementwise(orc):
-    y = np.concatenate([np.linspace(-6, 6, 2001), np.random.default_rng(1).standard_normal(2000) * 2]).astype(np.float32)
+def test_against_math_erfc_elementwise(orc):
+    y = np.concatenate([np.linspace(-12, 6, 3001), np.random.default_rng(1).standard_normal(2000) * 2]).astype(np.float32)
     g = orc.gelu(y, False)
     ref = np.array([np.float32(_gelu_math(float(v))) for v in y])
     assert np.array_equal(g, ref)
     gb = orc.gelu(y, True)
     assert np.array_equal(gb, orc.bf16_to_f32(orc.f32_to_bf16(ref)))
+    # the erf form of the same function agrees where 1 + erf does not cancel
+    mid = y > -2
+    erf_form = np.array([np.float32(0.5 * float(v) * (1.0 + math.erf(float(v) / math.sqrt(2.0)))) for v in y[mid]])
+    assert np.allclose(g[mid], erf_form, rtol=1e-6, atol=1e-12)
+    # and the negative tail keeps its relative accuracy (no cancellation)
+    assert g[0] < 0 and abs(g[0] / np.float32(-12 * 0.5 * math.erfc(12 / math.sqrt(2.0))) - 1) < 1e-6
 
 
 def test_chain_is_two_linears_with_gelu_between(orc):
