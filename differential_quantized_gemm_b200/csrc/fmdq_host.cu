@@ -221,10 +221,18 @@ int do_quantize(const dstar_mat* x_t, dstar_mat* x_prev, int lb, const dstar_til
                                   stream);
     if (e) return cuda_fail(e, "dynamic-base launch");
   }
+  // L2 prefetch of the next GEMM's operands: only what stays resident until the
+  // GEMM reads it (half of the 126 MB L2); a larger region would be evicted
+  // before use and only add HBM traffic
+  constexpr int64_t kPrefetchBudget = 64ll << 20;
   const dstar_mat* pf[2] = {pf_w, pf_y};
+  int64_t budget = kPrefetchBudget;
   for (int i = 0; i < 2; ++i) {
     if (pf[i] && pf[i]->data && pf[i]->rows > 0 && pf[i]->cols > 0) {
       const int64_t es = (int64_t)elem_size(pf[i]->dtype);
+      const int64_t bytes = pf[i]->rows * pf[i]->cols * es;
+      if (bytes > budget) continue;
+      budget -= bytes;
       q.prefetch[i] = L2Region{static_cast<const uint8_t*>(pf[i]->data), pf[i]->rows, pf[i]->cols * es,
                                pf[i]->ld * es};
     }

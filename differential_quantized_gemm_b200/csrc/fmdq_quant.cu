@@ -1,9 +1,12 @@
 // K1: the FMDQ quantizer (DSTAR section 3.1 steps 1-4; the paper's QPU,
 // section 4.2 "Design of QPU", stages 1-5).
 //
-// One 16-token tile is handled by a thread-block cluster of C CTAs (C = 1, 2,
-// 4 or 8, chosen so that small batches still fill every SM); CTA r owns a
-// contiguous range of channels.  Every thread owns pairs of adjacent channels
+// Two kernels share the per-tile stages.  For small batches one 16-token tile
+// is handled by a thread-block cluster of C CTAs (C = 1, 2, 4 or 8, chosen so
+// that small batches still fill every SM); CTA r owns a contiguous range of
+// channels.  For batches of at least two tiles per SM a persistent kernel
+// runs phase 1 of one tile and phase 2 of the previous one at the same time
+// (see quantize_persistent_kernel).  Every thread owns pairs of adjacent channels
 // and walks the 16 tokens, so a warp reads whole 128-byte row segments of X_t
 // and X_{t-1} and the per-channel max |dX| (stage 1: compare the magnitude
 // bits, sign dropped) stays inside the thread.  PoT (Eq. 3), the bit width
@@ -29,6 +32,21 @@ namespace cg = cooperative_groups;
 namespace fmdq {
 
 namespace {
+
+// Occupancy settings of the quantizer (compile-time; the defaults are the
+// measured best on B200): CTAs per SM the register budget is sized for,
+// whether phase 1 keeps the next channel pair's loads in flight, and the
+// channel count per CTA above which a tile is split over a cluster even when
+// the grid already fills the GPU (0: only to fill the GPU).
+#ifndef FMDQ_Q_MIN_BLOCKS
+#define FMDQ_Q_MIN_BLOCKS 2
+#endif
+#ifndef FMDQ_Q_PREFETCH
+#define FMDQ_Q_PREFETCH 1
+#endif
+#ifndef FMDQ_Q_SPLIT_K
+#define FMDQ_Q_SPLIT_K 0
+#endif
 
 constexpr int kQThreads = 256;
 constexpr int kQWarps = kQThreads / 32;
@@ -257,189 +275,187 @@ int quantize_cluster_size(int64_t M, int64_t K, int num_sms) {
   // about 1.5 CTAs per SM when the batch is small, at least 1024 channels per
   // CTA (below that the cluster exchanges cost more than the split gains)
   while (c < kMaxCluster && 2 * T * c < 3LL * num_sms && units / (2 * c) >= 32) c *= 2;
+  // a smaller share of channels per CTA lowers its shared memory, so more CTAs fit an SM
+  while (FMDQ_Q_SPLIT_K > 0 && c < kMaxCluster && K / c > FMDQ_Q_SPLIT_K && units / (2 * c) >= 32) c *= 2;
   return c;
 }
 
+// ------------------------------------------------------------------------
+// Per-tile stages, shared by the two quantizer kernels below.  `gt` is the
+// thread's index among the `NT` threads that run the stage together.
+
+// The call's constants of steps 1-2 (static or dynamic base).
+struct QConst {
+  int lb, t0, fb;
+  float beta;      // 2^lb
+  uint32_t dbits;  // dynamic base (fp32 bits), 1.0 when none
+  float dbase;
+  bool refresh;
+};
+
+template <bool DYN>
+__device__ __forceinline__ QConst quant_const(const QuantParams& p) {
+  QConst q;
+  q.lb = p.lb, q.t0 = p.t0, q.fb = p.force_bits;
+  q.beta = exp2_exact(q.lb);
+  q.dbits = 0x3F800000u;
+  if constexpr (DYN) {  // written by the first pass; all ones when no M_i was nonzero
+    q.dbits = *p.dyn_base;
+    if (q.dbits == 0xFFFFFFFFu) q.dbits = 0x3F800000u;
+  }
+  q.dbase = __uint_as_float(q.dbits);
+  q.refresh = !(p.flags & DSTAR_FLAG_NO_XPREV_REFRESH);
+  return q;
+}
+
+// Reductions phase 1 hands on: finest and coarsest FPoT, the plane-room
+// minima and the status flags of the thread's channels.
+struct P1Red {
+  int fmax, fmin, a1, a2, flags;
+};
+
+// Phase 1 (steps 1-3 of section 3.1; QPU stages 1-3) works on channel pairs:
+// a thread reads a pair's 16 token rows of X_t and X_{t-1} (a warp reads
+// 128-byte row segments), forms dX once (one fp32 subtraction), the magnitude
+// max, PoT, width, FPoT and the codes, and puts each channel's 16 codes into
+// shared memory as one 16-byte column; FPoT and width go to shared and global
+// memory, X_t into the x_prev cache.
+template <typename TIn>
+__device__ __forceinline__ void load_pair(const QuantParams& p, int64_t row0, int64_t c,
+                                          typename Pair<TIn>::Raw (&a)[kTile], typename Pair<TIn>::Raw (&b)[kTile]) {
+#pragma unroll
+  for (int i = 0; i < kTile; ++i) {
+    a[i] = Pair<TIn>::load(p.x_t, (row0 + i) * p.ld_xt + c);
+    b[i] = Pair<TIn>::load(p.x_prev, (row0 + i) * p.ld_xp + c);
+  }
+}
+
+// One channel pair (global channels c, c + 1; local lc, lc + 1) of tile t.
 template <typename TIn, bool DYN>
-__global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParams p, int C, int64_t kc_max) {
-  extern __shared__ __align__(16) uint8_t smem[];
+__device__ __forceinline__ void process_pair(const QuantParams& p, const QConst& qc, int64_t t, int64_t c, int lc,
+                                             const typename Pair<TIn>::Raw (&rt)[kTile],
+                                             const typename Pair<TIn>::Raw (&rp)[kTile], int8_t* s_code,
+                                             int8_t* s_fpot, int8_t* s_bits, P1Red& r) {
   using PR = Pair<TIn>;
-  cg::cluster_group cluster = cg::this_cluster();
-
   const int64_t K = p.K;
-  const int rank = (int)cluster.block_rank();
-  const int t = (int)(blockIdx.x / C);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t units = K / 32;
-  const int64_t k_lo = 32 * (rank * units / C), k_hi = 32 * ((rank + 1) * units / C);
-  const int Kc = (int)(k_hi - k_lo);
-
-  int8_t* s_code = reinterpret_cast<int8_t*>(smem);  // 16-byte slots: the 16 codes of a local channel
-  int8_t* s_fpot = s_code + 16 * kc_max;              // [Kc]
-  int8_t* s_bits = s_fpot + kc_max;                   // [Kc]
-  // [Kc / 32][kTagWin]: per 32-channel chunk and window tag, the ballot of the
-  // lanes carrying the tag and the warp's records of the tag in earlier chunks
-  uint2* s_tab = reinterpret_cast<uint2*>(s_bits + kc_max);
-  const int64_t tab_bytes = kc_max / 32 * kTagWin * 8;
-  QSmem& S = *reinterpret_cast<QSmem*>(smem + ((18 * kc_max + tab_bytes + 15) & ~(int64_t)15));
-
-  if (tid < kMaxMaskWords) S.mask[tid] = 0;
-  if (tid == 0) S.flags = 0;
-  pdl_launch_dependents();
-  pdl_wait();  // nothing of global memory is touched before the previous kernel completed
-  __syncthreads();
-
-  const int lb = p.lb, t0 = p.t0, fb = p.force_bits;
-  const float beta = exp2_exact(lb);
-  // dynamic base: written by the first pass; all ones when no M_i was nonzero
-  uint32_t dbits = 0x3F800000u;
+  const int64_t row0 = t * kTile;
+  if (qc.refresh) {
+#pragma unroll
+    for (int i = 0; i < kTile; ++i) PR::store(p.x_prev, (row0 + i) * p.ld_xp + c, rt[i]);
+  }
+  // Eq. 1 (one fp32 subtraction per element, kept) and stage 1 on the magnitude bits
+  float d0[kTile], d1[kTile];
+  uint32_t m0 = 0, m1 = 0;
+#pragma unroll
+  for (int i = 0; i < kTile; ++i) {
+    d0[i] = __fsub_rn(PR::lo(rt[i]), PR::lo(rp[i]));
+    d1[i] = __fsub_rn(PR::hi(rt[i]), PR::hi(rp[i]));
+    m0 = max(m0, __float_as_uint(d0[i]) & 0x7FFFFFFFu);
+    m1 = max(m1, __float_as_uint(d1[i]) & 0x7FFFFFFFu);
+  }
+  ColParams c0, c1;
   if constexpr (DYN) {
-    dbits = *p.dyn_base;
-    if (dbits == 0xFFFFFFFFu) dbits = 0x3F800000u;
+    c0 = col_params_dyn(m0, qc.dbits, qc.lb + qc.t0, qc.fb, r.flags);
+    c1 = col_params_dyn(m1, qc.dbits, qc.lb + qc.t0, qc.fb, r.flags);
+  } else {
+    c0 = col_params(m0, qc.lb, qc.beta, qc.t0, qc.fb, r.flags);
+    c1 = col_params(m1, qc.lb, qc.beta, qc.t0, qc.fb, r.flags);
   }
-  const float dbase = __uint_as_float(dbits);
-  const bool refresh = !(p.flags & DSTAR_FLAG_NO_XPREV_REFRESH);
-  const int64_t row0 = (int64_t)t * kTile;
-  const int npairs = Kc / 2;
-  int fmax = -1000, fmin = 1000, a1 = 1000, a2 = 1000;
-  int flags = 0;
-
-  // ---------------------------------------------------------------- phase 1
-  // bf16 inputs: the row words of a thread's next channel pair are requested
-  // before its current pair is processed, so two pairs' loads are in flight
-  // per thread (fp32 inputs would not fit the registers twice).
-  constexpr bool kAhead = sizeof(typename PR::Raw) == 4;
-  typename PR::Raw nt[kTile], np[kTile];
-  auto load_pair = [&](int pr, typename PR::Raw (&a)[kTile], typename PR::Raw (&b)[kTile]) {
-    const int64_t c = k_lo + 2 * pr;
+  // stage 3; a non-finite sub-channel has scale 0, and its NaN products convert to 0
+  const float s0 = c0.nonfinite ? 0.f : c0.scale, s1 = c1.nonfinite ? 0.f : c1.scale;
+  if constexpr (DYN) {  // dX / base first (one IEEE division), then the power-of-two scale
 #pragma unroll
-    for (int r = 0; r < kTile; ++r) {
-      a[r] = PR::load(p.x_t, (row0 + r) * p.ld_xt + c);
-      b[r] = PR::load(p.x_prev, (row0 + r) * p.ld_xp + c);
-    }
-  };
-  if (kAhead && tid < npairs) load_pair(tid, nt, np);
-  for (int pr = tid; pr < npairs; pr += kQThreads) {
-    const int lc = 2 * pr;
-    const int64_t c = k_lo + lc;
-    typename PR::Raw rt[kTile], rp[kTile];
-    if constexpr (kAhead) {
-#pragma unroll
-      for (int r = 0; r < kTile; ++r) rt[r] = nt[r], rp[r] = np[r];
-      if (pr + kQThreads < npairs) load_pair(pr + kQThreads, nt, np);
-    } else {
-      load_pair(pr, rt, rp);
-    }
-    if (refresh) {
-#pragma unroll
-      for (int r = 0; r < kTile; ++r) PR::store(p.x_prev, (row0 + r) * p.ld_xp + c, rt[r]);
-    }
-    // Eq. 1 (one fp32 subtraction per element, kept) and stage 1 on the magnitude bits
-    float d0[kTile], d1[kTile];
-    uint32_t m0 = 0, m1 = 0;
-#pragma unroll
-    for (int r = 0; r < kTile; ++r) {
-      d0[r] = __fsub_rn(PR::lo(rt[r]), PR::lo(rp[r]));
-      d1[r] = __fsub_rn(PR::hi(rt[r]), PR::hi(rp[r]));
-      m0 = max(m0, __float_as_uint(d0[r]) & 0x7FFFFFFFu);
-      m1 = max(m1, __float_as_uint(d1[r]) & 0x7FFFFFFFu);
-    }
-    ColParams c0, c1;
-    if constexpr (DYN) {
-      c0 = col_params_dyn(m0, dbits, lb + t0, fb, flags);
-      c1 = col_params_dyn(m1, dbits, lb + t0, fb, flags);
-    } else {
-      c0 = col_params(m0, lb, beta, t0, fb, flags);
-      c1 = col_params(m1, lb, beta, t0, fb, flags);
-    }
-    // stage 3; a non-finite sub-channel has scale 0, and its NaN products convert to 0
-    const float s0 = c0.nonfinite ? 0.f : c0.scale, s1 = c1.nonfinite ? 0.f : c1.scale;
-    if constexpr (DYN) {  // dX / base first (one IEEE division), then the power-of-two scale
-#pragma unroll
-      for (int r = 0; r < kTile; ++r) d0[r] = __fdiv_rn(d0[r], dbase), d1[r] = __fdiv_rn(d1[r], dbase);
-      m0 = __float_as_uint(__fdiv_rn(__uint_as_float(m0), dbase));
-      m1 = __float_as_uint(__fdiv_rn(__uint_as_float(m1), dbase));
-    }
-    uint32_t w0[4], w1[4];
-#pragma unroll
-    for (int R = 0; R < 4; ++R) {
-      int a[4], b[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        a[e] = __float2int_rn(__fmul_rn(d0[4 * R + e], s0));
-        b[e] = __float2int_rn(__fmul_rn(d1[4 * R + e], s1));
-      }
-      // low bytes of four codes, token 4R + e in byte e
-      w0[R] = __byte_perm(__byte_perm(a[0], a[1], 0x0040), __byte_perm(a[2], a[3], 0x0040), 0x5410);
-      w1[R] = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
-    }
-    // largest |code| of each channel: rne(M_i s_i) bounds every |rne(dX s_i)|
-    const int qa0 = c0.nonfinite ? 0 : __float2int_rn(__fmul_rn(__uint_as_float(m0), s0));
-    const int qa1 = c1.nonfinite ? 0 : __float2int_rn(__fmul_rn(__uint_as_float(m1), s1));
-    if (p.debug_codes) {
-#pragma unroll
-      for (int r = 0; r < kTile; ++r)
-        *reinterpret_cast<uint16_t*>(p.debug_codes + (row0 + r) * K + c) =
-            (uint16_t)(((w0[r >> 2] >> (8 * (r & 3))) & 0xFFu) | (((w1[r >> 2] >> (8 * (r & 3))) & 0xFFu) << 8));
-    }
-    *reinterpret_cast<uint4*>(s_code + 16 * code_slot(lc)) = make_uint4(w0[0], w0[1], w0[2], w0[3]);
-    *reinterpret_cast<uint4*>(s_code + 16 * code_slot(lc + 1)) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
-    auto two = [](int a, int b) { return (uint16_t)(((uint32_t)a & 0xFFu) | (((uint32_t)b & 0xFFu) << 8)); };
-    *reinterpret_cast<uint16_t*>(s_fpot + lc) = two(c0.fpot, c1.fpot);
-    *reinterpret_cast<uint16_t*>(s_bits + lc) = two(c0.bits, c1.bits);
-    *reinterpret_cast<uint16_t*>(p.fpot + (int64_t)t * K + c) = two(c0.fpot, c1.fpot);
-    *reinterpret_cast<uint16_t*>(p.bits + (int64_t)t * K + c) = two(c0.bits, c1.bits);
-    fmax = max(fmax, max(c0.fpot, c1.fpot));
-    fmin = min(fmin, min(c0.fpot, c1.fpot));
-    a1 = min(a1, min(c0.fpot + shift_room(qa0, false), c1.fpot + shift_room(qa1, false)));
-    a2 = min(a2, min(c0.fpot + shift_room(qa0, true), c1.fpot + shift_room(qa1, true)));
+    for (int i = 0; i < kTile; ++i) d0[i] = __fdiv_rn(d0[i], qc.dbase), d1[i] = __fdiv_rn(d1[i], qc.dbase);
+    m0 = __float_as_uint(__fdiv_rn(__uint_as_float(m0), qc.dbase));
+    m1 = __float_as_uint(__fdiv_rn(__uint_as_float(m1), qc.dbase));
   }
+  uint32_t w0[4], w1[4];
+#pragma unroll
+  for (int R = 0; R < 4; ++R) {
+    int a[4], b[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      a[e] = __float2int_rn(__fmul_rn(d0[4 * R + e], s0));
+      b[e] = __float2int_rn(__fmul_rn(d1[4 * R + e], s1));
+    }
+    // low bytes of four codes, token 4R + e in byte e
+    w0[R] = __byte_perm(__byte_perm(a[0], a[1], 0x0040), __byte_perm(a[2], a[3], 0x0040), 0x5410);
+    w1[R] = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
+  }
+  // largest |code| of each channel: rne(M_i s_i) bounds every |rne(dX s_i)|
+  const int qa0 = c0.nonfinite ? 0 : __float2int_rn(__fmul_rn(__uint_as_float(m0), s0));
+  const int qa1 = c1.nonfinite ? 0 : __float2int_rn(__fmul_rn(__uint_as_float(m1), s1));
+  if (p.debug_codes) {
+#pragma unroll
+    for (int i = 0; i < kTile; ++i)
+      *reinterpret_cast<uint16_t*>(p.debug_codes + (row0 + i) * K + c) =
+          (uint16_t)(((w0[i >> 2] >> (8 * (i & 3))) & 0xFFu) | (((w1[i >> 2] >> (8 * (i & 3))) & 0xFFu) << 8));
+  }
+  *reinterpret_cast<uint4*>(s_code + 16 * code_slot(lc)) = make_uint4(w0[0], w0[1], w0[2], w0[3]);
+  *reinterpret_cast<uint4*>(s_code + 16 * code_slot(lc + 1)) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+  auto two = [](int a, int b) { return (uint16_t)(((uint32_t)a & 0xFFu) | (((uint32_t)b & 0xFFu) << 8)); };
+  *reinterpret_cast<uint16_t*>(s_fpot + lc) = two(c0.fpot, c1.fpot);
+  *reinterpret_cast<uint16_t*>(s_bits + lc) = two(c0.bits, c1.bits);
+  *reinterpret_cast<uint16_t*>(p.fpot + t * K + c) = two(c0.fpot, c1.fpot);
+  *reinterpret_cast<uint16_t*>(p.bits + t * K + c) = two(c0.bits, c1.bits);
+  r.fmax = max(r.fmax, max(c0.fpot, c1.fpot));
+  r.fmin = min(r.fmin, min(c0.fpot, c1.fpot));
+  r.a1 = min(r.a1, min(c0.fpot + shift_room(qa0, false), c1.fpot + shift_room(qa1, false)));
+  r.a2 = min(r.a2, min(c0.fpot + shift_room(qa0, true), c1.fpot + shift_room(qa1, true)));
+}
 
-  // CTA reductions, then one exchange across the cluster
+// warp reduction of the phase-1 values (every lane gets the warp's result)
+__device__ __forceinline__ void warp_reduce(P1Red& r) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
-    fmax = max(fmax, __shfl_xor_sync(kFull, fmax, o));
-    fmin = min(fmin, __shfl_xor_sync(kFull, fmin, o));
-    a1 = min(a1, __shfl_xor_sync(kFull, a1, o));
-    a2 = min(a2, __shfl_xor_sync(kFull, a2, o));
-    flags |= __shfl_xor_sync(kFull, flags, o);
+    r.fmax = max(r.fmax, __shfl_xor_sync(kFull, r.fmax, o));
+    r.fmin = min(r.fmin, __shfl_xor_sync(kFull, r.fmin, o));
+    r.a1 = min(r.a1, __shfl_xor_sync(kFull, r.a1, o));
+    r.a2 = min(r.a2, __shfl_xor_sync(kFull, r.a2, o));
+    r.flags |= __shfl_xor_sync(kFull, r.flags, o);
   }
-  if (lane == 0) {
-    S.red[0][warp] = fmax, S.red[1][warp] = fmin, S.red[2][warp] = a1, S.red[3][warp] = a2;
-    if (flags) atomicOr(&S.flags, flags);
-  }
-  __syncthreads();
-  if (tid < 4) {
-    int v = S.red[tid][0];
-    for (int w = 1; w < kQWarps; ++w) v = tid == 0 ? max(v, S.red[tid][w]) : min(v, S.red[tid][w]);
-    S.xv[tid] = v;
-    if (tid == 0 && S.flags)
-      set_status(p.status, (S.flags & 1 ? DSTAR_STATUS_NONFINITE : 0u) | (S.flags & 2 ? DSTAR_STATUS_RANGE : 0u));
-  }
-  csync(cluster, C);
-  if (tid < 4 * C) {  // one remote read per thread, all in flight together
-    const int q = tid >> 2, u = tid & 3;
-    S.x[q][u] = (C > 1 ? cluster.map_shared_rank(&S, q) : &S)->xv[u];
-  }
-  __syncthreads();
-  int g = -1000, gmin = 1000, A1 = 1000, A2 = 1000;
-  for (int q = 0; q < C; ++q) {
-    g = max(g, S.x[q][0]), gmin = min(gmin, S.x[q][1]);
-    A1 = min(A1, S.x[q][2]), A2 = min(A2, S.x[q][3]);
-  }
-  // every v = q 2^(g - FPoT) must fit the split: g - FPoT <= room for each channel
-  const int planes = g <= A1 ? 1 : g <= A2 ? 2 : 3;
-  // HBM is idle from here on: pull the next GEMM's operands into L2
-  if (tid == 0) {
-    prefetch_region_share(p.prefetch[0], (int)blockIdx.x, (int)gridDim.x);
-    prefetch_region_share(p.prefetch[1], (int)blockIdx.x, (int)gridDim.x);
-  }
+}
 
-  // ------------------------------------------------- phase 2a: operand planes
-  // Four channels per thread: their 16-code columns, shifted, are transposed
-  // into 4-byte row words; a warp writes 128 contiguous bytes per row.
+// Phase 1 over channels [k_lo, k_lo + Kc) of tile t.  With bf16 inputs the
+// row words of the thread's next pair are requested before its current pair
+// is processed, so two pairs' loads are in flight per thread (fp32 inputs
+// would not fit the registers twice).
+template <typename TIn, bool DYN, int NT>
+__device__ __forceinline__ P1Red phase1(const QuantParams& p, const QConst& qc, int64_t t, int64_t k_lo, int Kc, int gt,
+                                        int8_t* s_code, int8_t* s_fpot, int8_t* s_bits) {
+  using Raw = typename Pair<TIn>::Raw;
+  const int64_t row0 = t * kTile;
+  const int npairs = Kc / 2;
+  P1Red r{-1000, 1000, 1000, 1000, 0};
+  constexpr bool kAhead = FMDQ_Q_PREFETCH && sizeof(Raw) == 4;
+  Raw nt[kTile], np[kTile];
+  if (kAhead && gt < npairs) load_pair<TIn>(p, row0, k_lo + 2 * gt, nt, np);
+  for (int pr = gt; pr < npairs; pr += NT) {
+    Raw rt[kTile], rp[kTile];
+    if constexpr (kAhead) {
+#pragma unroll
+      for (int i = 0; i < kTile; ++i) rt[i] = nt[i], rp[i] = np[i];
+      if (pr + NT < npairs) load_pair<TIn>(p, row0, k_lo + 2 * (pr + NT), nt, np);
+    } else {
+      load_pair<TIn>(p, row0, k_lo + 2 * pr, rt, rp);
+    }
+    process_pair<TIn, DYN>(p, qc, t, k_lo + 2 * pr, 2 * pr, rt, rp, s_code, s_fpot, s_bits, r);
+  }
+  warp_reduce(r);
+  return r;
+}
+
+// Phase 2a: the tensor-core operand planes of tile rows row0..row0+15,
+// channels [k_lo, k_lo + Kc).  Four channels per thread: their 16-code
+// columns, shifted by g - FPoT, are transposed into 4-byte row words; a warp
+// writes 128 contiguous bytes per row.  Chunks where plane 1 is nonzero are
+// marked in `mask` (shared memory).
+template <int NT>
+__device__ __forceinline__ void phase2_planes(const QuantParams& p, int64_t row0, int64_t k_lo, int Kc, int gt, int g,
+                                              int planes, const int8_t* s_code, const int8_t* s_fpot, uint32_t* mask) {
+  const int64_t K = p.K;
   if (planes == 1) {
-    for (int qd = tid; qd < Kc / 4; qd += kQThreads) {
+    for (int qd = gt; qd < Kc / 4; qd += NT) {
       const int lc = 4 * qd;
       const uint32_t f4 = *reinterpret_cast<const uint32_t*>(s_fpot + lc);
       uint32_t col[4][4];
@@ -462,7 +478,7 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParam
       }
     }
   } else if (planes == 2) {
-    for (int qd = tid; qd < Kc / 4; qd += kQThreads) {
+    for (int qd = gt; qd < Kc / 4; qd += NT) {
       const int lc = 4 * qd;
       uint32_t c0w[4][4], c1w[4][4];
       uint32_t nz = 0;
@@ -502,10 +518,140 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParam
       }
       if (nz) {
         const int chunk = (int)((k_lo + lc) / kChunkK);
-        atomicOr(&S.mask[chunk >> 5], 1u << (chunk & 31));
+        atomicOr(&mask[chunk >> 5], 1u << (chunk & 31));
       }
     }
   }
+}
+
+// Encoded stream, pass A for one window of kTagWin tags starting at tw, over
+// the warp's 32-channel chunks [ch_lo, ch_hi): per chunk, a warp bit
+// transpose of the lanes' tag masks gives every tag's lane ballot at once
+// (lane u: tag tw + u); the ballot and the warp's count of the tag before the
+// chunk go to the rank table.  Returns lane u's count of tag tw + u.
+__device__ __forceinline__ int count_window(int tw, int ch_lo, int ch_hi, int lane, const int8_t* s_fpot,
+                                            const int8_t* s_bits, uint2* s_tab) {
+  int cnt = 0;
+  for (int ch0 = ch_lo; ch0 < ch_hi; ch0 += kUA) {
+    uint32_t col[kUA];
+#pragma unroll
+    for (int u = 0; u < kUA; ++u) {
+      const int c = 32 * (ch0 + u) + lane;
+      const uint32_t m = ch0 + u < ch_hi ? tag_mask32(s_fpot[c], s_bits[c], tw) & ((1u << kTagWin) - 1u) : 0u;
+      col[u] = warp_bit_transpose(m, lane);
+    }
+#pragma unroll
+    for (int u = 0; u < kUA; ++u) {
+      if (ch0 + u < ch_hi && lane < kTagWin) {
+        s_tab[(ch0 + u) * kTagWin + lane] = make_uint2(col[u], (uint32_t)cnt);
+        cnt += __popc(col[u]);
+      }
+    }
+  }
+  return cnt;
+}
+
+// Encoded stream, pass B: every lane writes its channel's records of the
+// window; record of (tag, k) = the warp's first record of the tag (wb) + the
+// warp's count of the tag before the chunk + the set lanes below it in the
+// chunk's ballot.
+__device__ __forceinline__ void write_window(int tw, int ch_lo, int ch_hi, int lane, int64_t k_lo, const int* wb,
+                                             const int8_t* s_code, const int8_t* s_fpot, const int8_t* s_bits,
+                                             const uint2* s_tab, uint2* rec) {
+  const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll 2
+  for (int ch = ch_lo; ch < ch_hi; ++ch) {
+    const int c = 32 * ch + lane;
+    const int f = s_fpot[c], b = s_bits[c];
+    uint32_t words[4];
+    slice_words(*reinterpret_cast<const uint4*>(s_code + 16 * code_slot(c)), words);
+    const uint2* row = s_tab + ch * kTagWin;
+    const uint32_t meta_k = (uint32_t)(k_lo + c);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int ti = f - 2 * j - tw;  // window slot of slice j
+      if (2 * j < b && ti >= 0 && ti < kTagWin) {
+        const uint2 e = row[ti];
+        // the field j < b/2 of the b-bit pattern equals that of the 8-bit pattern
+        rec[wb[ti] + (int)e.y + __popc(e.x & lt)] =
+            make_uint2(words[j], meta_k | ((uint32_t)(uint8_t)(int8_t)(tw + ti) << 16) | ((uint32_t)j << 24));
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------------
+// K1 for small batches: one 16-token tile per cluster of C CTAs, CTA r owning
+// a contiguous range of channels; g_ref, plane count and per-tag record
+// counts are combined across the cluster through distributed shared memory.
+template <typename TIn, bool DYN>
+__global__ void __launch_bounds__(kQThreads, FMDQ_Q_MIN_BLOCKS) quantize_kernel(const QuantParams p, int C, int64_t kc_max) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  cg::cluster_group cluster = cg::this_cluster();
+
+  const int64_t K = p.K;
+  const int rank = (int)cluster.block_rank();
+  const int t = (int)(blockIdx.x / C);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t units = K / 32;
+  const int64_t k_lo = 32 * (rank * units / C), k_hi = 32 * ((rank + 1) * units / C);
+  const int Kc = (int)(k_hi - k_lo);
+
+  int8_t* s_code = reinterpret_cast<int8_t*>(smem);  // 16-byte slots: the 16 codes of a local channel
+  int8_t* s_fpot = s_code + 16 * kc_max;              // [Kc]
+  int8_t* s_bits = s_fpot + kc_max;                   // [Kc]
+  // [Kc / 32][kTagWin]: per 32-channel chunk and window tag, the ballot of the
+  // lanes carrying the tag and the warp's records of the tag in earlier chunks
+  uint2* s_tab = reinterpret_cast<uint2*>(s_bits + kc_max);
+  const int64_t tab_bytes = kc_max / 32 * kTagWin * 8;
+  QSmem& S = *reinterpret_cast<QSmem*>(smem + ((18 * kc_max + tab_bytes + 15) & ~(int64_t)15));
+
+  if (tid < kMaxMaskWords) S.mask[tid] = 0;
+  if (tid == 0) S.flags = 0;
+  pdl_launch_dependents();
+  pdl_wait();  // nothing of global memory is touched before the previous kernel completed
+  __syncthreads();
+
+  const QConst qc = quant_const<DYN>(p);
+  const int64_t row0 = (int64_t)t * kTile;
+
+  // ---------------------------------------------------------------- phase 1
+  const P1Red r1 = phase1<TIn, DYN, kQThreads>(p, qc, t, k_lo, Kc, tid, s_code, s_fpot, s_bits);
+
+  // CTA reductions, then one exchange across the cluster
+  if (lane == 0) {
+    S.red[0][warp] = r1.fmax, S.red[1][warp] = r1.fmin, S.red[2][warp] = r1.a1, S.red[3][warp] = r1.a2;
+    if (r1.flags) atomicOr(&S.flags, r1.flags);
+  }
+  __syncthreads();
+  if (tid < 4) {
+    int v = S.red[tid][0];
+    for (int w = 1; w < kQWarps; ++w) v = tid == 0 ? max(v, S.red[tid][w]) : min(v, S.red[tid][w]);
+    S.xv[tid] = v;
+    if (tid == 0 && S.flags)
+      set_status(p.status, (S.flags & 1 ? DSTAR_STATUS_NONFINITE : 0u) | (S.flags & 2 ? DSTAR_STATUS_RANGE : 0u));
+  }
+  csync(cluster, C);
+  if (tid < 4 * C) {  // one remote read per thread, all in flight together
+    const int q = tid >> 2, u = tid & 3;
+    S.x[q][u] = (C > 1 ? cluster.map_shared_rank(&S, q) : &S)->xv[u];
+  }
+  __syncthreads();
+  int g = -1000, gmin = 1000, A1 = 1000, A2 = 1000;
+  for (int q = 0; q < C; ++q) {
+    g = max(g, S.x[q][0]), gmin = min(gmin, S.x[q][1]);
+    A1 = min(A1, S.x[q][2]), A2 = min(A2, S.x[q][3]);
+  }
+  // every v = q 2^(g - FPoT) must fit the split: g - FPoT <= room for each channel
+  const int planes = g <= A1 ? 1 : g <= A2 ? 2 : 3;
+  // HBM is idle from here on: pull the next GEMM's operands into L2
+  if (tid == 0) {
+    prefetch_region_share(p.prefetch[0], (int)blockIdx.x, (int)gridDim.x);
+    prefetch_region_share(p.prefetch[1], (int)blockIdx.x, (int)gridDim.x);
+  }
+
+  // ------------------------------------------------- phase 2a: operand planes
+  phase2_planes<kQThreads>(p, row0, k_lo, Kc, tid, g, planes, s_code, s_fpot, S.mask);
 
   // ------------------------------------- phase 2b: FPoT-grouped encoded stream
   // Slice j of channel k carries tag FPoT(k) - 2j (j < bits/2).  Tags lie in
@@ -514,14 +660,10 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParam
   // contiguous run of 32-channel chunks (lane = channel).  The record of
   // (tag, k) lands after the tile's records of lower tags, then those of the
   // same tag in lower-ranked CTAs, lower warps of this CTA, earlier chunks of
-  // this warp and lower lanes of its chunk.  Pass A counts, and keeps per
-  // (chunk, tag) the ballot of the lanes carrying the tag with the warp's
-  // count of the tag before the chunk; pass B then places every record by
-  // itself: that count plus the set lanes below it in the ballot.
+  // this warp and lower lanes of its chunk.
   const int tlo = gmin - 6;
   const int nchunks = Kc / 32;
   const int ch_lo = warp * nchunks / kQWarps, ch_hi = (warp + 1) * nchunks / kQWarps;
-  const uint32_t lt = (1u << lane) - 1u;
   uint2* rec = p.records + (int64_t)t * p.record_cap;
   int total = 0;  // records of lower windows, all CTAs (kept by warp 0)
   bool first = true;
@@ -531,27 +673,7 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParam
       if (C > 1) cluster_wait();   // and every CTA with its remote reads of them
     }
     first = false;
-    // pass A: per chunk, the lane ballot of every window tag is a column of the
-    // bit matrix whose rows are the lanes' tag masks, so one warp transpose
-    // gives them all (lane u: tag tw + u); lane u also keeps this warp's count
-    // of its tag so far
-    int cnt = 0;
-    for (int ch0 = ch_lo; ch0 < ch_hi; ch0 += kUA) {
-      uint32_t col[kUA];
-#pragma unroll
-      for (int u = 0; u < kUA; ++u) {
-        const int c = 32 * (ch0 + u) + lane;
-        const uint32_t m = ch0 + u < ch_hi ? tag_mask32(s_fpot[c], s_bits[c], tw) & ((1u << kTagWin) - 1u) : 0u;
-        col[u] = warp_bit_transpose(m, lane);
-      }
-#pragma unroll
-      for (int u = 0; u < kUA; ++u) {
-        if (ch0 + u < ch_hi && lane < kTagWin) {
-          s_tab[(ch0 + u) * kTagWin + lane] = make_uint2(col[u], (uint32_t)cnt);
-          cnt += __popc(col[u]);
-        }
-      }
-    }
+    const int cnt = count_window(tw, ch_lo, ch_hi, lane, s_fpot, s_bits, s_tab);
     if (lane < kTagWin) S.warp_cnt[warp][lane] = cnt;
     __syncthreads();
     if (tid < kTagWin) {
@@ -597,27 +719,7 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParam
       S.wbase[warp][lane] = o;
     }
     __syncwarp();
-    // pass B: every lane writes its channel's records of the window
-    const int* wb = S.wbase[warp];
-#pragma unroll 2
-    for (int ch = ch_lo; ch < ch_hi; ++ch) {
-      const int c = 32 * ch + lane;
-      const int f = s_fpot[c], b = s_bits[c];
-      uint32_t words[4];
-      slice_words(*reinterpret_cast<const uint4*>(s_code + 16 * code_slot(c)), words);
-      const uint2* row = s_tab + ch * kTagWin;
-      const uint32_t meta_k = (uint32_t)(k_lo + c);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int ti = f - 2 * j - tw;  // window slot of slice j
-        if (2 * j < b && ti >= 0 && ti < kTagWin) {
-          const uint2 e = row[ti];
-          // the field j < b/2 of the b-bit pattern equals that of the 8-bit pattern
-          rec[wb[ti] + (int)e.y + __popc(e.x & lt)] =
-              make_uint2(words[j], meta_k | ((uint32_t)(uint8_t)(int8_t)(tw + ti) << 16) | ((uint32_t)j << 24));
-        }
-      }
-    }
+    write_window(tw, ch_lo, ch_hi, lane, k_lo, S.wbase[warp], s_code, s_fpot, s_bits, s_tab, rec);
   }
   if (rank == 0 && tid == 0) {
     p.g_ref[t] = g;
@@ -629,35 +731,235 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_kernel(const QuantParam
   if (C > 1) cluster_wait();  // no CTA leaves while another may still read its shared memory
 }
 
+// ------------------------------------------------------------------------
+// K1 for large batches: persistent (one CTA per SM) and warp-specialised.
+// With one CTA per tile, every CTA of a wave streams HBM in phase 1 and then
+// leaves it idle while it builds planes and records.  Here two groups of
+// eight warps work on consecutive tiles at once: group 1 runs phase 1 of a
+// tile into one of two shared-memory buffers while group 2 runs phases 2a
+// and 2b of the previous tile from the other, so each SM streams HBM and
+// encodes at the same time.  The per-tile arithmetic is that of the kernel
+// above (the same stage functions, with one CTA per tile); the buffers pass
+// between the groups through mbarriers (full: group 1 -> 2, empty: 2 -> 1)
+// whose waits are bounded.
+constexpr int kPGroup = 256;  // threads of each group
+constexpr int kPGroupWarps = kPGroup / 32;
+constexpr int kPThreads = 2 * kPGroup;
+constexpr int kBarG1 = 1, kBarG2 = 2;  // named barriers of the groups (0 is __syncthreads)
+
+struct PSmem {
+  uint64_t full[2], empty[2];
+  int abort;
+  int red[4][kPGroupWarps];
+  int xv[2][4];  // per buffer: finest FPoT, coarsest FPoT, min(FPoT + one-plane room), min(FPoT + two-plane room)
+  uint32_t mask[kMaxMaskWords];
+  int warp_cnt[kPGroupWarps][kTagWin];
+  int base[kTagWin];
+  int wbase[kPGroupWarps][kTagWin];
+};
+
+__device__ __forceinline__ void group_sync(int id) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "n"(kPGroup) : "memory");
+}
+
+template <typename TIn, bool DYN>
+__global__ void __launch_bounds__(kPThreads, 1) quantize_persistent_kernel(const QuantParams p) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int64_t K = p.K;
+  const int Kc = (int)K;
+  const int64_t T = p.M / kTile;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const bool g1 = tid < kPGroup;
+  const int gt = g1 ? tid : tid - kPGroup;  // thread index within the group
+  const int gw = gt >> 5;                   // warp index within the group
+  // buffer b: codes at 16 K b, FPoT at 32 K + 2 K b, widths right after the FPoTs
+  int8_t* const s_base = reinterpret_cast<int8_t*>(smem);
+  auto s_code = [&](int b) { return s_base + 16 * K * b; };
+  auto s_fpot = [&](int b) { return s_base + 32 * K + 2 * K * b; };
+  auto s_bits = [&](int b) { return s_base + 33 * K + 2 * K * b; };
+  uint2* s_tab = reinterpret_cast<uint2*>(smem + 36 * K);  // group 2 only
+  PSmem& S = *reinterpret_cast<PSmem*>(smem + ((36 * K + K / 32 * kTagWin * 8 + 15) & ~(int64_t)15));
+  volatile int* abort_flag = &S.abort;
+
+  if (tid == 0) {
+    for (int b = 0; b < 2; ++b) mbar_init(&S.full[b], kPGroup), mbar_init(&S.empty[b], kPGroup);
+    S.abort = 0;
+    fence_barrier_init();
+  }
+  pdl_launch_dependents();
+  pdl_wait();  // nothing of global memory is touched before the previous kernel completed
+  __syncthreads();
+  const QConst qc = quant_const<DYN>(p);
+  const int ntiles = T > (int64_t)blockIdx.x ? (int)((T - 1 - blockIdx.x) / gridDim.x) + 1 : 0;
+
+  if (g1) {
+    // ------------------------------------------------- group 1: phase 1
+    using Raw = typename Pair<TIn>::Raw;
+    constexpr bool kAhead = FMDQ_Q_PREFETCH && sizeof(Raw) == 4;
+    const int npairs = Kc / 2;
+    Raw nt[kTile], np[kTile];
+    if (kAhead && ntiles > 0 && gt < npairs) load_pair<TIn>(p, (int64_t)blockIdx.x * kTile, 2 * gt, nt, np);
+    for (int i = 0; i < ntiles; ++i) {
+      const int b = i & 1;
+      const int64_t t = blockIdx.x + (int64_t)i * gridDim.x;
+      // buffer b is free once group 2 has finished tile i - 2
+      if (gt == 0 && i >= 2 && !wait_parity(&S.empty[b], ((i >> 1) - 1) & 1, abort_flag, p.status, kWaitLimitNs))
+        *abort_flag = 1;
+      __syncwarp();
+      group_sync(kBarG1);  // also: every warp is done with the previous tile's reduction
+      if (*abort_flag) break;
+      // phase 1; the loads of the thread's first pair of the next tile are
+      // issued while its last pair of this tile is processed
+      P1Red r{-1000, 1000, 1000, 1000, 0};
+      for (int pr = gt; pr < npairs; pr += kPGroup) {
+        Raw rt[kTile], rp[kTile];
+        if constexpr (kAhead) {
+#pragma unroll
+          for (int j = 0; j < kTile; ++j) rt[j] = nt[j], rp[j] = np[j];
+          if (pr + kPGroup < npairs) load_pair<TIn>(p, t * kTile, 2 * (pr + kPGroup), nt, np);
+          else if (i + 1 < ntiles) load_pair<TIn>(p, (t + gridDim.x) * kTile, 2 * gt, nt, np);
+        } else {
+          load_pair<TIn>(p, t * kTile, 2 * pr, rt, rp);
+        }
+        process_pair<TIn, DYN>(p, qc, t, 2 * pr, 2 * pr, rt, rp, s_code(b), s_fpot(b), s_bits(b), r);
+      }
+      warp_reduce(r);
+      if (lane == 0) {
+        S.red[0][gw] = r.fmax, S.red[1][gw] = r.fmin, S.red[2][gw] = r.a1, S.red[3][gw] = r.a2;
+        if (r.flags)
+          set_status(p.status, (r.flags & 1 ? DSTAR_STATUS_NONFINITE : 0u) | (r.flags & 2 ? DSTAR_STATUS_RANGE : 0u));
+      }
+      group_sync(kBarG1);
+      if (gt < 4) {
+        int v = S.red[gt][0];
+        for (int w = 1; w < kPGroupWarps; ++w) v = gt == 0 ? max(v, S.red[gt][w]) : min(v, S.red[gt][w]);
+        S.xv[b][gt] = v;
+      }
+      mbar_arrive(&S.full[b]);  // every thread after its own writes of the tile
+    }
+    // this CTA no longer reads HBM: pull the next GEMM's operands into L2
+    if (gt == 0) {
+      prefetch_region_share(p.prefetch[0], (int)blockIdx.x, (int)gridDim.x);
+      prefetch_region_share(p.prefetch[1], (int)blockIdx.x, (int)gridDim.x);
+    }
+  } else {
+    // ------------------------------------- group 2: phases 2a and 2b
+    const int nchunks = Kc / 32;
+    const int ch_lo = gw * nchunks / kPGroupWarps, ch_hi = (gw + 1) * nchunks / kPGroupWarps;
+    for (int i = 0; i < ntiles; ++i) {
+      const int b = i & 1;
+      const int64_t t = blockIdx.x + (int64_t)i * gridDim.x;
+      if (gt == 0 && !wait_parity(&S.full[b], (i >> 1) & 1, abort_flag, p.status, kWaitLimitNs)) *abort_flag = 1;
+      __syncwarp();
+      group_sync(kBarG2);  // also: every warp is done with the previous tile
+      if (*abort_flag) break;
+      const int g = S.xv[b][0], gmin = S.xv[b][1], A1 = S.xv[b][2], A2 = S.xv[b][3];
+      const int planes = g <= A1 ? 1 : g <= A2 ? 2 : 3;
+      if (gt < kMaxMaskWords) S.mask[gt] = 0;
+      group_sync(kBarG2);
+      const int64_t row0 = t * kTile;
+      phase2_planes<kPGroup>(p, row0, 0, Kc, gt, g, planes, s_code(b), s_fpot(b), S.mask);
+      const int tlo = gmin - 6;
+      uint2* rec = p.records + t * p.record_cap;
+      int total = 0;  // records of lower windows (kept by warp 0)
+      for (int tw = tlo; tw <= g; tw += kTagWin) {
+        if (tw != tlo) group_sync(kBarG2);  // every warp is done with the previous window
+        const int cnt = count_window(tw, ch_lo, ch_hi, lane, s_fpot(b), s_bits(b), s_tab);
+        if (lane < kTagWin) S.warp_cnt[gw][lane] = cnt;
+        group_sync(kBarG2);  // counts written; every plane of the tile written (mask complete)
+        if (tw == tlo && gt < p.mask_words) p.mask1[t * p.mask_words + gt] = planes == 2 ? S.mask[gt] : 0u;
+        if (gw == 0) {
+          int all = 0;
+          if (lane < kTagWin)
+            for (int w = 0; w < kPGroupWarps; ++w) all += S.warp_cnt[w][lane];
+          int incl = all;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(kFull, incl, o);
+            if (lane >= o) incl += n;
+          }
+          if (lane < kTagWin) S.base[lane] = total + incl - all;
+          total += __shfl_sync(kFull, incl, 31);
+        }
+        group_sync(kBarG2);
+        if (lane < kTagWin) {
+          int o = S.base[lane];
+          for (int w = 0; w < gw; ++w) o += S.warp_cnt[w][lane];
+          S.wbase[gw][lane] = o;
+        }
+        __syncwarp();
+        write_window(tw, ch_lo, ch_hi, lane, 0, S.wbase[gw], s_code(b), s_fpot(b), s_bits(b), s_tab, rec);
+      }
+      if (gt == 0) {
+        p.g_ref[t] = g;
+        p.planes[t] = planes;
+        p.count[t] = total;
+      }
+      mbar_arrive(&S.empty[b]);  // buffer b may be refilled
+    }
+  }
+  __syncthreads();
+}
+
+size_t quantize_persistent_smem_bytes(int64_t K) {
+  size_t b = 36 * (size_t)K + (size_t)K / 32 * kTagWin * 8;
+  b = (b + 15) & ~(size_t)15;
+  return b + sizeof(PSmem);
+}
+
+// The persistent kernel takes batches of at least two tiles per SM whose
+// double buffers fit shared memory.
+bool use_persistent(int64_t M, int64_t K, int num_sms) {
+  return M / kTile >= 2LL * num_sms && quantize_persistent_smem_bytes(K) <= 227 * 1024;
+}
+
 int launch_quantize(const QuantParams& p, int in_bf16, int num_sms, void* stream) {
   const int64_t T = p.M / kTile;
   if (T == 0) return 0;
+  const bool dyn = p.dyn_base != nullptr;
+  cudaLaunchConfig_t cfg = {};
+  cfg.stream = (cudaStream_t)stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // overlap the launch with the previous kernel
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cudaError_t ce;
+  if (use_persistent(p.M, p.K, num_sms)) {
+    const void* fn = in_bf16 ? (dyn ? (const void*)quantize_persistent_kernel<__nv_bfloat16, true>
+                                    : (const void*)quantize_persistent_kernel<__nv_bfloat16, false>)
+                             : (dyn ? (const void*)quantize_persistent_kernel<float, true>
+                                    : (const void*)quantize_persistent_kernel<float, false>);
+    const int e = ensure_max_smem(fn, 227 * 1024);
+    if (e != 0) return e;
+    cfg.gridDim = dim3((unsigned)(T < num_sms ? T : num_sms), 1, 1);
+    cfg.blockDim = dim3(kPThreads, 1, 1);
+    cfg.dynamicSmemBytes = quantize_persistent_smem_bytes(p.K);
+    cfg.numAttrs = 1;
+    if (in_bf16) ce = dyn ? cudaLaunchKernelEx(&cfg, quantize_persistent_kernel<__nv_bfloat16, true>, p)
+                          : cudaLaunchKernelEx(&cfg, quantize_persistent_kernel<__nv_bfloat16, false>, p);
+    else ce = dyn ? cudaLaunchKernelEx(&cfg, quantize_persistent_kernel<float, true>, p)
+                  : cudaLaunchKernelEx(&cfg, quantize_persistent_kernel<float, false>, p);
+    if (ce != cudaSuccess) return (int)ce;
+    return (int)cudaGetLastError();
+  }
   const int C = quantize_cluster_size(p.M, p.K, num_sms);
   const int64_t units = p.K / 32;
   const int64_t kc_max = 32 * ((units + C - 1) / C);
   const size_t smem = quantize_smem_bytes(kc_max);
   const int smem_max = (int)quantize_smem_bytes(DSTAR_K_MAX);  // one setting serves every K
-  const bool dyn = p.dyn_base != nullptr;
   const void* fn = in_bf16 ? (dyn ? (const void*)quantize_kernel<__nv_bfloat16, true>
                                   : (const void*)quantize_kernel<__nv_bfloat16, false>)
                            : (dyn ? (const void*)quantize_kernel<float, true> : (const void*)quantize_kernel<float, false>);
   int e = ensure_max_smem(fn, smem_max);
   if (e != 0) return e;
-  cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(T * C), 1, 1);
   cfg.blockDim = dim3(kQThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
-  cfg.stream = (cudaStream_t)stream;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = C;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // overlap the launch with the previous kernel
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = C;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.numAttrs = 2;
-  cudaError_t ce;
   if (in_bf16) ce = dyn ? cudaLaunchKernelEx(&cfg, quantize_kernel<__nv_bfloat16, true>, p, C, kc_max)
                         : cudaLaunchKernelEx(&cfg, quantize_kernel<__nv_bfloat16, false>, p, C, kc_max);
   else ce = dyn ? cudaLaunchKernelEx(&cfg, quantize_kernel<float, true>, p, C, kc_max)

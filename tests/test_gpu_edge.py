@@ -147,3 +147,13 @@ def test_invalid_arguments_leave_buffers_untouched():
         nat.linear(d["x_t"], d["x_prev"], d["y_prev"], d["w_q"], d["w_scale"], 0.1, ws)
     torch.cuda.synchronize()
     assert torch.equal(before, d["y_prev"])
+
+
+def test_fp32_large_batch_takes_the_persistent_quantizer():
+    """fp32 inputs with enough 16-token tiles (>= 2 per SM) for the persistent,
+    warp-specialised quantizer; compared in full with the oracle."""
+    from gpu_helpers import full_parity
+    from differential_quantized_gemm_b200 import synth
+    inp = synth.make_layer(1, 0, M=16 * 2 * 152)
+    g, q, acc, y, exact = full_parity(inp)
+    assert exact > 0.999
