@@ -28,6 +28,12 @@ Parity status of each function (what pins it, see tests/test_oracle_pins.py):
                    against Python's math.erfc element by element, and
                    against math.erf away from the negative tail.
   ffn_gelu      -- composition of the pinned pieces above.
+  quant_rows    -- brute force per element, the 127 bound, the error bound.
+  masked_softmax -- rows sum to 1 over kept entries, pruned entries 0,
+                   agreement with a numpy softmax of the kept entries, shift
+                   invariance.
+  sar_attention -- composition of the pinned pieces; its dense-mask output
+                   within the quantization error of a plain fp64 attention.
 """
 from __future__ import annotations
 
@@ -74,6 +80,10 @@ def _load():
         lib.fmdq_orc_epilogue_dyn_f32.restype = None
         lib.fmdq_orc_gelu.argtypes = [P, i64, ci, P]
         lib.fmdq_orc_gelu.restype = None
+        lib.fmdq_orc_quant_rows.argtypes = [P, i64, i64, P, P]
+        lib.fmdq_orc_quant_rows.restype = None
+        lib.fmdq_orc_masked_softmax.argtypes = [P, i64, i64, P, i64, i64, P]
+        lib.fmdq_orc_masked_softmax.restype = None
         lib.fmdq_orc_set_threads.argtypes = [ci]
         lib.fmdq_orc_set_threads.restype = None
         lib.fmdq_orc_max_threads.restype = ci
@@ -270,6 +280,60 @@ def ffn_gelu(x_t, x_prev, y1_prev, w1, w1_scale, h_prev, y2_prev, w2, w2_scale, 
     h = gelu(y1, out_bf16)
     q2, acc2, y2 = linear(h, h_prev, y2_prev, w2, w2_scale, lb, t0, force_bits, out_bf16)
     return q1, acc1, y1, h, q2, acc2, y2
+
+
+def quant_rows(x: np.ndarray):
+    """Symmetric per-row int8: scale = max|row|/127, q = rne(x/scale); returns (q int8, scale fp32)."""
+    x = np.ascontiguousarray(x, np.float32)
+    rows, cols = x.shape
+    q = np.zeros((rows, cols), np.int8)
+    sc = np.zeros(rows, np.float32)
+    _load().fmdq_orc_quant_rows(_p(x), rows, cols, _p(q), _p(sc))
+    return q, sc
+
+
+def masked_softmax(s: np.ndarray, mask: np.ndarray, blk: int) -> np.ndarray:
+    """Row softmax over the kept blocks of a block mask (fp64, rounded to fp32); pruned entries 0."""
+    s = np.ascontiguousarray(s, np.float32)
+    rows, cols = s.shape
+    mask = np.ascontiguousarray(mask, np.uint8)
+    assert mask.shape == ((rows + blk - 1) // blk, (cols + blk - 1) // blk)
+    out = np.zeros((rows, cols), np.float32)
+    _load().fmdq_orc_masked_softmax(_p(s), rows, cols, _p(mask), blk, mask.shape[1], _p(out))
+    return out
+
+
+def sar_attention(q, k, v, mask, blk, lb_q, lb_p, scores_scale, p_cached=None):
+    """Attention of one head with INT8 FMDQ operands and sparse attention reuse
+    (sections 3.2 and 4.3).  q, k: [S x d]; v: [S x d]; mask [S/blk x S/blk].
+
+    Cached step (p_cached None):
+      K -> int8 per key (quant_rows); Q -> FMDQ with every width 8 and X_{t-1} = 0;
+      scores = dequant(acc(Q codes, K codes)) with w_scale = fl32(k_scale * scores_scale);
+      P = masked_softmax(scores); P -> FMDQ with every width 8 (the cached object).
+    Reused step: the cached quantized P.
+    Both: V^T -> int8 per head dimension; O = dequant(acc(P codes, V^T codes)).
+    Returns dict(qQ, kq, ks, acc_s, scores, p, qP, vq, vs, acc_o, out)."""
+    S, d = q.shape
+    res = {}
+    if p_cached is None:
+        kq, ks = quant_rows(k)
+        zeros_q = np.zeros_like(q, dtype=np.float32)
+        qQ = quantize(q, zeros_q, lb_q, 0, 8)
+        acc_s = acc_direct(qQ, kq)
+        w_s = (ks * np.float32(scores_scale)).astype(np.float32)
+        scores = epilogue_f32(acc_s, qQ.g_ref, lb_q, w_s, np.zeros((S, S), np.float32), False)
+        p = masked_softmax(scores, mask, blk)
+        qP = quantize(p, np.zeros_like(p), lb_p, 0, 8)
+        res.update(qQ=qQ, kq=kq, ks=ks, acc_s=acc_s, scores=scores, p=p, qP=qP)
+    else:
+        qP = p_cached
+        res.update(qP=qP)
+    vq, vs = quant_rows(np.ascontiguousarray(v.T))
+    acc_o = acc_direct(qP, vq)
+    out = epilogue_f32(acc_o, qP.g_ref, lb_p, vs, np.zeros((S, vq.shape[0]), np.float32), False)
+    res.update(vq=vq, vs=vs, acc_o=acc_o, out=out)
+    return res
 
 
 def n_threads() -> int:

@@ -547,6 +547,61 @@ void fmdq_orc_gelu(const float* y, int64_t n, int out_bf16, float* out) {
   }
 }
 
+/* ------------------------------------------------------------- attention */
+
+/*
+ * Symmetric int8 quantization of each row of a [rows x cols] fp32 matrix
+ * (the weight rule of section 5.1, A8W8, applied per row): scale = max|row| /
+ * 127 (one fp32 division), q = rne(x / scale) (one fp32 division, then
+ * round half to even), so |q| <= 127; an all-zero row gets scale 0 and codes 0.
+ * Used for the attention operands K (per key) and V (per head dimension),
+ * which section 4.3 runs in INT8.
+ */
+void fmdq_orc_quant_rows(const float* x, int64_t rows, int64_t cols, int8_t* q, float* scale) {
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < rows; ++r) {
+    float mx = 0.0f;
+    for (int64_t c = 0; c < cols; ++c) {
+      float a = fabsf(x[r * cols + c]);
+      if (a > mx) mx = a;
+    }
+    volatile float s = mx / 127.0f;
+    scale[r] = s;
+    for (int64_t c = 0; c < cols; ++c) {
+      if (mx == 0.0f) {
+        q[r * cols + c] = 0;
+      } else {
+        volatile float v = x[r * cols + c] / s;
+        q[r * cols + c] = (int8_t)nearbyintf(v);
+      }
+    }
+  }
+}
+
+/*
+ * Block-masked softmax over the rows of a [rows x cols] score matrix (section
+ * 3.2, Sparse Attention Reuse: pruned blocks of the score matrix are never
+ * computed).  Entry (r, c) takes part iff mask[(r / blk) * mask_cols + c / blk]
+ * is nonzero; P = exp(s - m) / sum over the row's kept entries, m their
+ * maximum, evaluated in fp64 and rounded to fp32; pruned entries are 0.  A
+ * row with no kept entry is all 0.
+ */
+void fmdq_orc_masked_softmax(const float* s, int64_t rows, int64_t cols, const uint8_t* mask, int64_t blk,
+                             int64_t mask_cols, float* p) {
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < rows; ++r) {
+    const uint8_t* mrow = mask + (r / blk) * mask_cols;
+    double m = -INFINITY;
+    for (int64_t c = 0; c < cols; ++c)
+      if (mrow[c / blk] && (double)s[r * cols + c] > m) m = (double)s[r * cols + c];
+    double sum = 0.0;
+    for (int64_t c = 0; c < cols; ++c)
+      if (mrow[c / blk]) sum += exp((double)s[r * cols + c] - m);
+    for (int64_t c = 0; c < cols; ++c)
+      p[r * cols + c] = mrow[c / blk] ? (float)(exp((double)s[r * cols + c] - m) / sum) : 0.0f;
+  }
+}
+
 /* bf16 helpers exposed for the tests (exact widening, RNE narrowing). */
 void fmdq_orc_bf16_to_f32(const uint16_t* h, int64_t n, float* f) {
   for (int64_t i = 0; i < n; ++i) f[i] = bf16_bits_to_float(h[i]);
