@@ -30,8 +30,10 @@ EXPORTED = [
     "dstar_fmdq_version", "dstar_fmdq_error_string", "dstar_fmdq_last_error", "dstar_fmdq_workspace_size",
     "dstar_fmdq_workspace_layout", "dstar_fmdq_workspace_init", "dstar_fmdq_linear", "dstar_fmdq_quantize",
     "dstar_fmdq_slice_gemm", "dstar_fmdq_status", "dstar_fmdq_selftest_wait", "dstar_fmdq_linear_noalloc",
-    "dstar_fmdq_ffn_gelu",
+    "dstar_fmdq_ffn_gelu", "dstar_sar_workspace_size", "dstar_sar_workspace_layout", "dstar_sar_workspace_init",
+    "dstar_sar_attention", "dstar_sar_status",
 ]
+SAR_BLOCK = 128
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
@@ -50,6 +52,16 @@ class WsLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in ("total", "status", "plane0", "plane1", "fpot", "bits", "g_ref",
                                                "planes", "count", "mask1", "records")] + \
                [("mask_words", ctypes.c_int64), ("record_cap", ctypes.c_int64), ("dyn_base", ctypes.c_size_t)]
+
+
+class SarCfg(ctypes.Structure):
+    _fields_ = [("heads", ctypes.c_int64), ("seq", ctypes.c_int64), ("head_dim", ctypes.c_int64),
+                ("block_mask", ctypes.c_void_p), ("scores_scale", ctypes.c_float), ("base_q", ctypes.c_float),
+                ("base_p", ctypes.c_float), ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
+
+
+class SarLayout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in ("total", "ws_p", "ws_q", "kq", "ks", "vqt", "vs", "scores", "probs")]
 
 
 class DstarError(RuntimeError):
@@ -85,6 +97,11 @@ def lib():
                                                 P]
         L.dstar_fmdq_ffn_gelu.argtypes = [MP, MP, MP, MP, P, MP, MP, MP, MP, P, ctypes.c_float,
                                           ctypes.POINTER(TileCfg), ctypes.POINTER(TileCfg), P]
+        L.dstar_sar_workspace_size.argtypes = [I64, I64, I64, ctypes.POINTER(ctypes.c_size_t)]
+        L.dstar_sar_workspace_layout.argtypes = [I64, I64, I64, ctypes.POINTER(SarLayout)]
+        L.dstar_sar_workspace_init.argtypes = [ctypes.POINTER(SarCfg), P]
+        L.dstar_sar_attention.argtypes = [MP, MP, MP, ctypes.POINTER(SarCfg), ctypes.c_int, MP, P]
+        L.dstar_sar_status.argtypes = [ctypes.POINTER(SarCfg), P, ctypes.POINTER(ctypes.c_uint32)]
         for name in EXPORTED[3:]:
             getattr(L, name).restype = ctypes.c_int
         _lib = L
@@ -227,6 +244,55 @@ def ffn_gelu(x_t, x_prev, y1_prev, w1, w1_scale, h_t, h_prev, y2_prev, w2, w2_sc
                                      *(ctypes.byref(v) for v in m[4:]), ctypes.c_void_p(w2_scale.data_ptr()),
                                      base_scale, ctypes.byref(c1), ctypes.byref(c2), _stream(stream)))
     return y2_prev
+
+
+class SarAttention:
+    """Sparse attention reuse with INT8 FMDQ operands (dstar_sar_attention):
+    `heads` problems of `seq` tokens and `head_dim` channels, a host block mask
+    [seq/128 x seq/128] (nonzero = kept), its caller-owned workspace."""
+
+    def __init__(self, heads: int, seq: int, head_dim: int, block_mask, scores_scale: float, base_q: float,
+                 base_p: float, device="cuda", stream=None):
+        import numpy as np
+        self.heads, self.seq, self.head_dim = heads, seq, head_dim
+        self.mask = np.ascontiguousarray(block_mask, dtype=np.uint8)
+        n = ctypes.c_size_t()
+        _check(lib().dstar_sar_workspace_size(heads, seq, head_dim, ctypes.byref(n)))
+        self.nbytes = n.value
+        buf = torch.empty(self.nbytes + 256, dtype=torch.uint8, device=device)
+        off = (-buf.data_ptr()) % 256
+        self.buf = buf[off:off + self.nbytes]
+        self.cfg = SarCfg(heads, seq, head_dim, self.mask.ctypes.data_as(ctypes.c_void_p), scores_scale, base_q,
+                          base_p, ctypes.c_void_p(self.buf.data_ptr()), self.nbytes)
+        self.layout = SarLayout()
+        _check(lib().dstar_sar_workspace_layout(heads, seq, head_dim, ctypes.byref(self.layout)))
+        _check(lib().dstar_sar_workspace_init(ctypes.byref(self.cfg), _stream(stream)))
+
+    def __call__(self, q, k, v, out, reuse: bool = False, stream=None):
+        mq, mk, mv, mo = mat(q), mat(k), mat(v), mat(out)
+        _check(lib().dstar_sar_attention(ctypes.byref(mq), ctypes.byref(mk), ctypes.byref(mv), ctypes.byref(self.cfg),
+                                         int(bool(reuse)), ctypes.byref(mo), _stream(stream)))
+        return out
+
+    def status(self, stream=None) -> int:
+        s = ctypes.c_uint32()
+        _check(lib().dstar_sar_status(ctypes.byref(self.cfg), _stream(stream), ctypes.byref(s)))
+        return s.value
+
+    def section(self, name: str, count: int, dtype):
+        off = getattr(self.layout, name)
+        nb = count * torch.tensor([], dtype=dtype).element_size()
+        return self.buf[off:off + nb].view(dtype)
+
+    def fmdq_sections(self, which: str) -> dict:
+        """The FMDQ workspace sections of P ('p') or of Q ('q')."""
+        R = self.heads * self.seq
+        K = self.seq if which == "p" else self.head_dim
+        off = getattr(self.layout, "ws_" + which)
+        ws = Workspace.__new__(Workspace)
+        ws.M, ws.K, ws.nbytes = R, K, workspace_size(R, K)
+        ws.buf = self.buf[off:off + ws.nbytes]
+        return ws.sections(R, K)
 
 
 def quantize(x_t, x_prev, base_scale: float, ws: Workspace, *, t0: int = 0, force_bits: int = 0, flags: int = 0,

@@ -14,7 +14,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 OUT_DIR = os.path.join(HERE, "_lib")
 LIB = os.path.join(OUT_DIR, "libdstar_fmdq.so")
-SOURCES = ["fmdq_host.cu", "fmdq_quant.cu", "fmdq_gemm.cu", "fmdq_noalloc.cu"]
+SOURCES = ["fmdq_host.cu", "fmdq_quant.cu", "fmdq_gemm.cu", "fmdq_noalloc.cu", "fmdq_attn.cu"]
 HEADERS = ["fmdq_device.cuh", "fmdq_internal.h"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -1,0 +1,150 @@
+// Element-wise kernels of sparse attention reuse with INT8 FMDQ operands
+// (DSTAR section 3.2 "Sparse Attention Reuse"; section 4.3 "Attention
+// Operation": every attention MMA runs in INT8, activations through FMDQ at
+// 8 bits).  The contractions themselves run in the FMDQ quantizer and the
+// slice GEMM (batched over heads, block-sparse); these kernels prepare the
+// weight-side operands and the softmax between the two products.
+#include <cuda_bf16.h>
+
+#include "fmdq_device.cuh"
+
+namespace fmdq {
+
+namespace {
+
+template <typename TIn>
+__device__ __forceinline__ float ld_f(const TIn* p) {
+  if constexpr (sizeof(TIn) == 2) return __bfloat162float(*p);
+  else return *p;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Symmetric int8 per row (the A8W8 weight rule of section 5.1 applied to the
+// key rows): scale = max|row| / 127, q = rne(x / scale), both fp32
+// divisions; an all-zero row gets scale 0 and codes 0.  scale_out = scale *
+// scale_mul (one fp32 product: the score scaling folded into the weights).
+// One warp per row.
+template <typename TIn>
+__global__ void __launch_bounds__(256) quant_rows_kernel(const TIn* __restrict__ x, int64_t ld, int64_t rows,
+                                                         int64_t cols, int8_t* __restrict__ q, int64_t ldq,
+                                                         float* __restrict__ scale_out, float scale_mul) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const TIn* xr = x + row * ld;
+  float mx = 0.f;
+  for (int64_t c = lane; c < cols; c += 32) mx = fmaxf(mx, fabsf(ld_f(xr + c)));
+  mx = warp_max(mx);
+  const float s = __fdiv_rn(mx, 127.f);
+  if (lane == 0) scale_out[row] = __fmul_rn(s, scale_mul);
+  for (int64_t c = lane; c < cols; c += 32)
+    q[row * ldq + c] = mx == 0.f ? (int8_t)0 : (int8_t)__float2int_rn(__fdiv_rn(ld_f(xr + c), s));
+}
+
+// The same rule per column of each head's V ([S x d] rows h S .. h S + S - 1),
+// written transposed: vqt[(h d + j) S + s] = rne(V[h S + s][j] / scale[h d + j]).
+// Block (h, 32-column group): a column maximum over the S rows, then each
+// thread writes the codes of its rows (consecutive threads: consecutive s).
+template <typename TIn>
+__global__ void __launch_bounds__(256) quant_cols_t_kernel(const TIn* __restrict__ v, int64_t ld, int64_t S,
+                                                           int64_t d, int8_t* __restrict__ vqt,
+                                                           float* __restrict__ scale) {
+  __shared__ float red[8][32];
+  __shared__ float sc[32], mxs[32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t h = blockIdx.x, j0 = 32 * (int64_t)blockIdx.y;
+  const TIn* base = v + h * S * ld + j0;
+  float mx = 0.f;
+  for (int64_t s = warp; s < S; s += 8) mx = fmaxf(mx, fabsf(ld_f(base + s * ld + lane)));
+  red[warp][lane] = mx;
+  __syncthreads();
+  if (warp == 0) {
+    float m = red[0][lane];
+    for (int w = 1; w < 8; ++w) m = fmaxf(m, red[w][lane]);
+    const float s = __fdiv_rn(m, 127.f);
+    mxs[lane] = m, sc[lane] = s;
+    scale[h * d + j0 + lane] = s;
+  }
+  __syncthreads();
+  for (int64_t s = threadIdx.x; s < S; s += 256) {
+    const TIn* row = base + s * ld;
+#pragma unroll 8
+    for (int j = 0; j < 32; ++j) {
+      const int8_t code = mxs[j] == 0.f ? (int8_t)0 : (int8_t)__float2int_rn(__fdiv_rn(ld_f(row + j), sc[j]));
+      vqt[(h * d + j0 + j) * S + s] = code;
+    }
+  }
+}
+
+// Softmax over the kept blocks of each score row (section 3.2: pruned blocks
+// of the score matrix are never computed); pruned entries become 0.  Row r
+// is query r mod S of its head; its mask row is bits[(r mod S) / 128] (bit c:
+// key block c kept).  One warp per row.  The pages leave the softmax's
+// precision open and P decides integer codes, so it is evaluated in fp64
+// (CUDA's double exp, fp64 sum and division) and rounded once to fp32.
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__global__ void __launch_bounds__(256) masked_softmax_kernel(const float* __restrict__ sc, float* __restrict__ pr,
+                                                             int64_t rows, int64_t S, const __grid_constant__ BlockMask mk) {
+  const int lane = threadIdx.x & 31;
+  const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (r >= rows) return;
+  const uint64_t keep = mk.bits[(r % S) / kBlockM];
+  const float* x = sc + r * S;
+  float m = -INFINITY;
+  for (int64_t c = lane; c < S; c += 32)
+    if ((keep >> (c / kBlockM)) & 1ull) m = fmaxf(m, x[c]);
+  const double md = (double)warp_max(m);
+  double l = 0.0;
+  for (int64_t c = lane; c < S; c += 32)
+    if ((keep >> (c / kBlockM)) & 1ull) l += exp((double)x[c] - md);
+  const double sum = warp_sum_d(l);
+  float* o = pr + r * S;
+  for (int64_t c = lane; c < S; c += 32)
+    o[c] = ((keep >> (c / kBlockM)) & 1ull) ? (float)(exp((double)x[c] - md) / sum) : 0.f;
+}
+
+}  // namespace
+
+int launch_quant_rows(const void* x, int64_t ld, int64_t rows, int64_t cols, int in_bf16, int8_t* q, int64_t ldq,
+                      float* scale, float scale_mul, void* stream) {
+  if (rows == 0) return 0;
+  const unsigned grid = (unsigned)((rows + 7) / 8);
+  if (in_bf16)
+    quant_rows_kernel<__nv_bfloat16><<<grid, 256, 0, (cudaStream_t)stream>>>(
+        static_cast<const __nv_bfloat16*>(x), ld, rows, cols, q, ldq, scale, scale_mul);
+  else
+    quant_rows_kernel<float><<<grid, 256, 0, (cudaStream_t)stream>>>(static_cast<const float*>(x), ld, rows, cols,
+                                                                      q, ldq, scale, scale_mul);
+  return (int)cudaGetLastError();
+}
+
+int launch_quant_cols_t(const void* v, int64_t ld, int64_t heads, int64_t S, int64_t d, int in_bf16, int8_t* vqt,
+                        float* scale, void* stream) {
+  if (heads == 0) return 0;
+  const dim3 grid((unsigned)heads, (unsigned)(d / 32));
+  if (in_bf16)
+    quant_cols_t_kernel<__nv_bfloat16><<<grid, 256, 0, (cudaStream_t)stream>>>(
+        static_cast<const __nv_bfloat16*>(v), ld, S, d, vqt, scale);
+  else
+    quant_cols_t_kernel<float><<<grid, 256, 0, (cudaStream_t)stream>>>(static_cast<const float*>(v), ld, S, d, vqt,
+                                                                        scale);
+  return (int)cudaGetLastError();
+}
+
+int launch_masked_softmax(const float* sc, float* pr, int64_t rows, int64_t S, const BlockMask& mk, void* stream) {
+  if (rows == 0) return 0;
+  masked_softmax_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, (cudaStream_t)stream>>>(sc, pr, rows, S, mk);
+  return (int)cudaGetLastError();
+}
+
+}  // namespace fmdq

@@ -202,7 +202,8 @@ __device__ void slice_stream_column(const uint2* recs, int cnt, const int8_t* bi
 #pragma unroll
   for (int i = 0; i < kTile; ++i) {
     const int64_t row = t * kTile + i;
-    const float y = epi(acc[i], true, p2, beta, ws, load_y<OUT_BF16>(y_prev, row * ld_yp + n));
+    // no y_prev: the output has no cached previous value (Y_{t-1} = 0)
+    const float y = epi(acc[i], true, p2, beta, ws, y_prev ? load_y<OUT_BF16>(y_prev, row * ld_yp + n) : 0.f);
     store_y<OUT_BF16>(y_out, row * ld_yo + n, y);
     if (y_distinct) store_y<OUT_BF16>(y_prev, row * ld_yp + n, y);
     if (h_out) store_y<OUT_BF16>(h_out, row * ld_h + n, gelu(stored_value<OUT_BF16>(y)));
@@ -216,7 +217,7 @@ __device__ void slice_stream_column(const uint2* recs, int cnt, const int8_t* bi
 // With GELU, the activation of the stored values also goes to hrow (this
 // lane's row of the activation output at the group's first column, global
 // memory), 16 bytes per chunk, for the first hchunks chunks (columns < N).
-template <bool OUT_BF16, bool WIDE, bool GELU>
+template <bool OUT_BF16, bool WIDE, bool GELU, bool ZERO_Y = false>
 __device__ __forceinline__ void epi_group(uint8_t* row, int swz, const float* ws32, const uint32_t (&d0)[32],
                                           const uint32_t (&d1)[32], bool wide_row, float p2, float beta,
                                           uint8_t* hrow, int hchunks) {
@@ -227,7 +228,7 @@ __device__ __forceinline__ void epi_group(uint8_t* row, int swz, const float* ws
 #pragma unroll
   for (int c = 0; c < kChunks; ++c) {
     uint4* cp = reinterpret_cast<uint4*>(row + 16 * (c ^ swz));
-    const uint4 yv = *cp;
+    const uint4 yv = ZERO_Y ? make_uint4(0u, 0u, 0u, 0u) : *cp;  // ZERO_Y: no cached output (Y_{t-1} = 0)
     const uint32_t yw[4] = {yv.x, yv.y, yv.z, yv.w};
     float wsv[E];
 #pragma unroll
@@ -284,11 +285,24 @@ __device__ __forceinline__ void epi_group(uint8_t* row, int swz, const float* ws
 
 size_t gemm_smem_bytes(int bn) { return bn == 256 ? GemmCfg<256, true>::kBytes : GemmCfg<128, true>::kBytes; }
 
-template <int BN, bool OUT_BF16, bool GELU>
+// The batched, block-sparse form takes a GemmSparse argument; the plain one
+// an empty struct.
+struct NoSparse {};
+template <bool S>
+struct SparseArg {
+  using T = NoSparse;
+};
+template <>
+struct SparseArg<true> {
+  using T = GemmSparse;
+};
+
+template <int BN, bool OUT_BF16, bool GELU, bool SPARSE>
 __global__ void __launch_bounds__(kGThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CUtensorMap tm_a1,
                 const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_yp,
-                const __grid_constant__ CUtensorMap tm_yo, const GemmParams p) {
+                const __grid_constant__ CUtensorMap tm_yo, const GemmParams p,
+                const __grid_constant__ typename SparseArg<SPARSE>::T sp) {
   using C = GemmCfg<BN, OUT_BF16>;
   using TOut = typename OutT<OUT_BF16>::T;
   extern __shared__ uint8_t smem_raw[];
@@ -309,7 +323,33 @@ __global__ void __launch_bounds__(kGThreads, 1)
   uint8_t* ysmem = smem + C::kOffY;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int num_tiles = p.tiles_m * p.tiles_n;
+  // Tile i of the launch -> (row block, column block); with SPARSE, tiles run
+  // head by head over the listed tiles of a head (all, when none is listed).
+  int num_tiles = p.tiles_m * p.tiles_n, rb_per_head = p.tiles_m, tiles_per_head = num_tiles;
+  if constexpr (SPARSE) {
+    rb_per_head = (int)(sp.rows_per_head / kBlockM);
+    tiles_per_head = sp.n_listed > 0 ? sp.n_listed : rb_per_head * p.tiles_n;
+    num_tiles = (int)sp.heads * tiles_per_head;
+  }
+  auto coords = [&](int i, int& rb, int& nb) {
+    if constexpr (SPARSE) {
+      const int head = i / tiles_per_head, j = i % tiles_per_head;
+      const int id = sp.n_listed > 0 ? (int)sp.list[j] : j;
+      rb = head * rb_per_head + id / p.tiles_n, nb = id % p.tiles_n;
+    } else {
+      rb = i / p.tiles_n, nb = i % p.tiles_n;
+    }
+  };
+  // first row of W for a tile (the head's weights with SPARSE)
+  auto w_row = [&](int rb, int nb) -> int {
+    if constexpr (SPARSE) return (int)((rb / rb_per_head) * sp.w_rows_per_head) + nb * BN;
+    else return nb * BN;
+  };
+  // K chunk c of plane 0 is read for row block rb
+  auto keep0 = [&](int rb, int c) -> bool {
+    if constexpr (SPARSE) return ((sp.chunk_keep[rb % rb_per_head] >> c) & 1ull) != 0;
+    else return true;
+  };
   const int my_tiles = num_tiles > (int)blockIdx.x ? (num_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
   const int T = (int)(p.M / kTile);
 
@@ -360,18 +400,21 @@ __global__ void __launch_bounds__(kGThreads, 1)
       // first stages are requested before waiting for it.
       uint32_t pre = 0;
       if (my_tiles > 0) {
-        const int nb0 = (int)blockIdx.x % p.tiles_n;
-        pre = (uint32_t)min(C::kStages, p.num_chunks);
-        for (uint32_t c = 0; c < pre; ++c) {
-          mbar_arrive_expect_tx(&full[c], C::kStageBytes);
-          tma_load_2d(stages + c * C::kStageBytes + kA0Bytes, &tm_w, &full[c], (int)c * kChunkK, nb0 * BN);
+        int rb0, nb0;
+        coords((int)blockIdx.x, rb0, nb0);
+        for (int c = 0; c < p.num_chunks && pre < (uint32_t)C::kStages; ++c) {
+          if (!keep0(rb0, c)) continue;
+          mbar_arrive_expect_tx(&full[pre], C::kStageBytes);
+          tma_load_2d(stages + pre * C::kStageBytes + kA0Bytes, &tm_w, &full[pre], c * kChunkK, w_row(rb0, nb0));
+          ++pre;
         }
       }
       pdl_wait();  // the operand planes are the previous kernel's output
       bool have_info = false;
       for (int slot = 0; slot < my_tiles && ok; ++slot) {
-        const int tile = (int)blockIdx.x + slot * (int)gridDim.x;
-        const int rb = tile / p.tiles_n, nb = tile % p.tiles_n;
+        int rb, nb;
+        coords((int)blockIdx.x + slot * (int)gridDim.x, rb, nb);
+        const int wr = w_row(rb, nb);
         for (int pass = 0; pass < 2 && ok; ++pass) {
           BlockInfo bi{};
           if (pass == 1) {  // plane 1 only where the block needs it
@@ -382,6 +425,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
           }
           const CUtensorMap* tm_a = pass == 0 ? &tm_a0 : &tm_a1;
           for (int c = 0; c < p.num_chunks; ++c) {
+            if (pass == 0 && !keep0(rb, c)) continue;
             if (pass == 1 && !chunk_has_plane1(bi, c)) continue;
             const int s = it % C::kStages;
             uint8_t* a = stages + s * C::kStageBytes;
@@ -396,7 +440,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
             }
             mbar_arrive_expect_tx(&full[s], C::kStageBytes);
             tma_load_2d(a, tm_a, &full[s], c * kChunkK, rb * kBlockM);
-            tma_load_2d(a + kA0Bytes, &tm_w, &full[s], c * kChunkK, nb * BN);
+            tma_load_2d(a + kA0Bytes, &tm_w, &full[s], c * kChunkK, wr);
             ++it;
           }
         }
@@ -414,8 +458,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
       uint32_t it = 0, slot_it = 0;
       bool ok = true, issued = false, have_info = false;
       for (int slot = 0; slot < my_tiles && ok; ++slot) {
-        const int tile = (int)blockIdx.x + slot * (int)gridDim.x;
-        const int rb = tile / p.tiles_n;
+        int rb, nb_unused;
+        coords((int)blockIdx.x + slot * (int)gridDim.x, rb, nb_unused);
         uint32_t acc0 = 0, acc1 = 0;
         int np = 1;
         for (int pass = 0; pass < 2 && ok; ++pass) {
@@ -437,6 +481,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
           const uint32_t d = tmem_base + acc * BN;
           bool first = true;
           for (int c = 0; c < p.num_chunks; ++c) {
+            if (pass == 0 && !keep0(rb, c)) continue;
             if (pass == 1 && !chunk_has_plane1(bi, c)) continue;
             const int s = it % C::kStages;
             if (!wait_parity(&full[s], (it / C::kStages) & 1, s_abort, p.status, kWaitLimitNs)) {
@@ -478,22 +523,34 @@ __global__ void __launch_bounds__(kGThreads, 1)
     // TMA swizzle of a 32 x 32 tile: 64-byte rows (bf16) use the 64-byte pattern,
     // 128-byte rows (fp32) the 128-byte one; chunk c of row r sits at chunk c ^ sw(r)
     auto sw = [](int r) { return OUT_BF16 ? ((r >> 1) & 3) : (r & 7); };
-    auto tile_rb = [&](int s) { return ((int)blockIdx.x + s * (int)gridDim.x) / p.tiles_n; };
-    auto tile_nb = [&](int s) { return ((int)blockIdx.x + s * (int)gridDim.x) % p.tiles_n; };
+    auto tile_rb = [&](int s) {
+      int rb, nb;
+      coords((int)blockIdx.x + s * (int)gridDim.x, rb, nb);
+      return rb;
+    };
+    auto tile_nb = [&](int s) {
+      int rb, nb;
+      coords((int)blockIdx.x + s * (int)gridDim.x, rb, nb);
+      return nb;
+    };
     // Everything a tile needs besides its accumulator is requested one tile
     // ahead: its y_prev boxes (each as soon as the previous tile's store has
     // read the box), its weight scales (shared memory, double-buffered) and
     // this lane's row data.
     auto weight_scale = [&](int s) -> float {
       const int64_t n = (int64_t)tile_nb(s) * BN + etid;
-      return (etid < BN && n < p.N) ? p.w_scale[n] : 0.f;
+      int64_t off = 0;  // the head's scales with SPARSE
+      if constexpr (SPARSE) off = (int64_t)(tile_rb(s) / rb_per_head) * p.N;
+      return (etid < BN && n < p.N) ? p.w_scale[off + n] : 0.f;
     };
     auto row_planes = [&](int s, int& pl, int& gref) {
       const int64_t row = (int64_t)tile_rb(s) * kBlockM + quarter * 32 + lane;
       pl = 3, gref = 0;
       if (row < p.M) pl = p.planes[row / kTile], gref = p.g_ref[row / kTile];
     };
+    // With SPARSE there is no cached output: Y_{t-1} = 0 is never read.
     auto load_y_box = [&](int s, int box) {  // lane 0
+      if constexpr (SPARSE) return;
       if (box == 0) mbar_arrive_expect_tx(&ybar[ew], C::kYWarpBytes);
       tma_load_2d(ybuf + box * C::kBoxBytes, &tm_yp, &ybar[ew], tile_nb(s) * BN + half * (BN / 2) + box * 32,
                   tile_rb(s) * kBlockM + quarter * 32);
@@ -561,12 +618,19 @@ __global__ void __launch_bounds__(kGThreads, 1)
             ok = wait_parity(&tm_full[acc_slot[q]], (si / C::kSlots) & 1, s_abort, p.status, kWaitLimitNs) ? 1 : 0;
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (lane == 0 && ok) ok = wait_parity(&ybar[ew], y_seen & 1, s_abort, p.status, kWaitLimitNs) ? 1 : 0;
-        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if constexpr (!SPARSE) {
+          if (lane == 0 && ok) ok = wait_parity(&ybar[ew], y_seen & 1, s_abort, p.status, kWaitLimitNs) ? 1 : 0;
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+        } else {
+          if (lane == 0) bulk_wait_read<0>();  // the previous tile's stores have read the boxes
+          __syncwarp();
+        }
         if (ok) {
           // the landed tiles are visible to the lanes that observe the barrier phase
-          mbar_try_wait(&ybar[ew], y_seen & 1);
-          ++y_seen;
+          if constexpr (!SPARSE) {
+            mbar_try_wait(&ybar[ew], y_seen & 1);
+            ++y_seen;
+          }
           tc_fence_after();
           const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
           const uint32_t col_half = half * (BN / 2);
@@ -621,7 +685,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
             if (row_ok) {
               int hch;
               uint8_t* hr = h_row(g, hch);
-              epi_group<OUT_BF16, false, GELU>(my_row + g * C::kBoxBytes, swz, ws_h + g * 32, d, d, false, p2, beta,
+              epi_group<OUT_BF16, false, GELU, SPARSE>(my_row + g * C::kBoxBytes, swz, ws_h + g * 32, d, d, false, p2, beta,
                                                hr, hch);
               if (p.debug_acc) debug_group(g, d, d, false);
             }
@@ -653,7 +717,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
               if (row_ok) {
                 int hch;
                 uint8_t* hr = h_row(g, hch);
-                epi_group<OUT_BF16, true, GELU>(my_row + g * C::kBoxBytes, swz, ws_h + g * 32, d0, d1, wide_row, p2,
+                epi_group<OUT_BF16, true, GELU, SPARSE>(my_row + g * C::kBoxBytes, swz, ws_h + g * 32, d0, d1, wide_row, p2,
                                                 beta, hr, hch);
                 if (p.debug_acc) debug_group(g, d0, d1, true);
               }
@@ -681,7 +745,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
             const int64_t n = n_base + c;
             if (n >= p.N) continue;
             slice_stream_column<OUT_BF16>(p.records + (int64_t)t * p.record_cap, p.count[t], p.bits + (int64_t)t * p.K,
-                                          p.g_ref[t], p.w_q + n * p.ld_w, t, n, p.lb, beta, ws_tile[c], p.y_prev, p.ld_yp,
+                                          p.g_ref[t], p.w_q + ((int64_t)w_row(rb, 0) + n) * p.ld_w, t, n, p.lb, beta,
+                                          ws_tile[c], SPARSE ? nullptr : p.y_prev, p.ld_yp,
                                           p.y_out, p.ld_yo, p.y_distinct, p.debug_acc, p.N, p.h_out, p.ld_h);
           }
         }
@@ -696,7 +761,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
     // y_prev boxes that were requested but not observed, and the last stores
     y_issued = __shfl_sync(0xffffffffu, y_issued, 0);
     if (lane == 0) {
-      if (y_issued > y_seen) wait_parity(&ybar[ew], (y_issued - 1) & 1, s_abort, p.status, kWaitLimitNs, true);
+      if (!SPARSE && y_issued > y_seen)
+        wait_parity(&ybar[ew], (y_issued - 1) & 1, s_abort, p.status, kWaitLimitNs, true);
       bulk_wait<0>();
     }
     __syncwarp();
@@ -747,13 +813,16 @@ __global__ void selftest_wait_kernel(uint32_t* status, uint64_t limit_ns) {
   }
 }
 
-template <int BN, bool BF, bool GELU>
-static int launch_gemm_t(const GemmParams& p, const CUtensorMap* m, int num_sms, void* stream) {
-  const int tiles = p.tiles_m * p.tiles_n;
+template <int BN, bool BF, bool GELU, bool SPARSE = false>
+static int launch_gemm_t(const GemmParams& p, const CUtensorMap* m, int num_sms, void* stream,
+                         const typename SparseArg<SPARSE>::T& sp = {}) {
+  int tiles = p.tiles_m * p.tiles_n;
+  if constexpr (SPARSE)
+    tiles = (int)sp.heads * (sp.n_listed > 0 ? sp.n_listed : (int)(sp.rows_per_head / kBlockM) * p.tiles_n);
   const int grid = tiles < num_sms ? tiles : num_sms;
   if (grid == 0) return 0;
   const int smem = GemmCfg<BN, BF>::kBytes;
-  const int e = ensure_max_smem((const void*)gemm_kernel<BN, BF, GELU>, smem);
+  const int e = ensure_max_smem((const void*)gemm_kernel<BN, BF, GELU, SPARSE>, smem);
   if (e != 0) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid, 1, 1);
@@ -765,7 +834,7 @@ static int launch_gemm_t(const GemmParams& p, const CUtensorMap* m, int num_sms,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t ce = cudaLaunchKernelEx(&cfg, gemm_kernel<BN, BF, GELU>, m[0], m[1], m[2], m[3], m[4], p);
+  const cudaError_t ce = cudaLaunchKernelEx(&cfg, gemm_kernel<BN, BF, GELU, SPARSE>, m[0], m[1], m[2], m[3], m[4], p, sp);
   if (ce != cudaSuccess) return (int)ce;
   return (int)cudaGetLastError();
 }
@@ -782,6 +851,10 @@ int launch_gemm(const GemmParams& p, const void* maps, int bn, int out_bf16, int
   const CUtensorMap* m = static_cast<const CUtensorMap*>(maps);
   return p.h_out ? launch_gemm_g<true>(p, m, bn, out_bf16, num_sms, stream)
                  : launch_gemm_g<false>(p, m, bn, out_bf16, num_sms, stream);
+}
+
+int launch_gemm_sparse(const GemmParams& p, const GemmSparse& sp, const void* maps, int num_sms, void* stream) {
+  return launch_gemm_t<128, false, false, true>(p, static_cast<const CUtensorMap*>(maps), num_sms, stream, sp);
 }
 
 int launch_slice_gemm(const SliceParams& p, int out_bf16, int num_sms, void* stream) {

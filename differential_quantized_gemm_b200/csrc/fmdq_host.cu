@@ -350,6 +350,87 @@ int check_gemm_args(const dstar_mat* w_q, const float* w_scale, dstar_mat* y_pre
   return DSTAR_OK;
 }
 
+// ------------------------------------------------------------ attention
+
+struct SarLayout {
+  size_t total, ws_p, ws_q, kq, ks, vqt, vs, scores, probs;
+};
+
+SarLayout sar_layout(int64_t G, int64_t S, int64_t d) {
+  SarLayout L{};
+  const int64_t R = G * S;
+  size_t o = 0;
+  L.ws_p = o, o = align256(o + ws_layout(R, S).total);
+  L.ws_q = o, o = align256(o + ws_layout(R, d).total);
+  L.kq = o, o = align256(o + (size_t)(R * d));
+  L.ks = o, o = align256(o + (size_t)R * 4);
+  L.vqt = o, o = align256(o + (size_t)(G * d * S));
+  L.vs = o, o = align256(o + (size_t)(G * d) * 4);
+  L.scores = o, o = align256(o + (size_t)(R * S) * 4);
+  L.probs = o, o = align256(o + (size_t)(R * S) * 4);
+  L.total = o;
+  return L;
+}
+
+int check_sar_sizes(int64_t G, int64_t S, int64_t d) {
+  if (G <= 0) return fail(DSTAR_ERR_INVALID_ARG, "heads must be positive");
+  if (S <= 0 || S % DSTAR_SAR_BLOCK != 0 || S / DSTAR_SAR_BLOCK > kSparseMaxRowBlocks)
+    return fail(DSTAR_ERR_INVALID_ARG, "seq must be a positive multiple of %d up to %d", DSTAR_SAR_BLOCK,
+                DSTAR_SAR_BLOCK * kSparseMaxRowBlocks);
+  if (d <= 0 || d % 32 != 0 || d > DSTAR_K_MAX)
+    return fail(DSTAR_ERR_INVALID_ARG, "head_dim must be a positive multiple of 32 up to %d", DSTAR_K_MAX);
+  return DSTAR_OK;
+}
+
+// One FMDQ workspace inside the attention workspace, as a tile_cfg with every width 8.
+dstar_tile_cfg sar_cfg_of(void* base, size_t off, int64_t M, int64_t K) {
+  dstar_tile_cfg c{};
+  c.tile_tokens = DSTAR_TILE_TOKENS;
+  c.force_bits = 8;
+  c.workspace = static_cast<uint8_t*>(base) + off;
+  c.workspace_bytes = ws_layout(M, K).total;
+  return c;
+}
+
+// The batched, block-sparse slice GEMM: operand planes of the FMDQ workspace
+// `c` (R rows, K columns), weights w [w_rows x K] (head h's rows start at h *
+// sp.w_rows_per_head), y [R x N] fp32 (Y_{t-1} = 0, not read).
+int do_gemm_sparse(const dstar_tile_cfg* c, int64_t R, int64_t K, const int8_t* w, int64_t w_rows, int64_t ldw,
+                   const float* w_scale, float* y, int64_t N, int64_t ldy, int lb, const GemmSparse& sp,
+                   const DevInfo& dev, void* stream) {
+  const WsLayout L = ws_layout(R, K);
+  CUtensorMap maps[5];
+  dstar_mat ym{y, DSTAR_F32, 0, R, N, ldy};
+  int r;
+  if ((r = make_map_i8(&maps[0], ws_ptr<void>(c, L.plane0), R, K, K, kBlockM)) != DSTAR_OK) return r;
+  if ((r = make_map_i8(&maps[1], ws_ptr<void>(c, L.plane1), R, K, K, kBlockM)) != DSTAR_OK) return r;
+  if ((r = make_map_i8(&maps[2], w, w_rows, K, ldw, 128)) != DSTAR_OK) return r;
+  if ((r = make_map_y(&maps[3], &ym)) != DSTAR_OK) return r;
+  if ((r = make_map_y(&maps[4], &ym)) != DSTAR_OK) return r;
+  GemmParams g{};
+  g.M = R, g.N = N, g.K = K;
+  g.lb = lb;
+  g.g_ref = ws_ptr<int32_t>(c, L.g_ref);
+  g.planes = ws_ptr<int32_t>(c, L.planes);
+  g.mask1 = ws_ptr<uint32_t>(c, L.mask1);
+  g.mask_words = L.mask_words;
+  g.w_scale = w_scale;
+  g.y_prev = y, g.ld_yp = ldy, g.y_out = y, g.ld_yo = ldy;
+  g.status = ws_ptr<uint32_t>(c, L.status);
+  g.tiles_m = (int)(R / kBlockM);
+  g.tiles_n = (int)((N + 127) / 128);
+  g.num_chunks = (int)((K + kChunkK - 1) / kChunkK);
+  g.w_q = w;
+  g.ld_w = ldw;
+  g.records = ws_ptr<const uint2>(c, L.records);
+  g.record_cap = L.record_cap;
+  g.count = ws_ptr<const int32_t>(c, L.count);
+  g.bits = ws_ptr<const int8_t>(c, L.bits);
+  const int e = launch_gemm_sparse(g, sp, maps, dev.sms, stream);
+  if (e) return cuda_fail(e, "sparse slice-GEMM launch");
+  return DSTAR_OK;
+}
+
 std::mutex g_attr_mu;
 struct AttrEntry {
   int dev;
@@ -571,6 +652,134 @@ int dstar_fmdq_ffn_gelu(const dstar_mat* x_t, dstar_mat* x_prev, dstar_mat* y1_p
                        n2 > 0 ? y2_prev : nullptr)) != DSTAR_OK)
     return r;
   if ((r = do_gemm(w2, w2_scale, y2_prev, lb, cfg2, y2_prev, M, N1, n2, dev, stream)) != DSTAR_OK) return r;
+  return ok();
+}
+
+int dstar_sar_workspace_size(int64_t heads, int64_t seq, int64_t head_dim, size_t* bytes) {
+  if (!bytes) return fail(DSTAR_ERR_INVALID_ARG, "bytes is NULL");
+  int r;
+  if ((r = check_sar_sizes(heads, seq, head_dim)) != DSTAR_OK) return r;
+  *bytes = sar_layout(heads, seq, head_dim).total;
+  return ok();
+}
+
+int dstar_sar_workspace_layout(int64_t heads, int64_t seq, int64_t head_dim, dstar_sar_layout* out) {
+  if (!out) return fail(DSTAR_ERR_INVALID_ARG, "out is NULL");
+  int r;
+  if ((r = check_sar_sizes(heads, seq, head_dim)) != DSTAR_OK) return r;
+  const SarLayout L = sar_layout(heads, seq, head_dim);
+  *out = dstar_sar_layout{L.total, L.ws_p, L.ws_q, L.kq, L.ks, L.vqt, L.vs, L.scores, L.probs};
+  return ok();
+}
+
+namespace {
+int check_sar_cfg(const dstar_sar_cfg* cfg, SarLayout* L) {
+  if (!cfg) return fail(DSTAR_ERR_INVALID_ARG, "cfg is NULL");
+  int r;
+  if ((r = check_sar_sizes(cfg->heads, cfg->seq, cfg->head_dim)) != DSTAR_OK) return r;
+  *L = sar_layout(cfg->heads, cfg->seq, cfg->head_dim);
+  if (!cfg->workspace) return fail(DSTAR_ERR_WORKSPACE, "workspace is NULL");
+  if (reinterpret_cast<uintptr_t>(cfg->workspace) & 255u) return fail(DSTAR_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  if (cfg->workspace_bytes < L->total)
+    return fail(DSTAR_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", cfg->workspace_bytes, L->total);
+  return DSTAR_OK;
+}
+}  // namespace
+
+int dstar_sar_workspace_init(const dstar_sar_cfg* cfg, void* stream) {
+  SarLayout L;
+  int r;
+  if ((r = check_sar_cfg(cfg, &L)) != DSTAR_OK) return r;
+  uint8_t* base = static_cast<uint8_t*>(cfg->workspace);
+  cudaError_t e = cudaMemsetAsync(base + L.ws_p, 0, 256, (cudaStream_t)stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(base + L.ws_q, 0, 256, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  return ok();
+}
+
+int dstar_sar_attention(const dstar_mat* q, const dstar_mat* k, const dstar_mat* v, const dstar_sar_cfg* cfg,
+                        int reuse, dstar_mat* out, void* stream) {
+  SarLayout L;
+  int r;
+  if ((r = check_sar_cfg(cfg, &L)) != DSTAR_OK) return r;
+  const int64_t G = cfg->heads, S = cfg->seq, d = cfg->head_dim, R = G * S, nb = S / DSTAR_SAR_BLOCK;
+  if (!q || !k || !v || !out) return fail(DSTAR_ERR_INVALID_ARG, "q, k, v or out is NULL");
+  if (!reuse) {
+    if ((r = check_mat(q, "q", R, d, true)) != DSTAR_OK) return r;
+    if ((r = check_mat(k, "k", R, d, true)) != DSTAR_OK) return r;
+    if (k->dtype != q->dtype) return fail(DSTAR_ERR_INVALID_ARG, "q and k must share a dtype");
+  }
+  if ((r = check_mat(v, "v", R, d, true)) != DSTAR_OK) return r;
+  if ((r = check_mat(out, "out", R, d, true)) != DSTAR_OK) return r;
+  if (out->dtype != DSTAR_F32) return fail(DSTAR_ERR_INVALID_ARG, "out must be F32");
+  if (!cfg->block_mask) return fail(DSTAR_ERR_INVALID_ARG, "block_mask is NULL");
+  if (!(cfg->scores_scale > 0.f) || !std::isfinite(cfg->scores_scale))
+    return fail(DSTAR_ERR_INVALID_ARG, "scores_scale must be positive and finite");
+  int lb_q = 0, lb_p = 0;
+  if ((r = base_log2(cfg->base_q, &lb_q)) != DSTAR_OK) return r;
+  if ((r = base_log2(cfg->base_p, &lb_p)) != DSTAR_OK) return r;
+  // the mask: per row block, the kept key blocks; the listed score tiles
+  GemmSparse sp_s{}, sp_o{};
+  BlockMask mk{};
+  int listed = 0;
+  for (int64_t a = 0; a < nb; ++a) {
+    for (int64_t b = 0; b < nb; ++b)
+      if (cfg->block_mask[a * nb + b]) {
+        mk.bits[a] |= 1ull << b;
+        sp_s.list[listed++] = (uint16_t)(a * nb + b);
+      }
+    if (!mk.bits[a]) return fail(DSTAR_ERR_INVALID_ARG, "block_mask row %lld keeps no block", (long long)a);
+  }
+  sp_s.heads = sp_o.heads = G;
+  sp_s.rows_per_head = sp_o.rows_per_head = S;
+  sp_s.w_rows_per_head = S, sp_o.w_rows_per_head = d;
+  sp_s.n_listed = listed == nb * nb ? 0 : listed;
+  sp_o.n_listed = 0;
+  for (int64_t a = 0; a < kSparseMaxRowBlocks; ++a) sp_s.chunk_keep[a] = ~0ull, sp_o.chunk_keep[a] = a < nb ? mk.bits[a] : 0;
+  DevInfo dev;
+  if ((r = device_info(&dev)) != DSTAR_OK) return r;
+  uint8_t* base = static_cast<uint8_t*>(cfg->workspace);
+  const dstar_tile_cfg cp = sar_cfg_of(base, L.ws_p, R, S);
+  const dstar_mat none{nullptr, q ? q->dtype : DSTAR_F32, 0, R, d, d};  // X_{t-1} = 0: the operands themselves
+  int e;
+  if (!reuse) {
+    const dstar_tile_cfg cq = sar_cfg_of(base, L.ws_q, R, d);
+    e = launch_quant_rows(k->data, k->ld, R, d, k->dtype == DSTAR_BF16, reinterpret_cast<int8_t*>(base + L.kq), d,
+                          reinterpret_cast<float*>(base + L.ks), cfg->scores_scale, stream);
+    if (e) return cuda_fail(e, "key quantization launch");
+    dstar_mat none_q = none;
+    if ((r = do_quantize(q, &none_q, lb_q, &cq, R, d, dev, stream)) != DSTAR_OK) return r;
+    if ((r = do_gemm_sparse(&cq, R, d, reinterpret_cast<const int8_t*>(base + L.kq), R, d,
+                            reinterpret_cast<const float*>(base + L.ks), reinterpret_cast<float*>(base + L.scores), S,
+                            S, lb_q, sp_s, dev, stream)) != DSTAR_OK)
+      return r;
+    e = launch_masked_softmax(reinterpret_cast<const float*>(base + L.scores), reinterpret_cast<float*>(base + L.probs),
+                              R, S, mk, stream);
+    if (e) return cuda_fail(e, "softmax launch");
+    const dstar_mat pm{base + L.probs, DSTAR_F32, 0, R, S, S};
+    dstar_mat none_p{nullptr, DSTAR_F32, 0, R, S, S};
+    if ((r = do_quantize(&pm, &none_p, lb_p, &cp, R, S, dev, stream)) != DSTAR_OK) return r;
+  }
+  e = launch_quant_cols_t(v->data, v->ld, G, S, d, v->dtype == DSTAR_BF16, reinterpret_cast<int8_t*>(base + L.vqt),
+                          reinterpret_cast<float*>(base + L.vs), stream);
+  if (e) return cuda_fail(e, "value quantization launch");
+  if ((r = do_gemm_sparse(&cp, R, S, reinterpret_cast<const int8_t*>(base + L.vqt), G * d, S,
+                          reinterpret_cast<const float*>(base + L.vs), static_cast<float*>(out->data), d, out->ld,
+                          lb_p, sp_o, dev, stream)) != DSTAR_OK)
+    return r;
+  return ok();
+}
+
+int dstar_sar_status(const dstar_sar_cfg* cfg, void* stream, uint32_t* status) {
+  SarLayout L;
+  int r;
+  if (!status) return fail(DSTAR_ERR_INVALID_ARG, "status is NULL");
+  if ((r = check_sar_cfg(cfg, &L)) != DSTAR_OK) return r;
+  uint32_t a = 0, b = 0;
+  uint8_t* base = static_cast<uint8_t*>(cfg->workspace);
+  if ((r = dstar_fmdq_status(base + L.ws_p, stream, &a)) != DSTAR_OK) return r;
+  if ((r = dstar_fmdq_status(base + L.ws_q, stream, &b)) != DSTAR_OK) return r;
+  *status = a | b;
   return ok();
 }
 

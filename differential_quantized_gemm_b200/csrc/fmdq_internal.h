@@ -30,7 +30,7 @@ struct L2Region {
 
 struct QuantParams {
   const void* x_t;
-  void* x_prev;
+  void* x_prev;  // nullptr: X_{t-1} = 0 (the operand itself is quantized; no refresh)
   int64_t ld_xt, ld_xp;
   int64_t M, K;
   int lb, t0, force_bits;
@@ -85,6 +85,26 @@ struct GemmParams {
   const int8_t* bits;
 };
 
+// Batched heads and block sparsity of the attention GEMMs (sparse attention
+// reuse): rows [h R, (h + 1) R) of the operand planes form head h, whose
+// weights are rows [h WR, (h + 1) WR) of W and whose weight scales are
+// w_scale[h N + n].  Within a head, only the listed 128 x 128 output tiles
+// are computed (local tile id = row block * tiles_n + column block), and
+// row block r reads only the K chunks set in chunk_keep[r].
+constexpr int kSparseMaxTiles = 1024;
+constexpr int kSparseMaxRowBlocks = 32;
+struct GemmSparse {
+  int64_t heads, rows_per_head, w_rows_per_head;
+  int n_listed;                  // listed tiles per head (0: every tile)
+  uint16_t list[kSparseMaxTiles];
+  uint64_t chunk_keep[kSparseMaxRowBlocks];  // all ones: every chunk
+};
+
+// A block mask of one head's score matrix: bit c of bits[r] = block (r, c) kept.
+struct BlockMask {
+  uint64_t bits[kSparseMaxRowBlocks];
+};
+
 struct SliceParams {
   int64_t M, N, K;
   int lb;
@@ -126,7 +146,16 @@ int launch_base_min(const void* x_t, const void* x_prev, int64_t ld_xt, int64_t 
 int quantize_cluster_size(int64_t M, int64_t K, int num_sms);
 int launch_gemm(const GemmParams& p, const void* maps /* CUtensorMap[5]: A0, A1, W, y_prev, y_out */, int bn,
                 int out_bf16, int num_sms, void* stream);
+// The batched, block-sparse form (fp32 outputs, 128-column tiles).
+int launch_gemm_sparse(const GemmParams& p, const GemmSparse& sp, const void* maps, int num_sms, void* stream);
 int launch_slice_gemm(const SliceParams& p, int out_bf16, int num_sms, void* stream);
+// attention operands: per-row int8 (scale_out = scale * scale_mul), per-column
+// int8 of each head's V written transposed, and the block-masked softmax
+int launch_quant_rows(const void* x, int64_t ld, int64_t rows, int64_t cols, int in_bf16, int8_t* q, int64_t ldq,
+                      float* scale_out, float scale_mul, void* stream);
+int launch_quant_cols_t(const void* v, int64_t ld, int64_t heads, int64_t S, int64_t d, int in_bf16, int8_t* vqt,
+                        float* scale, void* stream);
+int launch_masked_softmax(const float* sc, float* pr, int64_t rows, int64_t S, const BlockMask& mk, void* stream);
 int launch_selftest_wait(uint32_t* status, uint32_t spin_limit, void* stream);
 size_t quantize_smem_bytes(int64_t Kc);  // shared memory of a CTA owning Kc channels
 // Raise a kernel's dynamic shared-memory limit once per device (returns a

@@ -68,6 +68,7 @@ struct Pair<__nv_bfloat16> {
   // bf16 -> fp32 is exact: the bf16 bits are the high half of the fp32 word
   __device__ static float lo(Raw r) { return __uint_as_float(r << 16); }
   __device__ static float hi(Raw r) { return __uint_as_float(r & 0xFFFF0000u); }
+  __device__ static Raw zero() { return 0u; }
 };
 template <>
 struct Pair<float> {
@@ -80,6 +81,7 @@ struct Pair<float> {
   }
   __device__ static float lo(Raw r) { return __uint_as_float(r.x); }
   __device__ static float hi(Raw r) { return __uint_as_float(r.y); }
+  __device__ static Raw zero() { return make_uint2(0u, 0u); }
 };
 
 __device__ __forceinline__ float exp2_exact(int e) {  // 2^e for e in the normal range
@@ -304,7 +306,7 @@ __device__ __forceinline__ QConst quant_const(const QuantParams& p) {
     if (q.dbits == 0xFFFFFFFFu) q.dbits = 0x3F800000u;
   }
   q.dbase = __uint_as_float(q.dbits);
-  q.refresh = !(p.flags & DSTAR_FLAG_NO_XPREV_REFRESH);
+  q.refresh = !(p.flags & DSTAR_FLAG_NO_XPREV_REFRESH) && p.x_prev != nullptr;
   return q;
 }
 
@@ -323,10 +325,11 @@ struct P1Red {
 template <typename TIn>
 __device__ __forceinline__ void load_pair(const QuantParams& p, int64_t row0, int64_t c,
                                           typename Pair<TIn>::Raw (&a)[kTile], typename Pair<TIn>::Raw (&b)[kTile]) {
+  const bool diff = p.x_prev != nullptr;  // no x_prev: the operand itself is quantized (X_{t-1} = 0)
 #pragma unroll
   for (int i = 0; i < kTile; ++i) {
     a[i] = Pair<TIn>::load(p.x_t, (row0 + i) * p.ld_xt + c);
-    b[i] = Pair<TIn>::load(p.x_prev, (row0 + i) * p.ld_xp + c);
+    b[i] = diff ? Pair<TIn>::load(p.x_prev, (row0 + i) * p.ld_xp + c) : Pair<TIn>::zero();
   }
 }
 

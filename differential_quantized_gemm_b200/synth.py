@@ -252,3 +252,27 @@ class SweepChain:
 
 def sweep_chain(layer: int, steps: list[int], M: int = 8192, force_bits: int = 0) -> SweepChain:
     return SweepChain(layer, steps, M, force_bits)
+
+
+def attention_inputs(heads: int, seq: int, head_dim: int, pad_to: int, seed: int, keep: float = 0.5):
+    """Seeded Q, K, V for `heads` attention problems of `seq` tokens: N(0, 1)
+    in the first head_dim channels, zero padding up to pad_to (bf16 bit
+    patterns, [heads*seq x pad_to]); V of the next step (V plus a 0.05 N(0, 1)
+    change); and a block mask [seq/128 x seq/128] that keeps every diagonal
+    block and each other block with probability `keep` (the pages' masks come
+    from profiling trained models, which are not available)."""
+    rng = _rng(seed, 909)
+    R = heads * seq
+
+    def draw():
+        x = np.zeros((R, pad_to), np.float32)
+        x[:, :head_dim] = rng.standard_normal((R, head_dim), dtype=np.float32)
+        return x
+
+    q, k, v = draw(), draw(), draw()
+    v2 = v.copy()
+    v2[:, :head_dim] += 0.05 * rng.standard_normal((R, head_dim), dtype=np.float32)
+    nb = seq // 128
+    mask = (rng.random((nb, nb)) < keep).astype(np.uint8)
+    np.fill_diagonal(mask, 1)
+    return to_bf16_bits(q), to_bf16_bits(k), to_bf16_bits(v), to_bf16_bits(v2), mask

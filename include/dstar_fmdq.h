@@ -218,6 +218,66 @@ DSTAR_API int dstar_fmdq_ffn_gelu(const dstar_mat* x_t, dstar_mat* x_prev, dstar
                                   const dstar_tile_cfg* cfg1, const dstar_tile_cfg* cfg2, void* stream);
 
 /*
+ * Sparse attention reuse with INT8 FMDQ operands (section 3.2 "Sparse
+ * Attention Reuse"; section 4.3 "Attention Operation": every attention MMA
+ * in INT8, activations through FMDQ at 8 bits).  For each of `heads`
+ * independent problems (batch x head, stacked along the rows) of S tokens:
+ *   cached step (reuse == 0):
+ *     K -> int8 per key row (scale = max|row|/127, q = rne(k/scale));
+ *     Q -> FMDQ with every width 8 and X_{t-1} = 0 (base base_q);
+ *     scores = dequant(Q codes . K codes) * scores_scale, only on the blocks
+ *              the mask keeps (block size DSTAR_SAR_BLOCK; pruned blocks are
+ *              never computed);
+ *     P = softmax of each row over its kept blocks (fp32), 0 elsewhere;
+ *     P -> FMDQ with every width 8 and X_{t-1} = 0 (base base_p): this
+ *          quantized P is the cache, kept in the workspace;
+ *   reused step (reuse != 0): Q, K and the softmax are skipped and the P
+ *     cached by the last cached step on this workspace is used;
+ *   both: V -> int8 per head dimension; out = dequant(P codes . V codes),
+ *     reading only the kept blocks of P.
+ * Arguments
+ *   q, k, v  [heads*S x d] BF16 or F32 (one dtype), device; d a multiple of
+ *            32 (pad with zero channels; they change nothing)
+ *   out      [heads*S x d] F32, device: written
+ *   cfg      sizes, host block mask, scales and the caller-owned workspace of
+ *            dstar_sar_workspace_size bytes (256-byte aligned), initialised
+ *            once with dstar_sar_workspace_init
+ * S: a positive multiple of DSTAR_SAR_BLOCK up to 32 blocks; every mask row
+ * must keep at least one block.  Errors as dstar_fmdq_linear; status bits
+ * through dstar_sar_status.
+ */
+#define DSTAR_SAR_BLOCK 128
+typedef struct {
+  int64_t heads;             /* independent attention problems (batch x heads) */
+  int64_t seq;               /* S: tokens per problem */
+  int64_t head_dim;          /* d */
+  const uint8_t* block_mask; /* HOST [S/128 x S/128], row-major; nonzero = block kept */
+  float scores_scale;        /* multiplies Q K^T (1 / sqrt of the unpadded head dimension) */
+  float base_q, base_p;      /* static FMDQ bases of Q and of P (exact powers of two) */
+  void* workspace;
+  size_t workspace_bytes;
+} dstar_sar_cfg;
+
+/* Byte offsets of the attention workspace: ws_p and ws_q are FMDQ workspaces
+ * (dstar_fmdq_ws_layout inside) of P (rows heads*S, K = S: the cache of the
+ * reused steps) and of Q (K = d); kq int8 [heads*S x d] and ks fp32
+ * [heads*S] (the key scales times scores_scale); vqt int8 [heads*d x S] and
+ * vs fp32 [heads*d]; scores and probs fp32 [heads*S x S]. */
+typedef struct {
+  size_t total, ws_p, ws_q, kq, ks, vqt, vs, scores, probs;
+} dstar_sar_layout;
+
+DSTAR_API int dstar_sar_workspace_size(int64_t heads, int64_t seq, int64_t head_dim, size_t* bytes);
+DSTAR_API int dstar_sar_workspace_layout(int64_t heads, int64_t seq, int64_t head_dim, dstar_sar_layout* out);
+/* Clear the status words of a fresh attention workspace (enqueued on `stream`). */
+DSTAR_API int dstar_sar_workspace_init(const dstar_sar_cfg* cfg, void* stream);
+DSTAR_API int dstar_sar_attention(const dstar_mat* q, const dstar_mat* k, const dstar_mat* v, const dstar_sar_cfg* cfg,
+                                  int reuse, dstar_mat* out, void* stream);
+/* Synchronise `stream`, report and clear the status bits of the attention
+ * workspace described by cfg (both of its FMDQ stages). */
+DSTAR_API int dstar_sar_status(const dstar_sar_cfg* cfg, void* stream, uint32_t* status);
+
+/*
  * dstar_fmdq_linear for callers that cannot allocate device memory.  The
  * paper has no counterpart: this is a packaging choice of the library.
  *
