@@ -62,6 +62,8 @@ def parse(argv=None):
                          "copy: the quantizer copies X_t into one x_prev cache")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-next-rows", action="store_true",
+                    help="skip the chained FFN pair, the dynamic base and the sparse attention runs")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--mode", choices=["graph", "eager"], default="graph",
                     help="graph: each step replays a captured CUDA graph; eager: C-ABI calls per step")
@@ -846,6 +848,151 @@ def measure_sweep(args, torch, nat, L):
     return out
 
 
+def measure_dyn(args, torch, nat, L):
+    """The headline workload with the dynamic base (FMDQ-DYN): a first pass
+    finds min M_i, then the same quantizer and GEMM."""
+    cb = ConfigBench(args.config, args, 0, torch, nat, L)
+    for row in cb.sets:
+        for lay in row:
+            lay.cfg.flags |= nat.FLAG_DYNAMIC_BASE
+    stats = cb.warm_and_stats(args.warmup)
+    cb.capture()
+    steps = args.extra_steps
+    ms, _ = cb.timed(steps)
+    k1, k2 = cb.split_times(steps)
+    st = cb.status()
+    if st:
+        raise RuntimeError(f"device status {st} after the dynamic-base run")
+    dense = sum(s_["k2_dense"] for s_ in stats)
+    bases = [float(lay.ws.sections(lay.spec.M, lay.spec.K)["dyn_base"].cpu()[0]) for lay in cb.sets[0]]
+    out = {"what": "FMDQ-DYN (dynamic base = min M_i of the call, found by a first pass over X_t, X_{t-1})",
+           "value": job_tops(1, dense, ms / steps), "unit": "TOPS", "ms_per_step": ms / steps, "steps": steps,
+           "kernels": [{"layer": i.spec.name, "quantize_ms": round(a, 4), "slice_gemm_ms": round(b, 4)}
+                       for i, a, b in zip(cb.inputs, k1, k2)],
+           "bits_avg": [s_["bits_avg"] for s_ in stats], "dynamic_base": bases,
+           "gpu_launches_per_step": 3 * len(cb.inputs)}
+    cb.close()
+    return out
+
+
+def measure_ffn_gelu(args, torch, nat, L):
+    """The chained FFN pair of the headline workload with the GELU fused into
+    the first layer's epilogue (dstar_fmdq_ffn_gelu): X_t alternates between two
+    draws; every cache (x_prev, Y1, H, Y2) is carried by the library."""
+    from differential_quantized_gemm_b200 import synth
+    up = synth.make_layer(args.config, 0)
+    w2, s2 = synth.layer_weights(args.config, 1)
+    dev = "cuda"
+
+    def bf(a):
+        return torch.from_numpy(a).view(torch.bfloat16).to(dev)
+
+    xa, xb = bf(up.x_t), bf(up.x_prev)
+    x_prev = xb.clone()
+    y1 = bf(up.y_prev)
+    # H_{t-1} = GELU(Y1_{t-1}) and Y2_{t-1} = H_{t-1} W2_deq: the dense state of step 0 (not timed)
+    h_prev = torch.nn.functional.gelu(y1.float()).to(torch.bfloat16)
+    w1, ws1 = torch.from_numpy(up.w_q).to(dev), torch.from_numpy(up.w_scale).to(dev)
+    w2t, ws2 = torch.from_numpy(w2).to(dev), torch.from_numpy(s2).to(dev)
+    y2 = (h_prev.float() @ (w2t.float().t() * ws2[None, :])).to(torch.bfloat16)
+    h_t = torch.empty_like(h_prev)
+    M, K1, N1 = up.spec.M, up.spec.K, up.spec.N
+    wsa, wsb = nat.Workspace(M, K1), nat.Workspace(M, N1)
+    base = 2.0 ** up.spec.lb
+    stream = torch.cuda.current_stream()
+    graphs = []
+    cap = torch.cuda.Stream()
+    for x in (xa, xb):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            nat.ffn_gelu(x, x_prev, y1, w1, ws1, h_t, h_prev, y2, w2t, ws2, base, wsa, wsb)
+        graphs.append(g)
+    for _ in range(max(args.warmup, 4)):
+        for g in graphs:
+            g.replay()
+    torch.cuda.synchronize()
+    steps = args.extra_steps // 2 * 2
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):
+        graphs[i % 2].replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if nat.status(wsa) or nat.status(wsb):
+        raise RuntimeError("device status after the chained FFN pair")
+    ms = e0.elapsed_time(e1) / steps
+    layer_stats = []
+    for ws, K in ((wsa, K1), (wsb, N1)):
+        sec = ws.sections(M, K)
+        bits, planes = sec["bits"].float(), sec["planes"]
+        layer_stats.append({"bits_avg": float(bits.mean()),
+                            "planes_hist": [int((planes == 1).sum()), int((planes == 2).sum()),
+                                            int((planes > 2).sum())]})
+    dense = 2.0 * M * N1 * K1 + 2.0 * M * w2.shape[0] * N1
+    del graphs
+    torch.cuda.synchronize()
+    return {"what": "chained FFN pair, GELU fused into the first layer's epilogue (dstar_fmdq_ffn_gelu)",
+            "workload": synth.CONFIG_NAMES[args.config], "value": dense / (ms * 1e-3) / 1e12, "unit": "TOPS",
+            "ms_per_step": ms, "steps": steps, "gpu_launches_per_step": 4,
+            "layer_stats": layer_stats,
+            "note": "layer 2 quantizes the differential of GELU(Y1), wider than the independent draw of the "
+                    "headline's second layer (more 8-bit sub-channels and two-plane tiles)"}
+
+
+def measure_sar(args, torch, nat, L):
+    """Sparse attention reuse with INT8 FMDQ operands on the PixArt 1024px
+    attention: 2 x 16 heads of 4096 tokens, head dimension 72 (padded to 96),
+    a synthetic block mask keeping every diagonal block and half of the
+    others, the scores recomputed every second step (interval 2)."""
+    import math
+    from differential_quantized_gemm_b200 import synth
+    G, S, dh, d = 32, 4096, 72, 96
+    qb, kb, vb, v2b, mask = synth.attention_inputs(G, S, dh, d, seed=11, keep=0.5)
+
+    def dev(b):
+        return torch.from_numpy(b).view(torch.bfloat16).cuda()
+
+    q, k, v, v2 = dev(qb), dev(kb), dev(vb), dev(v2b)
+    out = torch.empty(G * S, d, dtype=torch.float32, device="cuda")
+    att = nat.SarAttention(G, S, d, mask, float(1.0 / math.sqrt(dh)), 2.0 ** -4, 2.0 ** -6)
+    stream = torch.cuda.current_stream()
+    cap = torch.cuda.Stream()
+    g_cached, g_reused = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_cached, stream=cap):
+        att(q, k, v, out)
+    with torch.cuda.graph(g_reused, stream=cap):
+        att(q, k, v2, out, reuse=True)
+    for _ in range(3):
+        g_cached.replay()
+        g_reused.replay()
+    torch.cuda.synchronize()
+    reps = max(4, min(40, args.extra_steps // 30))
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    tc, tr = [], []
+    for _ in range(reps):
+        ev[0].record(stream)
+        g_cached.replay()
+        ev[1].record(stream)
+        g_reused.replay()
+        ev[2].record(stream)
+        torch.cuda.synchronize()
+        tc.append(ev[0].elapsed_time(ev[1]))
+        tr.append(ev[1].elapsed_time(ev[2]))
+    if att.status():
+        raise RuntimeError("device status after the attention run")
+    kept = float(mask.mean())
+    dense = 4.0 * G * S * S * dh  # Q K^T and P V of full attention at the unpadded head dimension
+    c, r = statistics.median(tc), statistics.median(tr)
+    del g_cached, g_reused
+    torch.cuda.synchronize()
+    return {"what": "sparse attention reuse, INT8 FMDQ operands (dstar_sar_attention)",
+            "workload": f"PixArt 1024px attention: {G} heads x {S} tokens, head dim {dh} (padded to {d}), "
+                        f"{kept:.3f} of the 128x128 blocks kept, interval 2",
+            "cached_step_ms": c, "reused_step_ms": r, "ms_per_step": (c + r) / 2,
+            "value": dense / ((c + r) / 2 * 1e-3) / 1e12, "unit": "dense-equivalent attention TOPS",
+            "kept_block_fraction": kept, "reps": reps, "gpu_launches_per_step": 4.5}
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
 
@@ -901,13 +1048,17 @@ def run_ours(args, rank, world, local_rank):
     cb.close()
 
     # further workloads, on one GPU only (every rank would have to run them alike)
-    per_config, sweep = [], None
+    per_config, sweep, next_rows = [], None, None
     if world == 1:
         for c in [int(x) for x in args.extra_configs.split(",") if x.strip()]:
             if c != args.config:
                 per_config.append(measure_extra(c, args, torch, nat, L, peaks, peak_src))
         if args.sweep_steps > 0:
             sweep = measure_sweep(args, torch, nat, L)
+        if not args.no_next_rows:
+            next_rows = {"ffn_gelu": measure_ffn_gelu(args, torch, nat, L),
+                         "dynamic_base": measure_dyn(args, torch, nat, L),
+                         "sar_attention": measure_sar(args, torch, nat, L)}
 
     if rank != 0:
         return
@@ -935,7 +1086,7 @@ def run_ours(args, rank, world, local_rank):
         "slice_macs_per_s": sum(s["slice_macs"] for s in stats) / (ms_step * 1e-3),
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * nlayers * K,
         "clocks": clocks,
-        "per_config": per_config, "sweep": sweep,
+        "per_config": per_config, "sweep": sweep, "next_rows": next_rows,
         "kernel_sources": kernel_source_sha(),
         "timing": ("value: CUDA-graph replays of the captured dstar_fmdq_linear calls, one graph per cycle of "
                    f"{2 * args.sets} steps (every input set with both X_t); per-kernel times: a second timed "

@@ -151,12 +151,29 @@ __device__ __forceinline__ float gelu(float y) {
   return __fmul_rn(__fmul_rn(0.5f, y), erfcf(__fmul_rn(y, -0.70710678118654752f)));
 }
 
-// The stored Y_t as a float (bf16 outputs are rounded first), so that the
-// activation is a function of the cached output alone.
+}  // namespace
+
+// GELU of every bf16 value (the paper's vector unit computes GELU with
+// lookup tables): entry b holds GELU of the bf16 pattern b, evaluated in fp64
+// (CUDA's double erfc) and rounded to fp32, then to bf16.  Filled once per
+// CUDA context by gelu_table_kernel before the first GEMM that reads it.
+__device__ uint16_t g_gelu_bf16[65536];
+
+__global__ void gelu_table_kernel() {
+  const uint32_t b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= 65536u) return;
+  const double v = (double)__uint_as_float(b << 16);
+  const double g = 0.5 * v * erfc(-v * 0.70710678118654752440);
+  g_gelu_bf16[b] = __bfloat16_as_ushort(__float2bfloat16_rn((float)g));
+}
+
+namespace {
+
+// H = GELU(stored Y_t): the table for bf16 outputs, fp32 erfcf for fp32 ones.
 template <bool OUT_BF16>
-__device__ __forceinline__ float stored_value(float y) {
-  if constexpr (OUT_BF16) return __bfloat162float(__float2bfloat16_rn(y));
-  else return y;
+__device__ __forceinline__ float gelu_of_output(float y) {
+  if constexpr (OUT_BF16) return __bfloat162float(__ushort_as_bfloat16(g_gelu_bf16[__bfloat16_as_ushort(__float2bfloat16_rn(y))]));
+  else return gelu(y);
 }
 
 // The paper's accumulation order literally, for one 16-token tile and one
@@ -206,7 +223,7 @@ __device__ void slice_stream_column(const uint2* recs, int cnt, const int8_t* bi
     const float y = epi(acc[i], true, p2, beta, ws, y_prev ? load_y<OUT_BF16>(y_prev, row * ld_yp + n) : 0.f);
     store_y<OUT_BF16>(y_out, row * ld_yo + n, y);
     if (y_distinct) store_y<OUT_BF16>(y_prev, row * ld_yp + n, y);
-    if (h_out) store_y<OUT_BF16>(h_out, row * ld_h + n, gelu(stored_value<OUT_BF16>(y)));
+    if (h_out) store_y<OUT_BF16>(h_out, row * ld_h + n, gelu_of_output<OUT_BF16>(y));
     if (debug_acc) debug_acc[row * N + n] = acc[i];
   }
 }
@@ -260,12 +277,8 @@ __device__ __forceinline__ void epi_group(uint8_t* row, int swz, const float* ws
         if (c < hchunks) {
           uint32_t h[4];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162*>(&w[q]);
-            const __nv_bfloat162 g2 =
-                __floats2bfloat162_rn(gelu(__bfloat162float(b2.x)), gelu(__bfloat162float(b2.y)));
-            h[q] = *reinterpret_cast<const uint32_t*>(&g2);
-          }
+          for (int q = 0; q < 4; ++q)  // two table entries per word of stored values
+            h[q] = (uint32_t)g_gelu_bf16[w[q] & 0xFFFFu] | ((uint32_t)g_gelu_bf16[w[q] >> 16] << 16);
           *reinterpret_cast<uint4*>(hrow + 16 * c) = make_uint4(h[0], h[1], h[2], h[3]);
         }
       }
@@ -864,6 +877,11 @@ int launch_slice_gemm(const SliceParams& p, int out_bf16, int num_sms, void* str
   const int64_t grid = items < 4LL * num_sms ? items : 4LL * num_sms;
   if (out_bf16) slice_gemm_kernel<true><<<(unsigned)grid, 256, 0, (cudaStream_t)stream>>>(p);
   else slice_gemm_kernel<false><<<(unsigned)grid, 256, 0, (cudaStream_t)stream>>>(p);
+  return (int)cudaGetLastError();
+}
+
+int launch_gelu_table(void* stream) {
+  gelu_table_kernel<<<256, 256, 0, (cudaStream_t)stream>>>();
   return (int)cudaGetLastError();
 }
 

@@ -431,6 +431,44 @@ int do_gemm_sparse(const dstar_tile_cfg* c, int64_t R, int64_t K, const int8_t* 
   return DSTAR_OK;
 }
 
+// The bf16 GELU table of the slice GEMM is filled once per CUDA context (a
+// device reset or a new context loads the module again), before the first
+// GEMM that reads it, on that GEMM's stream.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+std::mutex g_gelu_mu;
+unsigned long long g_gelu_ctx[64] = {};
+int g_gelu_n = 0, g_gelu_next = 0;
+
+int ensure_gelu_table(void* stream) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+    return fail(DSTAR_ERR_CUDA, "cannot identify the current CUDA context");
+  std::lock_guard<std::mutex> lk(g_gelu_mu);
+  for (int i = 0; i < g_gelu_n; ++i)
+    if (g_gelu_ctx[i] == id) return DSTAR_OK;
+  const int e = launch_gelu_table(stream);
+  if (e) return cuda_fail(e, "GELU table launch");
+  g_gelu_ctx[g_gelu_next] = id;
+  g_gelu_next = (g_gelu_next + 1) % 64;
+  if (g_gelu_n < 64) ++g_gelu_n;
+  return DSTAR_OK;
+}
+
 std::mutex g_attr_mu;
 struct AttrEntry {
   int dev;
@@ -645,6 +683,7 @@ int dstar_fmdq_ffn_gelu(const dstar_mat* x_t, dstar_mat* x_prev, dstar_mat* y1_p
   DevInfo dev;
   if ((r = device_info(&dev)) != DSTAR_OK) return r;
   // layer 1, its epilogue also writing H_t = GELU(Y1_t)
+  if (h_t->dtype == DSTAR_BF16 && (r = ensure_gelu_table(stream)) != DSTAR_OK) return r;
   if ((r = do_quantize(x_t, x_prev, lb, cfg1, M, K1, dev, stream, w1, y1_prev)) != DSTAR_OK) return r;
   if ((r = do_gemm(w1, w1_scale, y1_prev, lb, cfg1, y1_prev, M, K1, N1, dev, stream, h_t)) != DSTAR_OK) return r;
   // layer 2 on the differential H_t - H_{t-1}

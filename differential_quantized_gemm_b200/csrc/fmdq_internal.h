@@ -157,6 +157,8 @@ int launch_quant_cols_t(const void* v, int64_t ld, int64_t heads, int64_t S, int
                         float* scale, void* stream);
 int launch_masked_softmax(const float* sc, float* pr, int64_t rows, int64_t S, const BlockMask& mk, void* stream);
 int launch_selftest_wait(uint32_t* status, uint32_t spin_limit, void* stream);
+// Fill the bf16 GELU table of the slice GEMM's activation output (enqueued on stream).
+int launch_gelu_table(void* stream);
 size_t quantize_smem_bytes(int64_t Kc);  // shared memory of a CTA owning Kc channels
 // Raise a kernel's dynamic shared-memory limit once per device (returns a
 // cudaError_t as int); later calls only look up the cache, so launches stay

@@ -201,8 +201,11 @@ DSTAR_API int dstar_fmdq_linear(const dstar_mat* x_t, dstar_mat* x_prev, dstar_m
  *                 cfg1 has DSTAR_FLAG_NO_XPREV_REFRESH)
  *   y1_prev       [M x N1] F32/BF16: layer 1's cache, updated in place to Y1_t
  *   w1 [N1 x K1] I8, w1_scale [N1]
- *   h_t           [M x N1], y1_prev's dtype: receives H_t (GELU of the stored
- *                 Y1_t value, 0.5 y erfc(-y / sqrt 2) in fp32, rounded to the dtype)
+ *   h_t           [M x N1], y1_prev's dtype: receives H_t = GELU of the stored
+ *                 Y1_t value, 0.5 y erfc(-y / sqrt 2): for bf16 from a table of
+ *                 every bf16 value (fp64, rounded to fp32 then bf16), filled
+ *                 once per CUDA context by the first call (make that call
+ *                 outside stream capture); for fp32 in fp32 with erfcf
  *   h_prev        [M x N1]: H_{t-1}; refreshed to H_t unless cfg2 has
  *                 DSTAR_FLAG_NO_XPREV_REFRESH (then the caller swaps h_t, h_prev)
  *   y2_prev       [M x N2] F32/BF16: layer 2's cache, updated in place to Y2_t

@@ -5,8 +5,9 @@ over consecutive steps with every cache carried on both sides:
 - layer 1 (codes, widths, FPoT, g_ref, encoded stream, int64 accumulators)
   bit-exact, Y1_t within the tolerance;
 - H_t = GELU(Y1_t) within one bf16 ulp of the oracle's fp64 GELU everywhere
-  and equal to it almost everywhere (CUDA's erfcf and the fp64 erfc round to
-  the same bf16 value except next to a rounding boundary);
+  and equal to it almost everywhere (the library's table is filled in fp64
+  with CUDA's erfc, the oracle's with the C library's: they round to the same
+  bf16 value except next to a rounding boundary);
 - layer 2: the GPU's and the oracle's inputs differ wherever their H differ,
   so its integer outputs are compared on every sub-channel (and every tile)
   whose inputs agree bit for bit, Y2_t within the tolerance everywhere.
@@ -102,7 +103,7 @@ def _chain(cfg, M, steps):
         hg = _f32(h_t)
         ulp = np.abs(_ordered(hg) - _ordered(h)) >> 16
         assert ulp.max() <= 1, ulp.max()
-        assert (hg == h).mean() > 0.999, (hg == h).mean()
+        assert (hg == h).mean() > 0.99999, (hg == h).mean()
         # H_{t-1} was refreshed to the GPU's H_t
         assert torch.equal(d["h_prev"], h_t)
         # layer 2: sub-channels whose 16 inputs (H_t and H_{t-1}) agree
