@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -243,11 +244,28 @@ int do_quantize(const dstar_mat* x_t, dstar_mat* x_prev, int lb, const dstar_til
 }
 
 // Output tile width: the one with the least wave-quantised work (ties -> 256).
+// Output tile width from a model of the mainloop: a 128-deep K chunk costs
+// the larger of its MMA cycles (BN / 2 at 8192 int8 MAC per clock) and its
+// operand bytes (128 x 128 + BN x 128) over the L2 -> shared-memory rate
+// (about 74 B per clock per SM with every SM loading); the busiest SM's tile
+// count times that cost decides.  256-wide tiles have fewer pipeline stages,
+// so they are taken only when the model gives them a clear (> 10 %) lead
+// (measured: PixArt QKV 53 -> 47 us with 256; the 16384 x 4608 -> 1152
+// down-projection, a 6 % model lead, ran 10 % slower).
+#ifndef FMDQ_BN_L2_MODEL
+#define FMDQ_BN_L2_MODEL 1
+#endif
 int choose_bn(int64_t M, int64_t N, int sms) {
   const int64_t tm = (M + kBlockM - 1) / kBlockM;
   const int64_t t256 = tm * ((N + 255) / 256), t128 = tm * ((N + 127) / 128);
-  const int64_t c256 = (t256 + sms - 1) / sms * 256, c128 = (t128 + sms - 1) / sms * 128;
-  return c128 < c256 ? 128 : 256;
+  if (!FMDQ_BN_L2_MODEL) {
+    const int64_t c256 = (t256 + sms - 1) / sms * 256, c128 = (t128 + sms - 1) / sms * 128;
+    return c128 < c256 ? 128 : 256;
+  }
+  auto chunk = [](int64_t bn) { return std::max<double>(bn / 2.0, (128.0 * 128 + bn * 128.0) / 74.0); };
+  const double c256 = (double)((t256 + sms - 1) / sms) * chunk(256);
+  const double c128 = (double)((t128 + sms - 1) / sms) * chunk(128);
+  return c256 < 0.9 * c128 ? 256 : 128;
 }
 
 int do_gemm(const dstar_mat* w_q, const float* w_scale, dstar_mat* y_prev, int lb, const dstar_tile_cfg* c,
