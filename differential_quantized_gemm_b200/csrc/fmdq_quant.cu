@@ -745,24 +745,32 @@ __global__ void __launch_bounds__(kQThreads, FMDQ_Q_MIN_BLOCKS) quantize_kernel(
 // above (the same stage functions, with one CTA per tile); the buffers pass
 // between the groups through mbarriers (full: group 1 -> 2, empty: 2 -> 1)
 // whose waits are bounded.
-constexpr int kPGroup = 256;  // threads of each group
-constexpr int kPGroupWarps = kPGroup / 32;
-constexpr int kPThreads = 2 * kPGroup;
+// Warps of each group (compile-time; 16 warps of 128 registers fill an SM).
+#ifndef FMDQ_P_G1_WARPS
+#define FMDQ_P_G1_WARPS 8
+#endif
+#ifndef FMDQ_P_G2_WARPS
+#define FMDQ_P_G2_WARPS 8
+#endif
+constexpr int kPG1Warps = FMDQ_P_G1_WARPS, kPG2Warps = FMDQ_P_G2_WARPS;
+constexpr int kPG1 = 32 * kPG1Warps, kPG2 = 32 * kPG2Warps;  // threads of each group
+constexpr int kPThreads = kPG1 + kPG2;
 constexpr int kBarG1 = 1, kBarG2 = 2;  // named barriers of the groups (0 is __syncthreads)
 
 struct PSmem {
   uint64_t full[2], empty[2];
   int abort;
-  int red[4][kPGroupWarps];
+  int red[4][kPG1Warps];
   int xv[2][4];  // per buffer: finest FPoT, coarsest FPoT, min(FPoT + one-plane room), min(FPoT + two-plane room)
   uint32_t mask[kMaxMaskWords];
-  int warp_cnt[kPGroupWarps][kTagWin];
+  int warp_cnt[kPG2Warps][kTagWin];
   int base[kTagWin];
-  int wbase[kPGroupWarps][kTagWin];
+  int wbase[kPG2Warps][kTagWin];
 };
 
+template <int NT>
 __device__ __forceinline__ void group_sync(int id) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "n"(kPGroup) : "memory");
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "n"(NT) : "memory");
 }
 
 template <typename TIn, bool DYN>
@@ -772,8 +780,8 @@ __global__ void __launch_bounds__(kPThreads, 1) quantize_persistent_kernel(const
   const int Kc = (int)K;
   const int64_t T = p.M / kTile;
   const int tid = threadIdx.x, lane = tid & 31;
-  const bool g1 = tid < kPGroup;
-  const int gt = g1 ? tid : tid - kPGroup;  // thread index within the group
+  const bool g1 = tid < kPG1;
+  const int gt = g1 ? tid : tid - kPG1;  // thread index within the group
   const int gw = gt >> 5;                   // warp index within the group
   // buffer b: codes at 16 K b, FPoT at 32 K + 2 K b, widths right after the FPoTs
   int8_t* const s_base = reinterpret_cast<int8_t*>(smem);
@@ -785,7 +793,7 @@ __global__ void __launch_bounds__(kPThreads, 1) quantize_persistent_kernel(const
   volatile int* abort_flag = &S.abort;
 
   if (tid == 0) {
-    for (int b = 0; b < 2; ++b) mbar_init(&S.full[b], kPGroup), mbar_init(&S.empty[b], kPGroup);
+    for (int b = 0; b < 2; ++b) mbar_init(&S.full[b], kPG1), mbar_init(&S.empty[b], kPG2);
     S.abort = 0;
     fence_barrier_init();
   }
@@ -809,17 +817,17 @@ __global__ void __launch_bounds__(kPThreads, 1) quantize_persistent_kernel(const
       if (gt == 0 && i >= 2 && !wait_parity(&S.empty[b], ((i >> 1) - 1) & 1, abort_flag, p.status, kWaitLimitNs))
         *abort_flag = 1;
       __syncwarp();
-      group_sync(kBarG1);  // also: every warp is done with the previous tile's reduction
+      group_sync<kPG1>(kBarG1);  // also: every warp is done with the previous tile's reduction
       if (*abort_flag) break;
       // phase 1; the loads of the thread's first pair of the next tile are
       // issued while its last pair of this tile is processed
       P1Red r{-1000, 1000, 1000, 1000, 0};
-      for (int pr = gt; pr < npairs; pr += kPGroup) {
+      for (int pr = gt; pr < npairs; pr += kPG1) {
         Raw rt[kTile], rp[kTile];
         if constexpr (kAhead) {
 #pragma unroll
           for (int j = 0; j < kTile; ++j) rt[j] = nt[j], rp[j] = np[j];
-          if (pr + kPGroup < npairs) load_pair<TIn>(p, t * kTile, 2 * (pr + kPGroup), nt, np);
+          if (pr + kPG1 < npairs) load_pair<TIn>(p, t * kTile, 2 * (pr + kPG1), nt, np);
           else if (i + 1 < ntiles) load_pair<TIn>(p, (t + gridDim.x) * kTile, 2 * gt, nt, np);
         } else {
           load_pair<TIn>(p, t * kTile, 2 * pr, rt, rp);
@@ -832,10 +840,10 @@ __global__ void __launch_bounds__(kPThreads, 1) quantize_persistent_kernel(const
         if (r.flags)
           set_status(p.status, (r.flags & 1 ? DSTAR_STATUS_NONFINITE : 0u) | (r.flags & 2 ? DSTAR_STATUS_RANGE : 0u));
       }
-      group_sync(kBarG1);
+      group_sync<kPG1>(kBarG1);
       if (gt < 4) {
         int v = S.red[gt][0];
-        for (int w = 1; w < kPGroupWarps; ++w) v = gt == 0 ? max(v, S.red[gt][w]) : min(v, S.red[gt][w]);
+        for (int w = 1; w < kPG1Warps; ++w) v = gt == 0 ? max(v, S.red[gt][w]) : min(v, S.red[gt][w]);
         S.xv[b][gt] = v;
       }
       mbar_arrive(&S.full[b]);  // every thread after its own writes of the tile
@@ -848,33 +856,33 @@ __global__ void __launch_bounds__(kPThreads, 1) quantize_persistent_kernel(const
   } else {
     // ------------------------------------- group 2: phases 2a and 2b
     const int nchunks = Kc / 32;
-    const int ch_lo = gw * nchunks / kPGroupWarps, ch_hi = (gw + 1) * nchunks / kPGroupWarps;
+    const int ch_lo = gw * nchunks / kPG2Warps, ch_hi = (gw + 1) * nchunks / kPG2Warps;
     for (int i = 0; i < ntiles; ++i) {
       const int b = i & 1;
       const int64_t t = blockIdx.x + (int64_t)i * gridDim.x;
       if (gt == 0 && !wait_parity(&S.full[b], (i >> 1) & 1, abort_flag, p.status, kWaitLimitNs)) *abort_flag = 1;
       __syncwarp();
-      group_sync(kBarG2);  // also: every warp is done with the previous tile
+      group_sync<kPG2>(kBarG2);  // also: every warp is done with the previous tile
       if (*abort_flag) break;
       const int g = S.xv[b][0], gmin = S.xv[b][1], A1 = S.xv[b][2], A2 = S.xv[b][3];
       const int planes = g <= A1 ? 1 : g <= A2 ? 2 : 3;
       if (gt < kMaxMaskWords) S.mask[gt] = 0;
-      group_sync(kBarG2);
+      group_sync<kPG2>(kBarG2);
       const int64_t row0 = t * kTile;
-      phase2_planes<kPGroup>(p, row0, 0, Kc, gt, g, planes, s_code(b), s_fpot(b), S.mask);
+      phase2_planes<kPG2>(p, row0, 0, Kc, gt, g, planes, s_code(b), s_fpot(b), S.mask);
       const int tlo = gmin - 6;
       uint2* rec = p.records + t * p.record_cap;
       int total = 0;  // records of lower windows (kept by warp 0)
       for (int tw = tlo; tw <= g; tw += kTagWin) {
-        if (tw != tlo) group_sync(kBarG2);  // every warp is done with the previous window
+        if (tw != tlo) group_sync<kPG2>(kBarG2);  // every warp is done with the previous window
         const int cnt = count_window(tw, ch_lo, ch_hi, lane, s_fpot(b), s_bits(b), s_tab);
         if (lane < kTagWin) S.warp_cnt[gw][lane] = cnt;
-        group_sync(kBarG2);  // counts written; every plane of the tile written (mask complete)
+        group_sync<kPG2>(kBarG2);  // counts written; every plane of the tile written (mask complete)
         if (tw == tlo && gt < p.mask_words) p.mask1[t * p.mask_words + gt] = planes == 2 ? S.mask[gt] : 0u;
         if (gw == 0) {
           int all = 0;
           if (lane < kTagWin)
-            for (int w = 0; w < kPGroupWarps; ++w) all += S.warp_cnt[w][lane];
+            for (int w = 0; w < kPG2Warps; ++w) all += S.warp_cnt[w][lane];
           int incl = all;
 #pragma unroll
           for (int o = 1; o < 32; o <<= 1) {
@@ -884,7 +892,7 @@ __global__ void __launch_bounds__(kPThreads, 1) quantize_persistent_kernel(const
           if (lane < kTagWin) S.base[lane] = total + incl - all;
           total += __shfl_sync(kFull, incl, 31);
         }
-        group_sync(kBarG2);
+        group_sync<kPG2>(kBarG2);
         if (lane < kTagWin) {
           int o = S.base[lane];
           for (int w = 0; w < gw; ++w) o += S.warp_cnt[w][lane];
