@@ -22,6 +22,16 @@ F32, BF16, I8 = 0, 1, 2
 FLAG_NO_XPREV_REFRESH = 1
 FLAG_SLICE_PATH = 2
 FLAG_DYNAMIC_BASE = 4
+# slice-GEMM tile forms (a tuning override in flags bits 8..10; 0 = the library's choice)
+TILE_128x128, TILE_128x256, TILE_PAIR_256x256, TILE_PAIR_256x128 = 1, 2, 3, 4
+TILE_SHIFT = 8
+
+
+def tile_flag(form: int) -> int:
+    """The flags bits that make a call use slice-GEMM tile form `form`."""
+    return int(form) << TILE_SHIFT
+
+
 TILE = 16
 POT_MAX = 32
 K_MAX = 8192
@@ -31,7 +41,7 @@ EXPORTED = [
     "dstar_fmdq_workspace_layout", "dstar_fmdq_workspace_init", "dstar_fmdq_linear", "dstar_fmdq_quantize",
     "dstar_fmdq_slice_gemm", "dstar_fmdq_status", "dstar_fmdq_selftest_wait", "dstar_fmdq_linear_noalloc",
     "dstar_fmdq_ffn_gelu", "dstar_sar_workspace_size", "dstar_sar_workspace_layout", "dstar_sar_workspace_init",
-    "dstar_sar_attention", "dstar_sar_status",
+    "dstar_sar_attention", "dstar_sar_status", "dstar_fmdq_gemm_tile",
 ]
 SAR_BLOCK = 128
 NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -102,6 +112,8 @@ def lib():
         L.dstar_sar_workspace_init.argtypes = [ctypes.POINTER(SarCfg), P]
         L.dstar_sar_attention.argtypes = [MP, MP, MP, ctypes.POINTER(SarCfg), ctypes.c_int, MP, P]
         L.dstar_sar_status.argtypes = [ctypes.POINTER(SarCfg), P, ctypes.POINTER(ctypes.c_uint32)]
+        L.dstar_fmdq_gemm_tile.argtypes = [I64, I64, I64, ctypes.c_int, ctypes.POINTER(ctypes.c_int),
+                                           ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
         for name in EXPORTED[3:]:
             getattr(L, name).restype = ctypes.c_int
         _lib = L
@@ -321,6 +333,14 @@ def status(ws: Workspace, stream=None) -> int:
     s = ctypes.c_uint32()
     _check(lib().dstar_fmdq_status(ctypes.c_void_p(ws.ptr), _stream(stream), ctypes.byref(s)))
     return s.value
+
+
+def gemm_tile(M: int, N: int, K: int, out_bf16: bool) -> tuple[int, int, bool]:
+    """(rows, columns, CTA pair) of the slice GEMM's output tiles for an M x N output with K channels."""
+    bm, bn, pair = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    _check(lib().dstar_fmdq_gemm_tile(ctypes.c_int64(M), ctypes.c_int64(N), ctypes.c_int64(K), int(bool(out_bf16)),
+                                      ctypes.byref(bm), ctypes.byref(bn), ctypes.byref(pair)))
+    return bm.value, bn.value, bool(pair.value)
 
 
 def selftest_wait(ws: Workspace, limit_us: int, stream=None):

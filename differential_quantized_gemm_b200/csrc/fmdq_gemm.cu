@@ -43,13 +43,23 @@ constexpr int kGThreads = 64 + 32 * kEpiWarps;     // producer warp, MMA warp, e
 constexpr int kA0Bytes = kBlockM * kChunkK;        // 16 KB
 constexpr int kMaxTileSlots = 32;                  // tiles per CTA whose block info is precomputed
 constexpr int kEpiBarrier = 1;                     // named barrier of the epilogue warps
-
-template <int BN, bool OUT_BF16>
+// PAIR: a cluster of two CTAs computes a 256 x BN tile with cta_group::2
+// MMAs, each CTA holding its 128 rows of A and half of the BN rows of W, so
+// every weight byte brought from L2 feeds twice the work without doubling one
+// SM's operand stages.
+// The mainloop is bound by the operand bytes in flight (loaded L2 latency
+// times rate), so every form takes as many stages as shared memory holds
+// beside the epilogue's y boxes: 6 x 32 KB (bf16 outputs), 5 x 32 KB (fp32)
+// and, in a pair, 8 x 24 KB (bf16) or 6 x 24 KB (fp32) fill the 227 KB of a
+// CTA; 128 x 256 tiles keep 3 x 48 KB beside their 64 KB of y boxes (4 x 32 KB
+// in a pair).
+template <int BN, bool OUT_BF16, bool PAIR = false>
 struct GemmCfg {
-  static constexpr int kStages = BN == 256 ? 3 : (OUT_BF16 ? 5 : 4);
-  static constexpr int kWBytes = BN * kChunkK;
+  static constexpr int kStages = PAIR ? (BN == 256 ? 4 : (OUT_BF16 ? 8 : 6)) : (BN == 256 ? 3 : (OUT_BF16 ? 6 : 5));
+  static constexpr int kWBytes = (PAIR ? BN / 2 : BN) * kChunkK;  // a CTA of a pair holds half of W's rows
   static constexpr int kStageBytes = kA0Bytes + kWBytes;
-  static constexpr int kSlots = 512 / BN;
+  static constexpr int kSlots = 512 / BN;                            // TMEM accumulator slots of BN columns
+  static_assert(kSlots >= 2, "a two-plane tile takes two accumulator slots");
   static constexpr int kHalfGroups = BN / 64;                        // 32-column groups per epilogue warp
   static constexpr int kOutBytes = OUT_BF16 ? 2 : 4;
   static constexpr int kBoxBytes = 32 * 32 * kOutBytes;              // one 32 x 32 tile of Y
@@ -65,6 +75,7 @@ struct GemmCfg {
   static constexpr int kOffStages = (kSmallBytes + 1023) & ~1023;
   static constexpr int kOffY = kOffStages + kStages * kStageBytes;
   static constexpr int kBytes = kOffY + kEpiWarps * kYWarpBytes + 1024;  // + base alignment slack
+  static_assert(kBytes <= 227 * 1024, "shared memory of one CTA");
 };
 
 struct BlockInfo {
@@ -73,15 +84,16 @@ struct BlockInfo {
   uint32_t mask[2];
 };
 
-// What the quantizer decided for a 128-row block (any thread, from global memory).
-__device__ __forceinline__ BlockInfo block_info_global(const GemmParams& p, int rb) {
+// What the quantizer decided for the token tiles [t0, t0 + n) of an output
+// tile's rows (any thread, from global memory).
+__device__ __forceinline__ BlockInfo block_info_global(const GemmParams& p, int t0, int n) {
   BlockInfo bi;
   bi.mask[0] = bi.mask[1] = 0;
   bi.any_slice = 0;
   const int T = (int)(p.M / kTile);
   int np = 0;
   bool any = false;
-  for (int t = rb * 8; t < min(rb * 8 + 8, T); ++t) {
+  for (int t = t0; t < min(t0 + n, T); ++t) {
     const int pl = p.planes[t];
     if (pl <= 2) {
       any = true;
@@ -296,7 +308,10 @@ __device__ __forceinline__ void epi_group(uint8_t* row, int swz, const float* ws
 
 }  // namespace
 
-size_t gemm_smem_bytes(int bn) { return bn == 256 ? GemmCfg<256, true>::kBytes : GemmCfg<128, true>::kBytes; }
+size_t gemm_smem_bytes(int bn, int pair) {
+  if (pair) return bn == 256 ? GemmCfg<256, true, true>::kBytes : GemmCfg<128, true, true>::kBytes;
+  return bn == 256 ? GemmCfg<256, true>::kBytes : GemmCfg<128, true>::kBytes;
+}
 
 // The batched, block-sparse form takes a GemmSparse argument; the plain one
 // an empty struct.
@@ -310,13 +325,22 @@ struct SparseArg<true> {
   using T = GemmSparse;
 };
 
-template <int BN, bool OUT_BF16, bool GELU, bool SPARSE>
+template <int BN, bool OUT_BF16, bool GELU, bool SPARSE, bool PAIR>
 __global__ void __launch_bounds__(kGThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CUtensorMap tm_a1,
                 const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_yp,
                 const __grid_constant__ CUtensorMap tm_yo, const GemmParams p,
                 const __grid_constant__ typename SparseArg<SPARSE>::T sp) {
-  using C = GemmCfg<BN, OUT_BF16>;
+  using C = GemmCfg<BN, OUT_BF16, PAIR>;
+  static_assert(!SPARSE || !PAIR, "the batched form uses 128-row tiles");
+  constexpr int BM = kBlockM * (PAIR ? 2 : 1);  // rows of an output tile
+  constexpr int kTilesPerBlock = BM / kTile;
+  // With PAIR, CTA crank of cluster `unit` owns rows [crank * 128, +128) of
+  // each tile; otherwise every CTA is its own unit.
+  const uint32_t crank = PAIR ? cluster_ctarank() : 0u;
+  const bool leader = crank == 0;
+  const int unit = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int units = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
   using TOut = typename OutT<OUT_BF16>::T;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -331,7 +355,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
   float* s_ws = reinterpret_cast<float*>(smem + C::kOffWs);
-  int4* s_info = reinterpret_cast<int4*>(smem + C::kOffInfo);  // {nplanes, any_slice, mask0, mask1}
+  int4* s_info = reinterpret_cast<int4*>(smem + C::kOffInfo);  // {nplanes, any_slice, mask0, mask1} per tile
   uint8_t* stages = smem + C::kOffStages;
   uint8_t* ysmem = smem + C::kOffY;
 
@@ -363,12 +387,15 @@ __global__ void __launch_bounds__(kGThreads, 1)
     if constexpr (SPARSE) return ((sp.chunk_keep[rb % rb_per_head] >> c) & 1ull) != 0;
     else return true;
   };
-  const int my_tiles = num_tiles > (int)blockIdx.x ? (num_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  const int my_tiles = num_tiles > unit ? (num_tiles - 1 - unit) / units + 1 : 0;
   const int T = (int)(p.M / kTile);
+  // first row of this CTA's rows of row block rb
+  auto row_of = [&](int rb) { return rb * BM + (int)crank * kBlockM; };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kStages; ++i) mbar_init(&full[i], 1), mbar_init(&empty[i], 1);
-    for (int i = 0; i < C::kSlots; ++i) mbar_init(&tm_full[i], 1), mbar_init(&tm_empty[i], kEpiWarps);
+    // with PAIR the even CTA's tm_empty counts both CTAs' epilogue warps
+    for (int i = 0; i < C::kSlots; ++i) mbar_init(&tm_full[i], 1), mbar_init(&tm_empty[i], (PAIR ? 2 : 1) * kEpiWarps);
     for (int i = 0; i < kEpiWarps; ++i) mbar_init(&ybar[i], 1);
     mbar_init(drain, 1);
     mbar_init(info_bar, 1);
@@ -383,11 +410,18 @@ __global__ void __launch_bounds__(kGThreads, 1)
   // set-up that does not touch memory written by the previous kernel
   for (int i = threadIdx.x; i < kMaxTileSlots; i += kGThreads) s_info[i] = make_int4(0, 0, 0, 0);
   if (warp == 1) {
-    tmem_alloc(s_tmem, 512);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(s_tmem, 512);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(s_tmem, 512);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  // with PAIR the peer's barriers and TMEM exist before either CTA signals the other
+  if constexpr (PAIR) cluster_sync();
+  else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
   pdl_launch_dependents();
@@ -401,7 +435,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
       bi.nplanes = (e.x == 2 && (e.z | e.w)) ? 2 : 1;
       return bi;
     }
-    return block_info_global(p, rb);
+    return block_info_global(p, rb * kTilesPerBlock, kTilesPerBlock);
   };
 
   if (warp == 0) {
@@ -409,16 +443,27 @@ __global__ void __launch_bounds__(kGThreads, 1)
     if (elect_one()) {
       uint32_t it = 0;
       bool ok = true;
+      // With PAIR both CTAs' loads complete on the even CTA's full barrier,
+      // which expects the bytes of both.
+      const uint32_t full_cl = PAIR ? cluster_smem_addr(full, 0) : 0u;
+      auto load = [&](void* dst, const CUtensorMap* m, int s, int x, int y) {
+        if constexpr (PAIR) tma_load_2d_pair(dst, m, full_cl + 8u * (uint32_t)s, x, y);
+        else tma_load_2d(dst, m, &full[s], x, y);
+      };
+      auto expect = [&](int s) {
+        if (leader) mbar_arrive_expect_tx(&full[s], (PAIR ? 2 : 1) * C::kStageBytes);
+      };
+      const int w_off = PAIR ? (int)crank * (BN / 2) : 0;  // this CTA's rows of the W tile
       // The weights do not depend on the previous kernel: the W tiles of the
       // first stages are requested before waiting for it.
       uint32_t pre = 0;
       if (my_tiles > 0) {
         int rb0, nb0;
-        coords((int)blockIdx.x, rb0, nb0);
+        coords(unit, rb0, nb0);
         for (int c = 0; c < p.num_chunks && pre < (uint32_t)C::kStages; ++c) {
           if (!keep0(rb0, c)) continue;
-          mbar_arrive_expect_tx(&full[pre], C::kStageBytes);
-          tma_load_2d(stages + pre * C::kStageBytes + kA0Bytes, &tm_w, &full[pre], c * kChunkK, w_row(rb0, nb0));
+          expect(pre);
+          load(stages + pre * C::kStageBytes + kA0Bytes, &tm_w, pre, c * kChunkK, w_row(rb0, nb0) + w_off);
           ++pre;
         }
       }
@@ -426,8 +471,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
       bool have_info = false;
       for (int slot = 0; slot < my_tiles && ok; ++slot) {
         int rb, nb;
-        coords((int)blockIdx.x + slot * (int)gridDim.x, rb, nb);
-        const int wr = w_row(rb, nb);
+        coords(unit + slot * units, rb, nb);
+        const int wr = w_row(rb, nb) + w_off;
         for (int pass = 0; pass < 2 && ok; ++pass) {
           BlockInfo bi{};
           if (pass == 1) {  // plane 1 only where the block needs it
@@ -443,7 +488,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
             const int s = it % C::kStages;
             uint8_t* a = stages + s * C::kStageBytes;
             if (it < pre) {  // the stage's W tile is already on its way
-              tma_load_2d(a, tm_a, &full[s], c * kChunkK, rb * kBlockM);
+              load(a, tm_a, s, c * kChunkK, row_of(rb));
               ++it;
               continue;
             }
@@ -451,28 +496,31 @@ __global__ void __launch_bounds__(kGThreads, 1)
               ok = false;
               break;
             }
-            mbar_arrive_expect_tx(&full[s], C::kStageBytes);
-            tma_load_2d(a, tm_a, &full[s], c * kChunkK, rb * kBlockM);
-            tma_load_2d(a + kA0Bytes, &tm_w, &full[s], c * kChunkK, wr);
+            expect(s);
+            load(a, tm_a, s, c * kChunkK, row_of(rb));
+            load(a + kA0Bytes, &tm_w, s, c * kChunkK, wr);
             ++it;
           }
         }
       }
       // drain: every stage filled must have landed before the block can exit
+      // (with PAIR the even CTA's barriers count both CTAs' loads, and the
+      // final cluster barrier holds the odd CTA until then)
       const uint32_t first = it > (uint32_t)C::kStages ? it - C::kStages : 0;
-      for (uint32_t j = first; j < it; ++j)
-        wait_parity(&full[j % C::kStages], (j / C::kStages) & 1, s_abort, p.status, kWaitLimitNs, true);
+      if (leader)
+        for (uint32_t j = first; j < it; ++j)
+          wait_parity(&full[j % C::kStages], (j / C::kStages) & 1, s_abort, p.status, kWaitLimitNs, true);
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
-    if (elect_one()) {
+    if (elect_one() && leader) {  // with PAIR the even CTA issues the pair's MMAs
       pdl_wait();  // block info beyond the shared-memory table is read from global memory
-      constexpr uint32_t idesc = idesc_i8(BN);
+      constexpr uint32_t idesc = idesc_i8(BN, PAIR ? 256 : 128);
       uint32_t it = 0, slot_it = 0;
       bool ok = true, issued = false, have_info = false;
       for (int slot = 0; slot < my_tiles && ok; ++slot) {
         int rb, nb_unused;
-        coords((int)blockIdx.x + slot * (int)gridDim.x, rb, nb_unused);
+        coords(unit + slot * units, rb, nb_unused);
         uint32_t acc0 = 0, acc1 = 0;
         int np = 1;
         for (int pass = 0; pass < 2 && ok; ++pass) {
@@ -505,22 +553,31 @@ __global__ void __launch_bounds__(kGThreads, 1)
             const uint64_t da = smem_desc_k_sw128(stages + s * C::kStageBytes);
             const uint64_t dw = smem_desc_k_sw128(stages + s * C::kStageBytes + kA0Bytes);
 #pragma unroll
-            for (int kk = 0; kk < kChunkK / 32; ++kk)
-              mma_i8(d, da + 2 * kk, dw + 2 * kk, idesc, (!first || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < kChunkK / 32; ++kk) {
+              if constexpr (PAIR) mma_i8_pair(d, da + 2 * kk, dw + 2 * kk, idesc, (!first || kk > 0) ? 1u : 0u);
+              else mma_i8(d, da + 2 * kk, dw + 2 * kk, idesc, (!first || kk > 0) ? 1u : 0u);
+            }
             first = false;
-            mma_commit(&empty[s]);
+            if constexpr (PAIR) mma_commit_pair_mc(&empty[s], 3);  // both CTAs may refill the stage
+            else mma_commit(&empty[s]);
             issued = true;
             ++it;
           }
         }
         if (!ok) break;
-        mma_commit(&tm_full[acc0]);
-        if (np == 2) mma_commit(&tm_full[acc1]);
+        if constexpr (PAIR) {  // both CTAs' epilogues read their halves of the slot
+          mma_commit_pair_mc(&tm_full[acc0], 3);
+          if (np == 2) mma_commit_pair_mc(&tm_full[acc1], 3);
+        } else {
+          mma_commit(&tm_full[acc0]);
+          if (np == 2) mma_commit(&tm_full[acc1]);
+        }
         slot_it += np;
       }
       // drain: all MMAs this thread issued complete before TMEM and SMEM go away
       if (issued) {
-        mma_commit(drain);
+        if constexpr (PAIR) mma_commit_pair(drain);
+        else mma_commit(drain);
         wait_parity(drain, 0, s_abort, p.status, kWaitLimitNs, true);
       }
     }
@@ -538,14 +595,16 @@ __global__ void __launch_bounds__(kGThreads, 1)
     auto sw = [](int r) { return OUT_BF16 ? ((r >> 1) & 3) : (r & 7); };
     auto tile_rb = [&](int s) {
       int rb, nb;
-      coords((int)blockIdx.x + s * (int)gridDim.x, rb, nb);
+      coords(unit + s * units, rb, nb);
       return rb;
     };
     auto tile_nb = [&](int s) {
       int rb, nb;
-      coords((int)blockIdx.x + s * (int)gridDim.x, rb, nb);
+      coords(unit + s * units, rb, nb);
       return nb;
     };
+    // the slot's tm_empty barrier: the even CTA's with PAIR
+    const uint32_t tm_empty_cl = PAIR ? cluster_smem_addr(tm_empty, 0) : 0u;
     // Everything a tile needs besides its accumulator is requested one tile
     // ahead: its y_prev boxes (each as soon as the previous tile's store has
     // read the box), its weight scales (shared memory, double-buffered) and
@@ -556,17 +615,18 @@ __global__ void __launch_bounds__(kGThreads, 1)
       if constexpr (SPARSE) off = (int64_t)(tile_rb(s) / rb_per_head) * p.N;
       return (etid < BN && n < p.N) ? p.w_scale[off + n] : 0.f;
     };
+    // this lane's row: plane count (3 beyond M) and g_ref
     auto row_planes = [&](int s, int& pl, int& gref) {
-      const int64_t row = (int64_t)tile_rb(s) * kBlockM + quarter * 32 + lane;
+      const int64_t row = (int64_t)row_of(tile_rb(s)) + quarter * 32 + lane;
       pl = 3, gref = 0;
       if (row < p.M) pl = p.planes[row / kTile], gref = p.g_ref[row / kTile];
     };
     // With SPARSE there is no cached output: Y_{t-1} = 0 is never read.
-    auto load_y_box = [&](int s, int box) {  // lane 0
+    auto load_y_box = [&](int s, int g) {  // lane 0
       if constexpr (SPARSE) return;
-      if (box == 0) mbar_arrive_expect_tx(&ybar[ew], C::kYWarpBytes);
-      tma_load_2d(ybuf + box * C::kBoxBytes, &tm_yp, &ybar[ew], tile_nb(s) * BN + half * (BN / 2) + box * 32,
-                  tile_rb(s) * kBlockM + quarter * 32);
+      if (g == 0) mbar_arrive_expect_tx(&ybar[ew], C::kYWarpBytes);
+      tma_load_2d(ybuf + g * C::kBoxBytes, &tm_yp, &ybar[ew], tile_nb(s) * BN + half * (BN / 2) + g * 32,
+                  row_of(tile_rb(s)) + quarter * 32);
     };
     uint32_t slot_it = 0;
     uint32_t y_issued = 0, y_seen = 0;  // batches of y_prev boxes requested (lane 0) / observed landed
@@ -583,10 +643,11 @@ __global__ void __launch_bounds__(kGThreads, 1)
       if (etid < BN) s_ws[etid] = weight_scale(0);
     }
     // block info of this CTA's first kMaxTileSlots tiles, loaded in parallel,
-    // then published to the producer and MMA threads
-    for (int i = etid; i < min(my_tiles, kMaxTileSlots) * 8; i += 32 * kEpiWarps) {
-      const int slot = i >> 3, sub = i & 7;
-      const int t = tile_rb(slot) * 8 + sub;
+    // then published to the producer and MMA threads (with PAIR both CTAs
+    // compute the same information for the tile's 256 rows)
+    for (int i = etid; i < min(my_tiles, kMaxTileSlots) * kTilesPerBlock; i += 32 * kEpiWarps) {
+      const int slot = i / kTilesPerBlock, sub = i % kTilesPerBlock;
+      const int t = tile_rb(slot) * kTilesPerBlock + sub;
       if (t < T) {
         const int pl = p.planes[t];
         int* e = reinterpret_cast<int*>(&s_info[slot]);
@@ -607,7 +668,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
       const BlockInfo bi = info(slot, rb);
       const int64_t n_base = (int64_t)nb * BN;
       const int64_t n_half = n_base + half * (BN / 2);
-      const int row0 = rb * kBlockM + quarter * 32;
+      const int row0 = row_of(rb) + quarter * 32;
       const float* ws_tile = s_ws + (slot & 1) * BN;
       float ws_next = 0.f;
       int pl_next = 3, gref_next = 0;
@@ -698,8 +759,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
             if (row_ok) {
               int hch;
               uint8_t* hr = h_row(g, hch);
-              epi_group<OUT_BF16, false, GELU, SPARSE>(my_row + g * C::kBoxBytes, swz, ws_h + g * 32, d, d, false, p2, beta,
-                                               hr, hch);
+              epi_group<OUT_BF16, false, GELU, SPARSE>(my_row + g * C::kBoxBytes, swz, ws_h + g * 32, d, d, false, p2,
+                                                       beta, hr, hch);
               if (p.debug_acc) debug_group(g, d, d, false);
             }
             store_group(g);
@@ -730,29 +791,35 @@ __global__ void __launch_bounds__(kGThreads, 1)
               if (row_ok) {
                 int hch;
                 uint8_t* hr = h_row(g, hch);
-                epi_group<OUT_BF16, true, GELU, SPARSE>(my_row + g * C::kBoxBytes, swz, ws_h + g * 32, d0, d1, wide_row, p2,
-                                                beta, hr, hch);
+                epi_group<OUT_BF16, true, GELU, SPARSE>(my_row + g * C::kBoxBytes, swz, ws_h + g * 32, d0, d1, wide_row,
+                                                        p2, beta, hr, hch);
                 if (p.debug_acc) debug_group(g, d0, d1, true);
               }
               store_group(g);
             }
           }
+          // the slot is free once this warp's TMEM reads are done (with PAIR
+          // the even CTA's barrier counts both CTAs' epilogue warps)
           tc_fence_before();
           __syncwarp();
           if (lane == 0)
-            for (int q = 0; q < bi.nplanes; ++q) mbar_arrive(&tm_empty[acc_slot[q]]);
+            for (int q = 0; q < bi.nplanes; ++q) {
+              if constexpr (PAIR) mbar_arrive_cluster(tm_empty_cl + 8u * acc_slot[q]);
+              else mbar_arrive(&tm_empty[acc_slot[q]]);
+            }
           slot_it += bi.nplanes;
         }
       }
 
-      // tiles of this row block whose operands need more than two planes:
-      // the slice stream, one output column per epilogue thread, after this
+      // this CTA's token tiles whose operands need more than two planes: the
+      // slice stream, one output column per epilogue thread, after this
       // tile's TMA stores have completed
       if (ok && bi.any_slice) {
         if (lane == 0) bulk_wait<0>();
         __syncwarp();
         epi_barrier();
-        for (int t = rb * 8; t < min(rb * 8 + 8, T); ++t) {
+        const int t0 = row_of(rb) / kTile;
+        for (int t = t0; t < min(t0 + kBlockM / kTile, T); ++t) {
           if (p.planes[t] <= 2) continue;
           for (int c = etid; c < BN; c += 32 * kEpiWarps) {
             const int64_t n = n_base + c;
@@ -782,11 +849,14 @@ __global__ void __launch_bounds__(kGThreads, 1)
   }
 
   tc_fence_before();
-  __syncthreads();
+  // with PAIR neither CTA leaves while the other's MMAs or loads may use its memory
+  if constexpr (PAIR) cluster_sync();
+  else __syncthreads();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, 512);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem_base, 512);
+    else tmem_dealloc(tmem_base, 512);
   }
 }
 
@@ -826,44 +896,58 @@ __global__ void selftest_wait_kernel(uint32_t* status, uint64_t limit_ns) {
   }
 }
 
-template <int BN, bool BF, bool GELU, bool SPARSE = false>
+template <int BN, bool BF, bool GELU, bool SPARSE = false, bool PAIR = false>
 static int launch_gemm_t(const GemmParams& p, const CUtensorMap* m, int num_sms, void* stream,
                          const typename SparseArg<SPARSE>::T& sp = {}) {
   int tiles = p.tiles_m * p.tiles_n;
   if constexpr (SPARSE)
     tiles = (int)sp.heads * (sp.n_listed > 0 ? sp.n_listed : (int)(sp.rows_per_head / kBlockM) * p.tiles_n);
-  const int grid = tiles < num_sms ? tiles : num_sms;
+  const int units = PAIR ? num_sms / 2 : num_sms;  // CTA pairs are clusters of two
+  const int grid = (tiles < units ? tiles : units) * (PAIR ? 2 : 1);
   if (grid == 0) return 0;
-  const int smem = GemmCfg<BN, BF>::kBytes;
-  const int e = ensure_max_smem((const void*)gemm_kernel<BN, BF, GELU, SPARSE>, smem);
+  const int smem = GemmCfg<BN, BF, PAIR>::kBytes;
+  const int e = ensure_max_smem((const void*)gemm_kernel<BN, BF, GELU, SPARSE, PAIR>, smem);
   if (e != 0) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid, 1, 1);
   cfg.blockDim = dim3(kGThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = (cudaStream_t)stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // overlap the launch with the quantizer
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = PAIR ? 2 : 1;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  const cudaError_t ce = cudaLaunchKernelEx(&cfg, gemm_kernel<BN, BF, GELU, SPARSE>, m[0], m[1], m[2], m[3], m[4], p, sp);
+  cfg.numAttrs = PAIR ? 2 : 1;
+  const cudaError_t ce =
+      cudaLaunchKernelEx(&cfg, gemm_kernel<BN, BF, GELU, SPARSE, PAIR>, m[0], m[1], m[2], m[3], m[4], p, sp);
   if (ce != cudaSuccess) return (int)ce;
   return (int)cudaGetLastError();
 }
 
 // maps: the A0, A1, W, y_prev and y_out tensor maps (CUtensorMap[5]).
 template <bool GELU>
-static int launch_gemm_g(const GemmParams& p, const CUtensorMap* m, int bn, int out_bf16, int num_sms, void* stream) {
-  if (out_bf16) return bn == 256 ? launch_gemm_t<256, true, GELU>(p, m, num_sms, stream)
-                                 : launch_gemm_t<128, true, GELU>(p, m, num_sms, stream);
-  return launch_gemm_t<128, false, GELU>(p, m, num_sms, stream);  // fp32 outputs use 128-column tiles
+static int launch_gemm_g(const GemmParams& p, const CUtensorMap* m, int bn, int pair, int out_bf16, int num_sms,
+                         void* stream) {
+  if (pair) {
+    if (!out_bf16) return launch_gemm_t<128, false, GELU, false, true>(p, m, num_sms, stream);
+    return bn == 256 ? launch_gemm_t<256, true, GELU, false, true>(p, m, num_sms, stream)
+                     : launch_gemm_t<128, true, GELU, false, true>(p, m, num_sms, stream);
+  }
+  if (out_bf16)
+    return bn == 256 ? launch_gemm_t<256, true, GELU>(p, m, num_sms, stream)
+                     : launch_gemm_t<128, true, GELU>(p, m, num_sms, stream);
+  return launch_gemm_t<128, false, GELU>(p, m, num_sms, stream);  // fp32 outputs: 128-column tiles
 }
 
-int launch_gemm(const GemmParams& p, const void* maps, int bn, int out_bf16, int num_sms, void* stream) {
+int launch_gemm(const GemmParams& p, const void* maps, int bn, int pair, int out_bf16, int num_sms, void* stream) {
   const CUtensorMap* m = static_cast<const CUtensorMap*>(maps);
-  return p.h_out ? launch_gemm_g<true>(p, m, bn, out_bf16, num_sms, stream)
-                 : launch_gemm_g<false>(p, m, bn, out_bf16, num_sms, stream);
+  if (!(bn == 128 || (bn == 256 && out_bf16))) return (int)cudaErrorInvalidValue;
+  return p.h_out ? launch_gemm_g<true>(p, m, bn, pair, out_bf16, num_sms, stream)
+                 : launch_gemm_g<false>(p, m, bn, pair, out_bf16, num_sms, stream);
 }
 
 int launch_gemm_sparse(const GemmParams& p, const GemmSparse& sp, const void* maps, int num_sms, void* stream) {

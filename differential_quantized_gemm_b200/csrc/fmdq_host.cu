@@ -164,8 +164,10 @@ int check_cfg(const dstar_tile_cfg* c, int64_t M, int64_t K) {
   if (c->force_bits != 0 && c->force_bits != 2 && c->force_bits != 4 && c->force_bits != 6 && c->force_bits != 8)
     return fail(DSTAR_ERR_INVALID_ARG, "force_bits must be 0, 2, 4, 6 or 8");
   if (c->thr0_log2 < -100 || c->thr0_log2 > 100) return fail(DSTAR_ERR_INVALID_ARG, "thr0_log2 out of [-100, 100]");
-  if (c->flags & ~(DSTAR_FLAG_NO_XPREV_REFRESH | DSTAR_FLAG_SLICE_PATH | DSTAR_FLAG_DYNAMIC_BASE))
+  if (c->flags & ~(DSTAR_FLAG_NO_XPREV_REFRESH | DSTAR_FLAG_SLICE_PATH | DSTAR_FLAG_DYNAMIC_BASE | DSTAR_FLAG_TILE_MASK))
     return fail(DSTAR_ERR_INVALID_ARG, "unknown flag bits 0x%x", c->flags);
+  if (((c->flags & DSTAR_FLAG_TILE_MASK) >> DSTAR_FLAG_TILE_SHIFT) > DSTAR_TILE_PAIR_256x128)
+    return fail(DSTAR_ERR_INVALID_ARG, "unknown tile form %u", (c->flags & DSTAR_FLAG_TILE_MASK) >> DSTAR_FLAG_TILE_SHIFT);
   const WsLayout L = ws_layout(M, K);
   if (!c->workspace) return fail(DSTAR_ERR_WORKSPACE, "workspace is NULL");
   if (reinterpret_cast<uintptr_t>(c->workspace) & 255u) return fail(DSTAR_ERR_WORKSPACE, "workspace must be 256-byte aligned");
@@ -243,29 +245,54 @@ int do_quantize(const dstar_mat* x_t, dstar_mat* x_prev, int lb, const dstar_til
   return DSTAR_OK;
 }
 
-// Output tile width: the one with the least wave-quantised work (ties -> 256).
-// Output tile width from a model of the mainloop: a 128-deep K chunk costs
-// the larger of its MMA cycles (BN / 2 at 8192 int8 MAC per clock) and its
-// operand bytes (128 x 128 + BN x 128) over the L2 -> shared-memory rate
-// (about 74 B per clock per SM with every SM loading); the busiest SM's tile
-// count times that cost decides.  256-wide tiles have fewer pipeline stages,
-// so they are taken only when the model gives them a clear (> 10 %) lead
-// (measured: PixArt QKV 53 -> 47 us with 256; the 16384 x 4608 -> 1152
-// down-projection, a 6 % model lead, ran 10 % slower).
-#ifndef FMDQ_BN_L2_MODEL
-#define FMDQ_BN_L2_MODEL 1
-#endif
-int choose_bn(int64_t M, int64_t N, int sms) {
-  const int64_t tm = (M + kBlockM - 1) / kBlockM;
-  const int64_t t256 = tm * ((N + 255) / 256), t128 = tm * ((N + 127) / 128);
-  if (!FMDQ_BN_L2_MODEL) {
-    const int64_t c256 = (t256 + sms - 1) / sms * 256, c128 = (t128 + sms - 1) / sms * 128;
-    return c128 < c256 ? 128 : 256;
+// Output tile shape from a model of one tile's period on an SM: the larger of
+// its mainloop and its epilogue (the two overlap through the TMEM slots).
+// Mainloop: the operand bytes in flight bound it -- with S stages of B bytes,
+// S - 1 are on their way while one is consumed, and the L2 -> shared-memory
+// rate an SM reaches grows with them (measured with every SM loading: about
+// 45 B per clock with 96 KB in flight, 60 with 160 KB, linear between, at
+// most 74) -- so a 128-deep K chunk costs the larger of its MMA cycles (the
+// SM's 128 rows x BN x 128 int8 MAC at 8192 per clock) and its bytes at that
+// rate.  Epilogue: about 1800 + 4800 cycles per 128 output columns of a
+// 128-row tile (y_prev in, Y_t out, TMEM reads), a fifth more in a pair whose
+// slots wait for both CTAs.  The busiest SM's (or pair's) tile count times
+// the period decides, ties to the earlier form.  Forms (stages): 128 x 128
+// (6 with bf16 outputs, 5 with fp32), 128 x 256 (3), and CTA pairs 256 x 256
+// (4; bf16 outputs) and 256 x 128 (8 with bf16 outputs, 6 with fp32), whose
+// SMs each hold 128 rows of A and half of W.
+struct TileShape {
+  int bm, bn, pair;
+};
+
+// form: a DSTAR_TILE_* value, 0 for the model's choice
+TileShape choose_tile(int64_t M, int64_t N, int64_t K, int sms, bool bf16, unsigned form = 0) {
+  switch (form) {
+    case DSTAR_TILE_128x128: return {128, 128, 0};
+    case DSTAR_TILE_128x256: return bf16 ? TileShape{128, 256, 0} : TileShape{128, 128, 0};
+    case DSTAR_TILE_PAIR_256x256: return bf16 ? TileShape{256, 256, 1} : TileShape{256, 128, 1};
+    case DSTAR_TILE_PAIR_256x128: return {256, 128, 1};
+    default: break;
   }
-  auto chunk = [](int64_t bn) { return std::max<double>(bn / 2.0, (128.0 * 128 + bn * 128.0) / 74.0); };
-  const double c256 = (double)((t256 + sms - 1) / sms) * chunk(256);
-  const double c128 = (double)((t128 + sms - 1) / sms) * chunk(128);
-  return c256 < 0.9 * c128 ? 256 : 128;
+  auto rate = [](double in_flight) { return std::min(74.0, 45.0 + (in_flight - 96.0 * 1024) / (64.0 * 1024) * 15.0); };
+  const double chunks = (double)((K + kChunkK - 1) / kChunkK);
+  auto cost = [&](int64_t bn, bool pair, int stages) {
+    const int64_t wrows = pair ? bn / 2 : bn;  // one SM's share of the W tile
+    const double bytes = (128 + wrows) * 128.0;
+    const double chunk = std::max<double>(128.0 * bn * 128.0 / 8192.0, bytes / rate((stages - 1) * bytes));
+    const double epi = (1800.0 + 4800.0 * bn / 128.0) * (pair ? 1.2 : 1.0);
+    const int64_t bm = pair ? 256 : 128, units = pair ? sms / 2 : sms;
+    const int64_t tiles = ((M + bm - 1) / bm) * ((N + bn - 1) / bn);
+    return (double)((tiles + units - 1) / units) * std::max(chunks * chunk, epi);
+  };
+  TileShape best{128, 128, 0};
+  double cb = cost(128, false, bf16 ? 6 : 5);
+  auto consider = [&](TileShape t, double c) {
+    if (c < cb) best = t, cb = c;
+  };
+  if (bf16) consider({128, 256, 0}, cost(256, false, 3));
+  if (bf16) consider({256, 256, 1}, cost(256, true, 4));
+  consider({256, 128, 1}, cost(128, true, bf16 ? 8 : 6));
+  return best;
 }
 
 int do_gemm(const dstar_mat* w_q, const float* w_scale, dstar_mat* y_prev, int lb, const dstar_tile_cfg* c,
@@ -281,12 +308,13 @@ int do_gemm(const dstar_mat* w_q, const float* w_scale, dstar_mat* y_prev, int l
   const uint32_t* dyn_base = dyn ? ws_ptr<const uint32_t>(c, L.dyn_base) : nullptr;
   if (dyn) lb = 0;
   if (!slice_all) {
-    const int bn = bf16 ? choose_bn(M, N, dev.sms) : 128;  // fp32 outputs use 128-column tiles
+    const TileShape ts = choose_tile(M, N, K, dev.sms, bf16, (c->flags & DSTAR_FLAG_TILE_MASK) >> DSTAR_FLAG_TILE_SHIFT);
+    const int bn = ts.bn;
     CUtensorMap maps[5];  // A0, A1, W, y_prev, y_out
     int r;
     if ((r = make_map_i8(&maps[0], ws_ptr<void>(c, L.plane0), M, K, K, kBlockM)) != DSTAR_OK) return r;
     if ((r = make_map_i8(&maps[1], ws_ptr<void>(c, L.plane1), M, K, K, kBlockM)) != DSTAR_OK) return r;
-    if ((r = make_map_i8(&maps[2], w_q->data, N, K, w_q->ld, bn)) != DSTAR_OK) return r;
+    if ((r = make_map_i8(&maps[2], w_q->data, N, K, w_q->ld, ts.pair ? bn / 2 : bn)) != DSTAR_OK) return r;
     if ((r = make_map_y(&maps[3], y_prev)) != DSTAR_OK) return r;
     if ((r = make_map_y(&maps[4], y_out)) != DSTAR_OK) return r;
     GemmParams g{};
@@ -308,7 +336,7 @@ int do_gemm(const dstar_mat* w_q, const float* w_scale, dstar_mat* y_prev, int l
     g.dyn_base = dyn_base;
     g.h_out = h_out ? h_out->data : nullptr;
     g.ld_h = h_out ? h_out->ld : 0;
-    g.tiles_m = (int)((M + kBlockM - 1) / kBlockM);
+    g.tiles_m = (int)((M + ts.bm - 1) / ts.bm);
     g.tiles_n = (int)((N + bn - 1) / bn);
     g.num_chunks = (int)((K + kChunkK - 1) / kChunkK);
     g.w_q = static_cast<const int8_t*>(w_q->data);
@@ -317,7 +345,7 @@ int do_gemm(const dstar_mat* w_q, const float* w_scale, dstar_mat* y_prev, int l
     g.record_cap = L.record_cap;
     g.count = ws_ptr<const int32_t>(c, L.count);
     g.bits = ws_ptr<const int8_t>(c, L.bits);
-    const int e = launch_gemm(g, maps, bn, bf16, dev.sms, stream);
+    const int e = launch_gemm(g, maps, bn, ts.pair, bf16, dev.sms, stream);
     if (e) return cuda_fail(e, "slice-GEMM launch");
     return DSTAR_OK;  // tiles needing the slice stream are handled inside the GEMM kernel
   }
@@ -846,6 +874,18 @@ int dstar_fmdq_status(void* workspace, void* stream, uint32_t* status) {
   if (e == cudaSuccess) e = cudaMemsetAsync(workspace, 0, sizeof(uint32_t), (cudaStream_t)stream);
   if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "reading the status word");
+  return ok();
+}
+
+int dstar_fmdq_gemm_tile(int64_t M, int64_t N, int64_t K, int out_bf16, int* bm, int* bn, int* pair) {
+  if (!bm || !bn) return fail(DSTAR_ERR_INVALID_ARG, "bm and bn must not be NULL");
+  if (M < 0 || N < 0 || K < 0) return fail(DSTAR_ERR_INVALID_ARG, "negative size");
+  DevInfo dev;
+  int r;
+  if ((r = device_info(&dev)) != DSTAR_OK) return r;
+  const TileShape ts = choose_tile(M, N, K, dev.sms, out_bf16 != 0);
+  *bm = ts.bm, *bn = ts.bn;
+  if (pair) *pair = ts.pair;
   return ok();
 }
 

@@ -144,8 +144,12 @@ int launch_quantize(const QuantParams& p, int in_bf16, int num_sms, void* stream
 int launch_base_min(const void* x_t, const void* x_prev, int64_t ld_xt, int64_t ld_xp, int64_t M, int64_t K,
                     int in_bf16, uint32_t* out, int num_sms, void* stream);
 int quantize_cluster_size(int64_t M, int64_t K, int num_sms);
+// Output tiles of 128 x bn in one CTA, or 256 x bn in a cluster of two CTAs
+// (pair); bn = 256 only with bf16 outputs.  tiles_m counts 128-row (256 with
+// pair) blocks.  The A0/A1 maps have 128-row boxes, the W map bn-row boxes
+// (bn / 2 with pair).
 int launch_gemm(const GemmParams& p, const void* maps /* CUtensorMap[5]: A0, A1, W, y_prev, y_out */, int bn,
-                int out_bf16, int num_sms, void* stream);
+                int pair, int out_bf16, int num_sms, void* stream);
 // The batched, block-sparse form (fp32 outputs, 128-column tiles).
 int launch_gemm_sparse(const GemmParams& p, const GemmSparse& sp, const void* maps, int num_sms, void* stream);
 int launch_slice_gemm(const SliceParams& p, int out_bf16, int num_sms, void* stream);
@@ -164,7 +168,7 @@ size_t quantize_smem_bytes(int64_t Kc);  // shared memory of a CTA owning Kc cha
 // cudaError_t as int); later calls only look up the cache, so launches stay
 // legal inside stream capture.
 int ensure_max_smem(const void* func, int bytes);
-size_t gemm_smem_bytes(int bn);
+size_t gemm_smem_bytes(int bn, int pair);
 
 // Record a one-line reason for dstar_fmdq_last_error() and return `code`.
 int report_error(int code, const char* msg);

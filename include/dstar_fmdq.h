@@ -87,6 +87,16 @@ extern "C" {
 #define DSTAR_FLAG_NO_XPREV_REFRESH 1u /* leave x_prev untouched (caller swaps buffers) */
 #define DSTAR_FLAG_SLICE_PATH 2u       /* compute every tile with the slice-stream kernel */
 #define DSTAR_FLAG_DYNAMIC_BASE 4u     /* FMDQ-DYN: base = min M_i of the call (see dstar_fmdq_linear) */
+/* Slice-GEMM output tile form, bits 8..10 of flags: 0 = the library's choice
+ * (dstar_fmdq_gemm_tile), else one form for the call -- a tuning override;
+ * results are the same bit for bit in every form.  The 256-column forms fall
+ * back to 128 columns with fp32 outputs. */
+#define DSTAR_FLAG_TILE_SHIFT 8
+#define DSTAR_FLAG_TILE_MASK (7u << DSTAR_FLAG_TILE_SHIFT)
+#define DSTAR_TILE_128x128 1u      /* one CTA */
+#define DSTAR_TILE_128x256 2u      /* one CTA; bf16 outputs */
+#define DSTAR_TILE_PAIR_256x256 3u /* a cluster of two CTAs (two SMs); bf16 outputs */
+#define DSTAR_TILE_PAIR_256x128 4u /* a cluster of two CTAs (two SMs) */
 
 /* limits of this implementation */
 #define DSTAR_TILE_TOKENS 16   /* tokens per sub-channel (the only supported tile) */
@@ -342,6 +352,19 @@ DSTAR_API int dstar_fmdq_quantize(const dstar_mat* x_t, dstar_mat* x_prev, float
  */
 DSTAR_API int dstar_fmdq_slice_gemm(const dstar_mat* w_q, const float* w_scale, dstar_mat* y_prev, float base_scale,
                           const dstar_tile_cfg* tile_cfg, dstar_mat* y_out, void* stream);
+
+/* The output tile shape the slice GEMM takes for an M x N output with K input
+ * channels on the current device (out_bf16: bf16 outputs): *bm x *bn, and
+ * *pair = 1 when a cluster of two CTAs (two SMs) computes each tile, 0 when
+ * one CTA does.
+ * Shapes: 128 x 128 and 128 x 256 in one CTA; 256 x 128 and 256 x 256 in a
+ * pair (the 256-column forms with bf16 outputs only).  It follows from the
+ * shape and the SM count alone (a model of the mainloop and the epilogue),
+ * not from the data.  Launches nothing.  `pair` may be NULL.
+ * Returns DSTAR_OK; DSTAR_ERR_INVALID_ARG for null bm/bn or negative sizes;
+ * DSTAR_ERR_UNSUPPORTED / DSTAR_ERR_CUDA when the current device cannot be
+ * queried or is not sm_100. */
+DSTAR_API int dstar_fmdq_gemm_tile(int64_t M, int64_t N, int64_t K, int out_bf16, int* bm, int* bn, int* pair);
 
 /* Synchronise `stream`, copy the workspace's sticky status word to *status
  * (DSTAR_STATUS_* bits, 0 when clean) and clear it. */
