@@ -41,7 +41,7 @@ EXPORTED = [
     "dstar_fmdq_workspace_layout", "dstar_fmdq_workspace_init", "dstar_fmdq_linear", "dstar_fmdq_quantize",
     "dstar_fmdq_slice_gemm", "dstar_fmdq_status", "dstar_fmdq_selftest_wait", "dstar_fmdq_linear_noalloc",
     "dstar_fmdq_ffn_gelu", "dstar_sar_workspace_size", "dstar_sar_workspace_layout", "dstar_sar_workspace_init",
-    "dstar_sar_attention", "dstar_sar_status", "dstar_fmdq_gemm_tile",
+    "dstar_sar_attention", "dstar_sar_status", "dstar_fmdq_gemm_tile", "dstar_fmdq_selftest_div",
 ]
 SAR_BLOCK = 128
 NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -112,6 +112,7 @@ def lib():
         L.dstar_sar_workspace_init.argtypes = [ctypes.POINTER(SarCfg), P]
         L.dstar_sar_attention.argtypes = [MP, MP, MP, ctypes.POINTER(SarCfg), ctypes.c_int, MP, P]
         L.dstar_sar_status.argtypes = [ctypes.POINTER(SarCfg), P, ctypes.POINTER(ctypes.c_uint32)]
+        L.dstar_fmdq_selftest_div.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P]
         L.dstar_fmdq_gemm_tile.argtypes = [I64, I64, I64, ctypes.c_int, ctypes.POINTER(ctypes.c_int),
                                            ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
         for name in EXPORTED[3:]:
@@ -341,6 +342,16 @@ def gemm_tile(M: int, N: int, K: int, out_bf16: bool) -> tuple[int, int, bool]:
     _check(lib().dstar_fmdq_gemm_tile(ctypes.c_int64(M), ctypes.c_int64(N), ctypes.c_int64(K), int(bool(out_bf16)),
                                       ctypes.byref(bm), ctypes.byref(bn), ctypes.byref(pair)))
     return bm.value, bn.value, bool(pair.value)
+
+
+def selftest_div(b: torch.Tensor, e_lo: int, e_hi: int, stream=None) -> int:
+    """dstar_fmdq_selftest_div: how many quotients a / b[i] of the dynamic-base
+    division differ from __fdiv_rn over all significands of a in [2^e_lo, 2^(e_hi+1))."""
+    assert b.is_cuda and b.dtype == torch.float32 and b.is_contiguous()
+    count = torch.zeros(1, dtype=torch.int64, device=b.device)
+    _check(lib().dstar_fmdq_selftest_div(ctypes.c_void_p(b.data_ptr()), int(b.numel()), int(e_lo), int(e_hi),
+                                         ctypes.c_void_p(count.data_ptr()), _stream(stream)))
+    return int(count.item())
 
 
 def selftest_wait(ws: Workspace, limit_us: int, stream=None):

@@ -889,6 +889,17 @@ int dstar_fmdq_gemm_tile(int64_t M, int64_t N, int64_t K, int out_bf16, int* bm,
   return ok();
 }
 
+int dstar_fmdq_selftest_div(const float* b, int n_b, int e_lo, int e_hi, unsigned long long* count, void* stream) {
+  if (!b || !count) return fail(DSTAR_ERR_INVALID_ARG, "b and count must not be NULL");
+  if (n_b < 0 || e_lo <= -127 || e_hi >= 128 || e_hi < e_lo) return fail(DSTAR_ERR_INVALID_ARG, "bad divisor count or exponents");
+  DevInfo dev;
+  int r;
+  if ((r = device_info(&dev)) != DSTAR_OK) return r;
+  const int e = launch_div_selftest(b, n_b, e_lo, e_hi, count, stream);
+  if (e) return cuda_fail(e, "division self-test launch");
+  return ok();
+}
+
 int dstar_fmdq_selftest_wait(void* workspace, uint32_t limit_us, void* stream) {
   if (!workspace) return fail(DSTAR_ERR_WORKSPACE, "workspace is NULL");
   DevInfo dev;

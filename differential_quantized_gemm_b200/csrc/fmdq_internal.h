@@ -144,6 +144,9 @@ int launch_quantize(const QuantParams& p, int in_bf16, int num_sms, void* stream
 int launch_base_min(const void* x_t, const void* x_prev, int64_t ld_xt, int64_t ld_xp, int64_t M, int64_t K,
                     int in_bf16, uint32_t* out, int num_sms, void* stream);
 int quantize_cluster_size(int64_t M, int64_t K, int num_sms);
+// Exhaustive comparison of the dynamic-base division with __fdiv_rn (see
+// dstar_fmdq_selftest_div).
+int launch_div_selftest(const float* b, int n_b, int e_lo, int e_hi, unsigned long long* count, void* stream);
 // Output tiles of 128 x bn in one CTA, or 256 x bn in a cluster of two CTAs
 // (pair); bn = 256 only with bf16 outputs.  tiles_m counts 128-row (256 with
 // pair) blocks.  The A0/A1 maps have 128-row boxes, the W map bn-row boxes

@@ -129,6 +129,35 @@ __device__ __forceinline__ int norm_float(uint32_t bits, uint32_t& sig) {
   return e - 127;
 }
 
+// a / b rounded to nearest for one divisor b shared by a whole call (the
+// dynamic base), from r = RN(1/b) (CUDA's __frcp_rn) and FMAs: y0 = RN(a r)
+// lies within 2 ulp of a/b; one Newton-Raphson correction with the exact
+// FMA residual, y1 = RN(y0 + (a - y0 b) r), makes it faithful; then
+// Markstein's theorem (IBM J. Res. Dev. 34(1), 1990: for a faithful y and a
+// correctly rounded reciprocal r, RN(y + (a - y b) r) is the correctly
+// rounded quotient, the residual being exact) gives q.  Used while b lies in
+// [2^-100, 2^100], where no product, residual or reciprocal leaves the
+// normal range for the quotients that decide codes; otherwise the IEEE
+// division itself.  dstar_fmdq_selftest_div compares it with __fdiv_rn.
+struct DivBy {
+  float b, r;
+  bool fast;
+};
+__device__ __forceinline__ DivBy div_by_setup(float b) {
+  DivBy d;
+  d.b = b;
+  d.r = __frcp_rn(b);
+  const float ab = fabsf(b);
+  d.fast = ab >= 0x1p-100f && ab <= 0x1p100f;
+  return d;
+}
+__device__ __forceinline__ float div_by(float a, const DivBy& d) {
+  if (!d.fast) return __fdiv_rn(a, d.b);
+  const float y0 = __fmul_rn(a, d.r);
+  const float y1 = __fmaf_rn(__fmaf_rn(-y0, d.b, a), d.r, y0);
+  return __fmaf_rn(__fmaf_rn(-y1, d.b, a), d.r, y1);
+}
+
 // Per-channel parameters with the dynamic base (FMDQ-DYN): PoT =
 // ceil(log2(M_i / base)) exactly, from the normalised exponents and
 // significands; the width from the predefined thresholds M_i <= 2^(thr + 2N)
@@ -366,11 +395,12 @@ __device__ __forceinline__ void process_pair(const QuantParams& p, const QConst&
   }
   // stage 3; a non-finite sub-channel has scale 0, and its NaN products convert to 0
   const float s0 = c0.nonfinite ? 0.f : c0.scale, s1 = c1.nonfinite ? 0.f : c1.scale;
-  if constexpr (DYN) {  // dX / base first (one IEEE division), then the power-of-two scale
+  if constexpr (DYN) {  // fl32(dX / base) first (correctly rounded), then the power-of-two scale
+    const DivBy dv = div_by_setup(qc.dbase);
 #pragma unroll
-    for (int i = 0; i < kTile; ++i) d0[i] = __fdiv_rn(d0[i], qc.dbase), d1[i] = __fdiv_rn(d1[i], qc.dbase);
-    m0 = __float_as_uint(__fdiv_rn(__uint_as_float(m0), qc.dbase));
-    m1 = __float_as_uint(__fdiv_rn(__uint_as_float(m1), qc.dbase));
+    for (int i = 0; i < kTile; ++i) d0[i] = div_by(d0[i], dv), d1[i] = div_by(d1[i], dv);
+    m0 = __float_as_uint(div_by(__uint_as_float(m0), dv));
+    m1 = __float_as_uint(div_by(__uint_as_float(m1), dv));
   }
   uint32_t w0[4], w1[4];
 #pragma unroll
@@ -1030,6 +1060,30 @@ __global__ void __launch_bounds__(256) base_min_kernel(const TIn* __restrict__ x
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) best = min(best, __shfl_xor_sync(0xffffffffu, best, o));
   if ((threadIdx.x & 31) == 0 && best != 0xFFFFFFFFu) atomicMin(out, best);
+}
+
+// Self-test of div_by against CUDA's __fdiv_rn: every a = (1 + m 2^-23) 2^e,
+// all 2^23 significands m and e in [e_lo, e_hi], divided by each of the n_b
+// divisors b[]; the number of results that differ in any bit is added to
+// *count.  Grid: (significand blocks, n_b, exponents).
+__global__ void __launch_bounds__(256) div_selftest_kernel(const float* __restrict__ b, int e_lo,
+                                                           unsigned long long* count) {
+  const DivBy d = div_by_setup(b[blockIdx.y]);
+  const int e = e_lo + (int)blockIdx.z;
+  unsigned long long bad = 0;
+  for (uint32_t m = blockIdx.x * blockDim.x + threadIdx.x; m < (1u << 23); m += gridDim.x * blockDim.x) {
+    const float a = __uint_as_float(((uint32_t)(e + 127) << 23) | m);
+    bad += __float_as_uint(div_by(a, d)) != __float_as_uint(__fdiv_rn(a, d.b));
+  }
+  for (int o = 16; o > 0; o >>= 1) bad += __shfl_xor_sync(0xffffffffu, bad, o);
+  if ((threadIdx.x & 31) == 0 && bad) atomicAdd(count, bad);
+}
+
+int launch_div_selftest(const float* b, int n_b, int e_lo, int e_hi, unsigned long long* count, void* stream) {
+  if (n_b <= 0 || e_hi < e_lo) return 0;
+  const dim3 grid(512, (unsigned)n_b, (unsigned)(e_hi - e_lo + 1));
+  div_selftest_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(b, e_lo, count);
+  return (int)cudaGetLastError();
 }
 
 int launch_base_min(const void* x_t, const void* x_prev, int64_t ld_xt, int64_t ld_xp, int64_t M, int64_t K,

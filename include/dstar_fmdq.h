@@ -377,6 +377,17 @@ DSTAR_API int dstar_fmdq_status(void* workspace, void* stream, uint32_t* status)
  * returns normally (the context stays usable). */
 DSTAR_API int dstar_fmdq_selftest_wait(void* workspace, uint32_t limit_us, void* stream);
 
+/* Device self-test of the division by the dynamic base (FMDQ-DYN divides every
+ * dX by one base per call with FMA corrections of a correctly rounded
+ * reciprocal instead of an IEEE division per element): for every
+ * a = (1 + m 2^-23) 2^e -- all 2^23 significands m, e_lo <= e <= e_hi
+ * (-126 < e < 128) -- and each of the n_b divisors b[i] (device memory), the
+ * quotient is compared bit for bit with CUDA's __fdiv_rn(a, b[i]); the number
+ * of differences is added to *count (device memory, 64-bit).  Enqueued on
+ * `stream`; DSTAR_ERR_INVALID_ARG for null pointers or exponents out of range. */
+DSTAR_API int dstar_fmdq_selftest_div(const float* b, int n_b, int e_lo, int e_hi, unsigned long long* count,
+                                      void* stream);
+
 /* Human-readable name of a return code; one-line reason for the last error of
  * the calling thread (empty when none). */
 DSTAR_API const char* dstar_fmdq_error_string(int code);
