@@ -36,10 +36,11 @@ def test_ragged_shapes(M, K, N):
     full_parity(_sub(base, M, K, N))
 
 
+@pytest.mark.parametrize("form", [0, nat.TILE_PAIR_256x128, nat.TILE_PAIR_256x256])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_distinct_output_refreshes_y_prev(dtype):
-    inp = synth.adversarial_layer(160, 256, 96, seed=6, spread=8, dtype=dtype)
-    g, q, acc, y, _ = full_parity(inp, y_distinct=True)
+def test_distinct_output_refreshes_y_prev(dtype, form):
+    inp = synth.adversarial_layer(400, 256, 272, seed=6, spread=8, dtype=dtype)
+    g, q, acc, y, _ = full_parity(inp, y_distinct=True, flags=nat.tile_flag(form))
     assert np.array_equal(g["y_prev_after"].float().cpu().numpy(), g["y"])
 
 

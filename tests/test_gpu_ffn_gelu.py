@@ -64,7 +64,7 @@ def _pair_inputs(cfg, M):
     return up, w2, ws2, y1p, hp, y2p
 
 
-def _chain(cfg, M, steps):
+def _chain(cfg, M, steps, flags=0):
     up, w2, ws2, y1p, hp, y2p = _pair_inputs(cfg, M)
     s = up.spec
     K1, N1, N2 = s.K, s.N, w2.shape[0]
@@ -87,7 +87,7 @@ def _chain(cfg, M, steps):
         c2 = torch.zeros(M, N1, dtype=torch.int8, device="cuda")
         a2 = torch.zeros(M, N2, dtype=torch.int64, device="cuda")
         nat.ffn_gelu(x_t, d["x_prev"], d["y1"], d["w1"], d["s1"], h_t, d["h_prev"], d["y2"], d["w2"], d["s2"],
-                     2.0 ** s.lb, ws1, wsb, debug1=(c1, a1), debug2=(c2, a2))
+                     2.0 ** s.lb, ws1, wsb, flags1=flags, flags2=flags, debug1=(c1, a1), debug2=(c2, a2))
         torch.cuda.synchronize()
         assert nat.status(ws1) == 0 and nat.status(wsb) == 0
         q1, acc1, y1, h, q2, acc2, y2 = oracle.ffn_gelu(x, x_prev_o, y1_o, up.w_q, up.w_scale, h_prev_o, y2_o,
@@ -139,6 +139,13 @@ def _chain(cfg, M, steps):
 
 def test_ffn_gelu_small_two_steps():
     _chain(2, 3 * 128 + 48, steps=2)
+
+
+@pytest.mark.parametrize("form", [nat.TILE_128x128, nat.TILE_128x256, nat.TILE_PAIR_256x256, nat.TILE_PAIR_256x128])
+def test_ffn_gelu_every_tile_form(form):
+    """Both layers in one forced tile form: the activation output of layer 1's
+    epilogue from single CTAs and from CTA pairs."""
+    _chain(2, 3 * 128 + 48, steps=1, flags=nat.tile_flag(form))
 
 
 def test_ffn_gelu_full_size_latte():
