@@ -296,10 +296,11 @@ def algorithmic_k2(spec, ws_sections, out_bytes=2):
     return dense_ops, issued, bytes_, int((planes > 2).sum())
 
 
-def kernel_rows(inputs, stats, k1_ms, k2_ms, peaks):
+def kernel_rows(inputs, stats, k1_ms, k2_ms, peaks, spread=None):
     """Per launch: time, achieved rate and fraction of the bound that applies
     (HBM for the quantizer; for the slice GEMM the larger of tensor and HBM
-    time at the measured peaks)."""
+    time at the measured peaks); with spread ({(kernel, layer index): (median,
+    min, max) ms}) also the spread of the sampled launches."""
     hbm = peaks["hbm_gbs"]
     i8 = peaks["bf16_tflops"] * INT8_PER_BF16
     kern = []
@@ -316,8 +317,10 @@ def kernel_rows(inputs, stats, k1_ms, k2_ms, peaks):
             kern.append(dict(kernel="slice_gemm", layer=name, ms=k2_ms[li], bound="hbm",
                              achieved=stt["k2_bytes"] / (k2_ms[li] * 1e-3) / 1e9, peak=hbm, unit="GB/s",
                              algorithmic=stt["k2_bytes"]))
-    for k in kern:
+    for i, k in enumerate(kern):
         k["frac"] = k["achieved"] / k["peak"]
+        if spread and (k["kernel"], i // 2) in spread:
+            k["ms_median"], k["ms_min"], k["ms_max"] = spread[(k["kernel"], i // 2)]
     return kern
 
 
@@ -567,7 +570,10 @@ class ConfigBench:
             self.graphs[s].replay()
 
     def split_times(self, K):
-        """Mean per-kernel times from replays of the split step (event nodes)."""
+        """Per-kernel times from replays of the split step (event nodes): the
+        mean over the last back-to-back cycle of every graph, returned, and in
+        self.split_stats the median, min and max over 10 more cycles whose
+        events are read after each replay."""
         torch, rt = self.torch, self.rt
         n = len(self.graphs)
         kp = max(n, min(K, 1200) // n * n)
@@ -584,6 +590,15 @@ class ConfigBench:
               for li in range(self.nlayers)]
         k2 = [statistics.fmean(el(self.gev[g][li][1], self.gev[g][li][2]) for g in range(n))
               for li in range(self.nlayers)]
+        samples = {}
+        for _ in range(10):
+            for g in range(n):
+                self.prof_graphs[g].replay()
+                torch.cuda.synchronize()
+                for li in range(self.nlayers):
+                    samples.setdefault(("quantize", li), []).append(el(self.gev[g][li][0], self.gev[g][li][1]))
+                    samples.setdefault(("slice_gemm", li), []).append(el(self.gev[g][li][1], self.gev[g][li][2]))
+        self.split_stats = {k: (statistics.median(v), min(v), max(v)) for k, v in samples.items()}
         return k1, k2
 
     def timed(self, K, dist=False, clocks_id=None, clocks_on=True):
@@ -721,7 +736,7 @@ def measure_extra(cfg, args, torch, nat, L, peaks, peak_src):
     if st:
         raise RuntimeError(f"device status {st} after workload {cfg}")
     dense = sum(s["k2_dense"] for s in stats)
-    kern = kernel_rows(cb.inputs, stats, k1, k2, peaks)
+    kern = kernel_rows(cb.inputs, stats, k1, k2, peaks, getattr(cb, "split_stats", None))
     out = {"workload": synth.CONFIG_NAMES[cfg], "value": job_tops(1, dense, ms / args.extra_steps), "unit": "TOPS",
            "ms_per_step": ms / args.extra_steps, "steps": args.extra_steps,
            "layers": [f"{i.spec.name} M={i.spec.M} K={i.spec.K} N={i.spec.N}" for i in cb.inputs],
@@ -1045,6 +1060,7 @@ def run_ours(args, rank, world, local_rank):
         raise RuntimeError(f"device status {st} after the benchmark")
     inputs = cb.inputs
     set_mb = cb.set_mb()
+    spread = getattr(cb, "split_stats", None)
     cb.close()
 
     # further workloads, on one GPU only (every rank would have to run them alike)
@@ -1063,7 +1079,7 @@ def run_ours(args, rank, world, local_rank):
     if rank != 0:
         return
 
-    kern = kernel_rows(inputs, stats, k1_ms, k2_ms, peaks)
+    kern = kernel_rows(inputs, stats, k1_ms, k2_ms, peaks, spread)
     roofline = roofline_of(kern, peak_src)
     cpu = None
     if not args.no_cpu_baseline:
