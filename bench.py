@@ -25,6 +25,7 @@ from __future__ import annotations
 import argparse
 import ctypes
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -81,10 +82,16 @@ def load_peaks():
 
 
 def kernel_source_sha():
+    """Hash of the kernel sources without their comments (a comment edit does
+    not make recorded counters stale; any code change does)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "differential_quantized_gemm_b200", "csrc")
     for f in sorted(os.listdir(csrc)):
-        h.update(open(os.path.join(csrc, f), "rb").read())
+        text = open(os.path.join(csrc, f), encoding="utf-8").read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        h.update(f.encode())
+        h.update("\n".join(line.rstrip() for line in text.splitlines() if line.strip()).encode())
     return h.hexdigest()[:16]
 
 

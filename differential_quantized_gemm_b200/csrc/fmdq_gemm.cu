@@ -14,12 +14,15 @@
 // ascending-FPoT shift-and-add produces -- then
 //   Y_t = Y_{t-1} + ((float)acc * 2^(-lb - g_ref)) * w_scale[n]   (fp32, in this order).
 //
-// Structure (one CTA per SM, persistent over 128 x BN output tiles):
+// Structure (one CTA per SM, persistent over 128 x BN output tiles; or, with
+// PAIR, one cluster of two CTAs per two SMs over 256 x BN tiles, each CTA
+// owning 128 rows):
 //   warp 0      TMA producer: per K chunk, a 128 x 128-byte tile of the operand
-//               plane and a BN x 128-byte tile of W; blocks that need the
-//               second plane run a second K pass over the chunks where it is
-//               nonzero
-//   warp 1      TMEM allocator and MMA issuer (one thread): M=128, N=BN, K=32
+//               plane and a BN x 128-byte tile of W (BN / 2 rows with PAIR);
+//               blocks that need the second plane run a second K pass over
+//               the chunks where it is nonzero
+//   warp 1      TMEM allocator and MMA issuer (one thread; the even CTA's with
+//               PAIR): M=128 (256 with PAIR), N=BN, K=32
 //   warps 2..9  epilogue, two warps per 32 TMEM lanes (rows), each half of the
 //               columns: TMA-load of its 32 x 32 tiles of y_prev into shared
 //               memory (issued before the accumulator is ready), tcgen05.ld,
@@ -29,7 +32,8 @@
 // slot, a two-plane tile two, so the epilogue of one tile overlaps the MMAs
 // of the next.  Tiles whose operands need more than two int8 planes are
 // computed by the epilogue warps along the slice stream.  Every wait is
-// bounded (wait_parity).
+// bounded (wait_parity).  The host picks BN and PAIR per call from a model of
+// the mainloop and the epilogue (choose_tile in fmdq_host.cu).
 #include <cuda_bf16.h>
 
 #include "fmdq_device.cuh"
