@@ -84,33 +84,81 @@ __global__ void __launch_bounds__(256) quant_cols_t_kernel(const TIn* __restrict
 // Softmax over the kept blocks of each score row (section 3.2: pruned blocks
 // of the score matrix are never computed); pruned entries become 0.  Row r
 // is query r mod S of its head; its mask row is bits[(r mod S) / 128] (bit c:
-// key block c kept).  One warp per row.  The pages leave the softmax's
-// precision open and P decides integer codes, so it is evaluated in fp64
-// (CUDA's double exp, fp64 sum and division) and rounded once to fp32.
+// key block c kept).  The pages leave the softmax's precision open and P
+// decides integer codes, so it is evaluated in fp64 (CUDA's double exp, fp64
+// sum and division) and rounded once to fp32.  One block of 256 threads per
+// row (S <= 4096): each thread holds the kept scores of columns
+// tid + 256 i in registers, so every score is read once and every exp is
+// evaluated once; the maximum and the sum are block reductions.
+constexpr int kSmThreads = 256;
+constexpr int kSmPer = 32 * kBlockM / kSmThreads;  // S <= 32 blocks of 128 columns
+
 __device__ __forceinline__ double warp_sum_d(double v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
 }
 
-__global__ void __launch_bounds__(256) masked_softmax_kernel(const float* __restrict__ sc, float* __restrict__ pr,
-                                                             int64_t rows, int64_t S, const __grid_constant__ BlockMask mk) {
-  const int lane = threadIdx.x & 31;
-  const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (r >= rows) return;
+__global__ void __launch_bounds__(kSmThreads) masked_softmax_kernel(const float* __restrict__ sc, float* __restrict__ pr,
+                                                                    int64_t S, const __grid_constant__ BlockMask mk) {
+  __shared__ float s_max[kSmThreads / 32];
+  __shared__ double s_sum[kSmThreads / 32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t r = blockIdx.x;
   const uint64_t keep = mk.bits[(r % S) / kBlockM];
   const float* x = sc + r * S;
+  float v[kSmPer];
+  uint32_t kept = 0;  // bit i: column tid + 256 i is kept
   float m = -INFINITY;
-  for (int64_t c = lane; c < S; c += 32)
-    if ((keep >> (c / kBlockM)) & 1ull) m = fmaxf(m, x[c]);
-  const double md = (double)warp_max(m);
+#pragma unroll
+  for (int i = 0; i < kSmPer; ++i) {
+    const int64_t c = threadIdx.x + (int64_t)kSmThreads * i;
+    v[i] = 0.f;
+    if (c < S && ((keep >> (c / kBlockM)) & 1ull)) {
+      v[i] = x[c];
+      kept |= 1u << i;
+      m = fmaxf(m, v[i]);
+    }
+  }
+  m = warp_max(m);
+  if (lane == 0) s_max[warp] = m;
+  __syncthreads();
+  m = s_max[0];
+#pragma unroll
+  for (int w = 1; w < kSmThreads / 32; ++w) m = fmaxf(m, s_max[w]);
+  const double md = (double)m;
+  double e[kSmPer];
   double l = 0.0;
-  for (int64_t c = lane; c < S; c += 32)
-    if ((keep >> (c / kBlockM)) & 1ull) l += exp((double)x[c] - md);
-  const double sum = warp_sum_d(l);
+#pragma unroll
+  for (int i = 0; i < kSmPer; ++i) {
+    e[i] = ((kept >> i) & 1u) ? exp((double)v[i] - md) : 0.0;
+    l += e[i];
+  }
+  l = warp_sum_d(l);
+  if (lane == 0) s_sum[warp] = l;
+  __syncthreads();
+  double sum = s_sum[0];
+#pragma unroll
+  for (int w = 1; w < kSmThreads / 32; ++w) sum += s_sum[w];
+  // e / sum for the row's one divisor: q0 = RN(e rs) with rs = RN(1/sum), one
+  // Newton-Raphson correction with the exact FMA residual (faithful), then
+  // Markstein's correction (IBM J. Res. Dev. 34(1), 1990), which gives the
+  // correctly rounded quotient; sum >= 1 (the maximum's own term is 1) and
+  // every e in [0, 1], so no step leaves the normal range but for e = 0.
+  const double rs = __drcp_rn(sum);
   float* o = pr + r * S;
-  for (int64_t c = lane; c < S; c += 32)
-    o[c] = ((keep >> (c / kBlockM)) & 1ull) ? (float)(exp((double)x[c] - md) / sum) : 0.f;
+#pragma unroll
+  for (int i = 0; i < kSmPer; ++i) {
+    const int64_t c = threadIdx.x + (int64_t)kSmThreads * i;
+    if (c >= S) continue;
+    float pv = 0.f;
+    if ((kept >> i) & 1u) {
+      const double q0 = __dmul_rn(e[i], rs);
+      const double q1 = __fma_rn(__fma_rn(-q0, sum, e[i]), rs, q0);
+      pv = (float)__fma_rn(__fma_rn(-q1, sum, e[i]), rs, q1);
+    }
+    o[c] = pv;
+  }
 }
 
 }  // namespace
@@ -143,7 +191,8 @@ int launch_quant_cols_t(const void* v, int64_t ld, int64_t heads, int64_t S, int
 
 int launch_masked_softmax(const float* sc, float* pr, int64_t rows, int64_t S, const BlockMask& mk, void* stream) {
   if (rows == 0) return 0;
-  masked_softmax_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, (cudaStream_t)stream>>>(sc, pr, rows, S, mk);
+  if (S > (int64_t)kSmThreads * kSmPer) return (int)cudaErrorInvalidValue;  // the host admits S <= 4096
+  masked_softmax_kernel<<<(unsigned)rows, kSmThreads, 0, (cudaStream_t)stream>>>(sc, pr, S, mk);
   return (int)cudaGetLastError();
 }
 
