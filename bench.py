@@ -81,12 +81,16 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+# the sources that decide the benchmarked step's kernels and their launches
+STEP_SOURCES = ("fmdq_device.cuh", "fmdq_gemm.cu", "fmdq_host.cu", "fmdq_internal.h", "fmdq_quant.cu")
+
+
 def kernel_source_sha():
-    """Hash of the kernel sources without their comments (a comment edit does
-    not make recorded counters stale; any code change does)."""
+    """Hash of the step's kernel sources without their comments (a comment
+    edit does not make recorded counters stale; any code change does)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "differential_quantized_gemm_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in STEP_SOURCES:
         text = open(os.path.join(csrc, f), encoding="utf-8").read()
         text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
         text = re.sub(r"//[^\n]*", "", text)
