@@ -2,7 +2,7 @@
 section 3.2 "Sparse Attention Reuse", section 4.3 "Attention Operation")
 against the oracle, head by head, through the C ABI (dstar_sar_attention):
 
-- cached step: the int8 keys and their scales, every integer output of Q's
+- cached step: the int8 keys and values and their scales, every integer output of Q's
   FMDQ (width, FPoT, g_ref, encoded stream) and the scores of every kept
   block bit-exact; the softmax (fp64 on both sides, rounded once to fp32;
   the library exp and the order of the sums may differ in the last fp64
@@ -52,6 +52,8 @@ def _run(G, S, dh, d, seed, heads_checked=None, keep=0.5):
     got = dict(out=out.cpu().numpy().copy(),
                kq=att.section("kq", R * d, torch.int8).view(R, d).cpu().numpy(),
                ks=att.section("ks", R, torch.float32).cpu().numpy(),
+               vqt=att.section("vqt", G * d * S, torch.int8).view(G * d, S).cpu().numpy(),
+               vs=att.section("vs", G * d, torch.float32).cpu().numpy(),
                scores=att.section("scores", R * S, torch.float32).view(R, S).clone(),  # on the device
                probs=att.section("probs", R * S, torch.float32).view(R, S).clone(),
                sq={n: t.cpu().numpy() for n, t in att.fmdq_sections("q").items() if n != "plane0" and n != "plane1"},
@@ -71,6 +73,9 @@ def _run(G, S, dh, d, seed, heads_checked=None, keep=0.5):
         # keys: int8 codes and scales (times the score scale)
         assert np.array_equal(got["kq"][rows], ref["kq"])
         assert np.array_equal(got["ks"][rows], (ref["ks"] * np.float32(scale)).astype(np.float32))
+        # values: int8 codes per column of the head's V, stored transposed, and their scales
+        assert np.array_equal(got["vqt"][h * d:(h + 1) * d], ref["vq"])
+        assert np.array_equal(got["vs"][h * d:(h + 1) * d], ref["vs"])
         # Q's FMDQ (every width 8, X_{t-1} = 0)
         tq = slice(h * T, (h + 1) * T)
         for name in ("fpot", "bits", "g_ref", "count"):
