@@ -164,9 +164,9 @@ def run_oracle_dyn(inp: synth.LayerInputs, y_prev_f32=None):
     return q, acc, y
 
 
-def dyn_parity(inp, debug=True):
-    """Dynamic base: GPU (DSTAR_FLAG_DYNAMIC_BASE) against the oracle, everything compared."""
-    g = run_gpu(inp, flags=nat.FLAG_DYNAMIC_BASE, debug=debug)
+def dyn_parity(inp, debug=True, flags=0):
+    """Dynamic base: GPU (DSTAR_FLAG_DYNAMIC_BASE, plus `flags`) against the oracle, everything compared."""
+    g = run_gpu(inp, flags=nat.FLAG_DYNAMIC_BASE | flags, debug=debug)
     q, acc, y = run_oracle_dyn(inp)
     assert g["status"] == 0, g["status"]
     base = float(g["ws"].sections(inp.spec.M, inp.spec.K)["dyn_base"].cpu()[0])

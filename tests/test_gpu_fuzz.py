@@ -2,8 +2,9 @@
 of the FMDQ differential linear) against the oracle: M, K and N drawn within
 the interface's rules (M % 16 == 0, K % 32 == 0, N % 16 == 0), bf16 or fp32,
 a random slice-GEMM tile form (one CTA or a CTA pair), a random dX spread
-(from one-plane tiles to the slice stream) and sometimes a distinct output.
-Every code, tag, record and accumulator bit-exact, Y_t within the bar."""
+(from one-plane tiles to the slice stream) and sometimes a distinct output;
+then with the dynamic base (FMDQ-DYN).  Every code, tag, record and
+accumulator bit-exact, Y_t within the bar."""
 import numpy as np
 import pytest
 import torch
@@ -11,7 +12,7 @@ import torch
 from differential_quantized_gemm_b200 import _native as nat
 from differential_quantized_gemm_b200 import synth
 
-from gpu_helpers import full_parity
+from gpu_helpers import dyn_parity, full_parity
 
 pytestmark = pytest.mark.gpu
 
@@ -44,3 +45,10 @@ def test_random_shape(i):
     g, q, acc, y, _ = full_parity(inp, flags=nat.tile_flag(form), y_distinct=distinct)
     if distinct:
         assert np.array_equal(g["y_prev_after"].float().cpu().numpy(), g["y"])
+
+
+@pytest.mark.parametrize("i", range(16))
+def test_random_shape_dynamic_base(i):
+    M, K, N, dtype, spread, form, _ = _case(100 + i)
+    inp = synth.adversarial_layer(M, K, N, seed=3000 + i, spread=spread, dtype=dtype)
+    dyn_parity(inp, flags=nat.tile_flag(form))
