@@ -121,9 +121,15 @@ __device__ __forceinline__ uint32_t cluster_smem_addr(const void* p, uint32_t ra
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-// Arrive (release, cluster scope) on an mbarrier given by its cluster address.
+// Arrive (relaxed, cluster scope) on an mbarrier given by its cluster
+// address.  Its one use frees a TMEM slot for the even CTA's MMAs: the
+// arriving warp's tcgen05.ld reads of the slot have completed at
+// tcgen05.wait::ld, and the MMA thread reads nothing else that the warp
+// wrote, so no release is needed.  A release at cluster scope would make the
+// arrive wait for all of the thread's outstanding memory operations
+// (measured: 2.5-3.6 K cycles per tile, which bounded the pair's epilogue).
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
 }
 // TMA load into this CTA's shared memory whose completion is counted on the
 // even CTA's barrier (bar_cluster: its cluster address).

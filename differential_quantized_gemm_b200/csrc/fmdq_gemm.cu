@@ -597,61 +597,56 @@ __global__ void __launch_bounds__(kGThreads, 1)
     // TMA swizzle of a 32 x 32 tile: 64-byte rows (bf16) use the 64-byte pattern,
     // 128-byte rows (fp32) the 128-byte one; chunk c of row r sits at chunk c ^ sw(r)
     auto sw = [](int r) { return OUT_BF16 ? ((r >> 1) & 3) : (r & 7); };
-    auto tile_rb = [&](int s) {
-      int rb, nb;
-      coords(unit + s * units, rb, nb);
-      return rb;
-    };
-    auto tile_nb = [&](int s) {
-      int rb, nb;
-      coords(unit + s * units, rb, nb);
-      return nb;
-    };
     // the slot's tm_empty barrier: the even CTA's with PAIR
     const uint32_t tm_empty_cl = PAIR ? cluster_smem_addr(tm_empty, 0) : 0u;
     // Everything a tile needs besides its accumulator is requested one tile
     // ahead: its y_prev boxes (each as soon as the previous tile's store has
     // read the box), its weight scales (shared memory, double-buffered) and
     // this lane's row data.
-    auto weight_scale = [&](int s) -> float {
-      const int64_t n = (int64_t)tile_nb(s) * BN + etid;
+    auto weight_scale = [&](int rb_s, int nb_s) -> float {
+      const int64_t n = (int64_t)nb_s * BN + etid;
       int64_t off = 0;  // the head's scales with SPARSE
-      if constexpr (SPARSE) off = (int64_t)(tile_rb(s) / rb_per_head) * p.N;
+      if constexpr (SPARSE) off = (int64_t)(rb_s / rb_per_head) * p.N;
       return (etid < BN && n < p.N) ? p.w_scale[off + n] : 0.f;
     };
     // this lane's row: plane count (3 beyond M) and g_ref
-    auto row_planes = [&](int s, int& pl, int& gref) {
-      const int64_t row = (int64_t)row_of(tile_rb(s)) + quarter * 32 + lane;
+    auto row_planes = [&](int rb_s, int& pl, int& gref) {
+      const int64_t row = (int64_t)row_of(rb_s) + quarter * 32 + lane;
       pl = 3, gref = 0;
       if (row < p.M) pl = p.planes[row / kTile], gref = p.g_ref[row / kTile];
     };
     // With SPARSE there is no cached output: Y_{t-1} = 0 is never read.
-    auto load_y_box = [&](int s, int g) {  // lane 0
+    auto load_y_box = [&](int rb_s, int nb_s, int g) {  // lane 0
       if constexpr (SPARSE) return;
       if (g == 0) mbar_arrive_expect_tx(&ybar[ew], C::kYWarpBytes);
-      tma_load_2d(ybuf + g * C::kBoxBytes, &tm_yp, &ybar[ew], tile_nb(s) * BN + half * (BN / 2) + g * 32,
-                  row_of(tile_rb(s)) + quarter * 32);
+      tma_load_2d(ybuf + g * C::kBoxBytes, &tm_yp, &ybar[ew], nb_s * BN + half * (BN / 2) + g * 32,
+                  row_of(rb_s) + quarter * 32);
     };
     uint32_t slot_it = 0;
     uint32_t y_issued = 0, y_seen = 0;  // batches of y_prev boxes requested (lane 0) / observed landed
     int ok = 1;
     pdl_wait();  // the quantizer's outputs and the cached output are read from here on
     const float beta = dyn_beta(p.dyn_base);
+    // this tile's coordinates and the next one's, advanced once per tile
+    int rb_c = 0, nb_c = 0;
+    if (my_tiles > 0) coords(unit, rb_c, nb_c);
     if (lane == 0 && my_tiles > 0) {
-      for (int g = 0; g < C::kHalfGroups; ++g) load_y_box(0, g);
+      for (int g = 0; g < C::kHalfGroups; ++g) load_y_box(rb_c, nb_c, g);
       ++y_issued;
     }
     int pl_cur = 3, gref_cur = 0;
     if (my_tiles > 0) {
-      row_planes(0, pl_cur, gref_cur);
-      if (etid < BN) s_ws[etid] = weight_scale(0);
+      row_planes(rb_c, pl_cur, gref_cur);
+      if (etid < BN) s_ws[etid] = weight_scale(rb_c, nb_c);
     }
     // block info of this CTA's first kMaxTileSlots tiles, loaded in parallel,
     // then published to the producer and MMA threads (with PAIR both CTAs
     // compute the same information for the tile's 256 rows)
     for (int i = etid; i < min(my_tiles, kMaxTileSlots) * kTilesPerBlock; i += 32 * kEpiWarps) {
       const int slot = i / kTilesPerBlock, sub = i % kTilesPerBlock;
-      const int t = tile_rb(slot) * kTilesPerBlock + sub;
+      int rb_s, nb_s;
+      coords(unit + slot * units, rb_s, nb_s);
+      const int t = rb_s * kTilesPerBlock + sub;
       if (t < T) {
         const int pl = p.planes[t];
         int* e = reinterpret_cast<int*>(&s_info[slot]);
@@ -667,8 +662,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
     // also after a timed-out wait (ok == 0), so no warp can be left waiting
     // at a barrier that another warp skipped.
     for (int slot = 0; slot < my_tiles; ++slot) {
-      const int rb = tile_rb(slot), nb = tile_nb(slot);
+      const int rb = rb_c, nb = nb_c;
       const bool has_next = slot + 1 < my_tiles;
+      int rb_n = 0, nb_n = 0;
+      if (has_next) coords(unit + (slot + 1) * units, rb_n, nb_n);
       const BlockInfo bi = info(slot, rb);
       const int64_t n_base = (int64_t)nb * BN;
       const int64_t n_half = n_base + half * (BN / 2);
@@ -677,8 +674,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
       float ws_next = 0.f;
       int pl_next = 3, gref_next = 0;
       if (has_next) {
-        ws_next = weight_scale(slot + 1);
-        row_planes(slot + 1, pl_next, gref_next);
+        ws_next = weight_scale(rb_n, nb_n);
+        row_planes(rb_n, pl_next, gref_next);
       }
 
       if (ok) {
@@ -732,11 +729,11 @@ __global__ void __launch_bounds__(kGThreads, 1)
               bulk_commit();
               if (has_next && g > 0) {
                 bulk_wait_read<1>();
-                load_y_box(slot + 1, g - 1);
+                load_y_box(rb_n, nb_n, g - 1);
               }
               if (has_next && g == C::kHalfGroups - 1) {
                 bulk_wait_read<0>();
-                load_y_box(slot + 1, g);
+                load_y_box(rb_n, nb_n, g);
                 ++y_issued;
               }
             }
@@ -839,6 +836,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
       // finished before the previous iteration's barrier
       if (has_next && etid < BN) s_ws[((slot + 1) & 1) * BN + etid] = ws_next;
       pl_cur = pl_next, gref_cur = gref_next;
+      rb_c = rb_n, nb_c = nb_n;
       epi_barrier();
     }
     // nothing of this warp's may still be in flight when the block exits:

@@ -253,9 +253,10 @@ int do_quantize(const dstar_mat* x_t, dstar_mat* x_prev, int lb, const dstar_til
 // 45 B per clock with 96 KB in flight, 60 with 160 KB, linear between, at
 // most 74) -- so a 128-deep K chunk costs the larger of its MMA cycles (the
 // SM's 128 rows x BN x 128 int8 MAC at 8192 per clock) and its bytes at that
-// rate.  Epilogue: about 1800 + 4800 cycles per 128 output columns of a
-// 128-row tile (y_prev in, Y_t out, TMEM reads), a fifth more in a pair whose
-// slots wait for both CTAs.  The busiest SM's (or pair's) tile count times
+// rate.  Epilogue: about 1400 + 3000 cycles per 128 output columns of an
+// SM's 128 rows (y_prev in, Y_t out, TMEM reads), in one CTA or a pair
+// (fitted so that the picks match the fastest measured form of each layer of
+// the DiT-XL/2, PixArt and Latte workloads).  The busiest SM's (or pair's) tile count times
 // the period decides, ties to the earlier form.  Forms (stages): 128 x 128
 // (6 with bf16 outputs, 5 with fp32), 128 x 256 (3), and CTA pairs 256 x 256
 // (4; bf16 outputs) and 256 x 128 (8 with bf16 outputs, 6 with fp32), whose
@@ -279,7 +280,7 @@ TileShape choose_tile(int64_t M, int64_t N, int64_t K, int sms, bool bf16, unsig
     const int64_t wrows = pair ? bn / 2 : bn;  // one SM's share of the W tile
     const double bytes = (128 + wrows) * 128.0;
     const double chunk = std::max<double>(128.0 * bn * 128.0 / 8192.0, bytes / rate((stages - 1) * bytes));
-    const double epi = (1800.0 + 4800.0 * bn / 128.0) * (pair ? 1.2 : 1.0);
+    const double epi = 1400.0 + 3000.0 * bn / 128.0;
     const int64_t bm = pair ? 256 : 128, units = pair ? sms / 2 : sms;
     const int64_t tiles = ((M + bm - 1) / bm) * ((N + bn - 1) / bn);
     return (double)((tiles + units - 1) / units) * std::max(chunks * chunk, epi);

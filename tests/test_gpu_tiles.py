@@ -30,9 +30,10 @@ def _build():
 
 
 def test_tile_shapes_of_the_workloads():
-    # the Latte FFN pair: 128 x 256 tiles for the up-projection (its epilogue
-    # bounds it), CTA pairs of 256 x 128 for the down-projection (K = 4608)
-    assert nat.gemm_tile(16384, 4608, 1152, True) == (128, 256, False)
+    # the Latte FFN pair: CTA pairs of 256 x 256 for the up-projection (every
+    # SM's 128 x 256 epilogue bounds it, with half the weight bytes per SM of
+    # a one-CTA tile), pairs of 256 x 128 for the down-projection (K = 4608)
+    assert nat.gemm_tile(16384, 4608, 1152, True) == (256, 256, True)
     assert nat.gemm_tile(16384, 1152, 4608, True) == (256, 128, True)
     valid = {(128, 128, False), (128, 256, False), (256, 256, True), (256, 128, True)}
     for M, N, K in [(2048, 4608, 1152), (2048, 1152, 4608), (8192, 3456, 1152), (432, 1152, 1152), (16, 16, 32)]:
