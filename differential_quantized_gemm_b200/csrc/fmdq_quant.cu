@@ -775,27 +775,25 @@ __global__ void __launch_bounds__(kQThreads, FMDQ_Q_MIN_BLOCKS) quantize_kernel(
 // above (the same stage functions, with one CTA per tile); the buffers pass
 // between the groups through mbarriers (full: group 1 -> 2, empty: 2 -> 1)
 // whose waits are bounded.
-// Warps of each group (compile-time; 16 warps of 128 registers fill an SM).
-#ifndef FMDQ_P_G1_WARPS
-#define FMDQ_P_G1_WARPS 8
-#endif
-#ifndef FMDQ_P_G2_WARPS
-#define FMDQ_P_G2_WARPS 8
-#endif
-constexpr int kPG1Warps = FMDQ_P_G1_WARPS, kPG2Warps = FMDQ_P_G2_WARPS;
-constexpr int kPG1 = 32 * kPG1Warps, kPG2 = 32 * kPG2Warps;  // threads of each group
-constexpr int kPThreads = kPG1 + kPG2;
+// Two forms, 16 warps of 128 registers per SM either way: one CTA of 8 + 8
+// warps, or two CTAs of 4 + 4 warps, whose group barriers take half the
+// threads and whose two tile streams cover each other's pipeline fill and
+// drain.  The second pays where an SM has few tiles (measured: PixArt's
+// 8192-token layers, 3.5 tiles per SM, 1-2 us faster per launch; the Latte
+// layers, 6.9 tiles per SM, 3 us slower per step) and needs two CTAs'
+// buffers in the SM's shared memory (inputs of up to about 2900 channels).
+constexpr int kPMaxWarps = 8;          // warps of a group, at most
 constexpr int kBarG1 = 1, kBarG2 = 2;  // named barriers of the groups (0 is __syncthreads)
 
 struct PSmem {
   uint64_t full[2], empty[2];
   int abort;
-  int red[4][kPG1Warps];
+  int red[4][kPMaxWarps];
   int xv[2][4];  // per buffer: finest FPoT, coarsest FPoT, min(FPoT + one-plane room), min(FPoT + two-plane room)
   uint32_t mask[kMaxMaskWords];
-  int warp_cnt[kPG2Warps][kTagWin];
+  int warp_cnt[kPMaxWarps][kTagWin];
   int base[kTagWin];
-  int wbase[kPG2Warps][kTagWin];
+  int wbase[kPMaxWarps][kTagWin];
 };
 
 template <int NT>
@@ -803,8 +801,11 @@ __device__ __forceinline__ void group_sync(int id) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "n"(NT) : "memory");
 }
 
-template <typename TIn, bool DYN>
-__global__ void __launch_bounds__(kPThreads, 1) quantize_persistent_kernel(const QuantParams p) {
+template <typename TIn, bool DYN, int kPG1Warps, int kPG2Warps, int kMinBlocks>
+__global__ void __launch_bounds__(32 * (kPG1Warps + kPG2Warps), kMinBlocks)
+    quantize_persistent_kernel(const QuantParams p) {
+  static_assert(kPG1Warps <= kPMaxWarps && kPG2Warps <= kPMaxWarps, "shared-memory tables");
+  constexpr int kPG1 = 32 * kPG1Warps, kPG2 = 32 * kPG2Warps;  // threads of each group
   extern __shared__ __align__(16) uint8_t smem[];
   const int64_t K = p.K;
   const int Kc = (int)K;
@@ -954,6 +955,31 @@ bool use_persistent(int64_t M, int64_t K, int num_sms) {
   return M / kTile >= 2LL * num_sms && quantize_persistent_smem_bytes(K) <= 227 * 1024;
 }
 
+// Two CTAs of the persistent kernel per SM: at most four tiles per SM, and
+// both CTAs fit the SM's 228 KB of shared memory, each with the 1 KB the
+// system reserves per CTA.
+bool persistent_two_per_sm(int64_t T, int64_t K, int num_sms) {
+  return T <= 4LL * num_sms && 2 * (quantize_persistent_smem_bytes(K) + 1024) <= 228 * 1024;
+}
+
+template <typename TIn, bool DYN>
+int launch_persistent(cudaLaunchConfig_t& cfg, const QuantParams& p, int64_t T, int num_sms) {
+  const bool two = persistent_two_per_sm(T, p.K, num_sms);
+  const void* fn = two ? (const void*)quantize_persistent_kernel<TIn, DYN, 4, 4, 2>
+                       : (const void*)quantize_persistent_kernel<TIn, DYN, 8, 8, 1>;
+  const int e = ensure_max_smem(fn, 227 * 1024);
+  if (e != 0) return e;
+  const int64_t ctas = (int64_t)num_sms * (two ? 2 : 1);
+  cfg.gridDim = dim3((unsigned)(T < ctas ? T : ctas), 1, 1);
+  cfg.blockDim = dim3(two ? 256 : 512, 1, 1);
+  cfg.dynamicSmemBytes = quantize_persistent_smem_bytes(p.K);
+  cfg.numAttrs = 1;
+  const cudaError_t ce = two ? cudaLaunchKernelEx(&cfg, quantize_persistent_kernel<TIn, DYN, 4, 4, 2>, p)
+                             : cudaLaunchKernelEx(&cfg, quantize_persistent_kernel<TIn, DYN, 8, 8, 1>, p);
+  if (ce != cudaSuccess) return (int)ce;
+  return (int)cudaGetLastError();
+}
+
 int launch_quantize(const QuantParams& p, int in_bf16, int num_sms, void* stream) {
   const int64_t T = p.M / kTile;
   if (T == 0) return 0;
@@ -966,22 +992,9 @@ int launch_quantize(const QuantParams& p, int in_bf16, int num_sms, void* stream
   cfg.attrs = attr;
   cudaError_t ce;
   if (use_persistent(p.M, p.K, num_sms)) {
-    const void* fn = in_bf16 ? (dyn ? (const void*)quantize_persistent_kernel<__nv_bfloat16, true>
-                                    : (const void*)quantize_persistent_kernel<__nv_bfloat16, false>)
-                             : (dyn ? (const void*)quantize_persistent_kernel<float, true>
-                                    : (const void*)quantize_persistent_kernel<float, false>);
-    const int e = ensure_max_smem(fn, 227 * 1024);
-    if (e != 0) return e;
-    cfg.gridDim = dim3((unsigned)(T < num_sms ? T : num_sms), 1, 1);
-    cfg.blockDim = dim3(kPThreads, 1, 1);
-    cfg.dynamicSmemBytes = quantize_persistent_smem_bytes(p.K);
-    cfg.numAttrs = 1;
-    if (in_bf16) ce = dyn ? cudaLaunchKernelEx(&cfg, quantize_persistent_kernel<__nv_bfloat16, true>, p)
-                          : cudaLaunchKernelEx(&cfg, quantize_persistent_kernel<__nv_bfloat16, false>, p);
-    else ce = dyn ? cudaLaunchKernelEx(&cfg, quantize_persistent_kernel<float, true>, p)
-                  : cudaLaunchKernelEx(&cfg, quantize_persistent_kernel<float, false>, p);
-    if (ce != cudaSuccess) return (int)ce;
-    return (int)cudaGetLastError();
+    if (in_bf16) return dyn ? launch_persistent<__nv_bfloat16, true>(cfg, p, T, num_sms)
+                            : launch_persistent<__nv_bfloat16, false>(cfg, p, T, num_sms);
+    return dyn ? launch_persistent<float, true>(cfg, p, T, num_sms) : launch_persistent<float, false>(cfg, p, T, num_sms);
   }
   const int C = quantize_cluster_size(p.M, p.K, num_sms);
   const int64_t units = p.K / 32;
