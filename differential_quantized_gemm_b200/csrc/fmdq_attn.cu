@@ -154,6 +154,11 @@ __global__ void __cluster_dims__(kColsCluster, 1, 1) __launch_bounds__(256)
 // tid + 256 i in registers, so every score is read once and every exp is
 // evaluated once; the maximum and the sum are block reductions.
 constexpr int kSmThreads = 256;
+// Four rows per SM at once (at most 64 registers a thread): a row's block waits
+// on its score loads and its two reductions, and more resident rows hide
+// that (measured on the 32-head, 4096-token step: 3.96 -> 3.03 ms with three
+// rows resident before).
+constexpr int kSmBlocks = 4;
 constexpr int kSmPer = 32 * kBlockM / kSmThreads;  // S <= 32 blocks of 128 columns
 
 __device__ __forceinline__ double warp_sum_d(double v) {
@@ -162,7 +167,7 @@ __device__ __forceinline__ double warp_sum_d(double v) {
   return v;
 }
 
-__global__ void __launch_bounds__(kSmThreads) masked_softmax_kernel(const float* __restrict__ sc, float* __restrict__ pr,
+__global__ void __launch_bounds__(kSmThreads, kSmBlocks) masked_softmax_kernel(const float* __restrict__ sc, float* __restrict__ pr,
                                                                     int64_t S, const __grid_constant__ BlockMask mk) {
   __shared__ float s_max[kSmThreads / 32];
   __shared__ double s_sum[kSmThreads / 32];
