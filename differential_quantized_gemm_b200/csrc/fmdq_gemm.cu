@@ -814,13 +814,15 @@ __global__ void __launch_bounds__(kGThreads, 1)
 
       // this CTA's token tiles whose operands need more than two planes: the
       // slice stream, one output column per epilogue thread, after this
-      // tile's TMA stores have completed
-      if (ok && bi.any_slice) {
+      // tile's TMA stores have completed.  Whether the barrier runs depends
+      // on the block info alone, the same in every warp, so a warp whose wait
+      // gave up (ok == 0) still takes it.
+      if (bi.any_slice) {
         if (lane == 0) bulk_wait<0>();
         __syncwarp();
         epi_barrier();
         const int t0 = row_of(rb) / kTile;
-        for (int t = t0; t < min(t0 + kBlockM / kTile, T); ++t) {
+        for (int t = ok ? t0 : T; t < min(t0 + kBlockM / kTile, T); ++t) {
           if (p.planes[t] <= 2) continue;
           for (int c = etid; c < BN; c += 32 * kEpiWarps) {
             const int64_t n = n_base + c;
